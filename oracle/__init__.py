@@ -1,0 +1,312 @@
+"""fp64 CPU oracle for CSA / HCA -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, the smoke check and the benchmark's CPU-baseline leg may import
+this package.  It shares no code with the CUDA library and never imports it.
+
+The arithmetic lives in hcsa_oracle.c (plain loops in double precision, see
+its header for the definitions and the passages they follow).  This module
+converts storage-format arrays to float64 (exact), runs the projections as a
+float64 library matmul, and assembles the per-query key lists:
+  * prefill: entries visible to query t are j < t // m (entry j is visible
+    iff m*j + m <= t); the raw window is tokens (t - window, t] inside [0, T);
+  * decode at position P (the new token): the cache holds entries formed by
+    tokens < P, the window ring holds token p in slot p % window and the gate /
+    indexer-key staging rings hold token p in slot p % width; the new token is
+    written into the rings first, an entry whose last token is P is formed,
+    and the query then sees entries j < P // m and tokens (P - window, P].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hcsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+ST_F64, ST_F32, ST_BF16 = 0, 1, 2
+
+_dp = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        V, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        lib.orc_round.argtypes = [V, I64, I]
+        lib.orc_compress.argtypes = [I64, I, I, I, V, I64, V, I64, V, V, I64, I, V, V, I]
+        lib.orc_pool_rows.argtypes = [I, I, V, I64, V, I64, V, I64, V, I]
+        lib.orc_index_scores.argtypes = [I, I, I, V, V, V, I64, V, V]
+        lib.orc_topk.argtypes = [I, V, I64, V, I, V, V, V]
+        lib.orc_attend.argtypes = [I, I, I, ctypes.c_double, V, I64, V, I, V, I, V, V, I64, V, I, V, I]
+        for f in ("orc_round", "orc_compress", "orc_pool_rows", "orc_index_scores", "orc_topk", "orc_attend"):
+            getattr(lib, f).restype = None
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def storage_code(dtype: str) -> int:
+    return {"f64": ST_F64, "f32": ST_F32, "bf16": ST_BF16}[dtype]
+
+
+def to_f64(a: np.ndarray) -> np.ndarray:
+    """Exact float64 value of a storage array (float32, float64 or bfloat16 bits as uint16)."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.asarray(a, dtype=np.float64)
+
+
+def round_to(a: np.ndarray, st: int) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float64).copy()
+    _load().orc_round(a.ctypes.data, a.size, st)
+    return a
+
+
+# ---------------------------------------------------------------- building blocks
+
+def project(x64: np.ndarray, W64: np.ndarray, st: int) -> np.ndarray:
+    """y = x W in float64 (library matmul), rounded to storage."""
+    return round_to(x64 @ W64, st)
+
+
+def compress(T, C, m, width, kv, ld_kv, g, ld_g, bias, ki, ld_ki, di, st, kv_base=None):
+    """Prefill pool over a sequence; kv/g/ki are float64 arrays (views via base + offsets)."""
+    N = -(-T // m)
+    entries = np.empty((N, C), np.float64)
+    idx = np.empty((N, di), np.float64) if ki is not None else None
+    _load().orc_compress(T, C, m, width, kv, ld_kv, g, ld_g, _p(bias), ki, ld_ki, di,
+                         _p(entries), _p(idx), st)
+    return entries, idx
+
+
+def pool_rows(kv_tok, g_tok, b_tok, nch, st):
+    n = kv_tok.shape[0]
+    out = np.empty(nch, np.float64)
+    kv_tok, g_tok, b_tok = (np.ascontiguousarray(a, np.float64) for a in (kv_tok, g_tok, b_tok))
+    _load().orc_pool_rows(n, nch, _p(kv_tok), kv_tok.shape[1], _p(g_tok), g_tok.shape[1], _p(b_tok),
+                          b_tok.shape[1], _p(out), st)
+    return out
+
+
+def index_scores(qi, w, keys, n_vis, Hi, di):
+    qi = np.ascontiguousarray(qi, np.float64)
+    w = np.ascontiguousarray(w, np.float64)
+    keys = np.ascontiguousarray(keys, np.float64)
+    n_vis = np.ascontiguousarray(n_vis, np.int64)
+    nq, N = qi.shape[0], keys.shape[0]
+    s = np.empty((nq, N), np.float64)
+    _load().orc_index_scores(nq, Hi, di, _p(qi), _p(w), _p(keys), N, _p(n_vis), _p(s))
+    return s
+
+
+def topk(scores, n_vis, k):
+    scores = np.ascontiguousarray(scores, np.float64)
+    n_vis = np.ascontiguousarray(n_vis, np.int64)
+    nq, N = scores.shape
+    sel = np.empty((nq, k), np.int32)
+    gap = np.empty(nq, np.float64)
+    kth = np.empty(nq, np.float64)
+    _load().orc_topk(nq, _p(scores), N, _p(n_vis), k, _p(sel), _p(gap), _p(kth))
+    return sel, gap, kth
+
+
+def attend(q, H, dh, scale, entries, sel, n_vis, raw, win_rows, st):
+    """q[nq, H*dh]; entries[N, C]; sel[nq, k] (or None => all j < n_vis); raw[R, >=C]; win_rows[nq, w]."""
+    q = np.ascontiguousarray(q, np.float64)
+    entries = np.ascontiguousarray(entries, np.float64)
+    raw = np.ascontiguousarray(raw, np.float64)
+    win_rows = np.ascontiguousarray(win_rows, np.int64)
+    nq = q.shape[0]
+    C = entries.shape[1] if entries.ndim == 2 and entries.shape[0] else 2 * dh
+    if entries.size == 0:
+        entries = np.zeros((1, C), np.float64)
+    out = np.empty((nq, H * dh), np.float64)
+    if sel is not None:
+        sel = np.ascontiguousarray(sel, np.int32)
+        nsel = sel.shape[1]
+        nv = None
+    else:
+        nsel = 0
+        nv = np.ascontiguousarray(n_vis, np.int64)
+    _load().orc_attend(nq, H, dh, float(scale), _p(q), q.shape[1], _p(entries), C, _p(sel), nsel, _p(nv),
+                       _p(raw), raw.shape[1], _p(win_rows), win_rows.shape[1], _p(out), st)
+    return out
+
+
+def prefill_window_rows(tpos, window):
+    tpos = np.asarray(tpos, np.int64)
+    r = tpos[:, None] - window + 1 + np.arange(window, dtype=np.int64)[None, :]
+    return np.where(r >= 0, r, -1)
+
+
+def prefill_n_vis(tpos, m, N):
+    return np.minimum(np.asarray(tpos, np.int64) // m, N)
+
+
+# ---------------------------------------------------------------- whole layer
+
+def _col_slices(spec):
+    cols, off = {}, 0
+    names = [("kv", spec.C), ("g", spec.C)]
+    if spec.kind == "csa":
+        names += [("ki", spec.di), ("qi", spec.Hi * spec.di), ("w", spec.Hi)]
+    names += [("q", spec.H * spec.dh)]
+    for n, w in names:
+        cols[n] = slice(off, off + w)
+        off += w
+    return cols
+
+
+def prefill(spec, inp, rows=None, chunk=8192):
+    """Run the whole layer on the oracle.
+
+    inp: storage arrays x[T,D], W_cat[D,ncat], B[width,C] (as produced by synth).
+    rows: query positions to evaluate (default: all).  Entries are always built
+    for the whole sequence.  Returns a dict of float64 arrays."""
+    st = storage_code(spec.dtype)
+    T, C, m = spec.T, spec.C, spec.m
+    cols = _col_slices(spec)
+    W = to_f64(inp["W_cat"])
+    B = to_f64(inp["B"])
+    csa = spec.kind == "csa"
+    pool_end = cols["ki"].stop if csa else cols["g"].stop
+    W_pool = np.ascontiguousarray(W[:, :pool_end])
+    ypool = np.empty((T, pool_end), np.float64)
+    for a in range(0, T, chunk):
+        ypool[a:a + chunk] = project(to_f64(inp["x"][a:a + chunk]), W_pool, st)
+    ld = pool_end
+    base = ypool.ctypes.data
+    ki_ptr = base + 8 * cols["ki"].start if csa else None
+    entries, idx = compress(T, C, m, spec.width, base, ld, base + 8 * C, ld, B, ki_ptr, ld,
+                            spec.di if csa else 0, st)
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    W_q = np.ascontiguousarray(W[:, pool_end:])
+    yq = project(to_f64(inp["x"][rows]), W_q, st)
+    off = pool_end
+    qcols = {n: slice(s.start - off, s.stop - off) for n, s in cols.items() if s.start >= off}
+    res = {"y_pool": ypool, "entries": entries, "idx_keys": idx, "rows": rows, "y_q": yq}
+    N = entries.shape[0]
+    n_vis = prefill_n_vis(rows, m, N)
+    res["n_vis"] = n_vis
+    if csa:
+        scores = index_scores(yq[:, qcols["qi"]], yq[:, qcols["w"]], idx, n_vis, spec.Hi, spec.di)
+        sel, gap, kth = topk(scores, n_vis, spec.topk)
+        res.update(scores=scores, sel=sel, gap=gap, kth=kth)
+    else:
+        sel = None
+    res["out"] = attend_rows(spec, res, yq[:, qcols["q"]], sel)
+    res["q"] = yq[:, qcols["q"]]
+    return res
+
+
+def attend_rows(spec, res, q, sel):
+    """Attention for res['rows'] given a selection (None = HCA dense); raw window = projected kv."""
+    st = storage_code(spec.dtype)
+    rows = res["rows"]
+    ypool = res["y_pool"]
+    win = prefill_window_rows(rows, spec.window)
+    return attend(q, spec.H, spec.dh, spec.scale, res["entries"], sel, res["n_vis"], ypool, win, st)
+
+
+def decode_step(spec, inp, P, seqs=None):
+    """One decode step of one layer for the sequences in `inp` (all at position P).
+
+    inp: storage arrays from synth.decode_inputs: W_cat, B, x[Ball, D] and the cache
+    for the selected sequences (entries[b,N,C], idx_keys[b,N,di], win_kv[b,win,C],
+    ring_g[b,width,C], ring_ki[b,width,di]).  seqs maps cache row b -> x row.
+    Returns dict with the updated rings/entries (float64) and per-sequence outputs."""
+    st = storage_code(spec.dtype)
+    csa = spec.kind == "csa"
+    m, Wd, win, C = spec.m, spec.width, spec.window, spec.C
+    if win < Wd:
+        raise ValueError("the window ring also stages the kv rows of the open pool: window >= width")
+    cols = _col_slices(spec)
+    nb = inp["entries"].shape[0]
+    seqs = list(range(nb)) if seqs is None else list(seqs)
+    x = to_f64(inp["x"][seqs])
+    y = project(x, to_f64(inp["W_cat"]), st)
+    Bm = to_f64(inp["B"])
+    entries = to_f64(inp["entries"])
+    win_kv = to_f64(inp["win_kv"]).copy()
+    ring_g = to_f64(inp["ring_g"]).copy()
+    idx = to_f64(inp["idx_keys"]) if csa else None
+    ring_ki = to_f64(inp["ring_ki"]).copy() if csa else None
+    Ncap = entries.shape[1]
+    new_entry = {}
+    outs, sels, gaps, scores_all = [], [], [], []
+    for b in range(nb):
+        yb = y[b]
+        win_kv[b, P % win] = yb[cols["kv"]]
+        ring_g[b, P % Wd] = yb[cols["g"]]
+        if csa:
+            ring_ki[b, P % Wd] = yb[cols["ki"]]
+        ent_b = entries[b]
+        idx_b = idx[b] if csa else None
+        if (P + 1) % m == 0:
+            j = (P + 1) // m - 1
+            lo = m * j - (Wd - m)
+            toks = [i for i in range(lo, m * j + m) if i >= 0]
+            kv_t = np.stack([win_kv[b, i % win] for i in toks])
+            g_t = np.stack([ring_g[b, i % Wd] for i in toks])
+            b_t = np.stack([Bm[i - lo] for i in toks])
+            e = pool_rows(kv_t, g_t, b_t, C, st)
+            new = {"j": j, "entry": e}
+            if csa:
+                ki_t = np.stack([ring_ki[b, i % Wd] for i in toks])
+                new["idx_key"] = pool_rows(ki_t, g_t, b_t, spec.di, st)
+            if j < Ncap:
+                ent_b = ent_b.copy()
+                ent_b[j] = e
+                if csa:
+                    idx_b = idx_b.copy()
+                    idx_b[j] = new["idx_key"]
+            new_entry[b] = new
+        n_vis = np.array([min(P // m, Ncap)], np.int64)
+        if csa:
+            sc = index_scores(yb[cols["qi"]][None], yb[cols["w"]][None], idx_b, n_vis, spec.Hi, spec.di)
+            sel, gap, kth = topk(sc, n_vis, spec.topk)
+            sels.append(sel[0])
+            gaps.append(gap[0])
+            scores_all.append(sc[0])
+        else:
+            sel = None
+        pos = P - win + 1 + np.arange(win)
+        wrows = np.where(pos >= 0, pos % win, -1)[None, :]
+        outs.append(attend(yb[cols["q"]][None], spec.H, spec.dh, spec.scale, ent_b, sel, n_vis,
+                           win_kv[b], wrows, st)[0])
+    res = {"y": y, "out": np.stack(outs), "win_kv": win_kv, "ring_g": ring_g, "new_entry": new_entry}
+    if csa:
+        res.update(sel=np.stack(sels), gap=np.array(gaps), scores=np.stack(scores_all), ring_ki=ring_ki)
+    return res
+
+
+def decode_attend_with_sel(spec, res, inp, P, sel_b, b):
+    """Recompute sequence b's decode output on a given selection (e.g. the GPU's)."""
+    st = storage_code(spec.dtype)
+    win = spec.window
+    cols = _col_slices(spec)
+    ent = to_f64(inp["entries"][b])
+    if b in res["new_entry"] and res["new_entry"][b]["j"] < ent.shape[0]:
+        ent = ent.copy()
+        ent[res["new_entry"][b]["j"]] = res["new_entry"][b]["entry"]
+    pos = P - win + 1 + np.arange(win)
+    wrows = np.where(pos >= 0, pos % win, -1)[None, :]
+    return attend(res["y"][b][cols["q"]][None], spec.H, spec.dh, spec.scale, ent, sel_b[None], None,
+                  res["win_kv"][b], wrows, st)[0]

@@ -1,0 +1,365 @@
+"""Pins for the CPU oracle: each oracle function is checked against something
+other than itself -- closed forms, special cases that reduce to a library
+routine (numpy, torch scaled_dot_product_attention), and brute force on tiny
+inputs.  CPU only."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+ST64 = 0
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ------------------------------------------------------------------ storage rounding
+
+def test_round_fp32_matches_numpy_cast(orc):
+    x = rng(0).standard_normal(10000) * 10.0 ** rng(1).integers(-20, 20, 10000)
+    np.testing.assert_array_equal(orc.round_to(x, orc.ST_F32), x.astype(np.float32).astype(np.float64))
+
+
+def test_round_bf16_matches_torch_on_float32_inputs(orc):
+    # values exactly representable in float32: torch's float32 -> bfloat16 cast is RNE
+    x = rng(2).standard_normal(20000).astype(np.float32)
+    x[:8] = [1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, -2.5, 1 + 2 ** -9, 255.5, 2 ** -130, -0.0]
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.round_to(x.astype(np.float64), orc.ST_BF16), ref)
+
+
+def test_round_bf16_ties_to_even(orc):
+    got = orc.round_to(np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -30]), orc.ST_BF16)
+    np.testing.assert_array_equal(got, [1.0, 1 + 2 ** -6, 1 + 2 ** -7])
+
+
+# ------------------------------------------------------------------ compressor
+
+def _compress(orc, kv, g, B, m, W, ki=None, st=ST64):
+    T, C = kv.shape
+    kv = np.ascontiguousarray(kv, np.float64)
+    g = np.ascontiguousarray(g, np.float64)
+    B = np.ascontiguousarray(B, np.float64)
+    di = ki.shape[1] if ki is not None else 0
+    kip = np.ascontiguousarray(ki, np.float64) if ki is not None else None
+    return orc.compress(T, C, m, W, kv.ctypes.data, C, g.ctypes.data, C, B,
+                        None if kip is None else kip.ctypes.data, di, di, st)
+
+
+@pytest.mark.parametrize("m,W,T", [(4, 8, 37), (128, 128, 300), (4, 8, 4), (2, 6, 9)])
+def test_compress_constant_gate_is_plain_mean(orc, m, W, T):
+    r = rng(3)
+    C = 6
+    kv = r.standard_normal((T, C))
+    g = np.zeros((T, C))
+    B = np.tile(r.standard_normal(C), (W, 1))          # constant along the pool axis
+    ent, _ = _compress(orc, kv, g, B, m, W)
+    N = -(-T // m)
+    assert ent.shape == (N, C)
+    for j in range(N):
+        lo, hi = max(m * j - (W - m), 0), min(m * j + m, T)
+        np.testing.assert_allclose(ent[j], kv[lo:hi].mean(axis=0), rtol=1e-13, atol=1e-14)
+
+
+def test_compress_width_one_is_identity(orc):
+    r = rng(4)
+    kv, g = r.standard_normal((50, 5)), r.standard_normal((50, 5))
+    ent, _ = _compress(orc, kv, g, r.standard_normal((1, 5)), 1, 1)
+    np.testing.assert_array_equal(ent, kv)
+
+
+def test_compress_bias_row_offset_and_edge_truncation(orc):
+    # one bias row dominates: entry j must equal the token at pool position r0,
+    # i.e. token m*j - (W-m) + r0, whenever that token lies inside [0, T)
+    m, W, T, C = 4, 8, 30, 3
+    r = rng(5)
+    kv, g = r.standard_normal((T, C)), np.zeros((T, C))
+    for r0 in range(W):
+        B = np.zeros((W, C))
+        B[r0] = 60.0
+        ent, _ = _compress(orc, kv, g, B, m, W)
+        for j in range(-(-T // m)):
+            tok = m * j - (W - m) + r0
+            lo, hi = max(m * j - (W - m), 0), min(m * j + m, T)
+            if lo <= tok < hi:
+                np.testing.assert_allclose(ent[j], kv[tok], rtol=1e-20, atol=1e-20)
+            else:   # dominating row outside the sequence: plain mean of the truncated pool
+                np.testing.assert_allclose(ent[j], kv[lo:hi].mean(axis=0), rtol=1e-12)
+
+
+def test_compress_is_per_channel_and_in_convex_hull(orc):
+    r = rng(6)
+    m, W, T, C = 4, 8, 64, 16
+    kv, g, B = r.standard_normal((T, C)), r.standard_normal((T, C)), r.standard_normal((W, C))
+    ent, _ = _compress(orc, kv, g, B, m, W)
+    for j in range(T // m):
+        lo, hi = max(m * j - 4, 0), m * j + 4
+        assert np.all(ent[j] <= kv[lo:hi].max(0) + 1e-12) and np.all(ent[j] >= kv[lo:hi].min(0) - 1e-12)
+    # shifting B by a per-channel constant changes nothing
+    ent2, _ = _compress(orc, kv, g, B + r.standard_normal(C)[None, :], m, W)
+    np.testing.assert_allclose(ent2, ent, rtol=1e-12, atol=1e-13)
+    # a gate that singles out one token in one channel only moves that channel
+    g2 = g.copy()
+    g2[9, 3] = 80.0
+    ent3, _ = _compress(orc, kv, g2, B, m, W)
+    j_hit = [j for j in range(T // m) if max(m * j - 4, 0) <= 9 < m * j + 4]
+    for j in j_hit:
+        assert ent3[j, 3] == pytest.approx(kv[9, 3], abs=1e-20)
+    mask = np.ones_like(ent, bool)
+    mask[j_hit, 3] = False
+    np.testing.assert_array_equal(ent3[mask], ent[mask])
+
+
+def test_indexer_keys_use_gate_channels_below_di(orc):
+    # the indexer-key pool reuses the gate of channel d for key dim d
+    m, W, T, C, di = 4, 8, 40, 8, 3
+    r = rng(7)
+    kv, ki = r.standard_normal((T, C)), r.standard_normal((T, di))
+    g = np.zeros((T, C))
+    for d in range(C):
+        g[10 + d, d] = 70.0        # channel d is dominated by token 10 + d
+    _, idx = _compress(orc, kv, g, np.zeros((W, C)), m, W, ki=ki)
+    for j in range(T // m):
+        lo, hi = max(m * j - 4, 0), min(m * j + 4, T)
+        for d in range(di):
+            tok = 10 + d
+            if lo <= tok < hi:
+                assert idx[j, d] == pytest.approx(ki[tok, d], abs=1e-20)
+            else:
+                assert idx[j, d] == pytest.approx(ki[lo:hi, d].mean(), rel=1e-12)
+
+
+# ------------------------------------------------------------------ indexer
+
+def test_indexer_one_head_unit_weight_is_relu_dot(orc):
+    r = rng(8)
+    q, k = r.standard_normal((5, 7)), r.standard_normal((11, 7))
+    s = orc.index_scores(q, np.ones((5, 1)), k, np.full(5, 11), 1, 7)
+    np.testing.assert_allclose(s, np.maximum(q @ k.T, 0.0), rtol=1e-13, atol=1e-14)
+
+
+def test_indexer_linear_in_head_weights_and_one_hot(orc):
+    # s is linear in w and equals relu(q_h . k) for w = e_h: together these fix the formula
+    r = rng(9)
+    Hi, di, N, nq = 4, 6, 20, 3
+    qi, k = r.standard_normal((nq, Hi * di)), r.standard_normal((N, di))
+    nv = np.full(nq, N)
+    w1, w2 = r.standard_normal((nq, Hi)), r.standard_normal((nq, Hi))
+    s = lambda w: orc.index_scores(qi, w, k, nv, Hi, di)
+    np.testing.assert_allclose(s(w1 + 2.5 * w2), s(w1) + 2.5 * s(w2), rtol=1e-12, atol=1e-12)
+    for h in range(Hi):
+        e = np.zeros((nq, Hi))
+        e[:, h] = 1.0
+        np.testing.assert_allclose(s(e), np.maximum(qi[:, h * di:(h + 1) * di] @ k.T, 0), rtol=1e-13,
+                                   atol=1e-14)
+
+
+def test_indexer_visibility(orc):
+    r = rng(10)
+    s = orc.index_scores(r.standard_normal((3, 8)), r.standard_normal((3, 2)), r.standard_normal((9, 4)),
+                         np.array([0, 4, 9]), 2, 4)
+    assert np.isnan(s[0]).all() and np.isnan(s[1, 4:]).all() and not np.isnan(s[1, :4]).any()
+    assert not np.isnan(s[2]).any()
+
+
+# ------------------------------------------------------------------ top-k
+
+def _lexsort_topk(s, n, k):
+    idx = np.lexsort((np.arange(n), -s[:n]))[:k]      # primary: score desc, secondary: index asc
+    return np.sort(idx)
+
+
+def test_topk_matches_lexsort_with_ties_and_signed_zero(orc):
+    r = rng(11)
+    nq, N, k = 40, 300, 17
+    s = r.integers(-5, 6, (nq, N)).astype(np.float64)     # many exact ties
+    s[s == 0] = np.where(r.random((s == 0).sum()) < 0.5, -0.0, 0.0)
+    nv = r.integers(0, N + 1, nq)
+    nv[:3] = [0, 5, k]
+    sel, gap, kth = orc.topk(s, nv, k)
+    for q in range(nq):
+        n = nv[q]
+        exp = _lexsort_topk(s[q], n, k)
+        np.testing.assert_array_equal(sel[q, :len(exp)], exp)
+        assert (sel[q, len(exp):] == -1).all()
+        if n > k:
+            srt = np.sort(s[q, :n])[::-1]
+            assert kth[q] == srt[k - 1]
+
+
+def test_topk_brute_force_subsets(orc):
+    r = rng(12)
+    for trial in range(30):
+        n, k = int(r.integers(1, 11)), int(r.integers(1, 5))
+        s = r.integers(-3, 4, n).astype(np.float64)
+        best = None
+        for sub in itertools.combinations(range(n), min(k, n)):
+            key = (-sum(s[list(sub)]), sub)
+            best = key if best is None or key < best else best
+        sel, _, _ = orc.topk(s[None, :], np.array([n]), k)
+        assert tuple(sel[0, :min(k, n)]) == best[1]
+
+
+# ------------------------------------------------------------------ attention
+
+def _sdpa(q, K, V, mask_bias, scale):
+    """torch SDPA in float64: q[H, d], K/V[n, d], mask_bias[n] added to the logits."""
+    qt = torch.from_numpy(q)[None, :, None, :]             # [1, H, 1, d]
+    Kt = torch.from_numpy(K)[None, None].expand(1, q.shape[0], -1, -1)
+    Vt = torch.from_numpy(V)[None, None].expand(1, q.shape[0], -1, -1)
+    bias = torch.from_numpy(mask_bias)[None, None, None, :]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=bias, scale=scale)
+    return o[0, :, 0, :].numpy()
+
+
+def _layer_inputs(r, T, C):
+    return r.standard_normal((T, C))
+
+
+@pytest.mark.parametrize("window", [128, 5])
+def test_attention_before_first_entry_is_window_attention(orc, window):
+    # t < m: no compressed entry is visible, only the causal raw window remains
+    r = rng(13)
+    T, H, dh = 4, 3, 8
+    kv = r.standard_normal((T, 2 * dh))
+    q = r.standard_normal((T, H * dh))
+    ent = r.standard_normal((1, 2 * dh))
+    win = orc.prefill_window_rows(np.arange(T), window)
+    out = orc.attend(q, H, dh, 0.3, ent, None, np.zeros(T, np.int64), kv, win, ST64)
+    for t in range(T):
+        bias = np.array([0.0 if max(0, t - window + 1) <= i <= t else -np.inf for i in range(T)])
+        ref = _sdpa(q[t].reshape(H, dh), kv[:, :dh], kv[:, dh:], bias, 0.3)
+        np.testing.assert_allclose(out[t].reshape(H, dh), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_hca_m1_zero_gate_is_full_attention_with_duplicate_bias(orc):
+    # m = 1, width 1, zero gate: entries are the raw tokens, entries j < t are visible,
+    # so tokens (t - win, t) appear twice: full causal attention with +ln 2 on them
+    r = rng(14)
+    T, H, dh, win = 40, 2, 4, 6
+    kv = r.standard_normal((T, 2 * dh))
+    q = r.standard_normal((T, H * dh))
+    ent, _ = _compress(orc, kv, np.zeros_like(kv), np.zeros((1, 2 * dh)), 1, 1)
+    nvis = orc.prefill_n_vis(np.arange(T), 1, T)
+    out = orc.attend(q, H, dh, 0.5, ent, None, nvis, kv, orc.prefill_window_rows(np.arange(T), win), ST64)
+    for t in range(T):
+        bias = np.full(T, -np.inf)
+        bias[:t + 1] = 0.0
+        lo = max(0, t - win + 1)
+        bias[lo:t] = math.log(2.0)
+        ref = _sdpa(q[t].reshape(H, dh), kv[:, :dh], kv[:, dh:], bias, 0.5)
+        np.testing.assert_allclose(out[t].reshape(H, dh), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_on_selection_matches_masked_sdpa(orc):
+    r = rng(15)
+    T, N, H, dh, win, k = 30, 9, 3, 4, 5, 4
+    kv = r.standard_normal((T, 2 * dh))
+    ent = r.standard_normal((N, 2 * dh))
+    q = r.standard_normal((T, H * dh))
+    sel = np.full((T, k), -1, np.int32)
+    for t in range(T):
+        c = np.sort(r.choice(N, size=int(r.integers(0, k + 1)), replace=False))
+        sel[t, :len(c)] = c
+    out = orc.attend(q, H, dh, 0.7, ent, sel, None, kv, orc.prefill_window_rows(np.arange(T), win), ST64)
+    K = np.concatenate([ent, kv])
+    for t in range(T):
+        bias = np.full(N + T, -np.inf)
+        bias[sel[t][sel[t] >= 0]] = 0.0
+        bias[N + max(0, t - win + 1):N + t + 1] = 0.0
+        ref = _sdpa(q[t].reshape(H, dh), K[:, :dh], K[:, dh:], bias, 0.7)
+        np.testing.assert_allclose(out[t].reshape(H, dh), ref, rtol=1e-12, atol=1e-13)
+
+
+def _small_csa(T=64, dtype="f32", topk=4, **kw):
+    import synth
+    base = dict(kind="csa", T=T, D=32, m=4, width=8, C=16, di=4, Hi=2, topk=topk, window=8, H=2, dh=8,
+                scale=0.35, dtype=dtype, seed=5)
+    base.update(kw)
+    return synth.LayerSpec(**base)
+
+
+def test_csa_with_k_at_least_visible_equals_dense_compressed_attention(orc):
+    import synth
+    spec = _small_csa(T=48, topk=64)
+    inp = synth.prefill_inputs(spec)
+    res = orc.prefill(spec, inp)
+    dense = orc.attend_rows(spec, res, res["q"], None)
+    np.testing.assert_array_equal(res["out"], dense)
+
+
+def test_csa_layer_small_against_masked_sdpa(orc):
+    # whole layer on a tiny sequence: attention output equals SDPA over [entries; raw tokens]
+    # with the selection and the causal window as the mask
+    import synth
+    spec = _small_csa(T=64, dtype="f32")
+    inp = synth.prefill_inputs(spec)
+    res = orc.prefill(spec, inp)
+    st = orc.ST_F32
+    ent, kv = res["entries"], res["y_pool"][:, :spec.C]
+    N, T, dh = ent.shape[0], spec.T, spec.dh
+    K = np.concatenate([ent, kv])
+    for t in range(T):
+        bias = np.full(N + T, -np.inf)
+        s = res["sel"][t]
+        bias[s[s >= 0]] = 0.0
+        bias[N + max(0, t - spec.window + 1):N + t + 1] = 0.0
+        ref = _sdpa(res["q"][t].reshape(spec.H, dh), K[:, :dh], K[:, dh:], bias, spec.scale)
+        np.testing.assert_allclose(res["out"][t], orc.round_to(ref.reshape(-1), st), rtol=0, atol=2e-7)
+        assert (s[s >= 0] < t // spec.m).all()
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_decode_steps_match_prefill(orc, kind):
+    """Decode at positions P..P+n-1 over a cache built from a prefill of P tokens reproduces the
+    prefill of P+n tokens (outputs, selections and newly completed entries)."""
+    import synth
+    if kind == "csa":
+        spec = _small_csa(T=0, dtype="f32")
+        P0, n = 37, 6
+    else:
+        spec = synth.LayerSpec(kind="hca", T=0, D=32, m=16, width=16, C=16, window=16, H=2, dh=8, scale=0.35,
+                               dtype="f32", seed=6)
+        P0, n = 29, 5
+    full = spec.replace(T=P0 + n)
+    inp = synth.prefill_inputs(full)
+    ref = orc.prefill(full, inp)
+    cols = orc._col_slices(spec)
+    m, W, win = spec.m, spec.width, spec.window
+    ypool = ref["y_pool"]
+    for step in range(n):
+        P = P0 + step
+        nc = P // m
+        ncap = nc + 2
+        cache = {"W_cat": inp["W_cat"], "B": inp["B"], "x": inp["x"][P:P + 1]}
+        ent = np.zeros((1, ncap, spec.C), np.float32)
+        ent[0, :nc] = ref["entries"][:nc]
+        cache["entries"] = ent
+        wk = np.zeros((1, win, spec.C), np.float32)
+        rg = np.zeros((1, W, spec.C), np.float32)
+        for p in range(max(0, P - win), P):
+            wk[0, p % win] = ypool[p, cols["kv"]]
+        for p in range(max(0, P - W), P):
+            rg[0, p % W] = ypool[p, cols["g"]]
+        cache["win_kv"], cache["ring_g"] = wk, rg
+        if kind == "csa":
+            ik = np.zeros((1, ncap, spec.di), np.float32)
+            ik[0, :nc] = ref["idx_keys"][:nc]
+            rk = np.zeros((1, W, spec.di), np.float32)
+            for p in range(max(0, P - W), P):
+                rk[0, p % W] = ypool[p, cols["ki"]]
+            cache["idx_keys"], cache["ring_ki"] = ik, rk
+        d = orc.decode_step(spec, cache, P)
+        np.testing.assert_allclose(d["out"][0], ref["out"][P], rtol=0, atol=1e-6)
+        if kind == "csa":
+            np.testing.assert_array_equal(d["sel"][0], ref["sel"][P])
+        if (P + 1) % m == 0:
+            j = (P + 1) // m - 1
+            np.testing.assert_allclose(d["new_entry"][0]["entry"], ref["entries"][j], rtol=0, atol=1e-6)
+        else:
+            assert 0 not in d["new_entry"]
