@@ -1,0 +1,493 @@
+"""Benchmark of the hybrid compressed attention path on B200.
+
+Default workload: one CSA layer prefill, bf16, T=131072, D=2048 (projection + compressor + lightning
+indexer/top-k + attention), inputs resident in HBM.  `value` is tokens/s over all ranks (each rank runs
+its own independent sequence: weak scaling, no collective on the data path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Other workloads (--workload): hca_prefill_T65536, csa_decode_B32_P262144, hybrid_decode_B4_P1048576.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "CSA/HCA prefill tokens/s and decode µs/step at 128K-1M ctx; % of HBM/TC roofline"
+
+WORKLOADS = {
+    "csa_prefill_T131072": ("prefill", "csa_bf16_t131072"),
+    "hca_prefill_T65536": ("prefill", "hca_bf16_t65536"),
+    "csa_decode_B32_P262144": ("decode", "csa_decode_b32_p262144"),
+    "hybrid_decode_B4_P1048576": ("decode", "hybrid_decode_b4_p1048576"),
+}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic work per call
+
+def prefill_work(spec):
+    """Algorithmic flops / bytes of each call of a prefill layer (visible pairs only)."""
+    T, m, k, win = spec.T, spec.m, spec.topk, spec.window
+    t = np.arange(T, dtype=np.float64)
+    vis = np.minimum(t // m, -(-T // m))
+    nwin = np.minimum(win, t + 1)
+    bpe = 2 if spec.dtype == "bf16" else 4
+    w = {}
+    ncols = 2 * spec.C + spec.H * spec.dh + (spec.di + spec.Hi * spec.di + spec.Hi if spec.kind == "csa" else 0)
+    w["hcsa_project"] = {"flops": 2.0 * T * spec.D * ncols}
+    N = -(-T // m)
+    pool_ch = spec.C + (spec.di if spec.kind == "csa" else 0)
+    w["compress"] = {"bytes": float(T * (2 * spec.C + (spec.di if spec.kind == "csa" else 0)) * bpe
+                                    + N * pool_ch * bpe)}
+    if spec.kind == "csa":
+        w["csa_index_topk"] = {"flops": float(vis.sum()) * spec.Hi * spec.di * 2.0}
+        nkeys = np.minimum(vis, k) + nwin
+    else:
+        nkeys = vis + nwin
+    w["attend"] = {"flops": float(nkeys.sum()) * spec.H * spec.dh * 4.0}
+    return w
+
+
+def decode_bytes(spec, B, N):
+    """Algorithmic HBM bytes of one decode step of one layer (weights + cache reads + writes)."""
+    bpe = 2
+    ncols = 2 * spec.C + spec.H * spec.dh + (spec.di + spec.Hi * spec.di + spec.Hi if spec.kind == "csa" else 0)
+    b = spec.D * ncols * bpe                                   # weights
+    if spec.kind == "csa":
+        b += B * N * spec.di * bpe                             # indexer key scan
+        b += B * (spec.topk + spec.window) * spec.C * bpe      # selected rows + window
+    else:
+        b += B * (N + spec.window) * spec.C * bpe              # all entries + window
+    b += B * spec.H * spec.dh * bpe * 2                        # q in, out
+    return float(b)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    def __init__(self, dev_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={dev_index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = sorted(sm)[len(sm) // 4:] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle timing (bounded sample)
+
+def oracle_prefill_rate(spec, inp, budget_rows=8):
+    """Oracle throughput (tokens/s) extrapolated from a bounded sample of the whole layer:
+    projection of 256 rows, the compressor over 1024 tokens, and index/top-k/attention for
+    `budget_rows` queries spread uniformly over the sequence."""
+    import oracle
+    st = oracle.storage_code(spec.dtype)
+    T = spec.T
+    W = oracle.to_f64(inp["W_cat"])
+    cols = oracle._col_slices(spec)
+    t0 = time.perf_counter()
+    nr = min(256, T)
+    y = oracle.project(oracle.to_f64(inp["x"][:nr]), W, st)
+    t_proj = (time.perf_counter() - t0) * T / nr
+    nt = min(1024, T)
+    t0 = time.perf_counter()
+    csa = spec.kind == "csa"
+    yp = np.ascontiguousarray(np.concatenate([y] * (-(-nt // nr)))[:nt])
+    base = yp.ctypes.data
+    oracle.compress(nt, spec.C, spec.m, spec.width, base, yp.shape[1], base + 8 * spec.C, yp.shape[1],
+                    oracle.to_f64(inp["B"]), base + 8 * cols["ki"].start if csa else None, yp.shape[1],
+                    spec.di if csa else 0, st)
+    t_comp = (time.perf_counter() - t0) * T / nt
+    # per-query work at uniformly spread positions, on synthetic stand-in rows of the right sizes
+    rows = ((np.arange(budget_rows) + 0.5) * T / budget_rows).astype(np.int64)
+    N = -(-T // spec.m)
+    rng = np.random.default_rng(0)
+    entries = rng.standard_normal((N, spec.C))
+    kvraw = rng.standard_normal((T, spec.C))
+    q = rng.standard_normal((budget_rows, spec.H * spec.dh))
+    nvis = np.minimum(rows // spec.m, N)
+    t0 = time.perf_counter()
+    if csa:
+        keys = rng.standard_normal((N, spec.di))
+        qi = rng.standard_normal((budget_rows, spec.Hi * spec.di))
+        w = rng.standard_normal((budget_rows, spec.Hi))
+        s = oracle.index_scores(qi, w, keys, nvis, spec.Hi, spec.di)
+        sel, _, _ = oracle.topk(s, nvis, spec.topk)
+    else:
+        sel = None
+    oracle.attend(q, spec.H, spec.dh, spec.scale, entries, sel, nvis, kvraw,
+                  oracle.prefill_window_rows(rows, spec.window), st)
+    t_q = (time.perf_counter() - t0) * T / budget_rows
+    total = t_proj + t_comp + t_q
+    sample = (f"projection of {nr} rows, compressor over {nt} tokens, indexer/top-k/attention for "
+              f"{budget_rows} queries spread over T={T}; whole-layer time extrapolated ({total:.1f} s)")
+    return T / total, sample
+
+
+def oracle_decode_rate(layers, B, N_list, P):
+    """Oracle µs/step from one sequence of each distinct layer shape, scaled to B sequences."""
+    import oracle
+    rng = np.random.default_rng(0)
+    total = 0.0
+    for spec, N in zip(layers, N_list):
+        st = oracle.storage_code(spec.dtype)
+        ncols = 2 * spec.C + spec.H * spec.dh + (spec.di + spec.Hi * spec.di + spec.Hi if spec.kind == "csa" else 0)
+        W = rng.standard_normal((spec.D, ncols))
+        x = rng.standard_normal((1, spec.D))
+        t0 = time.perf_counter()
+        y = oracle.project(x, W, st)
+        t_proj = time.perf_counter() - t0
+        entries = rng.standard_normal((N, spec.C))
+        win = rng.standard_normal((spec.window, spec.C))
+        nv = np.array([N], np.int64)
+        t0 = time.perf_counter()
+        if spec.kind == "csa":
+            keys = rng.standard_normal((N, spec.di))
+            s = oracle.index_scores(y[:, 2 * spec.C + spec.di:2 * spec.C + spec.di + spec.Hi * spec.di],
+                                    rng.standard_normal((1, spec.Hi)), keys, nv, spec.Hi, spec.di)
+            sel, _, _ = oracle.topk(s, nv, spec.topk)
+        else:
+            sel = None
+        wrows = (np.arange(spec.window, dtype=np.int64) % spec.window)[None]
+        oracle.attend(rng.standard_normal((1, spec.H * spec.dh)), spec.H, spec.dh, spec.scale, entries, sel, nv,
+                      win, wrows, st)
+        total += t_proj + (time.perf_counter() - t0) * B
+    return total * 1e6, f"one sequence per layer shape, N={N_list[0]} entries, scaled to B={B}"
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_prefill(args, spec_name, ws, rank):
+    import long_context_compressed_05_b200 as h
+    import synth
+    from tests._helpers import dev
+    spec = synth.PREFILL[spec_name]
+    if ws > 1:
+        spec = spec.replace(seed=spec.seed + 1000 * rank)   # independent sequence per rank
+    inp = synth.prefill_inputs(spec)
+    x, W, B = dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"])
+    layer = h.PrefillLayer(spec)
+    stream = torch.cuda.current_stream()
+    calls = ["hcsa_project", "compress"] + (["csa_index_topk"] if spec.kind == "csa" else []) + ["attend"]
+
+    def step(evs=None):
+        fns = [lambda: layer.project(x, W), lambda: layer.compress(B)]
+        if spec.kind == "csa":
+            fns.append(layer.index_topk)
+        fns.append(layer.attend)
+        for i, f in enumerate(fns):
+            if evs is not None:
+                evs[i][0].record(stream)
+            f()
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+           for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    barrier(ws)
+    torch.cuda.synchronize()
+    h.hcsa_launch_count(reset=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = h.hcsa_launch_count()
+    barrier(ws)
+    clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(e0.elapsed_time(e1), ws) / args.steps
+    phase_ms = {c: statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps))
+                for i, c in enumerate(calls)}
+    value = ws * spec.T / (ms / 1e3)
+    work = prefill_work(spec)
+    hbm, tc, tc_sus, src = peaks()
+    ours = {c: t for c, t in phase_ms.items() if c != "hcsa_project"}
+    dom = max(ours, key=ours.get)
+    wk = work[dom]
+    if "flops" in wk:
+        ach = wk["flops"] / (ours[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tc_sus, "unit": "TFLOP/s", "frac": ach / tc_sus,
+                "traffic": None, "kernel": dom, "peak_kind": f"{src} bf16 sustained"}
+    else:
+        ach = wk["bytes"] / (ours[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+                "kernel": dom, "peak_kind": f"{src} hbm"}
+    # end to end through the public API: pinned host x in, output back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        xh.copy_(x)
+        oh = torch.empty(layer.out.shape, dtype=layer.out.dtype, pin_memory=True)
+        ke = max(1, min(args.steps, 3))
+        torch.cuda.synchronize()
+        barrier(ws)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(ke):
+            x.copy_(xh, non_blocking=True)
+            layer.forward(x, W, B)
+            oh.copy_(layer.out, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(a0.elapsed_time(a1), ws) / ke
+        e2e = {"value": ws * spec.T / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size()}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, N(0,1/D) weights)",
+            "config": {"workload": f"{spec.kind}_prefill_bf16_T{spec.T}_D{spec.D}", "T": spec.T, "D": spec.D,
+                       "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh,
+                       "parallelism": f"replicas x{ws} (one sequence per GPU)",
+                       "l2": "inputs larger than L2 (x 0.5 GB, projections 9.7 GB)"},
+            "phase_ms": phase_ms, "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+    return line, (spec, inp)
+
+
+def run_decode(args, spec_name, ws, rank):
+    import long_context_compressed_05_b200 as h
+    import synth
+    from tests._helpers import dev
+    d = synth.DECODE[spec_name]
+    layers, Ws, Bs, xs = [], [], [], None
+    shared = {}
+    for li, spec in enumerate(d.layers):
+        inp = synth.decode_inputs(d, li)
+        cache = {k: dev(inp[k]) for k in ("entries", "win_kv", "ring_g", "idx_keys", "ring_ki") if k in inp}
+        n_cap = inp["entries"].shape[1]
+        layers.append(h.DecodeLayer(spec, d.B, n_cap, cache))
+        Ws.append(dev(inp["W_cat"]))
+        Bs.append(dev(inp["B"]))
+        if xs is None:
+            xs = dev(inp["x"])
+        del inp
+    pos = torch.full((d.B,), d.P, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for L, W, B in zip(layers, Ws, Bs):
+            L.step(xs, W, B, pos)   # each layer reads the same hidden state; pos is not advanced (idempotent)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    barrier(ws)
+    torch.cuda.synchronize()
+    h.hcsa_launch_count(reset=True)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = sampler.stop() if sampler else None
+    us = max_over_ranks(e0.elapsed_time(e1), ws) / args.steps * 1e3
+    # launches per step: count one eager step
+    h.hcsa_launch_count(reset=True)
+    step()
+    torch.cuda.synchronize()
+    launches = h.hcsa_launch_count() * args.steps
+    hbm, tc, tc_sus, src = peaks()
+    total_bytes = sum(decode_bytes(L.spec, d.B, L.p.n_cap) for L in layers)
+    ach = total_bytes / (us / 1e6) / 1e9
+    roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+            "kernel": "whole decode step (CUDA graph)", "peak_kind": f"{src} hbm"}
+    xh = torch.empty(xs.shape, dtype=xs.dtype, pin_memory=True)
+    xh.copy_(xs)
+    oh = torch.empty(layers[-1].out.shape, dtype=layers[-1].out.dtype, pin_memory=True)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        xs.copy_(xh, non_blocking=True)
+        g.replay()
+        oh.copy_(layers[-1].out, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    eus = max_over_ranks(a0.elapsed_time(a1), ws) / args.steps * 1e3
+    del g
+    line = {"metric": METRIC, "value": us, "unit": "us/step", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
+            "config": {"workload": spec_name, "B": d.B, "P": d.P, "layers": len(d.layers),
+                       "parallelism": f"replicas x{ws}", "l2": "working set larger than L2",
+                       "bytes_per_step": total_bytes},
+            "roofline": roof,
+            "e2e": {"value": eus, "unit": "us/step", "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                    "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+            "gpu_launches": launches, "clocks": clocks}
+    return line, (d, None)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="csa_prefill_T131072", choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    kind, name = WORKLOADS[args.workload]
+    ws, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import synth
+        cores = len(os.sched_getaffinity(0))
+        vals = []
+        if kind == "prefill":
+            spec = synth.PREFILL[name]
+            inp = synth.prefill_inputs(spec)
+            for i in range(args.warmup + args.steps):
+                v, sample = oracle_prefill_rate(spec, inp, budget_rows=4)
+                if i >= args.warmup:
+                    vals.append(v)
+            unit, hib = "tokens/s", True
+        else:
+            d = synth.DECODE[name]
+            Ns = [d.n_cache_entries(s) for s in d.layers]
+            for i in range(args.warmup + args.steps):
+                v, sample = oracle_decode_rate(list(d.layers), d.B, Ns, d.P)
+                if i >= args.warmup:
+                    vals.append(v)
+            unit, hib = "us/step", False
+        v = statistics.mean(vals)
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1,
+                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": hib,
+                          "dtype": "f64", "data": "synthetic", "config": {"workload": args.workload},
+                          "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+
+    if kind == "prefill":
+        line, (spec, inp) = run_prefill(args, name, ws, rank)
+    else:
+        line, (d, _) = run_decode(args, name, ws, rank)
+    if rank == 0:
+        if not args.no_cpu_baseline and ws == 1:
+            cores = len(os.sched_getaffinity(0))
+            if kind == "prefill":
+                v, sample = oracle_prefill_rate(spec, inp)
+                line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                        "sample": sample}
+            else:
+                Ns = [d.n_cache_entries(s) for s in d.layers]
+                v, sample = oracle_decode_rate(list(d.layers), d.B, Ns, d.P)
+                line["cpu_baseline"] = {"value": v, "unit": "us/step", "cores": cores, "kind": "oracle",
+                                        "sample": sample}
+        else:
+            line["cpu_baseline"] = None
+        print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

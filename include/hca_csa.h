@@ -1,0 +1,205 @@
+/*
+ * hca_csa.h -- C ABI of the B200 (sm_100a) hybrid compressed attention library.
+ *
+ * The operation is the attention layer of DeepSeek-V4 as described in
+ * "DeepSeek-V4: interleaved compressed attention with manifold-constrained
+ * hyper-connections" (TL;DR and the three-tier diagram: HCA 128-to-1, CSA
+ * 4-to-1 plus an indexer over a low-dimensional projection, an uncompressed
+ * recent window) and "DeepSeek-V4: ... KV cache ... compressed attention"
+ * (sections "CSA: compresion 4x mas recuperacion dispersa", "HCA: compresion
+ * 128x mas atencion densa", "Ventana deslizante"), with every step fixed as in
+ * the CSA fp32 T=2048 workload definition:
+ *
+ *   projections   kv = x W_kv, g = x W_g, ki = x W_ki, qi = x W_qi, w = x W_w, q = x W_q
+ *   compressor    entry j pools tokens i in [m j - (width - m), m j + m) within [0, T):
+ *                   c_j[c] = sum_i softmax_i(g[i,c] + B[i - m j + width - m, c]) kv[i,c]
+ *                 indexer key k_j[d] = the same pool over ki[i,d], gate channel d
+ *   indexer       s[t,j] = sum_h w[t,h] ReLU(qi[t,h,:] . k_j),  j visible iff m j + m <= t
+ *   top-k         the min(topk, visible) best s[t,j]; equal scores -> lower j first
+ *   attention     MQA over {selected entries} U {raw tokens (t - window, t]};
+ *                 key = first C/2 channels, value = last C/2; one softmax, scale tau
+ *   HCA           m = width = 128, every visible entry attended (no indexer)
+ *   decode        one new token per sequence over a compressed cache (the pages'
+ *                 problem statement: each decode step reads the past K/V)
+ *
+ * Conventions for every call
+ *   - All tensors are row-major and live in device memory owned by the caller.
+ *     The library allocates nothing (an internal cuBLAS handle per device is
+ *     the one exception, made on the first bf16 projection) and keeps one
+ *     device status word per device.
+ *   - Storage type is p->dtype: HCSA_F32 (fp32 storage; the kernels compute in
+ *     fp64) or HCSA_BF16 (bf16 storage; fp32 accumulation, tensor cores).
+ *   - Pointers must be 16-byte aligned; every leading dimension `ld_*` (in
+ *     elements) must keep rows 16-byte aligned.  Violations return
+ *     HCSA_ERR_ALIGN; wrong sizes return HCSA_ERR_SHAPE; a NULL tensor returns
+ *     HCSA_ERR_NULL; too little workspace returns HCSA_ERR_WORKSPACE.  Argument
+ *     errors are found on the host before anything is enqueued.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous, stream-ordered and deterministic.  Launch failures return
+ *     HCSA_ERR_CUDA.  Errors found by the kernels themselves (bounded waits
+ *     that gave up, out-of-range indices) are recorded in the device status
+ *     word and reported by hcsa_get_device_status().
+ *   - Entry selections `sel` are int32 [rows, topk], ascending entry index,
+ *     padded with -1 when fewer than topk entries are visible.
+ */
+#ifndef HCA_CSA_H
+#define HCA_CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HCSA_OK = 0,
+    HCSA_ERR_NULL = 1,
+    HCSA_ERR_SHAPE = 2,
+    HCSA_ERR_DTYPE = 3,
+    HCSA_ERR_ALIGN = 4,
+    HCSA_ERR_WORKSPACE = 5,
+    HCSA_ERR_CUDA = 6,
+    HCSA_ERR_TIMEOUT = 7,      /* a bounded device-side wait gave up */
+    HCSA_ERR_UNSUPPORTED = 8,  /* valid request this build does not implement */
+    HCSA_ERR_DEVICE = 9        /* a kernel's own bounds check fired */
+} hcsa_status;
+
+typedef enum { HCSA_F32 = 0, HCSA_BF16 = 1 } hcsa_dtype;
+
+typedef enum { HCSA_KIND_CSA = 0, HCSA_KIND_HCA = 1 } hcsa_kind;
+
+/* One struct describes a layer; each call reads the fields it needs. */
+typedef struct {
+    int32_t B;       /* sequences in a decode batch (prefill: 1) */
+    int32_t T;       /* tokens of the prefill sequence */
+    int32_t D;       /* model width */
+    int32_t m;       /* compression ratio (CSA 4, HCA 128) */
+    int32_t width;   /* pool width (CSA 8: overlapping; HCA = m) */
+    int32_t C;       /* compressed dim: key half C/2, value half C/2 */
+    int32_t di;      /* indexer key dim (CSA) */
+    int32_t Hi;      /* indexer heads (CSA) */
+    int32_t topk;    /* entries selected per query (CSA) */
+    int32_t window;  /* raw sliding window (tokens), >= width for decode */
+    int32_t H;       /* query heads */
+    int32_t dh;      /* head dim, must equal C/2 */
+    float scale;     /* softmax scale tau */
+    int32_t dtype;   /* hcsa_dtype */
+    int32_t n_cap;   /* decode: entry capacity per sequence of the cache arrays */
+} hcsa_params;
+
+/* Decode cache of one layer (device pointers, caller-owned).
+ * entries  [B, n_cap, C]        compressed entries, entry j of sequence b at row j
+ * idx_keys [B, n_cap, di]       indexer keys (CSA; NULL for HCA)
+ * win_kv   [B, window, C]       raw kv rows: token p in slot p % window
+ * ring_g   [B, width, C]        gate logits g = x W_g of token p in slot p % width
+ * ring_ki  [B, width, di]       indexer-key projections of token p in slot p % width (CSA)
+ * The window ring also stages the kv rows of the pool that is still open, which
+ * is why window >= width is required. */
+typedef struct {
+    void *entries;
+    void *idx_keys;
+    void *win_kv;
+    void *ring_g;
+    void *ring_ki;
+} hcsa_cache;
+
+/* Workspace queries: op selects the call. */
+typedef enum {
+    HCSA_OP_PROJECT = 0,
+    HCSA_OP_CSA_INDEX_TOPK = 1,
+    HCSA_OP_CSA_ATTEND = 2,
+    HCSA_OP_HCA_ATTEND = 3,
+    HCSA_OP_CSA_DECODE_INDEX_TOPK = 4,
+    HCSA_OP_CSA_DECODE_ATTEND = 5,
+    HCSA_OP_HCA_DECODE_ATTEND = 6
+} hcsa_op;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int32_t hcsa_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *hcsa_status_string(hcsa_status s);
+
+/* Bytes of scratch the call `op` needs for layer p (0 if none). */
+size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op);
+
+/* Number of projected columns for a layer of `kind`:
+ * CSA: C (kv) + C (g) + di (ki) + Hi*di (qi) + Hi (w) + H*dh (q);  HCA: C + C + H*dh. */
+int64_t hcsa_proj_cols(const hcsa_params *p, int32_t kind);
+
+/* Token projections (the "projection" step of the layer; a plain GEMM).
+ *   x     [rows, D]           (ld = D)
+ *   W_cat [D, ncols]          the concatenation [W_kv | W_g | W_ki | W_qi | W_w | W_q] (HCA: [W_kv | W_g | W_q])
+ *   y     [rows, ncols]       y = x W_cat rounded to the storage type; ncols = hcsa_proj_cols(p, kind)
+ * bf16: cuBLAS GEMM, fp32 accumulate; f32: fp64 accumulate.  ws may be NULL for f32. */
+hcsa_status hcsa_project(const hcsa_params *p, int32_t kind, int64_t rows, const void *x, const void *W_cat,
+                         void *y, void *ws, size_t ws_bytes, void *stream);
+
+/* CSA compressor (m, width = 8 overlapping pools), prefill of one sequence of p->T tokens.
+ *   kv [T, ld_kv] (C used), g [T, ld_g] (C used), ki [T, ld_ki] (di used), bias [width, C]
+ *   entries [N, C], idx_keys [N, di] with N = ceil(T / m) (edge pools are truncated to [0, T)). */
+hcsa_status csa_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
+                         const void *ki, int64_t ld_ki, const void *bias, void *entries, void *idx_keys,
+                         void *stream);
+
+/* HCA compressor (width = m, non-overlapping pools); as csa_compress without indexer keys. */
+hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
+                         const void *bias, void *entries, void *stream);
+
+/* CSA lightning indexer + top-k, causal prefill.
+ *   qi [T, ld_qi] (Hi*di used, head-major), w [T, ld_w] (Hi used), idx_keys [N, di]
+ *   sel [T, topk] int32: for query t the min(topk, t / m) best visible entries, ascending, -1 padded.
+ * ws: hcsa_workspace_bytes(p, HCSA_OP_CSA_INDEX_TOPK) bytes (materialised scores). */
+hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
+                           const void *idx_keys, int32_t *sel, void *ws, size_t ws_bytes, void *stream);
+
+/* CSA attention, causal prefill.
+ *   q [T, ld_q] (H*dh used, head-major), kv [T, ld_kv] raw window rows (C used), entries [N, C], sel [T, topk]
+ *   out [T, H*dh]: softmax over selected entries and raw tokens (t - window, t]. */
+hcsa_status csa_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
+                       const void *entries, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* HCA attention, causal prefill: every visible entry (j < t / m) plus the raw window. */
+hcsa_status hca_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
+                       const void *entries, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* Decode: append one new token per sequence to the cache.
+ *   pos [B] int32 (device): position of the new token of each sequence (not modified)
+ *   kv/g/ki [B, ld] the new token's projections (ki NULL for HCA), bias [width, C]
+ * Writes the rings; when pos[b] = m j + m - 1 the entry j is formed from the rings
+ * (and written if j < n_cap).  Callers advance pos themselves between steps. */
+hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                              const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
+                              int64_t ld_ki, const void *bias, void *stream);
+
+/* Decode: CSA indexer + top-k for the new token of each sequence over entries j < pos[b] / m.
+ *   qi [B, ld_qi], w [B, ld_w]; sel [B, topk]. */
+hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                  const void *qi, int64_t ld_qi, const void *w, int64_t ld_w, int32_t *sel,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/* Decode: CSA attention (split over keys, then a log-sum-exp combine).
+ *   q [B, ld_q], sel [B, topk]; out [B, H*dh].  Keys: selected entries U tokens (pos - window, pos]. */
+hcsa_status csa_decode_attend(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                              int64_t ld_q, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/* Decode: HCA attention over entries j < pos[b] / m and the raw window. */
+hcsa_status hca_decode_attend(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                              int64_t ld_q, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* Waits for `stream`, then returns and clears the device status word of the current device
+ * (HCSA_OK, HCSA_ERR_TIMEOUT or HCSA_ERR_DEVICE), or HCSA_ERR_CUDA if the wait itself failed. */
+hcsa_status hcsa_get_device_status(void *stream);
+
+/* Number of kernels this library enqueued on the calling host thread since the last reset
+ * (library GEMM kernels not included).  For launch accounting in benchmarks. */
+int64_t hcsa_launch_count(int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HCA_CSA_H */

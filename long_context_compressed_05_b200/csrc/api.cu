@@ -1,0 +1,284 @@
+// C ABI entry points of libhcsa.so: argument validation on the host, then the
+// kernel launches on the caller's stream.  See include/hca_csa.h for the
+// contract of every call.
+#include <stdio.h>
+
+#include "internal.cuh"
+
+namespace hcsa {
+
+static __device__ int g_status_word;
+static int *g_status_ptr[64];
+static thread_local int64_t g_launches = 0;
+
+int *device_status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = (int *)p;
+    }
+    return g_status_ptr[dev];
+}
+
+void count_launch(int n) { g_launches += n; }
+
+hcsa_status check_launch() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        fprintf(stderr, "hcsa: launch failed: %s\n", cudaGetErrorString(e));
+        return HCSA_ERR_CUDA;
+    }
+    return HCSA_OK;
+}
+
+}  // namespace hcsa
+
+using namespace hcsa;
+
+namespace {
+
+int esize(int dtype) { return dtype == HCSA_BF16 ? 2 : 4; }
+int vec(int dtype) { return dtype == HCSA_BF16 ? 8 : 4; }
+bool aligned(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool ld_ok(int dtype, int64_t ld, int64_t used) { return ld >= used && (ld * esize(dtype)) % 16 == 0; }
+
+#define HCSA_TRY(expr)                       \
+    do {                                     \
+        hcsa_status _s = (expr);             \
+        if (_s != HCSA_OK) return _s;        \
+    } while (0)
+
+hcsa_status check_common(const hcsa_params *p) {
+    if (!p) return HCSA_ERR_NULL;
+    if (p->dtype != HCSA_F32 && p->dtype != HCSA_BF16) return HCSA_ERR_DTYPE;
+    const int V = vec(p->dtype);
+    if (p->m < 1 || p->width < p->m || p->width > 512 || p->C < 2 || p->C % (2 * V) != 0) return HCSA_ERR_SHAPE;
+    if (p->H < 1 || p->dh != p->C / 2 || p->window < 1) return HCSA_ERR_SHAPE;
+    return HCSA_OK;
+}
+
+hcsa_status check_csa(const hcsa_params *p) {
+    HCSA_TRY(check_common(p));
+    if (p->di < 1 || p->di > p->C || p->di % vec(p->dtype) != 0 || p->Hi < 1 || p->topk < 1)
+        return HCSA_ERR_SHAPE;
+    return HCSA_OK;
+}
+
+hcsa_status check_decode(const hcsa_params *p, const hcsa_cache *c, const int32_t *pos, bool csa) {
+    if (!c || !pos || !c->entries || !c->win_kv || !c->ring_g) return HCSA_ERR_NULL;
+    if (csa && (!c->idx_keys || !c->ring_ki)) return HCSA_ERR_NULL;
+    if (p->B < 1 || p->n_cap < 1 || p->window < p->width) return HCSA_ERR_SHAPE;
+    if (!aligned(c->entries) || !aligned(c->win_kv) || !aligned(c->ring_g) || !aligned(pos)) return HCSA_ERR_ALIGN;
+    if (csa && (!aligned(c->idx_keys) || !aligned(c->ring_ki))) return HCSA_ERR_ALIGN;
+    return HCSA_OK;
+}
+
+int64_t n_entries(const hcsa_params *p) { return ((int64_t)p->T + p->m - 1) / p->m; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t hcsa_version(void) { return 100; }
+
+const char *hcsa_status_string(hcsa_status s) {
+    switch (s) {
+        case HCSA_OK: return "ok";
+        case HCSA_ERR_NULL: return "null pointer argument";
+        case HCSA_ERR_SHAPE: return "invalid shape or size";
+        case HCSA_ERR_DTYPE: return "unsupported storage dtype";
+        case HCSA_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
+        case HCSA_ERR_WORKSPACE: return "workspace too small";
+        case HCSA_ERR_CUDA: return "CUDA launch or runtime error";
+        case HCSA_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+        case HCSA_ERR_UNSUPPORTED: return "configuration not supported by this build";
+        case HCSA_ERR_DEVICE: return "device-side bounds check failed";
+    }
+    return "unknown status";
+}
+
+int64_t hcsa_proj_cols(const hcsa_params *p, int32_t kind) {
+    if (!p) return -1;
+    int64_t c = 2 * (int64_t)p->C + (int64_t)p->H * p->dh;
+    if (kind == HCSA_KIND_CSA) c += (int64_t)p->di + (int64_t)p->Hi * p->di + p->Hi;
+    return c;
+}
+
+size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op) {
+    if (!p) return 0;
+    switch (op) {
+        case HCSA_OP_PROJECT: return project_ws_bytes(p->dtype);
+        case HCSA_OP_CSA_INDEX_TOPK: return index_topk_ws_bytes(p->dtype, p->T, n_entries(p));
+        case HCSA_OP_CSA_ATTEND: return attend_ws_bytes(p->dtype, false, false, p->T, p->H, p->dh, p->topk,
+                                                        p->window, n_entries(p));
+        case HCSA_OP_HCA_ATTEND: return attend_ws_bytes(p->dtype, false, true, p->T, p->H, p->dh, 0, p->window,
+                                                        n_entries(p));
+        case HCSA_OP_CSA_DECODE_INDEX_TOPK: return index_topk_ws_bytes(p->dtype, p->B, p->n_cap);
+        case HCSA_OP_CSA_DECODE_ATTEND: return attend_ws_bytes(p->dtype, true, false, p->B, p->H, p->dh, p->topk,
+                                                               p->window, p->n_cap);
+        case HCSA_OP_HCA_DECODE_ATTEND: return attend_ws_bytes(p->dtype, true, true, p->B, p->H, p->dh, 0,
+                                                               p->window, p->n_cap);
+    }
+    return 0;
+}
+
+hcsa_status hcsa_project(const hcsa_params *p, int32_t kind, int64_t rows, const void *x, const void *W_cat,
+                         void *y, void *ws, size_t ws_bytes, void *stream) {
+    if (kind == HCSA_KIND_CSA) HCSA_TRY(check_csa(p));
+    else if (kind == HCSA_KIND_HCA) HCSA_TRY(check_common(p));
+    else return HCSA_ERR_SHAPE;
+    if (!x || !W_cat || !y) return HCSA_ERR_NULL;
+    if (rows < 0 || p->D < 1) return HCSA_ERR_SHAPE;
+    if (!aligned(x) || !aligned(W_cat) || !aligned(y)) return HCSA_ERR_ALIGN;
+    const int64_t nc = hcsa_proj_cols(p, kind);
+    if ((p->D * esize(p->dtype)) % 16 || (nc * esize(p->dtype)) % 16) return HCSA_ERR_ALIGN;
+    if (p->dtype == HCSA_BF16 && ws && ws_bytes < project_ws_bytes(p->dtype)) return HCSA_ERR_WORKSPACE;
+    return launch_project(p->dtype, rows, p->D, nc, x, W_cat, y, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+hcsa_status csa_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
+                         const void *ki, int64_t ld_ki, const void *bias, void *entries, void *idx_keys,
+                         void *stream) {
+    HCSA_TRY(check_csa(p));
+    if (!kv || !g || !ki || !bias || !entries || !idx_keys) return HCSA_ERR_NULL;
+    if (p->T < 0) return HCSA_ERR_SHAPE;
+    if (!aligned(kv) || !aligned(g) || !aligned(ki) || !aligned(bias) || !aligned(entries) || !aligned(idx_keys))
+        return HCSA_ERR_ALIGN;
+    if (!ld_ok(p->dtype, ld_kv, p->C) || !ld_ok(p->dtype, ld_g, p->C) || !ld_ok(p->dtype, ld_ki, p->di))
+        return HCSA_ERR_ALIGN;
+    return launch_compress(p->dtype, p->T, p->C, p->m, p->width, kv, ld_kv, g, ld_g, ki, ld_ki, p->di, bias,
+                           entries, idx_keys, (cudaStream_t)stream);
+}
+
+hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
+                         const void *bias, void *entries, void *stream) {
+    HCSA_TRY(check_common(p));
+    if (!kv || !g || !bias || !entries) return HCSA_ERR_NULL;
+    if (p->T < 0) return HCSA_ERR_SHAPE;
+    if (!aligned(kv) || !aligned(g) || !aligned(bias) || !aligned(entries)) return HCSA_ERR_ALIGN;
+    if (!ld_ok(p->dtype, ld_kv, p->C) || !ld_ok(p->dtype, ld_g, p->C)) return HCSA_ERR_ALIGN;
+    return launch_compress(p->dtype, p->T, p->C, p->m, p->width, kv, ld_kv, g, ld_g, nullptr, 0, 0, bias, entries,
+                           nullptr, (cudaStream_t)stream);
+}
+
+hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
+                           const void *idx_keys, int32_t *sel, void *ws, size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_csa(p));
+    if (!qi || !w || !idx_keys || !sel) return HCSA_ERR_NULL;
+    if (p->T < 0) return HCSA_ERR_SHAPE;
+    if (!aligned(qi) || !aligned(w) || !aligned(idx_keys) || !aligned(sel)) return HCSA_ERR_ALIGN;
+    if (ld_qi < (int64_t)p->Hi * p->di || ld_w < p->Hi) return HCSA_ERR_SHAPE;
+    if (!ws && p->T > 0) return HCSA_ERR_WORKSPACE;
+    if (ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
+    IndexArgs a{p->dtype, p->T, p->Hi, p->di, p->topk, p->m, n_entries(p), qi, ld_qi, w, ld_w, idx_keys,
+                nullptr, sel, ws, ws_bytes};
+    return launch_index_topk(a, (cudaStream_t)stream);
+}
+
+static hcsa_status attend_prefill(const hcsa_params *p, bool dense, const void *q, int64_t ld_q, const void *kv,
+                                  int64_t ld_kv, const void *entries, const int32_t *sel, void *out, void *ws,
+                                  size_t ws_bytes, void *stream) {
+    if (!q || !kv || !entries || !out || (!dense && !sel)) return HCSA_ERR_NULL;
+    if (p->T < 0) return HCSA_ERR_SHAPE;
+    if (!aligned(q) || !aligned(kv) || !aligned(entries) || !aligned(out)) return HCSA_ERR_ALIGN;
+    if (ld_q < (int64_t)p->H * p->dh || ld_kv < p->C) return HCSA_ERR_SHAPE;
+    AttendArgs a{};
+    a.dtype = p->dtype; a.rows = p->T; a.H = p->H; a.dh = p->dh; a.C = p->C; a.window = p->window; a.m = p->m;
+    a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = n_entries(p);
+    a.q = q; a.ld_q = ld_q; a.kv = kv; a.ld_kv = ld_kv; a.entries = entries; a.sel = sel; a.pos = nullptr;
+    a.out = out; a.ws = ws; a.ws_bytes = ws_bytes;
+    return launch_attend(a, (cudaStream_t)stream);
+}
+
+hcsa_status csa_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
+                       const void *entries, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
+                       void *stream) {
+    HCSA_TRY(check_csa(p));
+    return attend_prefill(p, false, q, ld_q, kv, ld_kv, entries, sel, out, ws, ws_bytes, stream);
+}
+
+hcsa_status hca_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
+                       const void *entries, void *out, void *ws, size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_common(p));
+    return attend_prefill(p, true, q, ld_q, kv, ld_kv, entries, nullptr, out, ws, ws_bytes, stream);
+}
+
+hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *kv,
+                              int64_t ld_kv, const void *g, int64_t ld_g, const void *ki, int64_t ld_ki,
+                              const void *bias, void *stream) {
+    const bool csa = ki != nullptr;
+    HCSA_TRY(csa ? check_csa(p) : check_common(p));
+    HCSA_TRY(check_decode(p, cache, pos, csa));
+    if (!kv || !g || !bias) return HCSA_ERR_NULL;
+    if (!aligned(kv) || !aligned(g) || !aligned(bias) || (csa && !aligned(ki))) return HCSA_ERR_ALIGN;
+    if (!ld_ok(p->dtype, ld_kv, p->C) || !ld_ok(p->dtype, ld_g, p->C) || (csa && !ld_ok(p->dtype, ld_ki, p->di)))
+        return HCSA_ERR_ALIGN;
+    return launch_cache_append(p->dtype, *p, *cache, pos, kv, ld_kv, g, ld_g, ki, ld_ki, bias,
+                               (cudaStream_t)stream);
+}
+
+hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                  const void *qi, int64_t ld_qi, const void *w, int64_t ld_w, int32_t *sel,
+                                  void *ws, size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_csa(p));
+    HCSA_TRY(check_decode(p, cache, pos, true));
+    if (!qi || !w || !sel) return HCSA_ERR_NULL;
+    if (!aligned(qi) || !aligned(w) || !aligned(sel)) return HCSA_ERR_ALIGN;
+    if (ld_qi < (int64_t)p->Hi * p->di || ld_w < p->Hi) return HCSA_ERR_SHAPE;
+    if (!ws || ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
+    IndexArgs a{p->dtype, p->B, p->Hi, p->di, p->topk, p->m, p->n_cap, qi, ld_qi, w, ld_w, cache->idx_keys,
+                pos, sel, ws, ws_bytes};
+    return launch_index_topk(a, (cudaStream_t)stream);
+}
+
+static hcsa_status attend_decode(const hcsa_params *p, bool dense, const hcsa_cache *cache, const int32_t *pos,
+                                 const void *q, int64_t ld_q, const int32_t *sel, void *out, void *ws,
+                                 size_t ws_bytes, void *stream) {
+    if (!q || !out || (!dense && !sel)) return HCSA_ERR_NULL;
+    if (!aligned(q) || !aligned(out)) return HCSA_ERR_ALIGN;
+    if (ld_q < (int64_t)p->H * p->dh) return HCSA_ERR_SHAPE;
+    const size_t need = hcsa_workspace_bytes(p, dense ? HCSA_OP_HCA_DECODE_ATTEND : HCSA_OP_CSA_DECODE_ATTEND);
+    if (need && (!ws || ws_bytes < need)) return HCSA_ERR_WORKSPACE;
+    AttendArgs a{};
+    a.dtype = p->dtype; a.rows = p->B; a.H = p->H; a.dh = p->dh; a.C = p->C; a.window = p->window; a.m = p->m;
+    a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = p->n_cap;
+    a.q = q; a.ld_q = ld_q; a.kv = cache->win_kv; a.ld_kv = p->C; a.entries = cache->entries; a.sel = sel;
+    a.pos = pos; a.out = out; a.ws = ws; a.ws_bytes = ws_bytes;
+    return launch_attend(a, (cudaStream_t)stream);
+}
+
+hcsa_status csa_decode_attend(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                              int64_t ld_q, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
+                              void *stream) {
+    HCSA_TRY(check_csa(p));
+    HCSA_TRY(check_decode(p, cache, pos, true));
+    return attend_decode(p, false, cache, pos, q, ld_q, sel, out, ws, ws_bytes, stream);
+}
+
+hcsa_status hca_decode_attend(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                              int64_t ld_q, void *out, void *ws, size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_common(p));
+    HCSA_TRY(check_decode(p, cache, pos, false));
+    return attend_decode(p, true, cache, pos, q, ld_q, nullptr, out, ws, ws_bytes, stream);
+}
+
+hcsa_status hcsa_get_device_status(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HCSA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return HCSA_ERR_CUDA;
+    if (v != 0) {
+        int zero = 0;
+        if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return HCSA_ERR_CUDA;
+    }
+    return (hcsa_status)v;
+}
+
+int64_t hcsa_launch_count(int32_t reset) {
+    int64_t v = g_launches;
+    if (reset) g_launches = 0;
+    return v;
+}
+
+}  // extern "C"

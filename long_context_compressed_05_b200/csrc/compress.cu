@@ -1,0 +1,191 @@
+// Learned gated-pool compressor (CSA m=4 over overlapping width-8 pools, HCA
+// m'=128 over non-overlapping pools), prefill and decode-append forms.
+//
+// Follows "DeepSeek-V4 ... KV cache compressed attention", sections "CSA:
+// compresion 4x" (learned pool over overlapping windows) and "HCA: compresion
+// 128x", with the pool fixed by the CSA workload definition: entry j pools
+// tokens [m j - (width - m), m j + m) within [0, T), per channel
+//   c_j[c] = sum_i softmax_i(g[i,c] + B[i - m j + width - m, c]) kv[i,c];
+// the indexer key of entry j is the same pool over ki with gate channel d.
+//
+// HBM-bound: one thread owns one 16-byte channel vector of one entry and
+// streams the pool's tokens with 16-byte loads (adjacent threads read
+// adjacent vectors of the same row, so every warp load is fully coalesced).
+// The softmax is a single-pass running max per channel.
+#include "internal.cuh"
+
+namespace hcsa {
+
+template <typename A, int V>
+struct PoolAcc {
+    A mx[V], z[V], acc[V];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int e = 0; e < V; ++e) { mx[e] = -INFINITY; z[e] = A(0); acc[e] = A(0); }
+    }
+    __device__ __forceinline__ void add(const A *gate, const A *bias, const A *val) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            A l = gate[e] + bias[e];
+            if (l > mx[e]) {
+                A sc = exp_acc(mx[e] - l);
+                acc[e] = acc[e] * sc + val[e];
+                z[e] = z[e] * sc + A(1);
+                mx[e] = l;
+            } else {
+                A p = exp_acc(l - mx[e]);
+                acc[e] += p * val[e];
+                z[e] += p;
+            }
+        }
+    }
+    __device__ __forceinline__ void result(A *out) const {
+#pragma unroll
+        for (int e = 0; e < V; ++e) out[e] = acc[e] / z[e];
+    }
+};
+
+template <typename S>
+__global__ void __launch_bounds__(256) compress_kernel(int64_t T, int C, int m, int width, const S *__restrict__ kv,
+                                                       int64_t ld_kv, const S *__restrict__ g, int64_t ld_g,
+                                                       const S *__restrict__ ki, int64_t ld_ki, int di,
+                                                       const S *__restrict__ bias, S *__restrict__ entries,
+                                                       S *__restrict__ idx_keys, int64_t N) {
+    using A = typename Traits<S>::A;
+    constexpr int V = Traits<S>::VEC;
+    const int slots_c = C / V;
+    const int slots = slots_c + (ki ? di / V : 0);
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= N * slots) return;
+    const int64_t j = gid / slots;
+    const int s = (int)(gid - j * slots);
+    const bool is_key = s >= slots_c;
+    const int c0 = (is_key ? s - slots_c : s) * V;   // value channel; also the gate channel
+    const S *val = is_key ? ki : kv;
+    const int64_t ld_val = is_key ? ld_ki : ld_kv;
+    const int64_t lo = (int64_t)m * j - (width - m);
+    const int64_t a = lo < 0 ? 0 : lo;
+    const int64_t b = (int64_t)m * j + m < T ? (int64_t)m * j + m : T;
+
+    PoolAcc<A, V> pa;
+    pa.init();
+#pragma unroll 4
+    for (int64_t i = a; i < b; ++i) {
+        A gv[V], bv[V], vv[V];
+        load_vec(g + i * ld_g + c0, gv);
+        load_vec(bias + (i - lo) * C + c0, bv);
+        load_vec(val + i * ld_val + c0, vv);
+        pa.add(gv, bv, vv);
+    }
+    A r[V];
+    pa.result(r);
+    if (is_key) store_vec(idx_keys + j * di + c0, r);
+    else store_vec(entries + j * C + c0, r);
+}
+
+hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
+                            const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
+                            void *entries, void *idx_keys, cudaStream_t st) {
+    const int64_t N = (T + m - 1) / m;
+    if (N == 0) return HCSA_OK;
+    const int threads = 256;
+    if (dtype == HCSA_BF16) {
+        using S = __nv_bfloat16;
+        const int64_t slots = C / 8 + (ki ? di / 8 : 0);
+        const int64_t blocks = (N * slots + threads - 1) / threads;
+        compress_kernel<S><<<(unsigned)blocks, threads, 0, st>>>(
+            T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di, (const S *)bias,
+            (S *)entries, (S *)idx_keys, N);
+    } else {
+        const int64_t slots = C / 4 + (ki ? di / 4 : 0);
+        const int64_t blocks = (N * slots + threads - 1) / threads;
+        compress_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
+            T, C, m, width, (const float *)kv, ld_kv, (const float *)g, ld_g, (const float *)ki, ld_ki, di,
+            (const float *)bias, (float *)entries, (float *)idx_keys, N);
+    }
+    count_launch();
+    return check_launch();
+}
+
+// ---------------------------------------------------------------- decode append
+// Sequence b's new token P = pos[b] is written into the rings; when P = m j + m - 1
+// entry j is formed from tokens [m j - (width - m), P] (earlier tokens from the
+// rings, token P straight from the inputs, so no thread waits on another's write).
+template <typename S>
+__global__ void __launch_bounds__(128) cache_append_kernel(
+    int C, int m, int width, int window, int di, int64_t n_cap, const int32_t *__restrict__ pos,
+    const S *__restrict__ kv_new, int64_t ld_kv, const S *__restrict__ g_new, int64_t ld_g,
+    const S *__restrict__ ki_new, int64_t ld_ki, const S *__restrict__ bias, S *entries, S *idx_keys, S *win_kv,
+    S *ring_g, S *ring_ki, int *status) {
+    using A = typename Traits<S>::A;
+    constexpr int V = Traits<S>::VEC;
+    const int b = blockIdx.y;
+    const int slots_c = C / V;
+    const int slots = slots_c + (ki_new ? di / V : 0);
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= slots) return;
+    const int64_t P = pos[b];
+    if (P < 0) { report(status, kStatusBounds); return; }
+    const bool is_key = s >= slots_c;
+    const int c0 = (is_key ? s - slots_c : s) * V;
+    const S *gnew = g_new + b * ld_g;
+    const S *vnew = is_key ? ki_new + b * ld_ki : kv_new + b * ld_kv;
+    // 1) ring writes (each thread writes its own 16-byte vector)
+    if (is_key) {
+        *reinterpret_cast<uint4 *>(ring_ki + ((int64_t)b * width + P % width) * di + c0) =
+            *reinterpret_cast<const uint4 *>(vnew + c0);
+    } else {
+        *reinterpret_cast<uint4 *>(win_kv + ((int64_t)b * window + P % window) * C + c0) =
+            *reinterpret_cast<const uint4 *>(vnew + c0);
+        *reinterpret_cast<uint4 *>(ring_g + ((int64_t)b * width + P % width) * C + c0) =
+            *reinterpret_cast<const uint4 *>(gnew + c0);
+    }
+    // 2) entry completion
+    if ((P + 1) % m != 0) return;
+    const int64_t j = (P + 1) / m - 1;
+    if (j >= n_cap) { report(status, kStatusBounds); return; }
+    const int64_t lo = (int64_t)m * j - (width - m);
+    PoolAcc<A, V> pa;
+    pa.init();
+    for (int64_t i = lo < 0 ? 0 : lo; i <= P; ++i) {
+        A gv[V], bv[V], vv[V];
+        const S *grow = (i == P) ? gnew : ring_g + ((int64_t)b * width + i % width) * C;
+        const S *vrow = (i == P) ? vnew
+                        : is_key ? ring_ki + ((int64_t)b * width + i % width) * di
+                                 : win_kv + ((int64_t)b * window + i % window) * C;
+        load_vec(grow + c0, gv);
+        load_vec(bias + (i - lo) * C + c0, bv);
+        load_vec(vrow + c0, vv);
+        pa.add(gv, bv, vv);
+    }
+    A r[V];
+    pa.result(r);
+    if (is_key) store_vec(idx_keys + ((int64_t)b * n_cap + j) * di + c0, r);
+    else store_vec(entries + ((int64_t)b * n_cap + j) * C + c0, r);
+}
+
+hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cache &c, const int32_t *pos,
+                                const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
+                                int64_t ld_ki, const void *bias, cudaStream_t st) {
+    const int V = dtype == HCSA_BF16 ? 8 : 4;
+    const int slots = p.C / V + (ki ? p.di / V : 0);
+    dim3 grid((slots + 127) / 128, p.B);
+    int *status = device_status_ptr();
+    if (dtype == HCSA_BF16) {
+        using S = __nv_bfloat16;
+        cache_append_kernel<S><<<grid, 128, 0, st>>>(
+            p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
+            (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
+            (S *)c.ring_ki, status);
+    } else {
+        using S = float;
+        cache_append_kernel<S><<<grid, 128, 0, st>>>(
+            p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
+            (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
+            (S *)c.ring_ki, status);
+    }
+    count_launch();
+    return check_launch();
+}
+
+}  // namespace hcsa

@@ -1,0 +1,116 @@
+// Internal declarations shared by the translation units of libhcsa.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hca_csa.h"
+
+namespace hcsa {
+
+// ---------------------------------------------------------------- storage / compute types
+// HCSA_F32 stores fp32 and computes in fp64; HCSA_BF16 stores bf16 and computes in fp32.
+template <typename S> struct Traits;
+template <> struct Traits<float> {
+    using A = double;
+    static constexpr int VEC = 4;  // elements per 16-byte vector
+};
+template <> struct Traits<__nv_bfloat16> {
+    using A = float;
+    static constexpr int VEC = 8;
+};
+
+__device__ __forceinline__ double to_acc(float v, double) { return (double)v; }
+__device__ __forceinline__ float to_acc(__nv_bfloat16 v, float) { return __bfloat162float(v); }
+
+__device__ __forceinline__ void store_val(float *p, double v) { *p = (float)v; }
+__device__ __forceinline__ void store_val(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// 16-byte vector load of VEC storage elements widened to the accumulation type.
+template <typename S, typename A>
+__device__ __forceinline__ void load_vec(const S *p, A *out) {
+    uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p));
+    const S *e = reinterpret_cast<const S *>(&raw);
+#pragma unroll
+    for (int i = 0; i < Traits<S>::VEC; ++i) out[i] = to_acc(e[i], A());
+}
+
+template <typename S, typename A>
+__device__ __forceinline__ void store_vec(S *p, const A *v) {
+    uint4 raw;
+    S *e = reinterpret_cast<S *>(&raw);
+#pragma unroll
+    for (int i = 0; i < Traits<S>::VEC; ++i) store_val(&e[i], v[i]);
+    *reinterpret_cast<uint4 *>(p) = raw;
+}
+
+__device__ __forceinline__ double exp_acc(double x) { return exp(x); }
+__device__ __forceinline__ float exp_acc(float x) { return expf(x); }
+
+// device status word codes (match hcsa_status)
+enum : int { kStatusOk = 0, kStatusTimeout = HCSA_ERR_TIMEOUT, kStatusBounds = HCSA_ERR_DEVICE };
+
+__device__ __forceinline__ void report(int *status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------- host side helpers
+int *device_status_ptr();           // lazily resolved per device; nullptr on failure
+void count_launch(int n = 1);
+hcsa_status check_launch();         // maps cudaGetLastError() to a status
+
+// ---------------------------------------------------------------- launchers
+// compressor (prefill): entries [N, C] (+ idx_keys [N, di] when ki != nullptr)
+hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
+                            const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
+                            void *entries, void *idx_keys, cudaStream_t st);
+
+hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cache &c, const int32_t *pos,
+                                const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
+                                int64_t ld_ki, const void *bias, cudaStream_t st);
+
+// indexer scores + top-k.  Prefill: rows = T queries of one sequence, n_vis(t) = min(t / m, N).
+// Decode: rows = B sequences, query b sees entries j < min(pos[b] / m, n_cap) of keys + b * n_cap * di.
+struct IndexArgs {
+    int dtype;
+    int64_t rows;        // queries
+    int Hi, di, topk, m;
+    int64_t N;           // entries per sequence (prefill: ceil(T/m); decode: n_cap)
+    const void *qi; int64_t ld_qi;
+    const void *w; int64_t ld_w;
+    const void *keys;    // [N, di] (prefill) or [B, n_cap, di] (decode)
+    const int32_t *pos;  // decode positions (nullptr: prefill, query t at position t)
+    int32_t *sel;
+    void *ws; size_t ws_bytes;
+};
+size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N);
+hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st);
+
+// attention.  Prefill (pos == nullptr): query t of one sequence, window rows kv[t-window+1 .. t].
+// Decode: query b at position pos[b], entries of sequence b, window ring win_kv[b].
+struct AttendArgs {
+    int dtype;
+    int64_t rows;
+    int H, dh, C, window, m, topk;
+    float scale;
+    bool dense;              // HCA: all visible entries instead of sel
+    int64_t N;               // entries per sequence (prefill: ceil(T/m); decode: n_cap)
+    const void *q; int64_t ld_q;
+    const void *kv; int64_t ld_kv;   // prefill raw rows [T, ld_kv] / decode ring base [B, window, C]
+    const void *entries;             // [N, C] or [B, n_cap, C]
+    const int32_t *sel;              // [rows, topk] (CSA)
+    const int32_t *pos;              // decode positions or nullptr
+    void *out;
+    void *ws; size_t ws_bytes;
+};
+size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, int dh, int topk, int window,
+                       int64_t N);
+hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st);
+
+// projection y[rows, ncols] = x[rows, D] W[D, ncols]
+size_t project_ws_bytes(int dtype);
+hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const void *x, const void *W, void *y,
+                           void *ws, size_t ws_bytes, cudaStream_t st);
+
+}  // namespace hcsa

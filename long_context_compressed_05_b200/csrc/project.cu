@@ -1,0 +1,96 @@
+// Token projections y = x W_cat (the layer's "low-dimensional projection"
+// inputs: kv, gate, indexer key / query / head weight and query columns).
+//
+// A plain dense GEMM.  bf16 storage runs it through cuBLAS (bf16 tensor
+// cores, fp32 accumulate, bf16 output); fp32 storage uses a tiled CUDA-core
+// kernel that accumulates in fp64 and rounds once to fp32.
+#include <cublas_v2.h>
+
+#include "internal.cuh"
+
+namespace hcsa {
+
+constexpr int kPT = 64;   // output tile (rows and cols)
+constexpr int kPK = 16;   // k step
+
+__global__ void __launch_bounds__(256) project_f64acc_kernel(int64_t rows, int D, int64_t ncols,
+                                                             const float *__restrict__ x,
+                                                             const float *__restrict__ W, float *__restrict__ y) {
+    __shared__ double sx[kPK][kPT + 1];
+    __shared__ double sw[kPK][kPT + 1];
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    const int64_t r0 = (int64_t)blockIdx.y * kPT, c0 = (int64_t)blockIdx.x * kPT;
+    double acc[4][4] = {};
+    for (int k0 = 0; k0 < D; k0 += kPK) {
+        for (int i = threadIdx.x; i < kPK * kPT; i += 256) {
+            int kk = i % kPK, rr = i / kPK;
+            int64_t r = r0 + rr;
+            sx[kk][rr] = (r < rows && k0 + kk < D) ? (double)x[r * D + k0 + kk] : 0.0;
+            int cc = i % kPT, k2 = i / kPT;
+            int64_t c = c0 + cc;
+            sw[k2][cc] = (c < ncols && k0 + k2 < D) ? (double)W[(int64_t)(k0 + k2) * ncols + c] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kPK; ++kk) {
+            double a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { a[i] = sx[kk][ty * 4 + i]; b[i] = sw[kk][tx * 4 + i]; }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int64_t r = r0 + ty * 4 + i;
+        if (r >= rows) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int64_t c = c0 + tx * 4 + j;
+            if (c < ncols) y[r * ncols + c] = (float)acc[i][j];
+        }
+    }
+}
+
+static cublasHandle_t g_handles[64];
+
+static cublasHandle_t handle_for_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!g_handles[dev]) {
+        cublasHandle_t h;
+        if (cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) return nullptr;
+        g_handles[dev] = h;
+    }
+    return g_handles[dev];
+}
+
+size_t project_ws_bytes(int dtype) { return dtype == HCSA_BF16 ? (size_t)32 << 20 : 0; }
+
+hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const void *x, const void *W, void *y,
+                           void *ws, size_t ws_bytes, cudaStream_t st) {
+    if (rows == 0 || ncols == 0) return HCSA_OK;
+    if (dtype == HCSA_F32) {
+        dim3 grid((unsigned)((ncols + kPT - 1) / kPT), (unsigned)((rows + kPT - 1) / kPT));
+        if (grid.y > 65535) return HCSA_ERR_UNSUPPORTED;
+        project_f64acc_kernel<<<grid, 256, 0, st>>>(rows, D, ncols, (const float *)x, (const float *)W, (float *)y);
+        count_launch();
+        return check_launch();
+    }
+    if (rows > INT32_MAX || ncols > INT32_MAX) return HCSA_ERR_UNSUPPORTED;
+    cublasHandle_t h = handle_for_device();
+    if (!h) return HCSA_ERR_CUDA;
+    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
+    if (ws && ws_bytes && cublasSetWorkspace(h, ws, ws_bytes) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
+    const float alpha = 1.0f, beta = 0.0f;
+    // row-major y[rows, ncols] = x[rows, D] W[D, ncols]  <=>  column-major y^T = W^T x^T
+    cublasStatus_t s = cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, (int)ncols, (int)rows, D, &alpha, W, CUDA_R_16BF,
+                                    (int)ncols, x, CUDA_R_16BF, D, &beta, y, CUDA_R_16BF, (int)ncols,
+                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+    return s == CUBLAS_STATUS_SUCCESS ? check_launch() : HCSA_ERR_CUDA;
+}
+
+}  // namespace hcsa

@@ -1,0 +1,141 @@
+"""Layer-level helpers over the C ABI: allocate device buffers with torch and
+issue the calls of one CSA / HCA layer (prefill) or one decode step, in order.
+
+Nothing here computes: every step is a call into libhcsa.so.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+__all__ = ["params_for", "torch_dtype", "PrefillLayer", "DecodeLayer"]
+
+
+def torch_dtype(dtype: str):
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def params_for(spec, *, T=None, B=1, n_cap=0) -> L.Params:
+    """Params from any object with the layer fields (kind, D, m, width, C, di, Hi, topk, window, H, dh, scale, dtype)."""
+    return L.make_params(T=spec.T if T is None else T, D=spec.D, m=spec.m, width=spec.width, C=spec.C,
+                         di=getattr(spec, "di", 0), Hi=getattr(spec, "Hi", 0), topk=getattr(spec, "topk", 0),
+                         window=spec.window, H=spec.H, dh=spec.dh, scale=spec.scale, dtype=spec.dtype, B=B,
+                         n_cap=n_cap)
+
+
+def _col_offsets(spec):
+    names = [("kv", spec.C), ("g", spec.C)]
+    if spec.kind == "csa":
+        names += [("ki", spec.di), ("qi", spec.Hi * spec.di), ("w", spec.Hi)]
+    names += [("q", spec.H * spec.dh)]
+    off, out = 0, {}
+    for n, w in names:
+        out[n] = (off, off + w)
+        off += w
+    return out, off
+
+
+class PrefillLayer:
+    """One CSA or HCA layer over a sequence of T tokens, buffers allocated once."""
+
+    def __init__(self, spec, device="cuda"):
+        self.spec = spec
+        self.csa = spec.kind == "csa"
+        self.kind = L.KIND_CSA if self.csa else L.KIND_HCA
+        self.p = params_for(spec)
+        dt = torch_dtype(spec.dtype)
+        T, N = spec.T, -(-spec.T // spec.m)
+        self.cols, ncols = _col_offsets(spec)
+        assert ncols == L.hcsa_proj_cols(self.p, self.kind)
+        self.y = torch.empty((T, ncols), dtype=dt, device=device)
+        self.entries = torch.empty((N, spec.C), dtype=dt, device=device)
+        self.out = torch.empty((T, spec.H * spec.dh), dtype=dt, device=device)
+        self.ws_proj = self._ws(L.OP_PROJECT, device)
+        if self.csa:
+            self.idx_keys = torch.empty((N, spec.di), dtype=dt, device=device)
+            self.sel = torch.empty((T, spec.topk), dtype=torch.int32, device=device)
+            self.ws_index = self._ws(L.OP_CSA_INDEX_TOPK, device)
+            self.ws_attend = self._ws(L.OP_CSA_ATTEND, device)
+        else:
+            self.ws_attend = self._ws(L.OP_HCA_ATTEND, device)
+
+    def _ws(self, op, device):
+        n = L.hcsa_workspace_bytes(self.p, op)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n else None
+
+    def view(self, name):
+        a, b = self.cols[name]
+        return self.y[:, a:b]
+
+    def project(self, x, W_cat):
+        L.hcsa_project(self.p, self.kind, x, W_cat, self.y, self.ws_proj)
+
+    def compress(self, bias):
+        if self.csa:
+            L.csa_compress(self.p, self.view("kv"), self.view("g"), self.view("ki"), bias, self.entries,
+                           self.idx_keys)
+        else:
+            L.hca_compress(self.p, self.view("kv"), self.view("g"), bias, self.entries)
+
+    def index_topk(self):
+        L.csa_index_topk(self.p, self.view("qi"), self.view("w"), self.idx_keys, self.sel, self.ws_index)
+
+    def attend(self, sel=None):
+        if self.csa:
+            L.csa_attend(self.p, self.view("q"), self.view("kv"), self.entries, self.sel if sel is None else sel,
+                         self.out, self.ws_attend)
+        else:
+            L.hca_attend(self.p, self.view("q"), self.view("kv"), self.entries, self.out, self.ws_attend)
+
+    def forward(self, x, W_cat, bias):
+        self.project(x, W_cat)
+        self.compress(bias)
+        if self.csa:
+            self.index_topk()
+        self.attend()
+        return self.out
+
+
+class DecodeLayer:
+    """One layer's decode step for B sequences over a caller-provided cache."""
+
+    def __init__(self, spec, B, n_cap, cache: dict, device="cuda"):
+        self.spec = spec
+        self.csa = spec.kind == "csa"
+        self.kind = L.KIND_CSA if self.csa else L.KIND_HCA
+        self.p = params_for(spec, T=0, B=B, n_cap=n_cap)
+        dt = torch_dtype(spec.dtype)
+        self.cols, ncols = _col_offsets(spec)
+        self.cache_t = cache
+        self.cache = L.make_cache(cache["entries"], cache["win_kv"], cache["ring_g"], cache.get("idx_keys"),
+                                  cache.get("ring_ki"))
+        self.y = torch.empty((B, ncols), dtype=dt, device=device)
+        self.out = torch.empty((B, spec.H * spec.dh), dtype=dt, device=device)
+        self.ws_proj = self._ws(L.OP_PROJECT, device)
+        if self.csa:
+            self.sel = torch.empty((B, spec.topk), dtype=torch.int32, device=device)
+            self.ws_index = self._ws(L.OP_CSA_DECODE_INDEX_TOPK, device)
+            self.ws_attend = self._ws(L.OP_CSA_DECODE_ATTEND, device)
+        else:
+            self.ws_attend = self._ws(L.OP_HCA_DECODE_ATTEND, device)
+
+    def _ws(self, op, device):
+        n = L.hcsa_workspace_bytes(self.p, op)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n else None
+
+    def view(self, name):
+        a, b = self.cols[name]
+        return self.y[:, a:b]
+
+    def step(self, x, W_cat, bias, pos):
+        L.hcsa_project(self.p, self.kind, x, W_cat, self.y, self.ws_proj)
+        L.hcsa_cache_append(self.p, self.cache, pos, self.view("kv"), self.view("g"),
+                            self.view("ki") if self.csa else None, bias)
+        if self.csa:
+            L.csa_decode_index_topk(self.p, self.cache, pos, self.view("qi"), self.view("w"), self.sel,
+                                    self.ws_index)
+            L.csa_decode_attend(self.p, self.cache, pos, self.view("q"), self.sel, self.out, self.ws_attend)
+        else:
+            L.hca_decode_attend(self.p, self.cache, pos, self.view("q"), self.out, self.ws_attend)
+        return self.out

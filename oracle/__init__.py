@@ -226,87 +226,92 @@ def attend_rows(spec, res, q, sel):
 
 
 def decode_step(spec, inp, P, seqs=None):
-    """One decode step of one layer for the sequences in `inp` (all at position P).
+    """One decode step of one layer.
 
-    inp: storage arrays from synth.decode_inputs: W_cat, B, x[Ball, D] and the cache
-    for the selected sequences (entries[b,N,C], idx_keys[b,N,di], win_kv[b,win,C],
-    ring_g[b,width,C], ring_ki[b,width,di]).  seqs maps cache row b -> x row.
-    Returns dict with the updated rings/entries (float64) and per-sequence outputs."""
+    inp: storage arrays as produced by synth.decode_inputs: W_cat, B, x[Ball, D] and the cache
+    entries[Ball,N,C], idx_keys[Ball,N,di], win_kv[Ball,win,C], ring_g[Ball,width,C], ring_ki[Ball,width,di].
+    P: position of the new token, one int or one per batch row.  seqs: the batch rows to evaluate
+    (default all).  Returns per-evaluated-row results (float64), in the order of seqs."""
     st = storage_code(spec.dtype)
     csa = spec.kind == "csa"
     m, Wd, win, C = spec.m, spec.width, spec.window, spec.C
     if win < Wd:
         raise ValueError("the window ring also stages the kv rows of the open pool: window >= width")
     cols = _col_slices(spec)
-    nb = inp["entries"].shape[0]
-    seqs = list(range(nb)) if seqs is None else list(seqs)
-    x = to_f64(inp["x"][seqs])
-    y = project(x, to_f64(inp["W_cat"]), st)
+    nb_all = inp["x"].shape[0]
+    seqs = list(range(nb_all)) if seqs is None else list(seqs)
+    Pv = np.broadcast_to(np.asarray(P, np.int64), (nb_all,))
     Bm = to_f64(inp["B"])
-    entries = to_f64(inp["entries"])
-    win_kv = to_f64(inp["win_kv"]).copy()
-    ring_g = to_f64(inp["ring_g"]).copy()
-    idx = to_f64(inp["idx_keys"]) if csa else None
-    ring_ki = to_f64(inp["ring_ki"]).copy() if csa else None
-    Ncap = entries.shape[1]
-    new_entry = {}
-    outs, sels, gaps, scores_all = [], [], [], []
-    for b in range(nb):
-        yb = y[b]
-        win_kv[b, P % win] = yb[cols["kv"]]
-        ring_g[b, P % Wd] = yb[cols["g"]]
+    W = to_f64(inp["W_cat"])
+    res = {"seqs": seqs, "y": [], "out": [], "win_kv": [], "ring_g": [], "ring_ki": [], "entries": [],
+           "new_entry": [], "sel": [], "gap": [], "scores": []}
+    for b in seqs:
+        Pb = int(Pv[b])
+        yb = project(to_f64(inp["x"][b:b + 1]), W, st)[0]
+        win_kv = to_f64(inp["win_kv"][b]).copy()
+        ring_g = to_f64(inp["ring_g"][b]).copy()
+        ent_b = to_f64(inp["entries"][b])
+        idx_b = to_f64(inp["idx_keys"][b]) if csa else None
+        ring_ki = to_f64(inp["ring_ki"][b]).copy() if csa else None
+        Ncap = ent_b.shape[0]
+        # append: the new token enters the rings
+        win_kv[Pb % win] = yb[cols["kv"]]
+        ring_g[Pb % Wd] = yb[cols["g"]]
         if csa:
-            ring_ki[b, P % Wd] = yb[cols["ki"]]
-        ent_b = entries[b]
-        idx_b = idx[b] if csa else None
-        if (P + 1) % m == 0:
-            j = (P + 1) // m - 1
+            ring_ki[Pb % Wd] = yb[cols["ki"]]
+        new = None
+        if (Pb + 1) % m == 0:       # the token closes entry j: pool tokens [m j - (width - m), m j + m)
+            j = (Pb + 1) // m - 1
             lo = m * j - (Wd - m)
             toks = [i for i in range(lo, m * j + m) if i >= 0]
-            kv_t = np.stack([win_kv[b, i % win] for i in toks])
-            g_t = np.stack([ring_g[b, i % Wd] for i in toks])
+            kv_t = np.stack([win_kv[i % win] for i in toks])
+            g_t = np.stack([ring_g[i % Wd] for i in toks])
             b_t = np.stack([Bm[i - lo] for i in toks])
-            e = pool_rows(kv_t, g_t, b_t, C, st)
-            new = {"j": j, "entry": e}
+            new = {"j": j, "entry": pool_rows(kv_t, g_t, b_t, C, st)}
             if csa:
-                ki_t = np.stack([ring_ki[b, i % Wd] for i in toks])
+                ki_t = np.stack([ring_ki[i % Wd] for i in toks])
                 new["idx_key"] = pool_rows(ki_t, g_t, b_t, spec.di, st)
             if j < Ncap:
                 ent_b = ent_b.copy()
-                ent_b[j] = e
+                ent_b[j] = new["entry"]
                 if csa:
                     idx_b = idx_b.copy()
                     idx_b[j] = new["idx_key"]
-            new_entry[b] = new
-        n_vis = np.array([min(P // m, Ncap)], np.int64)
+        n_vis = np.array([min(Pb // m, Ncap)], np.int64)
         if csa:
             sc = index_scores(yb[cols["qi"]][None], yb[cols["w"]][None], idx_b, n_vis, spec.Hi, spec.di)
-            sel, gap, kth = topk(sc, n_vis, spec.topk)
-            sels.append(sel[0])
-            gaps.append(gap[0])
-            scores_all.append(sc[0])
+            sel, gap, _ = topk(sc, n_vis, spec.topk)
+            res["sel"].append(sel[0])
+            res["gap"].append(gap[0])
+            res["scores"].append(sc[0])
         else:
             sel = None
-        pos = P - win + 1 + np.arange(win)
+        pos = Pb - win + 1 + np.arange(win)
         wrows = np.where(pos >= 0, pos % win, -1)[None, :]
-        outs.append(attend(yb[cols["q"]][None], spec.H, spec.dh, spec.scale, ent_b, sel, n_vis,
-                           win_kv[b], wrows, st)[0])
-    res = {"y": y, "out": np.stack(outs), "win_kv": win_kv, "ring_g": ring_g, "new_entry": new_entry}
+        res["out"].append(attend(yb[cols["q"]][None], spec.H, spec.dh, spec.scale, ent_b, sel, n_vis,
+                                 win_kv, wrows, st)[0])
+        res["y"].append(yb)
+        res["win_kv"].append(win_kv)
+        res["ring_g"].append(ring_g)
+        res["ring_ki"].append(ring_ki)
+        res["entries"].append(ent_b)
+        res["new_entry"].append(new)
+        res["P"] = Pv
+    res["out"] = np.stack(res["out"])
     if csa:
-        res.update(sel=np.stack(sels), gap=np.array(gaps), scores=np.stack(scores_all), ring_ki=ring_ki)
+        res["sel"] = np.stack(res["sel"])
+        res["gap"] = np.array(res["gap"])
     return res
 
 
-def decode_attend_with_sel(spec, res, inp, P, sel_b, b):
-    """Recompute sequence b's decode output on a given selection (e.g. the GPU's)."""
+def decode_attend_with_sel(spec, res, i, sel_row):
+    """Recompute the i-th evaluated row of a decode_step result on a given selection (e.g. the GPU's)."""
     st = storage_code(spec.dtype)
     win = spec.window
     cols = _col_slices(spec)
-    ent = to_f64(inp["entries"][b])
-    if b in res["new_entry"] and res["new_entry"][b]["j"] < ent.shape[0]:
-        ent = ent.copy()
-        ent[res["new_entry"][b]["j"]] = res["new_entry"][b]["entry"]
-    pos = P - win + 1 + np.arange(win)
+    b = res["seqs"][i]
+    Pb = int(res["P"][b])
+    pos = Pb - win + 1 + np.arange(win)
     wrows = np.where(pos >= 0, pos % win, -1)[None, :]
-    return attend(res["y"][b][cols["q"]][None], spec.H, spec.dh, spec.scale, ent, sel_b[None], None,
-                  res["win_kv"][b], wrows, st)[0]
+    return attend(res["y"][i][cols["q"]][None], spec.H, spec.dh, spec.scale, res["entries"][i],
+                  np.asarray(sel_row, np.int32)[None], None, res["win_kv"][i], wrows, st)[0]

@@ -133,10 +133,11 @@ def prefill_inputs(s: LayerSpec, rows=None) -> dict:
     return out
 
 
-def decode_inputs(d: DecodeSpec, layer_index: int, with_cache: bool = True, seqs=None) -> dict:
+def decode_inputs(d: DecodeSpec, layer_index: int, with_cache: bool = True, seqs=None, n_cap=None) -> dict:
     """Weights, new-token x[B,D] and (optionally) the cache of one layer of a decode workload.
 
-    seqs restricts the cache to a subset of sequences (for sampled checks)."""
+    seqs restricts the cache to a subset of sequences; n_cap overrides the entry capacity
+    (default: the P // m entries the prefix has formed)."""
     from . import normal
     s = d.layers[layer_index]
     kind = storage_kind(s)
@@ -145,7 +146,7 @@ def decode_inputs(d: DecodeSpec, layer_index: int, with_cache: bool = True, seqs
     out["W_cat"] = w_cat(s, out)
     out["x"] = normal(d.seed, 0, (d.B, s.D), 1.0, kind)
     if with_cache:
-        N = d.n_cache_entries(s)
+        N = d.n_cache_entries(s) if n_cap is None else n_cap
         seqs = list(range(d.B)) if seqs is None else list(seqs)
         dt = out["x"].dtype
         nb = len(seqs)

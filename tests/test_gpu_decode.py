@@ -1,0 +1,135 @@
+"""GPU parity of the decode path (cache append, indexer + top-k over the cache, split attention) against
+the fp64 oracle, and decode <-> prefill consistency, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._helpers import check_out, check_selection, dev, host64
+
+pytestmark = pytest.mark.gpu
+
+CSA_D = synth.LayerSpec(kind="csa", T=0, D=256, m=4, width=8, C=256, di=64, Hi=8, topk=64, window=128, H=8, dh=128,
+                        scale=128 ** -0.5, dtype="bf16", seed=31)
+HCA_D = synth.LayerSpec(kind="hca", T=0, D=256, m=128, width=128, C=256, window=128, H=4, dh=128,
+                        scale=128 ** -0.5, dtype="bf16", seed=32)
+
+
+def gpu_step(spec, inp, pos, n_cap):
+    from long_context_compressed_05_b200 import DecodeLayer, hcsa_get_device_status
+    cache = {k: dev(inp[k]) for k in ("entries", "win_kv", "ring_g", "idx_keys", "ring_ki") if k in inp}
+    B = inp["x"].shape[0]
+    layer = DecodeLayer(spec, B, n_cap, cache)
+    pos_t = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    layer.step(dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"]), pos_t)
+    torch.cuda.synchronize()
+    assert hcsa_get_device_status() == 0
+    return layer, cache
+
+
+def compare_step(spec, inp, layer, cache, P, seqs):
+    ref = oracle.decode_step(spec, inp, P, seqs=seqs)
+    f32 = spec.dtype == "f32"
+    for i, b in enumerate(seqs):
+        # cache side effects: the new token's rows and any completed entry
+        Pb = int(ref["P"][b])
+        np.testing.assert_allclose(host64(cache["win_kv"][b, Pb % spec.window]), ref["win_kv"][i][Pb % spec.window],
+                                   rtol=1e-6 if f32 else 2 ** -7, atol=1e-6)
+        ne = ref["new_entry"][i]
+        if ne is not None:
+            np.testing.assert_allclose(host64(cache["entries"][b, ne["j"]]), ne["entry"],
+                                       rtol=1e-6 if f32 else 2 ** -6, atol=1e-3 if not f32 else 1e-7)
+            if spec.kind == "csa":
+                np.testing.assert_allclose(host64(cache["idx_keys"][b, ne["j"]]), ne["idx_key"],
+                                           rtol=1e-6 if f32 else 2 ** -6, atol=1e-3 if not f32 else 1e-7)
+        if spec.kind == "csa":
+            sel = layer.sel[b].cpu().numpy()[None]
+            nv = np.array([min(Pb // spec.m, inp["entries"].shape[1])])
+            check_selection(sel, ref["sel"][i:i + 1], ref["gap"][i:i + 1], ref["scores"][i][None], nv, spec.topk,
+                            exact=f32)
+            ref_out = oracle.decode_attend_with_sel(spec, ref, i, sel[0])
+        else:
+            ref_out = ref["out"][i]
+        check_out(host64(layer.out[b]), ref_out, spec.dtype)
+
+
+@pytest.mark.parametrize("spec,pos,n_cap", [
+    (CSA_D, [515, 1023, 2000], 520),             # two appends close an entry
+    (CSA_D.replace(dtype="f32", seed=33), [7, 100, 403], 110),
+    (CSA_D, [3, 130, 259], 80),                   # no entry visible / fewer than k visible
+    (HCA_D, [255, 1000, 383], 16),                # HCA: 255 and 383 close entries 1 and 2
+    (HCA_D.replace(dtype="f32", seed=34), [127, 500, 64], 8),
+])
+def test_decode_small(spec, pos, n_cap):
+    d = synth.DecodeSpec(layers=(spec,), B=len(pos), P=max(pos), seed=spec.seed)
+    inp = synth.decode_inputs(d, 0, n_cap=n_cap)
+    layer, cache = gpu_step(spec, inp, pos, n_cap)
+    compare_step(spec, inp, layer, cache, np.array(pos), list(range(len(pos))))
+
+
+@pytest.mark.parametrize("kind,dtype", [("csa", "f32"), ("csa", "bf16"), ("hca", "bf16")])
+def test_decode_matches_prefill(kind, dtype):
+    """Decode steps over a cache built from a GPU prefill reproduce the GPU prefill of the longer sequence."""
+    from long_context_compressed_05_b200 import DecodeLayer, PrefillLayer
+    base = CSA_D if kind == "csa" else HCA_D.replace(m=16, width=16)
+    spec = base.replace(dtype=dtype)
+    P0, n = (301, 9) if kind == "csa" else (251, 8)
+    full = spec.replace(T=P0 + n)
+    inp = synth.prefill_inputs(full)
+    pre = PrefillLayer(full)
+    pre.forward(dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"]))
+    n_cap = (P0 + n) // spec.m + 2
+    dt = pre.entries.dtype
+    cache = {"entries": torch.zeros((1, n_cap, spec.C), dtype=dt, device="cuda"),
+             "win_kv": torch.zeros((1, spec.window, spec.C), dtype=dt, device="cuda"),
+             "ring_g": torch.zeros((1, spec.width, spec.C), dtype=dt, device="cuda")}
+    nc = P0 // spec.m
+    cache["entries"][0, :nc] = pre.entries[:nc]
+    for p in range(max(0, P0 - spec.window), P0):
+        cache["win_kv"][0, p % spec.window] = pre.view("kv")[p]
+    for p in range(max(0, P0 - spec.width), P0):
+        cache["ring_g"][0, p % spec.width] = pre.view("g")[p]
+    if kind == "csa":
+        cache["idx_keys"] = torch.zeros((1, n_cap, spec.di), dtype=dt, device="cuda")
+        cache["idx_keys"][0, :nc] = pre.idx_keys[:nc]
+        cache["ring_ki"] = torch.zeros((1, spec.width, spec.di), dtype=dt, device="cuda")
+        for p in range(max(0, P0 - spec.width), P0):
+            cache["ring_ki"][0, p % spec.width] = pre.view("ki")[p]
+    layer = DecodeLayer(spec, 1, n_cap, cache)
+    W, Bb = dev(inp["W_cat"]), dev(inp["B"])
+    x = dev(inp["x"])
+    for s in range(n):
+        P = P0 + s
+        layer.step(x[P:P + 1].contiguous(), W, Bb, torch.tensor([P], dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        if kind == "csa":
+            a, b = layer.sel[0].cpu().numpy(), pre.sel[P].cpu().numpy()
+            if dtype == "f32":
+                np.testing.assert_array_equal(a, b)
+            else:   # the one-row projection may round a few bf16 values differently from the T-row one
+                assert len(set(a.tolist()) ^ set(b.tolist())) <= 4
+        got, want = host64(layer.out[0]), host64(pre.out[P])
+        if dtype == "f32":
+            np.testing.assert_allclose(got, want, rtol=0, atol=1e-6)
+        else:
+            assert np.abs(got - want).max() <= 2e-2
+    # every entry completed during the steps equals the prefill's entry
+    for j in range(nc, (P0 + n) // spec.m):
+        np.testing.assert_allclose(host64(cache["entries"][0, j]), host64(pre.entries[j]), rtol=2 ** -6, atol=1e-3)
+
+
+@pytest.mark.parametrize("name", ["csa_decode_b32_p262144", "hybrid_decode_b4_p1048576"])
+def test_decode_full_size_sampled(name):
+    """Full-size decode workloads (all layers, all sequences on the GPU); the oracle checks sampled sequences."""
+    d = synth.DECODE[name]
+    seqs = [0, d.B - 1] if d.B > 2 else [0]
+    for li, spec in enumerate(d.layers):
+        if li >= 2 and li < len(d.layers) - 2:
+            continue   # the middle layers repeat the first two shapes; check first two and last two
+        inp = synth.decode_inputs(d, li)
+        n_cap = inp["entries"].shape[1]
+        layer, cache = gpu_step(spec, inp, [d.P] * d.B, n_cap)
+        compare_step(spec, inp, layer, cache, d.P, seqs)
+        del layer, cache
+        torch.cuda.empty_cache()

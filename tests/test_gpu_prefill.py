@@ -1,0 +1,100 @@
+"""GPU parity of the prefill path (projection, compressor, indexer + top-k, attention) against the
+fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._helpers import check_out, check_selection, dev, host64, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+CSA_SMALL = synth.LayerSpec(kind="csa", T=1003, D=256, m=4, width=8, C=256, di=64, Hi=8, topk=64, window=128, H=8,
+                            dh=128, scale=128 ** -0.5, dtype="bf16", seed=21)
+CSA_WIDE = synth.LayerSpec(kind="csa", T=700, D=512, m=4, width=8, C=1024, di=64, Hi=32, topk=128, window=128,
+                           H=4, dh=512, scale=512 ** -0.5, dtype="bf16", seed=22)
+HCA_SMALL = synth.LayerSpec(kind="hca", T=1500, D=256, m=128, width=128, C=256, window=128, H=4, dh=128,
+                            scale=128 ** -0.5, dtype="bf16", seed=23)
+HCA_F32 = HCA_SMALL.replace(dtype="f32", T=700, seed=24)
+
+CASES = {
+    "csa_f32_t2048": synth.PREFILL["csa_f32_t2048"],
+    "csa_bf16_small": CSA_SMALL,
+    "csa_bf16_wide": CSA_WIDE,
+    "hca_bf16_small": HCA_SMALL,
+    "hca_f32_small": HCA_F32,
+    # edge cases: no visible entry at all, a ragged tail, fewer visible entries than k everywhere
+    "csa_bf16_t3": CSA_SMALL.replace(T=3, seed=25),
+    "csa_bf16_t1": CSA_SMALL.replace(T=1, seed=26),
+    "csa_bf16_vis_lt_k": CSA_SMALL.replace(T=230, seed=27),
+    "csa_f32_ragged": synth.PREFILL["csa_f32_t2048"].replace(T=517, seed=28),
+    "hca_bf16_t100": HCA_SMALL.replace(T=100, seed=29),
+}
+
+
+def run_gpu(spec):
+    from long_context_compressed_05_b200 import PrefillLayer, hcsa_get_device_status
+    inp = synth.prefill_inputs(spec)
+    layer = PrefillLayer(spec)
+    layer.forward(dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"]))
+    torch.cuda.synchronize()
+    assert hcsa_get_device_status() == 0
+    return inp, layer
+
+
+def compare(spec, inp, layer, rows, ref):
+    f32 = spec.dtype == "f32"
+    cols = layer.cols
+    # projections (rounded storage): allow one storage ulp where accumulation order differs
+    y = host64(layer.y[torch.from_numpy(rows).cuda()])
+    pool_end = cols["ki"][1] if spec.kind == "csa" else cols["g"][1]
+    ypool_ref = ref["y_pool"][rows]
+    # fp32 accumulation error is absolute (~1e-6 for unit-scale terms); bf16 adds one storage ulp
+    rt, at = (1e-6, 1e-6) if f32 else (2 ** -7, 1e-5)
+    np.testing.assert_allclose(y[:, :pool_end], ypool_ref, rtol=rt, atol=at)
+    np.testing.assert_allclose(y[:, pool_end:], ref["y_q"], rtol=rt, atol=at)
+    # compressor
+    ent = host64(layer.entries)
+    # bf16: the pooled inputs may differ by a storage ulp (~4e-3 at unit scale)
+    rt, at = (1e-6, 1e-7) if f32 else (2 ** -6, 8e-3)
+    np.testing.assert_allclose(ent, ref["entries"], rtol=rt, atol=at)
+    if spec.kind == "csa":
+        np.testing.assert_allclose(host64(layer.idx_keys), ref["idx_keys"], rtol=rt, atol=at)
+        sel = layer.sel.cpu().numpy()[rows]
+        check_selection(sel, ref["sel"], ref["gap"], ref["scores"], ref["n_vis"], spec.topk, exact=f32)
+        ref_out = oracle.attend_rows(spec, ref, ref["q"], sel)     # oracle on the GPU's own selection
+    else:
+        ref_out = ref["out"]
+    out = host64(layer.out[torch.from_numpy(rows).cuda()])
+    return check_out(out, ref_out, spec.dtype)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_parity(name):
+    spec = CASES[name]
+    inp, layer = run_gpu(spec)
+    rows = np.arange(spec.T, dtype=np.int64)
+    ref = oracle.prefill(spec, inp, rows=rows)
+    compare(spec, inp, layer, rows, ref)
+
+
+def test_prefill_f32_sets_bit_exact_and_deterministic():
+    spec = synth.PREFILL["csa_f32_t2048"]
+    inp, layer = run_gpu(spec)
+    sel1, out1 = layer.sel.clone(), layer.out.clone()
+    layer.forward(dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"]))
+    torch.cuda.synchronize()
+    assert torch.equal(sel1, layer.sel) and torch.equal(out1, layer.out)
+    ref = oracle.prefill(spec, inp)
+    np.testing.assert_array_equal(layer.sel.cpu().numpy(), ref["sel"])
+
+
+@pytest.mark.parametrize("name", ["hca_bf16_t65536", "csa_bf16_t131072"])
+def test_prefill_full_size_sampled(name):
+    """Full-size workloads in the benchmark's launch configuration; the oracle checks sampled query rows."""
+    spec = synth.PREFILL[name]
+    inp, layer = run_gpu(spec)
+    rows = sample_rows(spec.T, spec.m, max(spec.topk, 1), n_random=24 if spec.kind == "csa" else 64)
+    ref = oracle.prefill(spec, inp, rows=rows)
+    compare(spec, inp, layer, rows, ref)

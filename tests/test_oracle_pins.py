@@ -362,4 +362,4 @@ def test_decode_steps_match_prefill(orc, kind):
             j = (P + 1) // m - 1
             np.testing.assert_allclose(d["new_entry"][0]["entry"], ref["entries"][j], rtol=0, atol=1e-6)
         else:
-            assert 0 not in d["new_entry"]
+            assert d["new_entry"][0] is None
