@@ -107,6 +107,9 @@ struct AttendArgs {
 size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, int dh, int topk, int window,
                        int64_t N);
 hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st);
+// tensor-core CSA prefill attention (H = 64, dh = 512, <= 640 keys, bf16)
+bool csa_attend_tc_supported(const AttendArgs &a);
+hcsa_status launch_csa_attend_tc(const AttendArgs &a, cudaStream_t st);
 
 // projection y[rows, ncols] = x[rows, D] W[D, ncols]
 size_t project_ws_bytes(int dtype);

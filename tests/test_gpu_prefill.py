@@ -17,6 +17,10 @@ CSA_WIDE = synth.LayerSpec(kind="csa", T=700, D=512, m=4, width=8, C=1024, di=64
 HCA_SMALL = synth.LayerSpec(kind="hca", T=1500, D=256, m=128, width=128, C=256, window=128, H=4, dh=128,
                             scale=128 ** -0.5, dtype="bf16", seed=23)
 HCA_F32 = HCA_SMALL.replace(dtype="f32", T=700, seed=24)
+# the shapes of the tensor-core attention kernel (64 heads of 512, <= 640 keys), at small D and T
+CSA_TC_K128 = synth.LayerSpec(kind="csa", T=900, D=256, m=4, width=8, C=1024, di=64, Hi=8, topk=128, window=128,
+                              H=64, dh=512, scale=512 ** -0.5, dtype="bf16", seed=41)
+CSA_TC_K512 = CSA_TC_K128.replace(T=2600, topk=512, seed=42)
 
 CASES = {
     "csa_f32_t2048": synth.PREFILL["csa_f32_t2048"],
@@ -30,7 +34,12 @@ CASES = {
     "csa_bf16_vis_lt_k": CSA_SMALL.replace(T=230, seed=27),
     "csa_f32_ragged": synth.PREFILL["csa_f32_t2048"].replace(T=517, seed=28),
     "hca_bf16_t100": HCA_SMALL.replace(T=100, seed=29),
+    "csa_bf16_tc_k128": CSA_TC_K128,
+    "csa_bf16_tc_k512": CSA_TC_K512,
+    "csa_bf16_tc_t5": CSA_TC_K128.replace(T=5, seed=43),
 }
+# query rows checked per case (default: all)
+SAMPLED = {"csa_bf16_tc_k128": 48, "csa_bf16_tc_k512": 48}
 
 
 def run_gpu(spec):
@@ -86,6 +95,8 @@ def test_prefill_parity(name):
     spec = CASES[name]
     inp, layer = run_gpu(spec)
     rows = np.arange(spec.T, dtype=np.int64)
+    if name in SAMPLED:
+        rows = sample_rows(spec.T, spec.m, spec.topk, n_random=SAMPLED[name], seed=spec.seed)
     ref = oracle.prefill(spec, inp, rows=rows)
     compare(spec, inp, layer, rows, ref)
 
