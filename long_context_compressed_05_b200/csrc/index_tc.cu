@@ -1,0 +1,445 @@
+// Lightning indexer on the tensor cores + register-resident exact top-k (bf16 storage).
+//
+// Operation ("DeepSeek-V4 ... KV cache compressed attention", section "CSA":
+// the Lightning Indexer scores the compressed blocks, the top-k are kept; fixed
+// by the CSA workload definition): s[t,j] = sum_h w[t,h] ReLU(qi[t,h,:] . k_j)
+// over visible entries (m j + m <= t); top-k keeps the min(k, visible) best,
+// equal scores to the lower j.
+//
+// Scores kernel.  The contraction has K = di = 64 only, so it is arranged to keep
+// the tensor core and the ReLU-weighted head reduction both busy:
+//   * A = 128 indexer keys (one TMEM lane each), B = TQ tokens x Hi heads of qi
+//     (TQ * Hi = 256 columns for prefill, Hi for decode), both loaded by TMA in the
+//     128-byte swizzled K-major layout (64 bf16 = one swizzle row);
+//   * 4 MMAs (K = 16 each) per key tile into one of two 256-column TMEM
+//     accumulators, so the epilogue of tile i overlaps the MMAs of tile i + 1;
+//   * 8 epilogue warps (two per TMEM lane quadrant, each owning half of the
+//     columns) read the accumulator, apply ReLU, weight by w and sum the heads in
+//     registers -- no cross-lane traffic -- and store fp32 scores coalesced.
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, warps 2..9 = epilogue.
+// Persistent CTAs walk a list of work units (prefill: one query tile each, the
+// heaviest causal tiles first; decode: (sequence, 8 key tiles)).
+//
+// Top-k kernel.  One CTA of 512 threads per query row keeps the row's scores in
+// registers (<= 32768), and finds the k-th largest order-preserving key with three
+// histogram passes (12 + 10 + 10 bits) over the registers, then writes the chosen
+// indices in ascending order with block scans; ties at the k-th value go to the
+// lowest j.
+#include <cub/block/block_scan.cuh>
+
+#include "tc_common.cuh"
+
+namespace hcsa {
+
+namespace {
+
+constexpr int kNS = 4;               // key-tile ring stages
+constexpr int kATile = 128 * 128;    // 128 keys x 64 bf16
+constexpr int kBTile = 256 * 128;    // up to 256 (token, head) rows x 64 bf16
+constexpr int kThreads = 320;        // 10 warps
+constexpr int kEpiThreads = 256;
+constexpr int kDecodeTilesPerUnit = 8;
+
+struct Args {
+    int64_t rows;        // prefill: T; decode: B
+    int64_t N;           // entries per sequence
+    int m, tq, ncols;    // tokens per unit, MMA N = tq * Hi
+    bool decode;
+    const int32_t *pos;
+    const __nv_bfloat16 *w;
+    int64_t ld_w;
+    float *scores;       // [rows, N]
+    int64_t n_units, n_qtiles;
+    int64_t dec_chunks;  // decode: units per sequence
+    int *status;
+};
+
+struct Unit {
+    int64_t b, r0;       // sequence, first query row
+    int kt0, kt1;        // key tiles [kt0, kt1)
+};
+
+__device__ __forceinline__ int64_t visible(const Args &a, int64_t row) {
+    int64_t p = a.decode ? (int64_t)a.pos[row] : row;
+    if (p < 0) return 0;
+    int64_t v = p / a.m;
+    return v < a.N ? v : a.N;
+}
+
+__device__ __forceinline__ Unit unit_of(const Args &a, int64_t u) {
+    Unit x;
+    if (!a.decode) {
+        const int64_t q = a.n_qtiles - 1 - u;   // heaviest first
+        x.b = 0;
+        x.r0 = q * a.tq;
+        int64_t last = x.r0 + a.tq - 1 < a.rows ? x.r0 + a.tq - 1 : a.rows - 1;
+        x.kt0 = 0;
+        x.kt1 = (int)((visible(a, last) + 127) / 128);
+    } else {
+        x.b = u / a.dec_chunks;
+        x.r0 = x.b;
+        const int c = (int)(u % a.dec_chunks);
+        const int nkt = (int)((visible(a, x.b) + 127) / 128);
+        x.kt0 = c * kDecodeTilesPerUnit;
+        x.kt1 = min(nkt, x.kt0 + kDecodeTilesPerUnit);
+    }
+    return x;
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kThreads, 1)
+index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
+                       Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;                       // kNS x 16 KB
+    uint8_t *sB = sA + kNS * kATile;          // 2 x 32 KB
+    float *sw = reinterpret_cast<float *>(sB + 2 * kBTile);   // 2 x 256 head weights
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 512);
+    uint64_t *a_full = bars, *a_empty = bars + kNS, *b_full = bars + 2 * kNS, *b_empty = b_full + 2;
+    uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNS; ++i) { tc::mbar_init(&a_full[i], 1); tc::mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1);
+            tc::mbar_init(&acc_full[i], 1); tc::mbar_init(&acc_empty[i], kEpiThreads / 32);
+        }
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t ia = 0, ib = 0;
+            for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+                const Unit x = unit_of(a, u);
+                if (x.kt0 >= x.kt1) continue;
+                const int bb = ib & 1;
+                if (ib >= 2) ok &= tc::mbar_wait(&b_empty[bb], ((ib >> 1) - 1) & 1, a.status);
+                tc::mbar_arrive_expect_tx(&b_full[bb], a.ncols * 128);
+                tc::tma_load_3d(tc::smem_u32(sB + bb * kBTile), &tm_qi, 0, 0, (int)x.r0, &b_full[bb]);
+                ++ib;
+                for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
+                    const int s = ia % kNS;
+                    if (ia >= kNS) ok &= tc::mbar_wait(&a_empty[s], ((ia / kNS) - 1) & 1, a.status);
+                    tc::mbar_arrive_expect_tx(&a_full[s], kATile);
+                    tc::tma_load_3d(tc::smem_u32(sA + s * kATile), &tm_keys, 0, kt * 128, (int)x.b, &a_full[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16(128, a.ncols, false, false);
+            uint32_t ia = 0, ib = 0, iacc = 0;
+            for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+                const Unit x = unit_of(a, u);
+                if (x.kt0 >= x.kt1) continue;
+                const int bb = ib & 1;
+                ok &= tc::mbar_wait(&b_full[bb], (ib >> 1) & 1, a.status);
+                const uint32_t bsm = tc::smem_u32(sB + bb * kBTile);
+                for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia, ++iacc) {
+                    const int s = ia % kNS, ab = iacc & 1;
+                    ok &= tc::mbar_wait(&a_full[s], (ia / kNS) & 1, a.status);
+                    if (iacc >= 2) ok &= tc::mbar_wait(&acc_empty[ab], ((iacc >> 1) - 1) & 1, a.status);
+                    tc::tc_fence_after();
+                    const uint32_t asm_ = tc::smem_u32(sA + s * kATile);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(tmem + ab * 256, tc::sdesc_sw128(asm_ + 32 * k, 16, 1024),
+                                     tc::sdesc_sw128(bsm + 32 * k, 16, 1024), idesc, k > 0);
+                    tc::mma_commit(&a_empty[s]);
+                    tc::mma_commit(&acc_full[ab]);
+                }
+                tc::mma_commit(&b_empty[bb]);
+                ++ib;
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue: ReLU, head weights, head sum
+        const int et = threadIdx.x - 64;              // 0..255
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int row = quad * 32 + lane;             // key within the tile (TMEM lane)
+        constexpr int TPH = 128 / HI > 0 ? 128 / HI : 1;   // tokens per half (prefill)
+        uint32_t iacc = 0, iu = 0;
+        for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+            const Unit x = unit_of(a, u);
+            if (x.kt0 >= x.kt1) continue;
+            float *w_s = sw + (iu & 1) * 256;
+            if (et < a.ncols) {
+                const int64_t r = x.r0 + et / HI;
+                w_s[et] = r < a.rows ? __bfloat162float(a.w[r * a.ld_w + et % HI]) : 0.f;
+            }
+            tc::named_bar_sync(1, kEpiThreads);
+            ++iu;
+            // rows (queries) of this half and their visible counts
+            const int ntok = a.ncols / HI;                       // tokens in the unit
+            const int tok0 = half * TPH;
+            int64_t vis[TPH];
+#pragma unroll
+            for (int i = 0; i < TPH; ++i) {
+                const int64_t r = x.r0 + tok0 + i;
+                vis[i] = (tok0 + i < ntok && r < a.rows) ? visible(a, r) : 0;
+            }
+            for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++iacc) {
+                const int ab = iacc & 1;
+                ok &= tc::mbar_wait(&acc_full[ab], (iacc >> 1) & 1, a.status);
+                tc::tc_fence_after();
+                float s[TPH];
+#pragma unroll
+                for (int i = 0; i < TPH; ++i) s[i] = 0.f;
+                const uint32_t tl = tmem + ab * 256 + ((uint32_t)(quad * 32) << 16);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int col0 = half * 128 + cc * 32;
+                    if (col0 < a.ncols) {
+                        float v[32];
+                        tc::tmem_ld32(tl + col0, v);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int c = cc * 32 + i;                // column within the half
+                            s[c / HI < TPH ? c / HI : TPH - 1] += w_s[col0 + i] * fmaxf(v[i], 0.f);
+                        }
+                    }
+                }
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
+                const int64_t j = (int64_t)kt * 128 + row;
+#pragma unroll
+                for (int i = 0; i < TPH; ++i)
+                    if (j < vis[i]) a.scores[(x.r0 + tok0 + i) * a.N + j] = s[i];
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_free(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ register-resident top-k
+constexpr int kTkThreads = 512;
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+    if (s == 0.0f) s = 0.0f;   // -0 and +0 compare equal
+    uint32_t b = __float_as_uint(s);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+template <int VPT>   // float4 vectors per thread: row capacity = 2048 * VPT
+__global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__restrict__ scores, int64_t N,
+                                                               int m, const int32_t *__restrict__ pos, int topk,
+                                                               int32_t *__restrict__ sel) {
+    using Scan = cub::BlockScan<int, kTkThreads>;
+    __shared__ typename Scan::TempStorage scan_tmp;
+    __shared__ int hist[4096];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_rem, s_eq_total;
+    const int tid = threadIdx.x;
+    const int64_t r = blockIdx.x;
+    int64_t p = pos ? (int64_t)pos[r] : r;
+    int64_t n = p < 0 ? 0 : (p / m < N ? p / m : N);
+    int32_t *out = sel + r * topk;
+    if (n <= topk) {
+        for (int i = tid; i < topk; i += kTkThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float *row = scores + r * N;
+    const bool vec_ok = (N & 3) == 0;   // rows start 16-byte aligned
+    uint32_t key[VPT * 4];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int64_t j0 = 4 * ((int64_t)tid + (int64_t)kTkThreads * i);
+        if (vec_ok && j0 + 3 < n) {
+            float4 v = __ldcs(reinterpret_cast<const float4 *>(row + j0));
+            key[4 * i] = order_key(v.x); key[4 * i + 1] = order_key(v.y);
+            key[4 * i + 2] = order_key(v.z); key[4 * i + 3] = order_key(v.w);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) key[4 * i + e] = (j0 + e < n) ? order_key(row[j0 + e]) : 0u;
+        }
+    }
+    // three histogram passes: bits [20,32), [10,20), [0,10)
+    uint32_t prefix = 0, mask = 0;
+    int rem = topk;
+    const int shifts[3] = {20, 10, 0};
+    const int widths[3] = {12, 10, 10};
+#pragma unroll
+    for (int pass = 0; pass < 3; ++pass) {
+        const int sh = shifts[pass], nb = 1 << widths[pass];
+        for (int i = tid; i < nb; i += kTkThreads) hist[i] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < VPT * 4; ++i)
+            if ((key[i] & mask) == prefix && key[i] != 0u) atomicAdd(&hist[(key[i] >> sh) & (nb - 1)], 1);
+        __syncthreads();
+        // suffix scan: thread tid owns bins [(nb/512) * (511 - tid), ...) so thread 0 holds the highest bins
+        const int per = nb / kTkThreads;
+        const int b0 = per * (kTkThreads - 1 - tid);
+        int local = 0;
+        for (int i = 0; i < per; ++i) local += hist[b0 + i];
+        int above, total;
+        Scan(scan_tmp).ExclusiveSum(local, above, total);
+        if (above < rem && above + local >= rem) {
+            int cum = above;
+            for (int i = per - 1; i >= 0; --i) {
+                const int c = hist[b0 + i];
+                if (cum + c >= rem) {
+                    s_prefix = prefix | ((uint32_t)(b0 + i) << sh);
+                    s_rem = rem - cum;
+                    break;
+                }
+                cum += c;
+            }
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        rem = s_rem;
+        mask |= (uint32_t)(nb - 1) << sh;
+        __syncthreads();
+    }
+    // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first)
+    int eq_local = 0;
+#pragma unroll
+    for (int i = 0; i < VPT * 4; ++i) eq_local += key[i] == prefix;
+    if (tid == 0) s_eq_total = 0;
+    __syncthreads();
+    if (eq_local) atomicAdd(&s_eq_total, eq_local);
+    __syncthreads();
+    const bool all_eq = s_eq_total <= rem;
+    int base_out = 0, base_eq = 0;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        int take[4], eq[4];
+        int eq_cnt = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            eq[e] = key[4 * i + e] == prefix;
+            eq_cnt += eq[e];
+        }
+        int eq_rank = 0, eq_sum = 0;
+        if (!all_eq) {
+            Scan(scan_tmp).ExclusiveSum(eq_cnt, eq_rank, eq_sum);
+            __syncthreads();
+        }
+        int cnt = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int t_eq = eq[e] && (all_eq || base_eq + eq_rank < rem);
+            eq_rank += eq[e];
+            take[e] = (key[4 * i + e] > prefix) || t_eq;
+            cnt += take[e];
+        }
+        int slot, total;
+        Scan(scan_tmp).ExclusiveSum(cnt, slot, total);
+        __syncthreads();
+        const int64_t j0 = 4 * ((int64_t)tid + (int64_t)kTkThreads * i);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (take[e]) {
+                if (base_out + slot < topk) out[base_out + slot] = (int32_t)(j0 + e);
+                ++slot;
+            }
+        base_out += total;
+        base_eq += eq_sum;
+    }
+}
+
+}  // namespace
+
+bool index_tc_supported(const IndexArgs &a) {
+    if (a.dtype != HCSA_BF16 || a.di != 64) return false;
+    if (!(a.Hi == 8 || a.Hi == 16 || a.Hi == 32 || a.Hi == 64)) return false;
+    if (a.pos && a.Hi < 16) return false;          // decode MMA N = Hi must be >= 16
+    if (((uintptr_t)a.qi & 15) || ((uintptr_t)a.keys & 15) || (a.ld_qi * 2) % 16) return false;
+    return a.N <= INT32_MAX && a.rows <= INT32_MAX;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int HI>
+static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, const CUtensorMap &tq, Args a,
+                                 cudaStream_t st) {
+    constexpr size_t smem = 1024 + kNS * kATile + 2 * kBTile + 512 * sizeof(float) + 16 * sizeof(uint64_t) + 16;
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return HCSA_ERR_CUDA;
+        configured = true;
+    }
+    const int64_t grid = a.n_units < num_sms() ? a.n_units : num_sms();
+    if (grid <= 0) return HCSA_OK;
+    index_scores_tc_kernel<HI><<<(unsigned)grid, kThreads, smem, st>>>(tk, tq, a);
+    count_launch();
+    return check_launch();
+}
+
+hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
+    const bool decode = ia.pos != nullptr;
+    const int64_t nseq = decode ? ia.rows : 1;
+    const int tq = decode ? 1 : 256 / ia.Hi;
+    CUtensorMap tk, tq_map;
+    if (!make_tmap_bf16_3d(&tk, ia.keys, 64, (uint64_t)ia.N, (uint64_t)nseq, 128, (uint64_t)ia.N * 128, 64, 128, 1,
+                           true))
+        return HCSA_ERR_CUDA;
+    if (!make_tmap_bf16_3d(&tq_map, ia.qi, 64, (uint64_t)ia.Hi, (uint64_t)ia.rows, 128, (uint64_t)ia.ld_qi * 2, 64,
+                           (uint32_t)ia.Hi, (uint32_t)tq, true))
+        return HCSA_ERR_CUDA;
+    Args a{};
+    a.rows = ia.rows; a.N = ia.N; a.m = ia.m; a.tq = tq; a.ncols = tq * ia.Hi; a.decode = decode; a.pos = ia.pos;
+    a.w = (const __nv_bfloat16 *)ia.w; a.ld_w = ia.ld_w; a.scores = (float *)ia.ws; a.status = device_status_ptr();
+    if (decode) {
+        const int64_t ntiles = (ia.N + 127) / 128;
+        a.dec_chunks = (ntiles + kDecodeTilesPerUnit - 1) / kDecodeTilesPerUnit;
+        a.n_units = ia.rows * a.dec_chunks;
+        a.n_qtiles = 0;
+    } else {
+        a.n_qtiles = (ia.rows + tq - 1) / tq;
+        a.n_units = a.n_qtiles;
+        a.dec_chunks = 0;
+    }
+    hcsa_status s;
+    switch (ia.Hi) {
+        case 8: s = launch_scores<8>(ia, tk, tq_map, a, st); break;
+        case 16: s = launch_scores<16>(ia, tk, tq_map, a, st); break;
+        case 32: s = launch_scores<32>(ia, tk, tq_map, a, st); break;
+        default: s = launch_scores<64>(ia, tk, tq_map, a, st); break;
+    }
+    if (s != HCSA_OK) return s;
+    // top-k over the materialised scores
+    if (ia.N <= 32768) {
+        const float *sc = (const float *)ia.ws;
+        if (ia.N <= 8192)
+            topk_regs_kernel<4><<<(unsigned)ia.rows, kTkThreads, 0, st>>>(sc, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+        else
+            topk_regs_kernel<16><<<(unsigned)ia.rows, kTkThreads, 0, st>>>(sc, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+        count_launch();
+        return check_launch();
+    }
+    return launch_topk_generic(ia, st);
+}
+
+}  // namespace hcsa

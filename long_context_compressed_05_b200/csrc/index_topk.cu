@@ -173,8 +173,16 @@ size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N) {
     return (size_t)rows * (size_t)N * (dtype == HCSA_BF16 ? sizeof(float) : sizeof(double));
 }
 
+hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st) {
+    if (a.dtype == HCSA_BF16) topk_kernel<float><<<(unsigned)a.rows, kTopkThreads, 0, st>>>(a);
+    else topk_kernel<double><<<(unsigned)a.rows, kTopkThreads, 0, st>>>(a);
+    count_launch();
+    return check_launch();
+}
+
 hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st) {
     if (a.rows == 0) return HCSA_OK;
+    if (index_tc_supported(a)) return launch_index_tc(a, st);
     const int qt = a.pos ? 1 : kQT;
     const size_t esz = a.dtype == HCSA_BF16 ? sizeof(float) : sizeof(double);
     const size_t smem = esz * ((size_t)qt * a.Hi * a.di + (size_t)qt * a.Hi + (size_t)kJT * (a.di + 1));
@@ -193,10 +201,7 @@ hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st) {
         }
         count_launch();
     }
-    if (a.dtype == HCSA_BF16) topk_kernel<float><<<(unsigned)a.rows, kTopkThreads, 0, st>>>(a);
-    else topk_kernel<double><<<(unsigned)a.rows, kTopkThreads, 0, st>>>(a);
-    count_launch();
-    return check_launch();
+    return launch_topk_generic(a, st);
 }
 
 }  // namespace hcsa

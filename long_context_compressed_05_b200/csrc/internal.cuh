@@ -86,6 +86,10 @@ struct IndexArgs {
 };
 size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N);
 hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st);
+hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st);
+// tensor-core indexer scores (bf16, di = 64) + register-resident top-k
+bool index_tc_supported(const IndexArgs &a);
+hcsa_status launch_index_tc(const IndexArgs &a, cudaStream_t st);
 
 // attention.  Prefill (pos == nullptr): query t of one sequence, window rows kv[t-window+1 .. t].
 // Decode: query b at position pos[b], entries of sequence b, window ring win_kv[b].
