@@ -190,6 +190,21 @@ hcsa_status csa_decode_attend(const hcsa_params *p, const hcsa_cache *cache, con
 hcsa_status hca_decode_attend(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
                               int64_t ld_q, void *out, void *ws, size_t ws_bytes, void *stream);
 
+/* Decode: csa_decode_index_topk without a caller workspace, for callers that cannot allocate
+ * device memory (for example code inside a serving engine or host framework that owns every
+ * device allocation and hands out no scratch).  The pages have no counterpart: this is an
+ * interface convenience, not part of the method.
+ * Arguments and results are those of csa_decode_index_topk.  The scores go to one fixed 8 MiB
+ * device array inside the library (held by every GPU that loads the library until exit), so
+ * B * n_cap may be at most 2,097,152 with bf16 storage or 1,048,576 with fp32 storage;
+ * larger requests return HCSA_ERR_WORKSPACE and launch nothing.  Allocates nothing.
+ * The first call on a device (with that device current) looks up the array's device address
+ * once; make that first call before any stream capture.  All calls share the array: calls
+ * that overlap on the GPU (other streams, other host threads) race on it. */
+hcsa_status csa_decode_index_topk_noalloc(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                          const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
+                                          int32_t *sel, void *stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the current device
  * (HCSA_OK, HCSA_ERR_TIMEOUT or HCSA_ERR_DEVICE), or HCSA_ERR_CUDA if the wait itself failed. */
 hcsa_status hcsa_get_device_status(void *stream);

@@ -26,7 +26,8 @@ STATUS = {0: "HCSA_OK", 1: "HCSA_ERR_NULL", 2: "HCSA_ERR_SHAPE", 3: "HCSA_ERR_DT
 # every entry point the header declares (checked by the CPU export test)
 EXPORTS = ["hcsa_version", "hcsa_status_string", "hcsa_workspace_bytes", "hcsa_proj_cols", "hcsa_project",
            "csa_compress", "hca_compress", "csa_index_topk", "csa_attend", "hca_attend", "hcsa_cache_append",
-           "csa_decode_index_topk", "csa_decode_attend", "hca_decode_attend", "hcsa_get_device_status",
+           "csa_decode_index_topk", "csa_decode_attend", "hca_decode_attend", "csa_decode_index_topk_noalloc",
+           "hcsa_get_device_status",
            "hcsa_launch_count"]
 
 
@@ -75,6 +76,7 @@ def load():
         "csa_decode_index_topk": (I32, [P, CP, V, V, I64, V, I64, V, V, SZ, V]),
         "csa_decode_attend": (I32, [P, CP, V, V, I64, V, V, V, SZ, V]),
         "hca_decode_attend": (I32, [P, CP, V, V, I64, V, V, SZ, V]),
+        "csa_decode_index_topk_noalloc": (I32, [P, CP, V, V, I64, V, I64, V, V]),
         "hcsa_get_device_status": (I32, [V]),
         "hcsa_launch_count": (I64, [I32]),
     }
@@ -192,6 +194,13 @@ def csa_decode_attend(p, cache: Cache, pos, q, sel, out, ws=None, stream=None):
 def hca_decode_attend(p, cache: Cache, pos, q, out, ws=None, stream=None):
     _check("hca_decode_attend", load().hca_decode_attend(ctypes.byref(p), ctypes.byref(cache), _ptr(pos), _ptr(q),
                                                          _ld(q), _ptr(out), _ptr(ws), _wsz(ws), _stream(stream)))
+
+
+def csa_decode_index_topk_noalloc(p, cache: Cache, pos, qi, w, sel, stream=None):
+    """csa_decode_index_topk with the scores in the library's fixed scratch array (no workspace)."""
+    _check("csa_decode_index_topk_noalloc", load().csa_decode_index_topk_noalloc(
+        ctypes.byref(p), ctypes.byref(cache), _ptr(pos), _ptr(qi), _ld(qi), _ptr(w), _ld(w), _ptr(sel),
+        _stream(stream)))
 
 
 def hcsa_get_device_status(stream=None) -> int:
