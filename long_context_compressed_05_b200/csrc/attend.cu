@@ -151,7 +151,17 @@ size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, 
 
 hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st) {
     if (a.rows == 0) return HCSA_OK;
-    if (csa_attend_tc_supported(a)) return launch_csa_attend_tc(a, st);
+    if (attend_tc_supported(a)) {
+        const int ns = attend_tc_segments(a);
+        if (ns > 1 &&
+            a.ws_bytes < attend_ws_bytes(a.dtype, true, a.dense, a.rows, a.H, a.dh, a.topk, a.window, a.N))
+            return HCSA_ERR_WORKSPACE;
+        hcsa_status s = launch_attend_tc(a, st);
+        if (s != HCSA_OK || ns == 1) return s;
+        combine_kernel<__nv_bfloat16><<<dim3((unsigned)a.rows, a.H), 128, 0, st>>>(a, ns);
+        count_launch();
+        return check_launch();
+    }
     if ((a.dh + 31) / 32 > kMaxEpl) return HCSA_ERR_UNSUPPORTED;
     const int ns = a.pos ? decode_splits(a.dense, a.topk, a.window, a.N) : 1;
     if (ns > 1 && a.ws_bytes < attend_ws_bytes(a.dtype, true, a.dense, a.rows, a.H, a.dh, a.topk, a.window, a.N))

@@ -1,86 +1,110 @@
-// CSA prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM).
+// MQA attention over compressed entries + the raw window on the 5th-generation tensor cores
+// (tcgen05 + TMEM, TMA row gathers), for 64 heads of dh = 512 (C = 1024), bf16 storage.
 //
-// Operation ("DeepSeek-V4 ... KV cache compressed attention", sections "CSA" and
-// "Ventana deslizante", fixed by the CSA workload definition): for query token t,
-// the keys are the selected compressed entries plus the raw tokens (t - 128, t];
-// key = first C/2 channels of a row, value = last C/2; every one of the H heads
-// shares those keys (MQA); one softmax over the union with scale tau.
+// Operation ("DeepSeek-V4 ... KV cache compressed attention", sections "CSA", "HCA" and
+// "Ventana deslizante", fixed by the CSA workload definition): the query of token t (or the
+// new token of a decode sequence) attends, with every head sharing the keys, to the selected
+// compressed entries (CSA) or to every visible entry (HCA) plus the raw tokens (t - 128, t];
+// key = first C/2 channels of a row, value = last C/2; one softmax with scale tau.
 //
-// Shape handled here: H = 64 heads, dh = C/2 = 512, at most 640 keys (top-k 512 +
-// window 128), bf16 storage.  One CTA (4 warps) per query token.
+// Work unit = (query, segment of its key list).  The key list is the entry part, padded to a
+// multiple of 128 keys, followed by one 128-key window tile.  A unit holds at most 5 tiles
+// (640 keys): prefill CSA is one unit per token (top-k 512 + window), decode splits every
+// sequence into one-tile units whose partial (accumulator, max, sum) are merged by the
+// log-sum-exp combine kernel.
 //
-// Layout choice: the MQA sharing makes the 64 heads the natural N of the MMA and
-// the keys its M, so S^T[key, head] = K . Q^T lands in TMEM with one key per lane
-// (5 tiles x 64 columns).  The softmax is exact and two-pass over all <= 640 keys
-// (per-head max across lanes via a warp transpose-reduction), which avoids any
-// rescaling of the output accumulator.  P^T is written to shared memory as a bf16
-// MN-major operand and O^T[dh, head] = V^T . P^T accumulates in the TMEM columns
-// the scores used (4 x 64 columns).  Gathered key / value rows stream through a
-// 6-stage ring of 16 KB chunks [128 rows x 64 bf16] in the 128-byte swizzled
-// layout, filled with 16-byte cp.async (8 threads per 128-byte row segment, so
-// every warp request covers whole L2 sectors); the MMA of chunk c overlaps the
-// loads of chunks c+1 .. c+4.
+// Per unit, with 128 keys on the TMEM lanes and the 64 heads as the MMA's N:
+//   S^T[key, head] = K . Q^T   tiles 0..3 in TMEM columns [0, 256), tile 4 in [256, 320)
+//   exact softmax over all keys of the unit (per-head max / sum across lanes)
+//   P^T (bf16) -> shared memory as an MN-major operand
+//   O^T[dh, head] = V^T . P^T  4 blocks of 128 dh in columns [256, 512)
+// Q is streamed in 64-dim chunks next to the key chunks, so the scores of the next unit
+// (columns [0, 256)) accumulate while this unit's P V runs and its output drains.
+//
+// Warp roles (persistent CTAs, 11 warps): warps 0-1 load (gathered entry rows and the decode
+// window ring with 16-byte cp.async whose completion arrives on the stage's mbarrier by itself;
+// Q chunks and the prefill window tile -- 128 consecutive raw rows -- with TMA box loads), warp 2 issues the MMAs, warps 3..10 run the softmax and the output
+// epilogue (two warps per TMEM lane quadrant, 32 heads each).  Gathered 128-byte row segments
+// are what bounds this kernel: the gather rate per SM, not the tensor core, sets its speed.
 #include "tc_common.cuh"
 
 namespace hcsa {
 
 namespace {
 
-constexpr int kH = 64;          // heads (MMA N)
-constexpr int kDh = 512;        // head dim = C / 2
-constexpr int kRowElems = 1024; // C
-constexpr int kKT = 128;        // keys per tile (MMA M)
-constexpr int kMaxTiles = 5;    // <= 640 keys
-constexpr int kNS = 6;          // ring stages (even: V chunk pairs sit in adjacent stages)
-constexpr int kStage = 16384;   // [128 rows x 128 bytes]
-constexpr int kUBytes = kMaxTiles * kKT * 128;   // P^T: 640 rows x 64 heads bf16 (Q needs 64 KB of it)
-constexpr int kThreads = 128;
+constexpr int kH = 64;
+constexpr int kDh = 512;
+constexpr int kC = 1024;
+constexpr int kKT = 128;          // keys per tile (MMA M)
+constexpr int kMaxTiles = 5;
+constexpr int kNS = 6;            // key/value ring stages (even: P V pairs sit in adjacent stages)
+constexpr int kStage = 16384;     // 128 rows x 64 bf16
+constexpr int kQStage = kH * 128; // 64 heads x 64 bf16
+constexpr int kPBytes = kMaxTiles * kKT * 128;
+constexpr int kProdThreads = 64;      // warps 0-1
+constexpr int kMmaWarp = 2;
+constexpr int kSoftWarp0 = 3;         // warps 3..10
+constexpr int kThreads = 352;
+constexpr int kSoftThreads = 256;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColB = 256;
 
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, kH, false, false);   // S^T = K . Q^T
 constexpr uint32_t kIdescPV = tc::idesc_bf16(128, kH, true, true);    // O^T = V^T . P^T
 
-struct Smem {
-    uint8_t *U, *ring;
-    const __nv_bfloat16 **rowptr;
-    float *red, *mx, *zinv;
-    uint64_t *empty, *s_done, *o_done;
-    uint32_t *tmem_slot;
-    int *abort_flag;
+struct Params {
+    bool decode, dense;
+    const __nv_bfloat16 *ent, *raw;   // entry rows (ld C) and raw window rows
+    int64_t ld_raw;
+    int64_t nq;          // queries (prefill T, decode B)
+    int64_t N;           // entries per sequence (prefill ceil(T/m), decode n_cap)
+    int m, topk, seg_tiles, nseg;
+    const int32_t *sel, *pos;
+    float scale, scale_log2;
+    __nv_bfloat16 *out;  // direct output [nq, H*dh] (nseg == 1)
+    float *part;         // partials: acc [nq][nseg][H][dh], then (max, sum) [nq][nseg][H][2]
+    int64_t n_units;
+    int *status;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t *raw) {
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-    Smem s;
-    s.U = base;
-    s.ring = base + kUBytes;
-    uint8_t *p = s.ring + kNS * kStage;
-    s.rowptr = reinterpret_cast<const __nv_bfloat16 **>(p);
-    p += sizeof(void *) * kMaxTiles * kKT;
-    s.red = reinterpret_cast<float *>(p);
-    p += sizeof(float) * 4 * kH;
-    s.mx = reinterpret_cast<float *>(p);
-    p += sizeof(float) * kH;
-    s.zinv = reinterpret_cast<float *>(p);
-    p += sizeof(float) * kH;
-    s.empty = reinterpret_cast<uint64_t *>(p);
-    s.s_done = s.empty + kNS;
-    s.o_done = s.s_done + 1;
-    p += sizeof(uint64_t) * (kNS + 2);
-    s.tmem_slot = reinterpret_cast<uint32_t *>(p);
-    s.abort_flag = reinterpret_cast<int *>(p + 4);
-    return s;
+struct Unit {
+    int64_t q, p, nvis;
+    int seg, E, t0, nt;
+};
+
+__device__ __forceinline__ Unit unit_of(const Params &a, int64_t u) {
+    Unit x;
+    x.q = u / a.nseg;
+    x.seg = (int)(u % a.nseg);
+    x.p = a.decode ? (int64_t)a.pos[x.q] : x.q;
+    x.nvis = x.p < 0 ? 0 : (x.p / a.m < a.N ? x.p / a.m : a.N);
+    x.E = a.dense ? (int)((x.nvis + kKT - 1) / kKT) * kKT : a.topk;
+    const int ntiles = x.E / kKT + 1;
+    x.t0 = x.seg * a.seg_tiles;
+    x.nt = ntiles - x.t0;
+    x.nt = x.nt < 0 ? 0 : (x.nt > a.seg_tiles ? a.seg_tiles : x.nt);
+    return x;
 }
 
-constexpr size_t kSmemBytes = 1024 + kUBytes + kNS * kStage + sizeof(void *) * kMaxTiles * kKT +
-                              sizeof(float) * 6 * kH + sizeof(uint64_t) * (kNS + 2) + 16;
+// Row of key kk (index into the query's key list) in the entry tensor (kk < E) or the raw tensor; -1 = masked.
+__device__ __forceinline__ int key_row(const Params &a, const Unit &x, int kk) {
+    if (kk < x.E) {
+        const int64_t j = a.dense ? (int64_t)kk : (int64_t)a.sel[x.q * a.topk + kk];
+        if (j < 0 || j >= x.nvis) return -1;
+        return (int)(a.decode ? x.q * a.N + j : j);
+    }
+    const int64_t pp = x.p - (kKT - 1) + (kk - x.E);
+    if (pp < 0) return -1;
+    return (int)(a.decode ? x.q * kKT + pp % kKT : pp);
+}
 
-// Per head, reduce 64 values across the 32 lanes of a warp (max or sum).  On return lane l holds
-// the warp-wide results for heads 2l and 2l+1 in v[0], v[1].
+__device__ __forceinline__ uint32_t s_col(int t) { return t < 4 ? (uint32_t)(t * kH) : kColB; }
+
 template <bool kMax>
-__device__ __forceinline__ void warp_transpose_reduce(float *v, int lane) {
+__device__ __forceinline__ float warp_transpose_reduce32(float *v, int lane) {
+    // 32 values per lane -> lane l holds the warp-wide reduction of value l
 #pragma unroll
-    for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+    for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
         const bool upper = (lane & o) != 0;
 #pragma unroll
         for (int i = 0; i < n; ++i) {
@@ -90,6 +114,7 @@ __device__ __forceinline__ void warp_transpose_reduce(float *v, int lane) {
             v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
         }
     }
+    return v[0];
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -98,197 +123,308 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-csa_attend_tc_kernel(const __nv_bfloat16 *__restrict__ q, int64_t ld_q, const __nv_bfloat16 *__restrict__ kv,
-                     int64_t ld_kv, const __nv_bfloat16 *__restrict__ entries, const int32_t *__restrict__ sel,
-                     int topk, int window, int64_t N, float scale_log2, __nv_bfloat16 *__restrict__ out,
-                     int *status) {
-    extern __shared__ uint8_t smem_raw[];
-    Smem sm = carve(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t t = blockIdx.x;
-    const int nk = topk + window;
-    const int ntiles = (nk + kKT - 1) / kKT;
-    const int nS = ntiles * 8, total = 2 * nS;
+__device__ __forceinline__ const __nv_bfloat16 *key_ptr(const Params &a, const Unit &x, int kk) {
+    const int row = key_row(a, x, kk);
+    if (row < 0) return nullptr;
+    return kk < x.E ? a.ent + (int64_t)row * kC : a.raw + (int64_t)row * a.ld_raw;
+}
 
-    // ---- key row pointers (nullptr = masked key: zero-filled, probability 0)
-    for (int kk = tid; kk < ntiles * kKT; kk += kThreads) {
-        const __nv_bfloat16 *ptr = nullptr;
-        if (kk < topk) {
-            const int32_t j = sel[t * topk + kk];
-            if (j >= 0 && j < N) ptr = entries + (int64_t)j * kRowElems;
-        } else if (kk < nk) {
-            const int64_t pp = t - window + 1 + (kk - topk);
-            if (pp >= 0) ptr = kv + pp * ld_kv;
-        }
-        sm.rowptr[kk] = ptr;
-    }
-    if (tid == 0) {
-        for (int s = 0; s < kNS; ++s) tc::mbar_init(&sm.empty[s], 1);
-        tc::mbar_init(sm.s_done, 1);
-        tc::mbar_init(sm.o_done, 1);
-        *sm.abort_flag = 0;
+struct Bars {
+    uint64_t rf[kNS], re[kNS], qf[2], qe[2];
+    uint64_t s_full, s_free, p_full, o_full, o_free, fin;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ent,
+                 const __grid_constant__ CUtensorMap tm_raw, Params a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sP = base;                         // P^T: 640 rows x 128 B
+    uint8_t *sRing = sP + kPBytes;              // kNS x 16 KB
+    uint8_t *sQ = sRing + kNS * kStage;         // 2 x 8 KB
+    float *red = reinterpret_cast<float *>(sQ + 2 * kQStage);   // [4][64]
+    float *mx = red + 4 * kH;                   // [64] scaled max
+    float *zinv = mx + kH;                      // [64]
+    float *znat = zinv + kH;                    // [64] sum
+    float *mnat = znat + kH;                    // [64] max logit in natural units (-inf: no valid key)
+    const __nv_bfloat16 **rowptr = reinterpret_cast<const __nv_bfloat16 **>(mnat + kH);   // [2][640]
+    Bars *bars = reinterpret_cast<Bars *>(rowptr + 2 * kMaxTiles * kKT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNS; ++i) { tc::mbar_init(&bars->rf[i], kProdThreads); tc::mbar_init(&bars->re[i], 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&bars->qf[i], 1); tc::mbar_init(&bars->qe[i], 1); }
+        tc::mbar_init(&bars->s_full, 1);
+        tc::mbar_init(&bars->o_full, 1);
+        tc::mbar_init(&bars->s_free, kSoftThreads / 32);
+        tc::mbar_init(&bars->p_full, kSoftThreads / 32);
+        tc::mbar_init(&bars->o_free, kSoftThreads / 32);
+        tc::mbar_init(&bars->fin, 1);
         tc::fence_mbar_init();
     }
-    if (warp == 0) tc::tmem_alloc(sm.tmem_slot, kTmemCols);
+    if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem = *sm.tmem_slot;
-    const uint32_t U = tc::smem_u32(sm.U), ring = tc::smem_u32(sm.ring);
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t P = tc::smem_u32(sP), ring = tc::smem_u32(sRing), Qs = tc::smem_u32(sQ);
+    bool ok = true;
 
-    // ---- loaders
-    auto load_q = [&]() {
-        const __nv_bfloat16 *qrow = q + t * ld_q;
-        for (int idx = tid; idx < kH * 64; idx += kThreads) {
-            const int h = idx >> 6, dc = (idx >> 3) & 7, g = idx & 7;
-            tc::cp_async16(U + dc * 8192 + tc::sw128_offset(h, g), qrow + h * kDh + dc * 64 + g * 8, true);
-        }
-    };
-    auto load_chunk = [&](int c) {
-        int kt, col;
-        if (c < nS) {
-            kt = c >> 3;
-            col = (c & 7) * 64;
-        } else {
-            const int v = c - nS, u = v >> 1;
-            kt = u >> 2;
-            col = kDh + (u & 3) * 128 + (v & 1) * 64;
-        }
-        const uint32_t st = ring + (c % kNS) * kStage;
-        const int g = tid & 7;
+    if (warp < kProdThreads / 32) {
+        // ------------------------------------------------ producers: cp.async gathers + TMA boxes
+        const int pt = threadIdx.x;
+        uint32_t ic = 0, iq = 0, iu = 0;
+        int32_t tma_use[kNS + 2];                        // thread 0: last use index of a stage filled by TMA
+        for (int i = 0; i < kNS + 2; ++i) tma_use[i] = -1;
+        for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+            const Unit x = unit_of(a, u);
+            if (x.nt <= 0) continue;
+            const __nv_bfloat16 **rp = rowptr + (iu & 1) * (kMaxTiles * kKT);
+            for (int kk = pt; kk < x.nt * kKT; kk += kProdThreads) rp[kk] = key_ptr(a, x, x.t0 * kKT + kk);
+            tc::named_bar_sync(2, kProdThreads);
+            ++iu;
+            auto load_chunk = [&](int t, int col) {
+                const int s = ic % kNS;
+                if (ic >= kNS) ok &= tc::mbar_wait(&bars->re[s], ((ic / kNS) - 1) & 1, a.status);
+                const bool tma_tile = !a.decode && (x.t0 + t) * kKT >= x.E;   // prefill window: 128 consecutive rows
+                if (tma_tile) {
+                    if (pt == 0) {
+                        tc::mbar_arrive_expect_tx(&bars->rf[s], kStage);
+                        tc::tma_load_2d(ring + s * kStage, &tm_raw, col, (int)(x.p - (kKT - 1)), &bars->rf[s]);
+                        tma_use[s] = (int32_t)(ic / kNS);
+                    } else {
+                        tc::mbar_arrive(&bars->rf[s]);
+                    }
+                } else {
+                    const int g = pt & 7;
+                    const __nv_bfloat16 *const *rows = rp + t * kKT;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int row = i * 16 + (tid >> 3);
-            const __nv_bfloat16 *p = sm.rowptr[kt * kKT + row];
-            tc::cp_async16(st + tc::sw128_offset(row, g), p ? p + col + g * 8 : entries, p != nullptr);
+                    for (int i = 0; i < 16; ++i) {
+                        const int row = i * 8 + (pt >> 3);
+                        const __nv_bfloat16 *p = rows[row];
+                        tc::cp_async16(ring + s * kStage + tc::sw128_offset(row, g), p ? p + col + g * 8 : a.ent,
+                                       p != nullptr);
+                    }
+                    tc::cp_async_arrive_noinc(&bars->rf[s]);
+                }
+                ++ic;
+            };
+            auto load_q = [&](int dc) {
+                const int qb = iq & 1;
+                if (pt == 0) {
+                    if (iq >= 2) ok &= tc::mbar_wait(&bars->qe[qb], ((iq >> 1) - 1) & 1, a.status);
+                    tc::mbar_arrive_expect_tx(&bars->qf[qb], kQStage);
+                    tc::tma_load_3d(Qs + qb * kQStage, &tm_q, dc * 64, 0, (int)x.q, &bars->qf[qb]);
+                    tma_use[kNS + qb] = (int32_t)(iq >> 1);
+                }
+                ++iq;
+            };
+            const int n1 = x.nt < 4 ? x.nt : 4;
+            for (int dc = 0; dc < 8; ++dc) {          // S phase 1: tiles 0..3
+                load_q(dc);
+                for (int t = 0; t < n1; ++t) load_chunk(t, dc * 64);
+            }
+            if (x.nt == 5)
+                for (int dc = 0; dc < 8; ++dc) {      // S phase 2: tile 4
+                    load_q(dc);
+                    load_chunk(4, dc * 64);
+                }
+            for (int t = 0; t < x.nt; ++t)            // P V: value halves, 64-dh chunks in pairs
+                for (int c = 0; c < 8; ++c) load_chunk(t, kDh + c * 64);
         }
-    };
-
-    load_q();
-    load_chunk(0);
-    tc::cp_async_commit();
-    for (int c = 1; c <= kNS - 3; ++c) {
-        if (c < total) load_chunk(c);
-        tc::cp_async_commit();
-    }
-
-    for (int c = 0; c < total; ++c) {
-        const int cn = c + kNS - 2;
-        if (cn < total) {
-            if (cn >= kNS && !tc::mbar_wait(&sm.empty[cn % kNS], ((cn - kNS) / kNS) & 1, status)) *sm.abort_flag = 1;
-            load_chunk(cn);
+        tc::cp_async_wait_all();
+        if (!ok && pt == 0) {
+            // abandoned run: let every TMA load this thread issued land before the CTA exits
+            for (int i = 0; i < kNS + 2; ++i)
+                if (tma_use[i] >= 0)
+                    tc::mbar_wait(i < kNS ? &bars->rf[i] : &bars->qf[i - kNS], (uint32_t)tma_use[i] & 1, nullptr);
         }
-        tc::cp_async_commit();
-        tc::cp_async_wait<kNS - 2>();
-
-        if (c == nS) {
-            // ---- softmax over all keys: S^T tiles in TMEM -> P^T (bf16) in shared memory
-            if (!tc::mbar_wait(sm.s_done, 0, status)) *sm.abort_flag = 1;
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t ic = 0, iq = 0, iu = 0;
+            for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+                const Unit x = unit_of(a, u);
+                if (x.nt <= 0) continue;
+                const int n1 = x.nt < 4 ? x.nt : 4;
+                if (iu >= 1) ok &= tc::mbar_wait(&bars->s_free, (iu - 1) & 1, a.status);
+                for (int dc = 0; dc < 8; ++dc) {
+                    const int qb = iq & 1;
+                    ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                    for (int t = 0; t < n1; ++t, ++ic) {
+                        const int s = ic % kNS;
+                        ok &= tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
+                        tc::fence_async_smem();   // cp.async data (generic proxy) -> MMA (async proxy)
+                        tc::tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_bf16(tmem + s_col(t), tc::sdesc_sw128(ring + s * kStage + 32 * k, 16, 1024),
+                                         tc::sdesc_sw128(Qs + qb * kQStage + 32 * k, 16, 1024), kIdescS,
+                                         (dc | k) != 0);
+                        tc::mma_commit(&bars->re[s]);
+                    }
+                    tc::mma_commit(&bars->qe[qb]);
+                    ++iq;
+                }
+                if (x.nt == 5) {
+                    if (iu >= 1) ok &= tc::mbar_wait(&bars->o_free, (iu - 1) & 1, a.status);
+                    for (int dc = 0; dc < 8; ++dc, ++ic, ++iq) {
+                        const int qb = iq & 1, s = ic % kNS;
+                        ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                        ok &= tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
+                        tc::fence_async_smem();
+                        tc::tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_bf16(tmem + kColB, tc::sdesc_sw128(ring + s * kStage + 32 * k, 16, 1024),
+                                         tc::sdesc_sw128(Qs + qb * kQStage + 32 * k, 16, 1024), kIdescS,
+                                         (dc | k) != 0);
+                        tc::mma_commit(&bars->re[s]);
+                        tc::mma_commit(&bars->qe[qb]);
+                    }
+                }
+                tc::mma_commit(&bars->s_full);
+                ok &= tc::mbar_wait(&bars->p_full, iu & 1, a.status);
+                tc::tc_fence_after();
+                for (int t = 0; t < x.nt; ++t)
+                    for (int dp = 0; dp < 4; ++dp, ic += 2) {
+                        const int s0 = ic % kNS, s1 = (ic + 1) % kNS;
+                        ok &= tc::mbar_wait(&bars->rf[s0], (ic / kNS) & 1, a.status);
+                        ok &= tc::mbar_wait(&bars->rf[s1], ((ic + 1) / kNS) & 1, a.status);
+                        tc::fence_async_smem();
+                        tc::tc_fence_after();
+                        const uint32_t av = ring + s0 * kStage, bp = P + t * kKT * 128;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            tc::mma_bf16(tmem + kColB + dp * kH, tc::sdesc_sw128(av + 2048 * k, kStage, 1024),
+                                         tc::sdesc_sw128(bp + 2048 * k, kStage, 1024), kIdescPV, (t | k) != 0);
+                        tc::mma_commit(&bars->re[s0]);
+                        tc::mma_commit(&bars->re[s1]);
+                    }
+                tc::mma_commit(&bars->o_full);
+                ++iu;
+            }
+            // every MMA issued by this thread has completed before TMEM is released
+            tc::mma_commit(&bars->fin);
+            tc::mbar_wait(&bars->fin, 0, a.status);
+        }
+    } else {
+        // ------------------------------------------------ softmax + output epilogue (8 warps)
+        const int et = threadIdx.x - kSoftWarp0 * 32;
+        const int quad = warp & 3, hh = (warp - kSoftWarp0) >> 2;
+        const int r = quad * 32 + lane;                  // key row in a tile; dh row in an output block
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        uint32_t iu = 0;
+        for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+            const Unit x = unit_of(a, u);
+            const int64_t slot = x.q * a.nseg + x.seg;
+            if (x.nt <= 0) {
+                if (a.part && et < kH) {
+                    float *pml = a.part + a.nq * (int64_t)a.nseg * kH * kDh;
+                    pml[(slot * kH + et) * 2] = -INFINITY;
+                    pml[(slot * kH + et) * 2 + 1] = 0.f;
+                }
+                continue;
+            }
+            bool valid[kMaxTiles];
+#pragma unroll
+            for (int t = 0; t < kMaxTiles; ++t) valid[t] = t < x.nt && key_row(a, x, (x.t0 + t) * kKT + r) >= 0;
+            ok &= tc::mbar_wait(&bars->s_full, iu & 1, a.status);
             tc::tc_fence_after();
-            const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-            float m[kH];
+            float v[32];
 #pragma unroll
-            for (int h = 0; h < kH; ++h) m[h] = -INFINITY;
-            for (int kt = 0; kt < ntiles; ++kt) {
-                float s[kH];
-                tc::tmem_ld32(tl + kt * kH, s);
-                tc::tmem_ld32(tl + kt * kH + 32, s + 32);
+            for (int i = 0; i < 32; ++i) v[i] = -INFINITY;
+            for (int t = 0; t < x.nt; ++t) {
+                float s[32];
+                tc::tmem_ld32(tl + s_col(t) + hh * 32, s);
                 tc::tmem_ld_wait();
-                if (sm.rowptr[kt * kKT + tid]) {
+                if (valid[t]) {
 #pragma unroll
-                    for (int h = 0; h < kH; ++h) m[h] = fmaxf(m[h], s[h]);
+                    for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], s[i]);
                 }
             }
-            warp_transpose_reduce<true>(m, lane);
-            sm.red[warp * kH + 2 * lane] = m[0];
-            sm.red[warp * kH + 2 * lane + 1] = m[1];
-            __syncthreads();
-            if (tid < kH) {
-                float mm = fmaxf(fmaxf(sm.red[tid], sm.red[kH + tid]), fmaxf(sm.red[2 * kH + tid], sm.red[3 * kH + tid]));
-                sm.mx[tid] = mm * scale_log2;
+            red[quad * kH + hh * 32 + lane] = warp_transpose_reduce32<true>(v, lane);
+            tc::named_bar_sync(1, kSoftThreads);
+            if (et < kH) {
+                const float mm = fmaxf(fmaxf(red[et], red[kH + et]), fmaxf(red[2 * kH + et], red[3 * kH + et]));
+                mx[et] = mm == -INFINITY ? 0.f : mm * a.scale_log2;
+                mnat[et] = mm == -INFINITY ? -INFINITY : mm * a.scale;
             }
-            __syncthreads();
-            float z[kH];
+            tc::named_bar_sync(1, kSoftThreads);
+            float mloc[32];
 #pragma unroll
-            for (int h = 0; h < kH; ++h) z[h] = 0.f;
-            for (int kt = 0; kt < ntiles; ++kt) {
-                float s[kH];
-                tc::tmem_ld32(tl + kt * kH, s);
-                tc::tmem_ld32(tl + kt * kH + 32, s + 32);
+            for (int i = 0; i < 32; ++i) { mloc[i] = mx[hh * 32 + i]; v[i] = 0.f; }
+            for (int t = 0; t < x.nt; ++t) {
+                float s[32];
+                tc::tmem_ld32(tl + s_col(t) + hh * 32, s);
                 tc::tmem_ld_wait();
-                const bool valid = sm.rowptr[kt * kKT + tid] != nullptr;
-                const int R = kt * kKT + tid;
+                const bool vt = valid[t];
+                const uint32_t rowaddr = P + (uint32_t)(t * kKT + r) * 128u;
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
+                for (int g = 0; g < 4; ++g) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int h0 = g * 8 + 2 * e;
-                        float p0 = valid ? ex2(fmaf(s[h0], scale_log2, -sm.mx[h0])) : 0.f;
-                        float p1 = valid ? ex2(fmaf(s[h0 + 1], scale_log2, -sm.mx[h0 + 1])) : 0.f;
-                        z[h0] += p0;
-                        z[h0 + 1] += p1;
+                        const float p0 = vt ? ex2(fmaf(s[h0], a.scale_log2, -mloc[h0])) : 0.f;
+                        const float p1 = vt ? ex2(fmaf(s[h0 + 1], a.scale_log2, -mloc[h0 + 1])) : 0.f;
+                        v[h0] += p0;
+                        v[h0 + 1] += p1;
                         __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                         w[e] = *reinterpret_cast<uint32_t *>(&pr);
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(U + tc::sw128_offset(R, g)),
+                    const uint32_t gg = (uint32_t)(hh * 4 + g);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowaddr + ((gg ^ (uint32_t)(r & 7)) << 4)),
                                  "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                                  : "memory");
                 }
             }
-            warp_transpose_reduce<false>(z, lane);
-            __syncthreads();   // everyone is done reading red[] (max pass)
-            sm.red[warp * kH + 2 * lane] = z[0];
-            sm.red[warp * kH + 2 * lane + 1] = z[1];
-            __syncthreads();
-            if (tid < kH) sm.zinv[tid] = 1.f / (sm.red[tid] + sm.red[kH + tid] + sm.red[2 * kH + tid] + sm.red[3 * kH + tid]);
             tc::tc_fence_before();
-        }
-        tc::fence_async_smem();
-        __syncthreads();
-        if (*sm.abort_flag) break;
-
-        if (tid == 0) {
-            tc::tc_fence_after();
-            if (c < nS) {
-                const int kt = c >> 3, dc = c & 7;
-                const uint32_t a = ring + (c % kNS) * kStage, b = U + dc * 8192;
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    tc::mma_bf16(tmem + kt * kH, tc::sdesc_sw128(a + 32 * k, 16, 1024),
-                                 tc::sdesc_sw128(b + 32 * k, 16, 1024), kIdescS, (dc | k) != 0);
-                tc::mma_commit(&sm.empty[c % kNS]);
-                if (c == nS - 1) tc::mma_commit(sm.s_done);
-            } else if ((c - nS) & 1) {
-                const int u = (c - nS) >> 1, kt = u >> 2, dp = u & 3;
-                const uint32_t a = ring + ((c - 1) % kNS) * kStage, b = U + kt * kKT * 128;
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc::mma_bf16(tmem + dp * kH, tc::sdesc_sw128(a + 2048 * k, kStage, 1024),
-                                 tc::sdesc_sw128(b + 2048 * k, kStage, 1024), kIdescPV, (kt | k) != 0);
-                tc::mma_commit(&sm.empty[(c - 1) % kNS]);
-                tc::mma_commit(&sm.empty[c % kNS]);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->s_free);
+            const float zsum = warp_transpose_reduce32<false>(v, lane);
+            tc::named_bar_sync(1, kSoftThreads);     // everyone is done with red[] from the max pass
+            red[quad * kH + hh * 32 + lane] = zsum;
+            tc::named_bar_sync(1, kSoftThreads);
+            if (et < kH) {
+                const float Z = red[et] + red[kH + et] + red[2 * kH + et] + red[3 * kH + et];
+                zinv[et] = Z > 0.f ? 1.f / Z : 0.f;
+                znat[et] = Z;
             }
-            if (c == total - 1) tc::mma_commit(sm.o_done);
-        }
-    }
-    tc::cp_async_wait<0>();
-
-    // ---- epilogue: O^T[dh, head] / Z[head] -> out[t, head, dh]
-    if (!*sm.abort_flag) {
-        if (tc::mbar_wait(sm.o_done, 0, status)) {
+            tc::fence_async_smem();
+            tc::named_bar_sync(1, kSoftThreads);
+            if (lane == 0) tc::mbar_arrive(&bars->p_full);
+            // ---- output
+            ok &= tc::mbar_wait(&bars->o_full, iu & 1, a.status);
             tc::tc_fence_after();
-            const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-            __nv_bfloat16 *orow = out + t * (int64_t)kH * kDh;
             for (int dp = 0; dp < 4; ++dp) {
-                float o[kH];
-                tc::tmem_ld32(tl + dp * kH, o);
-                tc::tmem_ld32(tl + dp * kH + 32, o + 32);
+                float o[32];
+                tc::tmem_ld32(tl + kColB + dp * kH + hh * 32, o);
                 tc::tmem_ld_wait();
+                const int dh = dp * 128 + r;
+                if (a.part == nullptr) {
+                    __nv_bfloat16 *orow = a.out + x.q * (int64_t)kH * kDh + dh;
 #pragma unroll
-                for (int h = 0; h < kH; ++h) orow[h * kDh + dp * 128 + tid] = __float2bfloat16_rn(o[h] * sm.zinv[h]);
+                    for (int i = 0; i < 32; ++i) {
+                        const int h = hh * 32 + i;
+                        orow[(int64_t)h * kDh] = __float2bfloat16_rn(o[i] * zinv[h]);
+                    }
+                } else {
+                    float *pacc = a.part + slot * (int64_t)kH * kDh + dh;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) pacc[(int64_t)(hh * 32 + i) * kDh] = o[i];
+                }
             }
+            if (a.part && et < kH) {
+                float *pml = a.part + a.nq * (int64_t)a.nseg * kH * kDh;
+                pml[(slot * kH + et) * 2] = mnat[et];
+                pml[(slot * kH + et) * 2 + 1] = znat[et];
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->o_free);
+            ++iu;
         }
     }
     tc::tc_fence_before();
@@ -299,26 +435,82 @@ csa_attend_tc_kernel(const __nv_bfloat16 *__restrict__ q, int64_t ld_q, const __
     }
 }
 
-}  // namespace
+constexpr size_t kSmemBytes = 1024 + kPBytes + kNS * kStage + 2 * kQStage + sizeof(float) * 8 * kH +
+                              sizeof(void *) * 2 * kMaxTiles * kKT + sizeof(Bars) + 16;
 
-bool csa_attend_tc_supported(const AttendArgs &a) {
-    return a.dtype == HCSA_BF16 && a.pos == nullptr && !a.dense && a.H == kH && a.dh == kDh && a.C == kRowElems &&
-           a.topk >= 1 && a.topk + a.window <= kMaxTiles * kKT;
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
 }
 
-hcsa_status launch_csa_attend_tc(const AttendArgs &a, cudaStream_t st) {
+}  // namespace
+
+bool attend_tc_supported(const AttendArgs &a) {
+    if (a.dtype != HCSA_BF16 || a.H != kH || a.dh != kDh || a.C != kC || a.window != kKT) return false;
+    if (a.ld_q % 8 || (a.pos == nullptr && a.ld_kv % 8)) return false;
+    if (a.N > INT32_MAX / 2 || a.rows * (a.pos ? a.N : 1) > INT32_MAX) return false;
+    if (!a.dense) {
+        if (a.topk % kKT) return false;
+        if (a.pos == nullptr && a.topk / kKT + 1 > kMaxTiles) return false;
+    } else if (a.pos == nullptr && (a.N + kKT - 1) / kKT + 1 > kMaxTiles) {
+        return false;
+    }
+    return true;
+}
+
+int attend_tc_segments(const AttendArgs &a) {
+    if (a.pos == nullptr) return 1;
+    const int64_t e = a.dense ? (a.N + kKT - 1) / kKT * kKT : a.topk;
+    return (int)(e / kKT + 1);
+}
+
+hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(csa_attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytes) != cudaSuccess)
+        if (cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+            cudaSuccess)
             return HCSA_ERR_CUDA;
         configured = true;
     }
-    const float scale_log2 = a.scale * 1.4426950408889634f;
-    csa_attend_tc_kernel<<<(unsigned)a.rows, kThreads, kSmemBytes, st>>>(
-        (const __nv_bfloat16 *)a.q, a.ld_q, (const __nv_bfloat16 *)a.kv, a.ld_kv,
-        (const __nv_bfloat16 *)a.entries, a.sel, a.topk, a.window, a.N, scale_log2, (__nv_bfloat16 *)a.out,
-        device_status_ptr());
+    const bool decode = a.pos != nullptr;
+    CUtensorMap tq, te, tr;
+    const uint64_t ent_rows = decode ? (uint64_t)a.rows * a.N : (uint64_t)a.N;
+    if (!make_tmap_bf16_3d(&tq, a.q, kDh, kH, (uint64_t)a.rows, kDh * 2, (uint64_t)a.ld_q * 2, 64, kH, 1, true))
+        return HCSA_ERR_CUDA;
+    if (!make_tmap_bf16_2d(&te, a.entries, kC, ent_rows, kC * 2, 64, 1, true)) return HCSA_ERR_CUDA;
+    if (decode) {
+        tr = te;   // unused: decode window rows are gathered from the ring
+    } else if (!make_tmap_bf16_2d(&tr, a.kv, kC, (uint64_t)a.rows, (uint64_t)a.ld_kv * 2, 64, kKT, true)) {
+        return HCSA_ERR_CUDA;
+    }
+    Params p{};
+    p.ent = (const __nv_bfloat16 *)a.entries;
+    p.raw = (const __nv_bfloat16 *)a.kv;
+    p.ld_raw = decode ? kC : a.ld_kv;
+    p.decode = decode;
+    p.dense = a.dense;
+    p.nq = a.rows;
+    p.N = a.N;
+    p.m = a.m;
+    p.topk = a.topk;
+    p.nseg = attend_tc_segments(a);
+    p.seg_tiles = decode ? 1 : kMaxTiles;
+    p.sel = a.sel;
+    p.pos = a.pos;
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.out = (__nv_bfloat16 *)a.out;
+    p.part = p.nseg > 1 ? (float *)a.ws : nullptr;
+    p.n_units = a.rows * p.nseg;
+    p.status = device_status_ptr();
+    const int64_t grid = p.n_units < num_sms() ? p.n_units : num_sms();
+    attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tq, te, tr, p);
     count_launch();
     return check_launch();
 }

@@ -111,9 +111,10 @@ struct AttendArgs {
 size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, int dh, int topk, int window,
                        int64_t N);
 hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st);
-// tensor-core CSA prefill attention (H = 64, dh = 512, <= 640 keys, bf16)
-bool csa_attend_tc_supported(const AttendArgs &a);
-hcsa_status launch_csa_attend_tc(const AttendArgs &a, cudaStream_t st);
+// tensor-core MQA attention (H = 64, dh = 512, window 128, bf16): prefill CSA, decode CSA and HCA
+bool attend_tc_supported(const AttendArgs &a);
+int attend_tc_segments(const AttendArgs &a);     // key segments per query (> 1: partials + combine)
+hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st);
 
 // projection y[rows, ncols] = x[rows, D] W[D, ncols]
 size_t project_ws_bytes(int dtype);

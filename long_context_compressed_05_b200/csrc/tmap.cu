@@ -33,4 +33,19 @@ bool make_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0,
+                       uint32_t b1, bool swizzle128) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {s1};
+    cuuint32_t box[2] = {b0, b1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace hcsa

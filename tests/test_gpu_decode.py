@@ -14,6 +14,9 @@ CSA_D = synth.LayerSpec(kind="csa", T=0, D=256, m=4, width=8, C=256, di=64, Hi=8
                         scale=128 ** -0.5, dtype="bf16", seed=31)
 HCA_D = synth.LayerSpec(kind="hca", T=0, D=256, m=128, width=128, C=256, window=128, H=4, dh=128,
                         scale=128 ** -0.5, dtype="bf16", seed=32)
+# the tensor-core attention shapes (64 heads of 512, key segments of 128 merged by the combine kernel)
+CSA_TC = CSA_D.replace(C=1024, H=64, dh=512, Hi=32, topk=128, scale=512 ** -0.5, seed=35)
+HCA_TC = HCA_D.replace(C=1024, H=64, dh=512, scale=512 ** -0.5, seed=36)
 
 
 def gpu_step(spec, inp, pos, n_cap):
@@ -60,6 +63,8 @@ def compare_step(spec, inp, layer, cache, P, seqs):
     (CSA_D, [3, 130, 259], 80),                   # no entry visible / fewer than k visible
     (HCA_D, [255, 1000, 383], 16),                # HCA: 255 and 383 close entries 1 and 2
     (HCA_D.replace(dtype="f32", seed=34), [127, 500, 64], 8),
+    (CSA_TC, [515, 1023, 60], 300),               # P = 60: 15 visible < k and a partial window
+    (HCA_TC, [255, 3000, 100], 30),               # 255 closes entry 1; 100: window only
 ])
 def test_decode_small(spec, pos, n_cap):
     d = synth.DecodeSpec(layers=(spec,), B=len(pos), P=max(pos), seed=spec.seed)
