@@ -194,10 +194,12 @@ hcsa_status hca_decode_attend(const hcsa_params *p, const hcsa_cache *cache, con
  * device memory (for example code inside a serving engine or host framework that owns every
  * device allocation and hands out no scratch).  The pages have no counterpart: this is an
  * interface convenience, not part of the method.
- * Arguments and results are those of csa_decode_index_topk.  The scores go to one fixed 8 MiB
- * device array inside the library (held by every GPU that loads the library until exit), so
- * B * n_cap may be at most 2,097,152 with bf16 storage or 1,048,576 with fp32 storage;
- * larger requests return HCSA_ERR_WORKSPACE and launch nothing.  Allocates nothing.
+ * Arguments and results are those of csa_decode_index_topk.  Its scratch (the scores, plus 49,168
+ * bytes per sequence for the multi-block selection when n_cap > 32768) goes to one fixed 8 MiB
+ * device array inside the library (held by every GPU that loads the library until exit):
+ * hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK) must be at most 8 MiB -- with bf16
+ * storage B * n_cap <= 2,097,152 while n_cap <= 32768 -- or the call returns HCSA_ERR_WORKSPACE
+ * and launches nothing.  Allocates nothing.
  * The first call on a device (with that device current) looks up the array's device address
  * once; make that first call before any stream capture.  All calls share the array: calls
  * that overlap on the GPU (other streams, other host threads) race on it. */

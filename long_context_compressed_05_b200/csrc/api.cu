@@ -115,7 +115,11 @@ size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op) {
                                                         p->window, n_entries(p));
         case HCSA_OP_HCA_ATTEND: return attend_ws_bytes(p->dtype, false, true, p->T, p->H, p->dh, 0, p->window,
                                                         n_entries(p));
-        case HCSA_OP_CSA_DECODE_INDEX_TOPK: return index_topk_ws_bytes(p->dtype, p->B, p->n_cap);
+        case HCSA_OP_CSA_DECODE_INDEX_TOPK: {
+            size_t b = index_topk_ws_bytes(p->dtype, p->B, p->n_cap);
+            if (p->dtype == HCSA_BF16 && p->n_cap > 32768) b = ((b + 255) & ~(size_t)255) + topk_rows_ws_bytes(p->B);
+            return b;
+        }
         case HCSA_OP_CSA_DECODE_ATTEND: return attend_ws_bytes(p->dtype, true, false, p->B, p->H, p->dh, p->topk,
                                                                p->window, p->n_cap);
         case HCSA_OP_HCA_DECODE_ATTEND: return attend_ws_bytes(p->dtype, true, true, p->B, p->H, p->dh, 0,
@@ -173,7 +177,7 @@ hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, 
     if (!ws && p->T > 0) return HCSA_ERR_WORKSPACE;
     if (ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
     IndexArgs a{p->dtype, p->T, p->Hi, p->di, p->topk, p->m, n_entries(p), qi, ld_qi, w, ld_w, idx_keys,
-                nullptr, sel, ws, ws_bytes};
+                nullptr, sel, ws, ws_bytes, nullptr};
     return launch_index_topk(a, (cudaStream_t)stream);
 }
 
@@ -229,7 +233,7 @@ hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache,
     if (ld_qi < (int64_t)p->Hi * p->di || ld_w < p->Hi) return HCSA_ERR_SHAPE;
     if (!ws || ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
     IndexArgs a{p->dtype, p->B, p->Hi, p->di, p->topk, p->m, p->n_cap, qi, ld_qi, w, ld_w, cache->idx_keys,
-                pos, sel, ws, ws_bytes};
+                pos, sel, ws, ws_bytes, nullptr};
     return launch_index_topk(a, (cudaStream_t)stream);
 }
 

@@ -104,33 +104,74 @@ __global__ void __launch_bounds__(kHeadsPerCta * 32) attend_kernel(AttendArgs a,
     if (lane == 0) { pml[slot * 2] = mx; pml[slot * 2 + 1] = z; }
 }
 
+// Log-sum-exp merge of the per-split partials of one (row, head): weights exp(m_s - M) / Z are computed
+// once per CTA in shared memory, then every thread merges one output element across the splits.
 template <typename S>
-__global__ void combine_kernel(AttendArgs a, int nsplit) {
+__global__ void __launch_bounds__(512) combine_kernel(AttendArgs a, int nsplit) {
     using A = typename Traits<S>::A;
+    extern __shared__ __align__(16) unsigned char comb_smem[];
+    A *wgt = reinterpret_cast<A *>(comb_smem);      // [nsplit]
+    A *red = wgt + nsplit;                          // [blockDim.x]
     const int64_t r = blockIdx.x;
     const int h = blockIdx.y;
     const A *pacc = reinterpret_cast<const A *>(a.ws);
     const A *pml = pacc + a.rows * (int64_t)nsplit * a.H * a.dh;
-    A M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) {
-        A m = pml[((r * nsplit + s) * a.H + h) * 2];
-        M = m > M ? m : M;
+    A mloc = -INFINITY;
+    for (int s = threadIdx.x; s < nsplit; s += blockDim.x) {
+        const A m = pml[((r * nsplit + s) * a.H + h) * 2];
+        wgt[s] = m;
+        mloc = m > mloc ? m : mloc;
     }
-    A Z = A(0);
-    for (int s = 0; s < nsplit; ++s) {
-        const int64_t slot = (r * nsplit + s) * a.H + h;
-        A m = pml[slot * 2];
-        if (m != -INFINITY) Z += exp_acc(m - M) * pml[slot * 2 + 1];
+    red[threadIdx.x] = mloc;
+    __syncthreads();
+    for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+        if (threadIdx.x < o) red[threadIdx.x] = red[threadIdx.x + o] > red[threadIdx.x] ? red[threadIdx.x + o] : red[threadIdx.x];
+        __syncthreads();
     }
+    const A M = red[0];
+    __syncthreads();
+    A zloc = A(0);
+    for (int s = threadIdx.x; s < nsplit; s += blockDim.x) {
+        const A m = wgt[s];
+        const A e = m == -INFINITY ? A(0) : exp_acc(m - M);
+        wgt[s] = e;
+        zloc += e * pml[((r * nsplit + s) * a.H + h) * 2 + 1];
+    }
+    red[threadIdx.x] = zloc;
+    __syncthreads();
+    for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+        if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+        __syncthreads();
+    }
+    const A Z = red[0];
+    const A zi = Z > A(0) ? A(1) / Z : A(0);
     S *o = reinterpret_cast<S *>(a.out) + r * (int64_t)a.H * a.dh + (int64_t)h * a.dh;
+    const A *base = pacc + ((r * nsplit) * a.H + h) * (int64_t)a.dh;
+    const int64_t sstride = (int64_t)a.H * a.dh;
     for (int d = threadIdx.x; d < a.dh; d += blockDim.x) {
         A acc = A(0);
+#pragma unroll 4
         for (int s = 0; s < nsplit; ++s) {
-            const int64_t slot = (r * nsplit + s) * a.H + h;
-            A m = pml[slot * 2];
-            if (m != -INFINITY) acc += exp_acc(m - M) * pacc[slot * a.dh + d];
+            const A wv = wgt[s];
+            if (wv != A(0)) acc += wv * base[s * sstride + d];
         }
-        store_val(&o[d], Z > A(0) ? acc / Z : A(0));
+        store_val(&o[d], acc * zi);
+    }
+}
+
+static void launch_combine(const AttendArgs &a, int ns, cudaStream_t st) {
+    int threads = 32;
+    while (threads < a.dh && threads < 512) threads <<= 1;
+    const size_t esz = a.dtype == HCSA_BF16 ? sizeof(float) : sizeof(double);
+    const size_t smem = esz * ((size_t)ns + threads);
+    if (a.dtype == HCSA_BF16) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        combine_kernel<__nv_bfloat16><<<dim3((unsigned)a.rows, a.H), threads, smem, st>>>(a, ns);
+    } else {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(combine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        combine_kernel<float><<<dim3((unsigned)a.rows, a.H), threads, smem, st>>>(a, ns);
     }
 }
 
@@ -158,7 +199,7 @@ hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st) {
             return HCSA_ERR_WORKSPACE;
         hcsa_status s = launch_attend_tc(a, st);
         if (s != HCSA_OK || ns == 1) return s;
-        combine_kernel<__nv_bfloat16><<<dim3((unsigned)a.rows, a.H), 128, 0, st>>>(a, ns);
+        launch_combine(a, ns, st);
         count_launch();
         return check_launch();
     }
@@ -168,13 +209,9 @@ hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st) {
         return HCSA_ERR_WORKSPACE;
     if (ns > 65535) return HCSA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)a.rows, (a.H + kHeadsPerCta - 1) / kHeadsPerCta, ns);
-    if (a.dtype == HCSA_BF16) {
-        attend_kernel<__nv_bfloat16><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns);
-        if (ns > 1) combine_kernel<__nv_bfloat16><<<dim3((unsigned)a.rows, a.H), 128, 0, st>>>(a, ns);
-    } else {
-        attend_kernel<float><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns);
-        if (ns > 1) combine_kernel<float><<<dim3((unsigned)a.rows, a.H), 128, 0, st>>>(a, ns);
-    }
+    if (a.dtype == HCSA_BF16) attend_kernel<__nv_bfloat16><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns);
+    else attend_kernel<float><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns);
+    if (ns > 1) launch_combine(a, ns, st);
     count_launch(ns > 1 ? 2 : 1);
     return check_launch();
 }

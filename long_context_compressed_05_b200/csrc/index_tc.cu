@@ -439,6 +439,15 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         count_launch();
         return check_launch();
     }
+    if (topk_rows_supported(ia)) {
+        // scratch for the multi-CTA select sits after the scores
+        uint8_t *scratch = (uint8_t *)ia.ws + (((size_t)ia.rows * ia.N * sizeof(float) + 255) & ~(size_t)255);
+        hcsa_status s2 = launch_topk_rows(ia, scratch, st);
+        if (s2 != HCSA_OK) return s2;
+        IndexArgs fb = ia;                       // rows whose threshold bucket overflowed the candidate list
+        fb.only_rows = (const int32_t *)(scratch + (size_t)ia.rows * 4096 * sizeof(uint32_t));
+        return launch_topk_generic(fb, st);
+    }
     return launch_topk_generic(ia, st);
 }
 

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
     __shared__ int s_base_eq, s_base_out;
 
     const int64_t r = blockIdx.x;
+    if (a.only_rows && a.only_rows[4 * r + 3] == 0) return;
     const int64_t p = a.pos ? a.pos[r] : r;
     const int64_t n = p < 0 ? 0 : (p / a.m < a.N ? p / a.m : a.N);
     const int k = a.topk;

@@ -83,8 +83,13 @@ struct IndexArgs {
     const int32_t *pos;  // decode positions (nullptr: prefill, query t at position t)
     int32_t *sel;
     void *ws; size_t ws_bytes;
+    const int32_t *only_rows;   // if set: the generic select handles only rows r with only_rows[4 r + 3] != 0
 };
 size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N);
+// multi-CTA exact top-k for long decode rows (N > 32768); scratch after the scores
+bool topk_rows_supported(const IndexArgs &a);
+size_t topk_rows_ws_bytes(int64_t rows);
+hcsa_status launch_topk_rows(const IndexArgs &a, void *scratch, cudaStream_t st);
 hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st);
 hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st);
 // tensor-core indexer scores (bf16, di = 64) + register-resident top-k
