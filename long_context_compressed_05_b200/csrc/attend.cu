@@ -145,17 +145,25 @@ __global__ void __launch_bounds__(512) combine_kernel(AttendArgs a, int nsplit) 
     }
     const A Z = red[0];
     const A zi = Z > A(0) ? A(1) / Z : A(0);
+    // compact the splits that hold keys (an empty split's accumulator is never written)
+    int *idx = reinterpret_cast<int *>(red + blockDim.x);
+    __shared__ int n_live;
+    if (threadIdx.x == 0) {
+        int c = 0;
+        for (int s = 0; s < nsplit; ++s)
+            if (wgt[s] != A(0)) { idx[c] = s; wgt[c] = wgt[s] * zi; ++c; }
+        n_live = c;
+    }
+    __syncthreads();
+    const int nl = n_live;
     S *o = reinterpret_cast<S *>(a.out) + r * (int64_t)a.H * a.dh + (int64_t)h * a.dh;
     const A *base = pacc + ((r * nsplit) * a.H + h) * (int64_t)a.dh;
     const int64_t sstride = (int64_t)a.H * a.dh;
     for (int d = threadIdx.x; d < a.dh; d += blockDim.x) {
         A acc = A(0);
-#pragma unroll 4
-        for (int s = 0; s < nsplit; ++s) {
-            const A wv = wgt[s];
-            if (wv != A(0)) acc += wv * base[s * sstride + d];
-        }
-        store_val(&o[d], acc * zi);
+#pragma unroll 16
+        for (int i = 0; i < nl; ++i) acc += wgt[i] * base[idx[i] * sstride + d];
+        store_val(&o[d], acc);
     }
 }
 
@@ -163,7 +171,7 @@ static void launch_combine(const AttendArgs &a, int ns, cudaStream_t st) {
     int threads = 32;
     while (threads < a.dh && threads < 512) threads <<= 1;
     const size_t esz = a.dtype == HCSA_BF16 ? sizeof(float) : sizeof(double);
-    const size_t smem = esz * ((size_t)ns + threads);
+    const size_t smem = esz * ((size_t)ns + threads) + sizeof(int) * (size_t)ns;
     if (a.dtype == HCSA_BF16) {
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -187,11 +187,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             auto load_chunk = [&](int t, int col) {
                 const int s = ic % kNS;
                 if (ic >= kNS) ok &= tc::mbar_wait(&bars->re[s], ((ic / kNS) - 1) & 1, a.status);
-                const bool tma_tile = !a.decode && (x.t0 + t) * kKT >= x.E;   // prefill window: 128 consecutive rows
-                if (tma_tile) {
+                const int kt = x.t0 + t;
+                // 128 consecutive rows: the prefill window, or a dense (HCA) entry tile inside the visible range
+                const bool win_tile = !a.decode && kt * kKT >= x.E;
+                const bool ent_tile = a.dense && (int64_t)(kt + 1) * kKT <= x.nvis;
+                if (win_tile || ent_tile) {
                     if (pt == 0) {
                         tc::mbar_arrive_expect_tx(&bars->rf[s], kStage);
-                        tc::tma_load_2d(ring + s * kStage, &tm_raw, col, (int)(x.p - (kKT - 1)), &bars->rf[s]);
+                        if (win_tile)
+                            tc::tma_load_2d(ring + s * kStage, &tm_raw, col, (int)(x.p - (kKT - 1)), &bars->rf[s]);
+                        else
+                            tc::tma_load_2d(ring + s * kStage, &tm_ent, col,
+                                            (int)((a.decode ? x.q * a.N : 0) + (int64_t)kt * kKT), &bars->rf[s]);
                         tma_use[s] = (int32_t)(ic / kNS);
                     } else {
                         tc::mbar_arrive(&bars->rf[s]);
@@ -483,7 +490,7 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     const uint64_t ent_rows = decode ? (uint64_t)a.rows * a.N : (uint64_t)a.N;
     if (!make_tmap_bf16_3d(&tq, a.q, kDh, kH, (uint64_t)a.rows, kDh * 2, (uint64_t)a.ld_q * 2, 64, kH, 1, true))
         return HCSA_ERR_CUDA;
-    if (!make_tmap_bf16_2d(&te, a.entries, kC, ent_rows, kC * 2, 64, 1, true)) return HCSA_ERR_CUDA;
+    if (!make_tmap_bf16_2d(&te, a.entries, kC, ent_rows, kC * 2, 64, kKT, true)) return HCSA_ERR_CUDA;
     if (decode) {
         tr = te;   // unused: decode window rows are gathered from the ring
     } else if (!make_tmap_bf16_2d(&tr, a.kv, kC, (uint64_t)a.rows, (uint64_t)a.ld_kv * 2, 64, kKT, true)) {

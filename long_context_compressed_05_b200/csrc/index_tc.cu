@@ -33,7 +33,7 @@ namespace hcsa {
 
 namespace {
 
-constexpr int kNS = 4;               // key-tile ring stages
+constexpr int kNS = 8;               // key-tile ring stages
 constexpr int kATile = 128 * 128;    // 128 keys x 64 bf16
 constexpr int kBTile = 256 * 128;    // up to 256 (token, head) rows x 64 bf16
 constexpr int kThreads = 320;        // 10 warps

@@ -59,7 +59,19 @@ __global__ void __launch_bounds__(kThreads) rows_hist_kernel(RowArgs a) {
     __syncthreads();
     const float *row = a.scores + r * a.N;
     const int64_t e = s0 + kSlice < n ? s0 + kSlice : n;
-    for (int64_t j = s0 + threadIdx.x; j < e; j += kThreads) atomicAdd(&h[okey(row[j]) >> 20], 1u);
+    if ((a.N & 3) == 0 && e - s0 == kSlice) {   // full slice, 16-byte aligned: vector loads
+        const float4 *v = reinterpret_cast<const float4 *>(row + s0);
+#pragma unroll 4
+        for (int i = threadIdx.x; i < kSlice / 4; i += kThreads) {
+            const float4 x = v[i];
+            atomicAdd(&h[okey(x.x) >> 20], 1u);
+            atomicAdd(&h[okey(x.y) >> 20], 1u);
+            atomicAdd(&h[okey(x.z) >> 20], 1u);
+            atomicAdd(&h[okey(x.w) >> 20], 1u);
+        }
+    } else {
+        for (int64_t j = s0 + threadIdx.x; j < e; j += kThreads) atomicAdd(&h[okey(row[j]) >> 20], 1u);
+    }
     __syncthreads();
     uint32_t *g = a.hist + r * kBins;
     for (int i = threadIdx.x; i < kBins; i += kThreads)
@@ -108,29 +120,48 @@ __global__ void __launch_bounds__(kThreads) rows_collect_kernel(RowArgs a) {
     uint64_t *cand = a.cand + r * kCap;
     const int64_t e = s0 + kSlice < n ? s0 + kSlice : n;
     const int lane = threadIdx.x & 31;
-    for (int64_t base = s0; base < e; base += kThreads) {
-        const int64_t j = base + threadIdx.x;
-        uint32_t k = 0;
-        bool take = false;
-        if (j < e) {
-            k = okey(row[j]);
-            take = (k >> 20) >= bucket;
-        }
+    auto push = [&](uint32_t k, int64_t j, bool take) {
         const uint32_t m = __ballot_sync(0xffffffffu, take);
-        if (!m) continue;
+        if (!m) return;
         int slot = 0;
         if (lane == 0) slot = atomicAdd(&a.meta[r * 4 + 2], __popc(m));
         slot = __shfl_sync(0xffffffffu, slot, 0) + __popc(m & ((1u << lane) - 1u));
         if (take && slot < kCap) cand[slot] = ((uint64_t)k << 32) | (uint32_t)j;
+    };
+    if ((a.N & 3) == 0 && e - s0 == kSlice) {
+        const float4 *v = reinterpret_cast<const float4 *>(row + s0);
+        for (int i = threadIdx.x; i < kSlice / 4; i += kThreads) {
+            const float4 x = v[i];
+            const int64_t j = s0 + 4 * (int64_t)i;
+            const uint32_t k0 = okey(x.x), k1 = okey(x.y), k2 = okey(x.z), k3 = okey(x.w);
+            if (!__any_sync(0xffffffffu, (k0 >> 20) >= bucket || (k1 >> 20) >= bucket || (k2 >> 20) >= bucket ||
+                                             (k3 >> 20) >= bucket))
+                continue;
+            push(k0, j, (k0 >> 20) >= bucket);
+            push(k1, j + 1, (k1 >> 20) >= bucket);
+            push(k2, j + 2, (k2 >> 20) >= bucket);
+            push(k3, j + 3, (k3 >> 20) >= bucket);
+        }
+    } else {
+        for (int64_t base = s0; base < e; base += kThreads) {
+            const int64_t j = base + threadIdx.x;
+            uint32_t k = 0;
+            bool take = false;
+            if (j < e) {
+                k = okey(row[j]);
+                take = (k >> 20) >= bucket;
+            }
+            push(k, j, take);
+        }
     }
 }
 
-// bitonic sort of kCap 64-bit values in shared memory, descending
-__device__ void sort_desc(uint64_t *v) {
-    for (int size = 2; size <= kCap; size <<= 1)
+// bitonic sort of n (power of two) 64-bit values in shared memory, descending
+__device__ void sort_desc(uint64_t *v, int n) {
+    for (int size = 2; size <= n; size <<= 1)
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             __syncthreads();
-            for (int i = threadIdx.x; i < kCap / 2; i += blockDim.x) {
+            for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
                 const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
                 const bool desc = (lo & size) == 0;
                 const uint64_t x = v[lo], y = v[hi];
@@ -151,8 +182,10 @@ __global__ void __launch_bounds__(1024) rows_select_kernel(RowArgs a) {
     }
     if (a.meta[r * 4 + 3]) return;   // finished by the single-CTA select
     const int cnt = a.meta[r * 4 + 2];
+    int n2 = 1;
+    while (n2 < cnt) n2 <<= 1;
     // (key desc, index asc): store key << 32 | ~index so a descending sort puts lower indices first
-    for (int i = threadIdx.x; i < kCap; i += blockDim.x) {
+    for (int i = threadIdx.x; i < n2; i += blockDim.x) {
         uint64_t x = 0;
         if (i < cnt) {
             const uint64_t c = a.cand[r * kCap + i];
@@ -160,10 +193,13 @@ __global__ void __launch_bounds__(1024) rows_select_kernel(RowArgs a) {
         }
         v[i] = x;
     }
-    sort_desc(v);
+    sort_desc(v, n2);
     // the first topk entries are the selection; re-sort their indices ascending (as descending ~index)
-    for (int i = threadIdx.x; i < kCap; i += blockDim.x) v[i] = i < a.topk ? (uint64_t)(uint32_t)v[i] : 0;
-    sort_desc(v);   // ~index descending == index ascending
+    int k2 = 1;
+    while (k2 < a.topk) k2 <<= 1;
+    __syncthreads();
+    for (int i = threadIdx.x; i < k2; i += blockDim.x) v[i] = i < a.topk ? (uint64_t)(uint32_t)v[i] : 0;
+    sort_desc(v, k2);   // ~index descending == index ascending
     for (int i = threadIdx.x; i < a.topk; i += blockDim.x) out[i] = (int32_t)(~(uint32_t)v[i]);
 }
 
