@@ -471,10 +471,17 @@ bool attend_tc_supported(const AttendArgs &a) {
     return true;
 }
 
+// Decode splits each sequence's key list into units: one tile per unit for CSA (the gathered rows
+// are the bottleneck, so spread them over as many SMs as possible), four for HCA (contiguous
+// entry tiles load fast; fewer units write fewer partials).
+static int decode_seg_tiles(const AttendArgs &a) { return a.dense ? 4 : 1; }
+
 int attend_tc_segments(const AttendArgs &a) {
     if (a.pos == nullptr) return 1;
     const int64_t e = a.dense ? (a.N + kKT - 1) / kKT * kKT : a.topk;
-    return (int)(e / kKT + 1);
+    const int64_t tiles = e / kKT + 1;
+    const int st = decode_seg_tiles(a);
+    return (int)((tiles + st - 1) / st);
 }
 
 hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
@@ -507,7 +514,7 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.m = a.m;
     p.topk = a.topk;
     p.nseg = attend_tc_segments(a);
-    p.seg_tiles = decode ? 1 : kMaxTiles;
+    p.seg_tiles = decode ? decode_seg_tiles(a) : kMaxTiles;
     p.sel = a.sel;
     p.pos = a.pos;
     p.scale = a.scale;

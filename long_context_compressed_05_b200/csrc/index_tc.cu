@@ -44,6 +44,7 @@ struct Args {
     int64_t rows;        // prefill: T; decode: B
     int64_t N;           // entries per sequence
     int m, tq, ncols;    // tokens per unit, MMA N = tq * Hi
+    int nbuf, stride;    // TMEM accumulators (2 x 256 columns, or 4 x 128 when ncols <= 128)
     bool decode;
     const int32_t *pos;
     const __nv_bfloat16 *w;
@@ -97,16 +98,14 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
     float *sw = reinterpret_cast<float *>(sB + 2 * kBTile);   // 2 x 256 head weights
     uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 512);
     uint64_t *a_full = bars, *a_empty = bars + kNS, *b_full = bars + 2 * kNS, *b_empty = b_full + 2;
-    uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNS; ++i) { tc::mbar_init(&a_full[i], 1); tc::mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1);
-            tc::mbar_init(&acc_full[i], 1); tc::mbar_init(&acc_empty[i], kEpiThreads / 32);
-        }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1); }
+        for (int i = 0; i < 4; ++i) { tc::mbar_init(&acc_full[i], 1); tc::mbar_init(&acc_empty[i], kEpiThreads / 32); }
         tc::fence_mbar_init();
     }
     if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
@@ -148,14 +147,15 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 ok &= tc::mbar_wait(&b_full[bb], (ib >> 1) & 1, a.status);
                 const uint32_t bsm = tc::smem_u32(sB + bb * kBTile);
                 for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia, ++iacc) {
-                    const int s = ia % kNS, ab = iacc & 1;
+                    const int s = ia % kNS, ab = iacc % a.nbuf;
                     ok &= tc::mbar_wait(&a_full[s], (ia / kNS) & 1, a.status);
-                    if (iacc >= 2) ok &= tc::mbar_wait(&acc_empty[ab], ((iacc >> 1) - 1) & 1, a.status);
+                    if (iacc >= (uint32_t)a.nbuf)
+                        ok &= tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
                     tc::tc_fence_after();
                     const uint32_t asm_ = tc::smem_u32(sA + s * kATile);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(tmem + ab * 256, tc::sdesc_sw128(asm_ + 32 * k, 16, 1024),
+                        tc::mma_bf16(tmem + ab * a.stride, tc::sdesc_sw128(asm_ + 32 * k, 16, 1024),
                                      tc::sdesc_sw128(bsm + 32 * k, 16, 1024), idesc, k > 0);
                     tc::mma_commit(&a_empty[s]);
                     tc::mma_commit(&acc_full[ab]);
@@ -166,10 +166,15 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
         }
     } else {
         // ------------------------------------------------ epilogue: ReLU, head weights, head sum
+        // Prefill (256 columns): the two warp groups split the columns of every tile.  Decode (<= 128
+        // columns): the groups take alternate tiles, each reading all columns.
         const int et = threadIdx.x - 64;              // 0..255
         const int quad = warp & 3, half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;             // key within the tile (TMEM lane)
-        constexpr int TPH = 128 / HI > 0 ? 128 / HI : 1;   // tokens per half (prefill)
+        const bool split = a.ncols <= 128;
+        constexpr int TPH = 128 / HI > 0 ? 128 / HI : 1;   // tokens per 128 columns
+        const int tok_base = split ? 0 : half * TPH;
+        const int col_base = split ? 0 : half * 128;
         uint32_t iacc = 0, iu = 0;
         for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
             const Unit x = unit_of(a, u);
@@ -181,44 +186,43 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
             }
             tc::named_bar_sync(1, kEpiThreads);
             ++iu;
-            // rows (queries) of this half and their visible counts
             const int ntok = a.ncols / HI;                       // tokens in the unit
-            const int tok0 = half * TPH;
             int64_t vis[TPH];
 #pragma unroll
             for (int i = 0; i < TPH; ++i) {
-                const int64_t r = x.r0 + tok0 + i;
-                vis[i] = (tok0 + i < ntok && r < a.rows) ? visible(a, r) : 0;
+                const int64_t r = x.r0 + tok_base + i;
+                vis[i] = (tok_base + i < ntok && r < a.rows) ? visible(a, r) : 0;
             }
             for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++iacc) {
-                const int ab = iacc & 1;
-                ok &= tc::mbar_wait(&acc_full[ab], (iacc >> 1) & 1, a.status);
+                if (split && (int)(iacc & 1) != half) continue;
+                const int ab = iacc % a.nbuf;
+                ok &= tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
                 tc::tc_fence_after();
                 float s[TPH];
 #pragma unroll
                 for (int i = 0; i < TPH; ++i) s[i] = 0.f;
-                const uint32_t tl = tmem + ab * 256 + ((uint32_t)(quad * 32) << 16);
+                const uint32_t tl = tmem + ab * a.stride + ((uint32_t)(quad * 32) << 16);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    const int col0 = half * 128 + cc * 32;
+                    const int col0 = col_base + cc * 32;
                     if (col0 < a.ncols) {
                         float v[32];
                         tc::tmem_ld32(tl + col0, v);
                         tc::tmem_ld_wait();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            const int c = cc * 32 + i;                // column within the half
+                            const int c = cc * 32 + i;                // column within this group's 128
                             s[c / HI < TPH ? c / HI : TPH - 1] += w_s[col0 + i] * fmaxf(v[i], 0.f);
                         }
                     }
                 }
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
+                if (lane == 0) tc::mbar_arrive_cnt(&acc_empty[ab], split ? 2 : 1);
                 const int64_t j = (int64_t)kt * 128 + row;
 #pragma unroll
                 for (int i = 0; i < TPH; ++i)
-                    if (j < vis[i]) a.scores[(x.r0 + tok0 + i) * a.N + j] = s[i];
+                    if (j < vis[i]) a.scores[(x.r0 + tok_base + i) * a.N + j] = s[i];
             }
         }
     }
@@ -382,7 +386,7 @@ static int num_sms() {
 template <int HI>
 static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, const CUtensorMap &tq, Args a,
                                  cudaStream_t st) {
-    constexpr size_t smem = 1024 + kNS * kATile + 2 * kBTile + 512 * sizeof(float) + 16 * sizeof(uint64_t) + 16;
+    constexpr size_t smem = 1024 + kNS * kATile + 2 * kBTile + 512 * sizeof(float) + (2 * kNS + 12) * sizeof(uint64_t) + 16;
     static bool configured = false;
     if (!configured) {
         if (cudaFuncSetAttribute(index_scores_tc_kernel<HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -410,6 +414,8 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         return HCSA_ERR_CUDA;
     Args a{};
     a.rows = ia.rows; a.N = ia.N; a.m = ia.m; a.tq = tq; a.ncols = tq * ia.Hi; a.decode = decode; a.pos = ia.pos;
+    a.nbuf = a.ncols <= 128 ? 4 : 2;
+    a.stride = a.ncols <= 128 ? 128 : 256;
     a.w = (const __nv_bfloat16 *)ia.w; a.ld_w = ia.ld_w; a.scores = (float *)ia.ws; a.status = device_status_ptr();
     if (decode) {
         const int64_t ntiles = (ia.N + 127) / 128;

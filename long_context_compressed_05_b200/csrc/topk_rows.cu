@@ -11,8 +11,9 @@
 //               keys are in higher buckets.
 //   3. collect: each CTA appends (key, index) of every key in that bucket or above to the row's
 //               candidate list (one atomic per warp).
-//   4. select:  one CTA per row sorts the candidates by (key desc, index asc) in shared memory,
-//               keeps the first k and sorts their indices ascending.
+//   4. select:  one CTA per row refines the threshold inside the bucket (two 10-bit histogram passes
+//               over the candidates), marks the chosen indices in a bitmap of the row and emits them in
+//               ascending order with a block scan over the bitmap words.
 // The candidate list holds at most `cap` entries per row; a row whose threshold bucket overflows
 // it is finished by the generic single-CTA select instead.
 #include "internal.cuh"
@@ -156,57 +157,145 @@ __global__ void __launch_bounds__(kThreads) rows_collect_kernel(RowArgs a) {
     }
 }
 
-// bitonic sort of n (power of two) 64-bit values in shared memory, descending
-__device__ void sort_desc(uint64_t *v, int n) {
-    for (int size = 2; size <= n; size <<= 1)
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            __syncthreads();
-            for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
-                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const uint64_t x = v[lo], y = v[hi];
-                if ((x < y) == desc) { v[lo] = y; v[hi] = x; }
-            }
-        }
-    __syncthreads();
-}
+constexpr int kSelThreads = 1024;
+constexpr int kMaxRow = 1 << 18;   // rows up to 262144 entries use the shared-memory bitmap
 
-__global__ void __launch_bounds__(1024) rows_select_kernel(RowArgs a) {
-    extern __shared__ uint64_t v[];   // kCap
+// Exact selection among the candidates of one row, then the indices in ascending order:
+//   two 10-bit histogram passes over the low 20 key bits of the threshold-bucket candidates give the
+//   k-th largest key K* and how many keys equal to K* are taken (lowest index first); every chosen
+//   index is set in a bitmap of the row, and a block scan over the bitmap words emits them in order.
+__global__ void __launch_bounds__(kSelThreads) rows_select_kernel(RowArgs a) {
+    extern __shared__ uint32_t sm[];
+    uint32_t *bitmap = sm;                       // kMaxRow / 32 words
+    uint32_t *hist = bitmap + kMaxRow / 32;      // 1024 bins
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_rem, s_eq_cnt, s_base;
+    __shared__ uint32_t eq_idx[64];
+    __shared__ uint32_t warp_sums[kSelThreads / 32];
     const int64_t r = blockIdx.x;
     const int64_t n = row_n(a, r);
     int32_t *out = a.sel + r * a.topk;
+    const int tid = threadIdx.x;
     if (n <= a.topk) {
-        for (int i = threadIdx.x; i < a.topk; i += blockDim.x) out[i] = i < n ? i : -1;
+        for (int i = tid; i < a.topk; i += kSelThreads) out[i] = i < n ? i : -1;
         return;
     }
     if (a.meta[r * 4 + 3]) return;   // finished by the single-CTA select
     const int cnt = a.meta[r * 4 + 2];
-    int n2 = 1;
-    while (n2 < cnt) n2 <<= 1;
-    // (key desc, index asc): store key << 32 | ~index so a descending sort puts lower indices first
-    for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        uint64_t x = 0;
-        if (i < cnt) {
-            const uint64_t c = a.cand[r * kCap + i];
-            x = (c & 0xFFFFFFFF00000000ull) | (uint32_t)(~(uint32_t)c);
+    const uint32_t bucket = (uint32_t)a.meta[r * 4 + 0];
+    const uint64_t *cand = a.cand + r * kCap;
+    // refine the threshold inside the bucket: bits [10, 20), then [0, 10)
+    uint32_t prefix = bucket << 20, mask = 0xFFF00000u;
+    int rem = a.topk - a.meta[r * 4 + 1];
+    for (int pass = 0; pass < 2; ++pass) {
+        const int sh = pass == 0 ? 10 : 0;
+        for (int i = tid; i < 1024; i += kSelThreads) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < cnt; i += kSelThreads) {
+            const uint32_t k = (uint32_t)(cand[i] >> 32);
+            if ((k & mask) == prefix) atomicAdd(&hist[(k >> sh) & 1023u], 1u);
         }
-        v[i] = x;
+        __syncthreads();
+        if (tid < 32) {   // one warp scans the 1024 bins from the top
+            uint32_t local = 0;
+            for (int i = 0; i < 32; ++i) local += hist[1023 - (tid * 32 + i)];
+            uint32_t incl = local;
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += y;
+            }
+            const uint32_t excl = incl - local;
+            if (excl < (uint32_t)rem && incl >= (uint32_t)rem) {
+                uint32_t cum = excl;
+                for (int i = 0; i < 32; ++i) {
+                    const int bin = 1023 - (tid * 32 + i);
+                    if (cum + hist[bin] >= (uint32_t)rem) {
+                        s_prefix = prefix | ((uint32_t)bin << sh);
+                        s_rem = rem - (int)cum;
+                        break;
+                    }
+                    cum += hist[bin];
+                }
+            }
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        rem = s_rem;
+        mask |= 1023u << sh;
+        __syncthreads();
     }
-    sort_desc(v, n2);
-    // the first topk entries are the selection; re-sort their indices ascending (as descending ~index)
-    int k2 = 1;
-    while (k2 < a.topk) k2 <<= 1;
+    // prefix = K*: keys above are taken, plus the `rem` lowest indices among keys equal to K*
+    for (int i = tid; i < (int)((n + 31) / 32); i += kSelThreads) bitmap[i] = 0;
+    if (tid == 0) s_eq_cnt = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < k2; i += blockDim.x) v[i] = i < a.topk ? (uint64_t)(uint32_t)v[i] : 0;
-    sort_desc(v, k2);   // ~index descending == index ascending
-    for (int i = threadIdx.x; i < a.topk; i += blockDim.x) out[i] = (int32_t)(~(uint32_t)v[i]);
+    for (int i = tid; i < cnt; i += kSelThreads) {
+        const uint64_t c = cand[i];
+        const uint32_t k = (uint32_t)(c >> 32), j = (uint32_t)c;
+        if (k > prefix) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+        else if (k == prefix) {
+            const int e = atomicAdd(&s_eq_cnt, 1);
+            if (e < 64) eq_idx[e] = j;
+        }
+    }
+    __syncthreads();
+    if (s_eq_cnt > 64) {
+        // too many keys tie at the threshold to rank here: hand the row to the single-CTA select
+        if (tid == 0) a.meta[r * 4 + 3] = 1;
+        return;
+    }
+    if (tid == 0) {
+        int ne = s_eq_cnt < 64 ? s_eq_cnt : 64;
+        // take the `rem` lowest indices among the equal keys (selection by repeated minimum; ne is small)
+        for (int t = 0; t < rem && t < ne; ++t) {
+            int best = t;
+            for (int q = t + 1; q < ne; ++q)
+                if (eq_idx[q] < eq_idx[best]) best = q;
+            const uint32_t tmp = eq_idx[t];
+            eq_idx[t] = eq_idx[best];
+            eq_idx[best] = tmp;
+            bitmap[eq_idx[t] >> 5] |= 1u << (eq_idx[t] & 31);
+        }
+    }
+    __syncthreads();
+    // ascending emission: each thread owns a contiguous range of bitmap words
+    const int nw = (int)((n + 31) / 32);
+    const int per = (nw + kSelThreads - 1) / kSelThreads;
+    const int w0 = tid * per;
+    int local = 0;
+    for (int w = w0; w < w0 + per && w < nw; ++w) local += __popc(bitmap[w]);
+    int incl = local;
+    const int lane = tid & 31, wid = tid >> 5;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[wid] = (uint32_t)incl;
+    __syncthreads();
+    if (wid == 0) {
+        int v = lane < kSelThreads / 32 ? (int)warp_sums[lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += y;
+        }
+        if (lane < kSelThreads / 32) warp_sums[lane] = (uint32_t)v;
+    }
+    __syncthreads();
+    int pos = incl - local + (wid > 0 ? (int)warp_sums[wid - 1] : 0);
+    for (int w = w0; w < w0 + per && w < nw; ++w) {
+        uint32_t bits = bitmap[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (pos < a.topk) out[pos] = w * 32 + b;
+            ++pos;
+        }
+    }
 }
 
 }  // namespace
 
 bool topk_rows_supported(const IndexArgs &a) {
-    return a.pos != nullptr && a.dtype == HCSA_BF16 && a.topk <= 2048 && a.N > 32768 && a.N <= INT32_MAX;
+    return a.pos != nullptr && a.dtype == HCSA_BF16 && a.topk <= kCap && a.N > 32768 && a.N <= kMaxRow;
 }
 
 size_t topk_rows_ws_bytes(int64_t rows) {
@@ -235,14 +324,15 @@ hcsa_status launch_topk_rows(const IndexArgs &ia, void *extra, cudaStream_t st) 
     rows_hist_kernel<<<g2, kThreads, 0, st>>>(a);
     rows_bucket_kernel<<<(unsigned)ia.rows, kThreads, 0, st>>>(a);
     rows_collect_kernel<<<g2, kThreads, 0, st>>>(a);
+    constexpr size_t sel_smem = (kMaxRow / 32 + 1024) * sizeof(uint32_t);
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(rows_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(kCap * sizeof(uint64_t))) != cudaSuccess)
+        if (cudaFuncSetAttribute(rows_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem) !=
+            cudaSuccess)
             return HCSA_ERR_CUDA;
         configured = true;
     }
-    rows_select_kernel<<<(unsigned)ia.rows, 1024, kCap * sizeof(uint64_t), st>>>(a);
+    rows_select_kernel<<<(unsigned)ia.rows, kSelThreads, sel_smem, st>>>(a);
     count_launch(4);
     return check_launch();
 }
