@@ -181,7 +181,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const Unit x = unit_of(a, u);
             if (x.nt <= 0) continue;
             const __nv_bfloat16 **rp = rowptr + (iu & 1) * (kMaxTiles * kKT);
-            for (int kk = pt; kk < x.nt * kKT; kk += kProdThreads) rp[kk] = key_ptr(a, x, x.t0 * kKT + kk);
+            {
+                // all selection indices of the unit are loaded before any is used (independent loads in flight)
+                constexpr int kPer = kMaxTiles * kKT / kProdThreads;   // 10
+                int32_t jsel[kPer];
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int kk = x.t0 * kKT + pt + i * kProdThreads;
+                    jsel[i] = (pt + i * kProdThreads < x.nt * kKT && !a.dense && kk < x.E) ? __ldg(&a.sel[x.q * a.topk + kk])
+                                                                                      : 0;
+                }
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int loc = pt + i * kProdThreads;
+                    if (loc >= x.nt * kKT) break;
+                    const int kk = x.t0 * kKT + loc;
+                    const __nv_bfloat16 *ptr = nullptr;
+                    if (kk < x.E) {
+                        const int64_t j = a.dense ? (int64_t)kk : (int64_t)jsel[i];
+                        if (j >= 0 && j < x.nvis) ptr = a.ent + ((a.decode ? x.q * a.N : 0) + j) * (int64_t)kC;
+                    } else {
+                        const int64_t pp = x.p - (kKT - 1) + (kk - x.E);
+                        if (pp >= 0) ptr = a.raw + (a.decode ? x.q * kKT + pp % kKT : pp) * a.ld_raw;
+                    }
+                    rp[loc] = ptr;
+                }
+            }
             tc::named_bar_sync(2, kProdThreads);
             ++iu;
             auto load_chunk = [&](int t, int col) {
@@ -335,8 +360,28 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 continue;
             }
             bool valid[kMaxTiles];
+            {
+                int32_t jsel[kMaxTiles];
 #pragma unroll
-            for (int t = 0; t < kMaxTiles; ++t) valid[t] = t < x.nt && key_row(a, x, (x.t0 + t) * kKT + r) >= 0;
+                for (int t = 0; t < kMaxTiles; ++t) {
+                    const int kk = (x.t0 + t) * kKT + r;
+                    jsel[t] = (t < x.nt && !a.dense && kk < x.E) ? __ldg(&a.sel[x.q * a.topk + kk]) : 0;
+                }
+#pragma unroll
+                for (int t = 0; t < kMaxTiles; ++t) {
+                    const int kk = (x.t0 + t) * kKT + r;
+                    bool v = false;
+                    if (t < x.nt) {
+                        if (kk < x.E) {
+                            const int64_t j = a.dense ? (int64_t)kk : (int64_t)jsel[t];
+                            v = j >= 0 && j < x.nvis;
+                        } else {
+                            v = x.p - (kKT - 1) + (kk - x.E) >= 0;
+                        }
+                    }
+                    valid[t] = v;
+                }
+            }
             ok &= tc::mbar_wait(&bars->s_full, iu & 1, a.status);
             tc::tc_fence_after();
             float v[32];

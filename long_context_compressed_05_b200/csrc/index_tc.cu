@@ -22,9 +22,9 @@
 //
 // Top-k kernel.  One CTA of 512 threads per query row keeps the row's scores in
 // registers (<= 32768), and finds the k-th largest order-preserving key with three
-// histogram passes (12 + 10 + 10 bits) over the registers, then writes the chosen
-// indices in ascending order with block scans; ties at the k-th value go to the
-// lowest j.
+// histogram passes (12 + 10 + 10 bits) over the registers; the chosen indices are
+// marked in a shared-memory bitmap of the row (ties at the k-th value: lowest j) and
+// emitted in ascending order with one block scan over the bitmap words.
 #include <cub/block/block_scan.cuh>
 
 #include "tc_common.cuh"
@@ -38,7 +38,7 @@ constexpr int kATile = 128 * 128;    // 128 keys x 64 bf16
 constexpr int kBTile = 256 * 128;    // up to 256 (token, head) rows x 64 bf16
 constexpr int kThreads = 320;        // 10 warps
 constexpr int kEpiThreads = 256;
-constexpr int kDecodeTilesPerUnit = 8;
+constexpr int kDecodeTilesPerUnit = 32;
 
 struct Args {
     int64_t rows;        // prefill: T; decode: B
@@ -250,6 +250,8 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
     using Scan = cub::BlockScan<int, kTkThreads>;
     __shared__ typename Scan::TempStorage scan_tmp;
     __shared__ int hist[4096];
+    __shared__ uint32_t bitmap[1024];   // rows of up to 32768 entries
+    __shared__ uint32_t eq_idx[64];
     __shared__ uint32_t s_prefix;
     __shared__ int s_rem, s_eq_total;
     const int tid = threadIdx.x;
@@ -315,50 +317,67 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
         mask |= (uint32_t)(nb - 1) << sh;
         __syncthreads();
     }
-    // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first)
-    int eq_local = 0;
-#pragma unroll
-    for (int i = 0; i < VPT * 4; ++i) eq_local += key[i] == prefix;
+    // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first).
+    // Mark the chosen indices in a bitmap of the row, then emit them in ascending order with one scan.
+    const int nw = (int)((n + 31) / 32);
+    for (int i = tid; i < nw; i += kTkThreads) bitmap[i] = 0;
     if (tid == 0) s_eq_total = 0;
     __syncthreads();
-    if (eq_local) atomicAdd(&s_eq_total, eq_local);
-    __syncthreads();
-    const bool all_eq = s_eq_total <= rem;
-    int base_out = 0, base_eq = 0;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        int take[4], eq[4];
-        int eq_cnt = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            eq[e] = key[4 * i + e] == prefix;
-            eq_cnt += eq[e];
-        }
-        int eq_rank = 0, eq_sum = 0;
-        if (!all_eq) {
-            Scan(scan_tmp).ExclusiveSum(eq_cnt, eq_rank, eq_sum);
-            __syncthreads();
-        }
-        int cnt = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            int t_eq = eq[e] && (all_eq || base_eq + eq_rank < rem);
-            eq_rank += eq[e];
-            take[e] = (key[4 * i + e] > prefix) || t_eq;
-            cnt += take[e];
-        }
-        int slot, total;
-        Scan(scan_tmp).ExclusiveSum(cnt, slot, total);
-        __syncthreads();
-        const int64_t j0 = 4 * ((int64_t)tid + (int64_t)kTkThreads * i);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (take[e]) {
-                if (base_out + slot < topk) out[base_out + slot] = (int32_t)(j0 + e);
-                ++slot;
+            const uint32_t kv = key[4 * i + e];
+            const int64_t j = 4 * ((int64_t)tid + (int64_t)kTkThreads * i) + e;
+            if (kv > prefix) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+            else if (kv == prefix && kv != 0u) {
+                const int q = atomicAdd(&s_eq_total, 1);
+                if (q < 64) eq_idx[q] = (uint32_t)j;
             }
-        base_out += total;
-        base_eq += eq_sum;
+        }
+    }
+    __syncthreads();
+    if (s_eq_total > 64) {
+        // many equal keys at the threshold: mark the lowest `rem` of them by scanning the row in order
+        if (tid < 32) {
+            int taken = 0;
+            for (int64_t base = 0; base < n && taken < rem; base += 32) {
+                const int64_t j = base + tid;
+                bool eq = false;
+                if (j < n) eq = order_key(row[j]) == prefix;
+                const uint32_t m = __ballot_sync(0xffffffffu, eq);
+                const int before = __popc(m & ((1u << tid) - 1u));
+                if (eq && taken + before < rem) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                taken += __popc(m);
+            }
+        }
+    } else if (tid == 0) {
+        const int ne = s_eq_total;
+        for (int t = 0; t < rem && t < ne; ++t) {   // repeated minimum over the few equal keys
+            int best = t;
+            for (int q = t + 1; q < ne; ++q)
+                if (eq_idx[q] < eq_idx[best]) best = q;
+            const uint32_t tmp = eq_idx[t];
+            eq_idx[t] = eq_idx[best];
+            eq_idx[best] = tmp;
+            atomicOr(&bitmap[eq_idx[t] >> 5], 1u << (eq_idx[t] & 31));
+        }
+    }
+    __syncthreads();
+    const int per = (nw + kTkThreads - 1) / kTkThreads;
+    const int w0 = tid * per;
+    int local = 0;
+    for (int w = w0; w < w0 + per && w < nw; ++w) local += __popc(bitmap[w]);
+    int slot, total;
+    Scan(scan_tmp).ExclusiveSum(local, slot, total);
+    for (int w = w0; w < w0 + per && w < nw; ++w) {
+        uint32_t bits = bitmap[w];
+        while (bits) {
+            const int bpos = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (slot < topk) out[slot] = w * 32 + bpos;
+            ++slot;
+        }
     }
 }
 
