@@ -47,6 +47,12 @@ def peaks():
 
 # ------------------------------------------------------------------ algorithmic work per call
 
+# DRAM bytes per query token of the tensor-core attention kernel (query rows in, output rows out; the
+# gathered key/value rows are served by L2), from an ncu capture of the same kernel at T=8192 with
+# dram__bytes_read.sum + dram__bytes_write.sum = 1076.4 MB; linear in T.
+ATTEND_TC_DRAM_BYTES_PER_TOKEN = 1076.4e6 / 8192
+
+
 def prefill_work(spec):
     """Algorithmic flops / bytes of each call of a prefill layer (visible pairs only)."""
     T, m, k, win = spec.T, spec.m, spec.topk, spec.window
@@ -251,6 +257,8 @@ def run_prefill(args, spec_name, ws, rank):
     import synth
     from tests._helpers import dev
     spec = synth.PREFILL[spec_name]
+    if args.tokens:
+        spec = spec.replace(T=args.tokens)
     if ws > 1:
         spec = spec.replace(seed=spec.seed + 1000 * rank)   # independent sequence per rank
     inp = synth.prefill_inputs(spec)
@@ -300,8 +308,11 @@ def run_prefill(args, spec_name, ws, rank):
     wk = work[dom]
     if "flops" in wk:
         ach = wk["flops"] / (ours[dom] / 1e3) / 1e12
+        traffic = None
+        if dom == "attend" and spec.kind == "csa" and spec.H == 64 and spec.dh == 512:
+            traffic = ATTEND_TC_DRAM_BYTES_PER_TOKEN * spec.T
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_sus, "unit": "TFLOP/s", "frac": ach / tc_sus,
-                "traffic": None, "kernel": dom, "peak_kind": f"{src} bf16 sustained"}
+                "traffic": traffic, "kernel": dom, "peak_kind": f"{src} bf16 sustained"}
     else:
         ach = wk["bytes"] / (ours[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
@@ -343,6 +354,9 @@ def run_decode(args, spec_name, ws, rank):
     import synth
     from tests._helpers import dev
     d = synth.DECODE[spec_name]
+    if args.batch:
+        import dataclasses
+        d = dataclasses.replace(d, B=args.batch)
     layers, Ws, Bs, xs = [], [], [], None
     shared = {}
     for li, spec in enumerate(d.layers):
@@ -430,6 +444,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="override T of a prefill workload (profiling small cases)")
+    ap.add_argument("--batch", type=int, default=0, help="override B of a decode workload (profiling small cases)")
     args = ap.parse_args()
     kind, name = WORKLOADS[args.workload]
     ws, rank, local = dist_setup()
