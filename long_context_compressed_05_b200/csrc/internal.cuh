@@ -120,6 +120,9 @@ hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st);
 bool attend_tc_supported(const AttendArgs &a);
 int attend_tc_segments(const AttendArgs &a);     // key segments per query (> 1: partials + combine)
 hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st);
+// tensor-core HCA prefill attention over query blocks (dh = 128, C = 256, H | 128, window 128, bf16)
+bool hca_attend_tc_supported(const AttendArgs &a);
+hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st);
 
 // projection y[rows, ncols] = x[rows, D] W[D, ncols]
 size_t project_ws_bytes(int dtype);
