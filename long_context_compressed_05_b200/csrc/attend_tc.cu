@@ -516,15 +516,25 @@ bool attend_tc_supported(const AttendArgs &a) {
     return true;
 }
 
-// Decode splits each sequence's key list into units: one tile per unit for CSA (the gathered rows
-// are the bottleneck, so spread them over as many SMs as possible), four for HCA (contiguous
-// entry tiles load fast; fewer units write fewer partials).
-static int decode_seg_tiles(const AttendArgs &a) { return a.dense ? 4 : 1; }
+static int64_t decode_tiles(const AttendArgs &a) {
+    const int64_t e = a.dense ? (a.N + kKT - 1) / kKT * kKT : a.topk;
+    return e / kKT + 1;
+}
+
+// Decode splits each sequence's key list into units of equal tile counts.  Every SM streams its
+// units at a rate of its own, so the step takes as long as the busiest SM: use the fewest tiles per
+// unit that still fit all units in one wave over the SMs (fewer, longer units write fewer partials
+// for the merge); when no split fits one wave, take the longest units.
+static int decode_seg_tiles(const AttendArgs &a) {
+    const int64_t tiles = decode_tiles(a);
+    for (int s = 1; s <= kMaxTiles; ++s)
+        if (a.rows * ((tiles + s - 1) / s) <= num_sms()) return s;
+    return kMaxTiles;
+}
 
 int attend_tc_segments(const AttendArgs &a) {
     if (a.pos == nullptr) return 1;
-    const int64_t e = a.dense ? (a.N + kKT - 1) / kKT * kKT : a.topk;
-    const int64_t tiles = e / kKT + 1;
+    const int64_t tiles = decode_tiles(a);
     const int st = decode_seg_tiles(a);
     return (int)((tiles + st - 1) / st);
 }

@@ -33,12 +33,13 @@ namespace hcsa {
 
 namespace {
 
-constexpr int kNS = 8;               // key-tile ring stages
+constexpr int kNS = 8;               // key-tile ring stages (prefill)
+constexpr int kNSDec = 12;           // decode: more tiles in flight (the keys stream from HBM)
 constexpr int kATile = 128 * 128;    // 128 keys x 64 bf16
 constexpr int kBTile = 256 * 128;    // up to 256 (token, head) rows x 64 bf16
+constexpr int kBTileDec = 64 * 128;  // decode: one token, Hi <= 64 heads
 constexpr int kThreads = 320;        // 10 warps
 constexpr int kEpiThreads = 256;
-constexpr int kDecodeTilesPerUnit = 32;
 
 struct Args {
     int64_t rows;        // prefill: T; decode: B
@@ -50,8 +51,9 @@ struct Args {
     const __nv_bfloat16 *w;
     int64_t ld_w;
     float *scores;       // [rows, N]
-    int64_t n_units, n_qtiles;
-    int64_t dec_chunks;  // decode: units per sequence
+    uint32_t *hist;      // decode: per-row histogram of the top 12 key bits of the scores, or nullptr
+    int64_t n_units, n_qtiles;   // prefill: query tiles; decode: (sequence, key tile) pairs
+    int64_t tps;         // decode: key tiles per sequence (ceil(N / 128))
     int *status;
 };
 
@@ -69,41 +71,75 @@ __device__ __forceinline__ int64_t visible(const Args &a, int64_t row) {
 
 __device__ __forceinline__ Unit unit_of(const Args &a, int64_t u) {
     Unit x;
-    if (!a.decode) {
-        const int64_t q = a.n_qtiles - 1 - u;   // heaviest first
-        x.b = 0;
-        x.r0 = q * a.tq;
-        int64_t last = x.r0 + a.tq - 1 < a.rows ? x.r0 + a.tq - 1 : a.rows - 1;
-        x.kt0 = 0;
-        x.kt1 = (int)((visible(a, last) + 127) / 128);
-    } else {
-        x.b = u / a.dec_chunks;
-        x.r0 = x.b;
-        const int c = (int)(u % a.dec_chunks);
-        const int nkt = (int)((visible(a, x.b) + 127) / 128);
-        x.kt0 = c * kDecodeTilesPerUnit;
-        x.kt1 = min(nkt, x.kt0 + kDecodeTilesPerUnit);
-    }
+    const int64_t q = a.n_qtiles - 1 - u;   // heaviest first
+    x.b = 0;
+    x.r0 = q * a.tq;
+    int64_t last = x.r0 + a.tq - 1 < a.rows ? x.r0 + a.tq - 1 : a.rows - 1;
+    x.kt0 = 0;
+    x.kt1 = (int)((visible(a, last) + 127) / 128);
     return x;
 }
 
-template <int HI>
+// Work iteration, the same in every warp role.  Prefill: persistent CTAs take query tiles round-robin.
+// Decode: CTA c takes an equal contiguous share [g0, g1) of the (sequence, key tile) pairs in
+// sequence-major order; its units are the pieces of that share inside each sequence (usually one or two).
+struct Iter {
+    int64_t u, g, g1;
+};
+
+__device__ __forceinline__ Iter iter_begin(const Args &a) {
+    Iter it;
+    it.u = blockIdx.x;
+    it.g = (int64_t)blockIdx.x * a.n_units / gridDim.x;
+    it.g1 = (int64_t)(blockIdx.x + 1) * a.n_units / gridDim.x;
+    return it;
+}
+
+__device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
+    if (!a.decode) {
+        while (it.u < a.n_units) {
+            x = unit_of(a, it.u);
+            it.u += gridDim.x;
+            if (x.kt0 < x.kt1) return true;
+        }
+        return false;
+    }
+    while (it.g < it.g1) {
+        const int64_t b = it.g / a.tps;
+        const int64_t end = it.g1 < (b + 1) * a.tps ? it.g1 : (b + 1) * a.tps;
+        const int nkt = (int)((visible(a, b) + 127) / 128);
+        x.b = b;
+        x.r0 = b;
+        x.kt0 = (int)(it.g - b * a.tps);
+        x.kt1 = min(nkt, (int)(end - b * a.tps));
+        it.g = end;
+        if (x.kt0 < x.kt1) return true;
+    }
+    return false;
+}
+
+template <int HI, bool DEC>
 __global__ void __launch_bounds__(kThreads, 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
                        Args a) {
+    // decode: key tiles that share one 128-column TMEM accumulator (Hi columns each)
+    constexpr int kTPB = 128 / HI < 4 ? 128 / HI : 4;
+    constexpr int NS = DEC ? kNSDec : kNS;
+    constexpr int BT = DEC ? kBTileDec : kBTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = base;                       // kNS x 16 KB
-    uint8_t *sB = sA + kNS * kATile;          // 2 x 32 KB
-    float *sw = reinterpret_cast<float *>(sB + 2 * kBTile);   // 2 x 256 head weights
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 512);
-    uint64_t *a_full = bars, *a_empty = bars + kNS, *b_full = bars + 2 * kNS, *b_empty = b_full + 2;
+    uint8_t *sA = base;                       // NS x 16 KB
+    uint8_t *sB = sA + NS * kATile;           // 2 x BT
+    float *sw = reinterpret_cast<float *>(sB + 2 * BT);   // prefill: 2 x 256 head weights
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sw + (DEC ? 0 : 512));
+    uint64_t *a_full = bars, *a_empty = bars + NS, *b_full = bars + 2 * NS, *b_empty = b_full + 2;
     uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 4);
+    uint32_t *shist = tmem_slot + 4;          // decode: [4096] key-bit histogram of the current unit
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNS; ++i) { tc::mbar_init(&a_full[i], 1); tc::mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < NS; ++i) { tc::mbar_init(&a_full[i], 1); tc::mbar_init(&a_empty[i], 1); }
         for (int i = 0; i < 2; ++i) { tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1); }
         for (int i = 0; i < 4; ++i) { tc::mbar_init(&acc_full[i], 1); tc::mbar_init(&acc_empty[i], kEpiThreads / 32); }
         tc::fence_mbar_init();
@@ -119,17 +155,16 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t ia = 0, ib = 0;
-            for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
-                const Unit x = unit_of(a, u);
-                if (x.kt0 >= x.kt1) continue;
+            Unit x;
+            for (Iter it = iter_begin(a); ok && iter_next(a, it, x);) {
                 const int bb = ib & 1;
                 if (ib >= 2) ok &= tc::mbar_wait(&b_empty[bb], ((ib >> 1) - 1) & 1, a.status);
                 tc::mbar_arrive_expect_tx(&b_full[bb], a.ncols * 128);
-                tc::tma_load_3d(tc::smem_u32(sB + bb * kBTile), &tm_qi, 0, 0, (int)x.r0, &b_full[bb]);
+                tc::tma_load_3d(tc::smem_u32(sB + bb * BT), &tm_qi, 0, 0, (int)x.r0, &b_full[bb]);
                 ++ib;
                 for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
-                    const int s = ia % kNS;
-                    if (ia >= kNS) ok &= tc::mbar_wait(&a_empty[s], ((ia / kNS) - 1) & 1, a.status);
+                    const int s = ia % NS;
+                    if (ia >= NS) ok &= tc::mbar_wait(&a_empty[s], ((ia / NS) - 1) & 1, a.status);
                     tc::mbar_arrive_expect_tx(&a_full[s], kATile);
                     tc::tma_load_3d(tc::smem_u32(sA + s * kATile), &tm_keys, 0, kt * 128, (int)x.b, &a_full[s]);
                 }
@@ -140,15 +175,49 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16(128, a.ncols, false, false);
             uint32_t ia = 0, ib = 0, iacc = 0;
-            for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
-                const Unit x = unit_of(a, u);
-                if (x.kt0 >= x.kt1) continue;
+            Unit x;
+            for (Iter it = iter_begin(a); ok && iter_next(a, it, x);) {
                 const int bb = ib & 1;
                 ok &= tc::mbar_wait(&b_full[bb], (ib >> 1) & 1, a.status);
-                const uint32_t bsm = tc::smem_u32(sB + bb * kBTile);
-                for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia, ++iacc) {
-                    const int s = ia % kNS, ab = iacc % a.nbuf;
-                    ok &= tc::mbar_wait(&a_full[s], (ia / kNS) & 1, a.status);
+                const uint32_t bsm = tc::smem_u32(sB + bb * BT);
+                if (DEC) {
+                    // Decode: kTPB consecutive tiles share one accumulator (HI columns each).  Every tile is a
+                    // chain of 4 dependent MMAs (K = 16 each) whose latency, not the tensor pipe, sets the pace,
+                    // so the K steps of two tiles are interleaved (two independent chains in flight).
+                    for (int kt = x.kt0; kt < x.kt1 && ok; kt += 2, ia += 2) {
+                        const int slot = (kt - x.kt0) % kTPB;
+                        const bool two = kt + 1 < x.kt1;   // pairs start at even slots: both in one accumulator
+                        const int s0 = ia % NS, s1 = (ia + 1) % NS, ab = iacc % a.nbuf;
+                        ok &= tc::mbar_wait(&a_full[s0], (ia / NS) & 1, a.status);
+                        if (two) ok &= tc::mbar_wait(&a_full[s1], ((ia + 1) / NS) & 1, a.status);
+                        if (slot == 0 && iacc >= (uint32_t)a.nbuf)
+                            ok &= tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
+                        tc::tc_fence_after();
+                        const uint32_t a0 = tc::smem_u32(sA + s0 * kATile), a1 = tc::smem_u32(sA + s1 * kATile);
+                        const uint32_t d0 = tmem + ab * a.stride + slot * HI;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t bd = tc::sdesc_sw128(bsm + 32 * k, 16, 1024);
+                            tc::mma_bf16(d0, tc::sdesc_sw128(a0 + 32 * k, 16, 1024), bd, idesc, k > 0);
+                            if (two) tc::mma_bf16(d0 + HI, tc::sdesc_sw128(a1 + 32 * k, 16, 1024), bd, idesc, k > 0);
+                        }
+                        tc::mma_commit(&a_empty[s0]);
+                        if (two) tc::mma_commit(&a_empty[s1]);
+                        const int last = kt + (two ? 1 : 0);
+                        if ((slot + (two ? 1 : 0)) == kTPB - 1 || last == x.kt1 - 1) {
+                            tc::mma_commit(&acc_full[ab]);
+                            ++iacc;
+                        }
+                    }
+                    if (!ok) break;
+                    ia -= (uint32_t)((x.kt1 - x.kt0) & 1);   // an odd tile count used one stage, not two
+                    tc::mma_commit(&b_empty[bb]);
+                    ++ib;
+                    continue;
+                }
+                for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
+                    const int s = ia % NS, ab = iacc % a.nbuf;
+                    ok &= tc::mbar_wait(&a_full[s], (ia / NS) & 1, a.status);
                     if (iacc >= (uint32_t)a.nbuf)
                         ok &= tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
                     tc::tc_fence_after();
@@ -159,32 +228,97 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                                      tc::sdesc_sw128(bsm + 32 * k, 16, 1024), idesc, k > 0);
                     tc::mma_commit(&a_empty[s]);
                     tc::mma_commit(&acc_full[ab]);
+                    ++iacc;
                 }
                 tc::mma_commit(&b_empty[bb]);
                 ++ib;
             }
         }
+    } else if (DEC) {
+        // ------------------------------------------------ decode epilogue: one token, Hi columns per tile
+        // The two warp groups take alternate accumulators; each holds up to kTPB key tiles.
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int row = quad * 32 + lane;
+        const int et = threadIdx.x - 64;              // 0..255
+        const bool hist = a.hist != nullptr;
+        if (hist)
+            for (int i = et; i < 4096; i += kEpiThreads) shist[i] = 0;
+        uint32_t iacc = 0;
+        Unit x;
+        for (Iter it = iter_begin(a); iter_next(a, it, x);) {
+            // with the histogram the epilogue warps meet at barriers: they leave the loop together
+            if (hist) ok = tc::named_bar_and(1, kEpiThreads, ok);
+            if (!ok) break;
+            float wr[HI];
+#pragma unroll
+            for (int h = 0; h < HI; ++h) wr[h] = __bfloat162float(a.w[x.b * a.ld_w + h]);
+            const int64_t vis = visible(a, x.b);
+            float *srow = a.scores + x.b * a.N;
+            const int nbat = (x.kt1 - x.kt0 + kTPB - 1) / kTPB;
+            for (int bi = 0; bi < nbat && ok; ++bi, ++iacc) {
+                if ((int)(iacc & 1) != half) continue;
+                const int ab = iacc % a.nbuf;
+                ok &= tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
+                tc::tc_fence_after();
+                const int kt0 = x.kt0 + bi * kTPB;
+                const int nt = min(kTPB, x.kt1 - kt0);
+                const uint32_t tl = tmem + ab * a.stride + ((uint32_t)(quad * 32) << 16);
+                float sc[kTPB];
+#pragma unroll
+                for (int t = 0; t < kTPB; ++t) sc[t] = 0.f;
+#pragma unroll
+                for (int c0 = 0; c0 < kTPB * HI; c0 += 32) {   // 32 columns: part of a tile, or 32 / HI tiles
+                    if (c0 / HI < nt) {
+                        float v[32];
+                        tc::tmem_ld32(tl + c0, v);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) sc[(c0 + i) / HI] += wr[(c0 + i) % HI] * fmaxf(v[i], 0.f);
+                    }
+                }
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive_cnt(&acc_empty[ab], 2);
+#pragma unroll
+                for (int t = 0; t < kTPB; ++t) {
+                    const int64_t j = (int64_t)(kt0 + t) * 128 + row;
+                    if (t < nt && j < vis) {
+                        srow[j] = sc[t];
+                        if (hist) atomicAdd(&shist[score_order_key(sc[t]) >> 20], 1u);
+                    }
+                }
+            }
+            if (hist) {   // add the unit's counts into its row's histogram
+                tc::named_bar_sync(1, kEpiThreads);
+                uint32_t *g = a.hist + x.b * 4096;
+                for (int i = et; i < 4096; i += kEpiThreads) {
+                    const uint32_t c = shist[i];
+                    if (c) {
+                        atomicAdd(&g[i], c);
+                        shist[i] = 0;
+                    }
+                }
+            }
+        }
     } else {
         // ------------------------------------------------ epilogue: ReLU, head weights, head sum
-        // Prefill (256 columns): the two warp groups split the columns of every tile.  Decode (<= 128
-        // columns): the groups take alternate tiles, each reading all columns.
+        // The two warp groups split the 256 columns of every tile.
         const int et = threadIdx.x - 64;              // 0..255
         const int quad = warp & 3, half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;             // key within the tile (TMEM lane)
-        const bool split = a.ncols <= 128;
         constexpr int TPH = 128 / HI > 0 ? 128 / HI : 1;   // tokens per 128 columns
-        const int tok_base = split ? 0 : half * TPH;
-        const int col_base = split ? 0 : half * 128;
+        const int tok_base = half * TPH;
+        const int col_base = half * 128;
         uint32_t iacc = 0, iu = 0;
-        for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
-            const Unit x = unit_of(a, u);
-            if (x.kt0 >= x.kt1) continue;
+        Unit x;
+        for (Iter it = iter_begin(a); iter_next(a, it, x);) {
             float *w_s = sw + (iu & 1) * 256;
             if (et < a.ncols) {
                 const int64_t r = x.r0 + et / HI;
                 w_s[et] = r < a.rows ? __bfloat162float(a.w[r * a.ld_w + et % HI]) : 0.f;
             }
-            tc::named_bar_sync(1, kEpiThreads);
+            ok = tc::named_bar_and(1, kEpiThreads, ok);   // all epilogue warps leave together on a failed wait
+            if (!ok) break;
             ++iu;
             const int ntok = a.ncols / HI;                       // tokens in the unit
             int64_t vis[TPH];
@@ -194,7 +328,6 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 vis[i] = (tok_base + i < ntok && r < a.rows) ? visible(a, r) : 0;
             }
             for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++iacc) {
-                if (split && (int)(iacc & 1) != half) continue;
                 const int ab = iacc % a.nbuf;
                 ok &= tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
                 tc::tc_fence_after();
@@ -218,7 +351,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 }
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive_cnt(&acc_empty[ab], split ? 2 : 1);
+                if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
                 const int64_t j = (int64_t)kt * 128 + row;
 #pragma unroll
                 for (int i = 0; i < TPH; ++i)
@@ -237,11 +370,6 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
 // ------------------------------------------------------------------ register-resident top-k
 constexpr int kTkThreads = 512;
 
-__device__ __forceinline__ uint32_t order_key(float s) {
-    if (s == 0.0f) s = 0.0f;   // -0 and +0 compare equal
-    uint32_t b = __float_as_uint(s);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
 
 template <int VPT>   // float4 vectors per thread: row capacity = 2048 * VPT
 __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__restrict__ scores, int64_t N,
@@ -271,11 +399,11 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
         const int64_t j0 = 4 * ((int64_t)tid + (int64_t)kTkThreads * i);
         if (vec_ok && j0 + 3 < n) {
             float4 v = __ldcs(reinterpret_cast<const float4 *>(row + j0));
-            key[4 * i] = order_key(v.x); key[4 * i + 1] = order_key(v.y);
-            key[4 * i + 2] = order_key(v.z); key[4 * i + 3] = order_key(v.w);
+            key[4 * i] = score_order_key(v.x); key[4 * i + 1] = score_order_key(v.y);
+            key[4 * i + 2] = score_order_key(v.z); key[4 * i + 3] = score_order_key(v.w);
         } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) key[4 * i + e] = (j0 + e < n) ? order_key(row[j0 + e]) : 0u;
+            for (int e = 0; e < 4; ++e) key[4 * i + e] = (j0 + e < n) ? score_order_key(row[j0 + e]) : 0u;
         }
     }
     // three histogram passes: bits [20,32), [10,20), [0,10)
@@ -344,7 +472,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
             for (int64_t base = 0; base < n && taken < rem; base += 32) {
                 const int64_t j = base + tid;
                 bool eq = false;
-                if (j < n) eq = order_key(row[j]) == prefix;
+                if (j < n) eq = score_order_key(row[j]) == prefix;
                 const uint32_t m = __ballot_sync(0xffffffffu, eq);
                 const int before = __popc(m & ((1u << tid) - 1u));
                 if (eq && taken + before < rem) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
@@ -402,20 +530,23 @@ static int num_sms() {
     return n;
 }
 
-template <int HI>
+template <int HI, bool DEC>
 static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, const CUtensorMap &tq, Args a,
                                  cudaStream_t st) {
-    constexpr size_t smem = 1024 + kNS * kATile + 2 * kBTile + 512 * sizeof(float) + (2 * kNS + 12) * sizeof(uint64_t) + 16;
+    constexpr int NS = DEC ? kNSDec : kNS;
+    constexpr size_t smem = 1024 + NS * kATile + 2 * (DEC ? kBTileDec : kBTile) + (DEC ? 0 : 512 * sizeof(float)) +
+                            (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 0);
+    static_assert(smem <= 232448, "shared memory per CTA");
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return HCSA_ERR_CUDA;
         configured = true;
     }
     const int64_t grid = a.n_units < num_sms() ? a.n_units : num_sms();
     if (grid <= 0) return HCSA_OK;
-    index_scores_tc_kernel<HI><<<(unsigned)grid, kThreads, smem, st>>>(tk, tq, a);
+    index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, kThreads, smem, st>>>(tk, tq, a);
     count_launch();
     return check_launch();
 }
@@ -436,22 +567,37 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
     a.nbuf = a.ncols <= 128 ? 4 : 2;
     a.stride = a.ncols <= 128 ? 128 : 256;
     a.w = (const __nv_bfloat16 *)ia.w; a.ld_w = ia.ld_w; a.scores = (float *)ia.ws; a.status = device_status_ptr();
+    // long decode rows: multi-CTA select, whose histogram the scores kernel fills; scratch after the scores
+    const bool rows_path = ia.N > 32768 && topk_rows_supported(ia);
+    uint8_t *scratch = (uint8_t *)ia.ws + (((size_t)ia.rows * ia.N * sizeof(float) + 255) & ~(size_t)255);
+    a.hist = nullptr;
+    if (rows_path) {
+        if (topk_rows_begin(ia, scratch, st) != HCSA_OK) return HCSA_ERR_CUDA;
+        a.hist = reinterpret_cast<uint32_t *>(scratch);
+    }
     if (decode) {
-        const int64_t ntiles = (ia.N + 127) / 128;
-        a.dec_chunks = (ntiles + kDecodeTilesPerUnit - 1) / kDecodeTilesPerUnit;
-        a.n_units = ia.rows * a.dec_chunks;
+        a.tps = (ia.N + 127) / 128;
+        a.n_units = ia.rows * a.tps;
         a.n_qtiles = 0;
     } else {
         a.n_qtiles = (ia.rows + tq - 1) / tq;
         a.n_units = a.n_qtiles;
-        a.dec_chunks = 0;
+        a.tps = 0;
     }
     hcsa_status s;
-    switch (ia.Hi) {
-        case 8: s = launch_scores<8>(ia, tk, tq_map, a, st); break;
-        case 16: s = launch_scores<16>(ia, tk, tq_map, a, st); break;
-        case 32: s = launch_scores<32>(ia, tk, tq_map, a, st); break;
-        default: s = launch_scores<64>(ia, tk, tq_map, a, st); break;
+    if (decode) {
+        switch (ia.Hi) {
+            case 16: s = launch_scores<16, true>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, true>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, true>(ia, tk, tq_map, a, st); break;
+        }
+    } else {
+        switch (ia.Hi) {
+            case 8: s = launch_scores<8, false>(ia, tk, tq_map, a, st); break;
+            case 16: s = launch_scores<16, false>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, false>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, false>(ia, tk, tq_map, a, st); break;
+        }
     }
     if (s != HCSA_OK) return s;
     // top-k over the materialised scores
@@ -464,13 +610,11 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         count_launch();
         return check_launch();
     }
-    if (topk_rows_supported(ia)) {
-        // scratch for the multi-CTA select sits after the scores
-        uint8_t *scratch = (uint8_t *)ia.ws + (((size_t)ia.rows * ia.N * sizeof(float) + 255) & ~(size_t)255);
+    if (rows_path) {
         hcsa_status s2 = launch_topk_rows(ia, scratch, st);
         if (s2 != HCSA_OK) return s2;
-        IndexArgs fb = ia;                       // rows whose threshold bucket overflowed the candidate list
-        fb.only_rows = (const int32_t *)(scratch + (size_t)ia.rows * 4096 * sizeof(uint32_t));
+        IndexArgs fb = ia;                       // rows flagged by the multi-CTA select
+        fb.only_rows = topk_rows_flags(ia, scratch);
         return launch_topk_generic(fb, st);
     }
     return launch_topk_generic(ia, st);

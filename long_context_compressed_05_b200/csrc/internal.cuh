@@ -86,10 +86,21 @@ struct IndexArgs {
     const int32_t *only_rows;   // if set: the generic select handles only rows r with only_rows[4 r + 3] != 0
 };
 size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N);
-// multi-CTA exact top-k for long decode rows (N > 32768); scratch after the scores
+// multi-CTA exact top-k for long decode rows (N > 32768); scratch after the scores.  The scratch starts
+// with the rows' histograms of the top 12 bits of score_order_key ([rows][4096] uint32, filled by the
+// indexer), then [rows][4] int32 counters whose element 3 flags rows left to the generic select.
 bool topk_rows_supported(const IndexArgs &a);
 size_t topk_rows_ws_bytes(int64_t rows);
+hcsa_status topk_rows_begin(const IndexArgs &a, void *scratch, cudaStream_t st);   // zero histograms + counters
+const int32_t *topk_rows_flags(const IndexArgs &a, const void *scratch);
 hcsa_status launch_topk_rows(const IndexArgs &a, void *scratch, cudaStream_t st);
+
+// order-preserving key of a score: larger score -> larger key; -0.0 and +0.0 map to the same key
+__device__ __forceinline__ uint32_t score_order_key(float s) {
+    if (s == 0.0f) s = 0.0f;
+    const uint32_t b = __float_as_uint(s);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
 hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st);
 hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st);
 // tensor-core indexer scores (bf16, di = 64) + register-resident top-k

@@ -138,3 +138,29 @@ def test_decode_full_size_sampled(name):
         compare_step(spec, inp, layer, cache, d.P, seqs)
         del layer, cache
         torch.cuda.empty_cache()
+
+
+def test_decode_long_rows_select():
+    """Decode rows longer than 32768 entries take the multi-CTA select: a full row, a ragged last slice,
+    a row with fewer visible entries than k, and a row whose indexer keys repeat 50 distinct vectors (hundreds
+    of scores tie at the threshold: lowest indices first, via the single-CTA fallback).  Besides oracle parity,
+    the selection must be exactly the top-k of the kernel's own fp32 scores (a property of the select itself)."""
+    spec = CSA_TC.replace(seed=37)
+    n_cap = 40000
+    pos = [4 * n_cap, 4 * 35001 + 1, 4 * 100, 4 * 39000 + 3]
+    d = synth.DecodeSpec(layers=(spec,), B=len(pos), P=max(pos), seed=spec.seed)
+    inp = synth.decode_inputs(d, 0, n_cap=n_cap)
+    keys = inp["idx_keys"]
+    keys[3] = keys[3][np.arange(n_cap) % 50]
+    layer, cache = gpu_step(spec, inp, pos, n_cap)
+    compare_step(spec, inp, layer, cache, np.array(pos), list(range(len(pos))))
+    scores = layer.ws_index[: len(pos) * n_cap * 4].view(torch.float32).view(len(pos), n_cap).cpu().numpy()
+    sel = layer.sel.cpu().numpy()
+    for b, P in enumerate(pos):
+        n = min(P // spec.m, n_cap)
+        s = scores[b, :n].astype(np.float64)
+        s[s == 0] = 0.0
+        order = np.lexsort((np.arange(n), -s))[: min(spec.topk, n)]
+        want = np.full(spec.topk, -1, dtype=np.int64)
+        want[: len(order)] = np.sort(order)
+        np.testing.assert_array_equal(sel[b], want)
