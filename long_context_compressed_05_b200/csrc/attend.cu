@@ -104,55 +104,57 @@ __global__ void __launch_bounds__(kHeadsPerCta * 32) attend_kernel(AttendArgs a,
     if (lane == 0) { pml[slot * 2] = mx; pml[slot * 2 + 1] = z; }
 }
 
-// Log-sum-exp merge of the per-split partials of one (row, head): weights exp(m_s - M) / Z are computed
-// once per CTA in shared memory, then every thread merges one output element across the splits.
+// Log-sum-exp merge of the per-split partials of one (row, head).  Warp 0 computes the weights
+// exp(m_s - M) / Z of the splits that hold keys (compacted in split order, with warp reductions only),
+// then every thread merges one output element across those splits.
 template <typename S>
 __global__ void __launch_bounds__(512) combine_kernel(AttendArgs a, int nsplit) {
     using A = typename Traits<S>::A;
     extern __shared__ __align__(16) unsigned char comb_smem[];
-    A *wgt = reinterpret_cast<A *>(comb_smem);      // [nsplit]
-    A *red = wgt + nsplit;                          // [blockDim.x]
+    A *wgt = reinterpret_cast<A *>(comb_smem);                 // [nsplit]
+    int *idx = reinterpret_cast<int *>(wgt + nsplit);          // [nsplit]
+    __shared__ int n_live;
     const int64_t r = blockIdx.x;
     const int h = blockIdx.y;
     const A *pacc = reinterpret_cast<const A *>(a.ws);
     const A *pml = pacc + a.rows * (int64_t)nsplit * a.H * a.dh;
-    A mloc = -INFINITY;
-    for (int s = threadIdx.x; s < nsplit; s += blockDim.x) {
-        const A m = pml[((r * nsplit + s) * a.H + h) * 2];
-        wgt[s] = m;
-        mloc = m > mloc ? m : mloc;
-    }
-    red[threadIdx.x] = mloc;
-    __syncthreads();
-    for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-        if (threadIdx.x < o) red[threadIdx.x] = red[threadIdx.x + o] > red[threadIdx.x] ? red[threadIdx.x + o] : red[threadIdx.x];
-        __syncthreads();
-    }
-    const A M = red[0];
-    __syncthreads();
-    A zloc = A(0);
-    for (int s = threadIdx.x; s < nsplit; s += blockDim.x) {
-        const A m = wgt[s];
-        const A e = m == -INFINITY ? A(0) : exp_acc(m - M);
-        wgt[s] = e;
-        zloc += e * pml[((r * nsplit + s) * a.H + h) * 2 + 1];
-    }
-    red[threadIdx.x] = zloc;
-    __syncthreads();
-    for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-        if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-        __syncthreads();
-    }
-    const A Z = red[0];
-    const A zi = Z > A(0) ? A(1) / Z : A(0);
-    // compact the splits that hold keys (an empty split's accumulator is never written)
-    int *idx = reinterpret_cast<int *>(red + blockDim.x);
-    __shared__ int n_live;
-    if (threadIdx.x == 0) {
-        int c = 0;
-        for (int s = 0; s < nsplit; ++s)
-            if (wgt[s] != A(0)) { idx[c] = s; wgt[c] = wgt[s] * zi; ++c; }
-        n_live = c;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        A M = -INFINITY;
+        for (int s = lane; s < nsplit; s += 32) {
+            const A m = pml[((r * nsplit + s) * a.H + h) * 2];
+            M = m > M ? m : M;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const A y = __shfl_xor_sync(0xffffffffu, M, o);
+            M = y > M ? y : M;
+        }
+        A zl = A(0);
+        int live_total = 0;
+        for (int s0 = 0; s0 < nsplit; s0 += 32) {
+            const int s = s0 + lane;
+            A e = A(0);
+            if (s < nsplit) {
+                const A m = pml[((r * nsplit + s) * a.H + h) * 2];
+                e = m == -INFINITY ? A(0) : exp_acc(m - M);
+                zl += e * pml[((r * nsplit + s) * a.H + h) * 2 + 1];
+            }
+            const bool live = e != A(0);   // an empty split's accumulator is never written
+            const uint32_t b = __ballot_sync(0xffffffffu, live);
+            if (live) {
+                const int q = live_total + __popc(b & ((1u << lane) - 1u));
+                idx[q] = s;
+                wgt[q] = e;
+            }
+            live_total += __popc(b);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) zl += __shfl_xor_sync(0xffffffffu, zl, o);
+        const A zi = zl > A(0) ? A(1) / zl : A(0);
+        __syncwarp();
+        for (int q = lane; q < live_total; q += 32) wgt[q] *= zi;
+        if (lane == 0) n_live = live_total;
     }
     __syncthreads();
     const int nl = n_live;
@@ -171,7 +173,7 @@ static void launch_combine(const AttendArgs &a, int ns, cudaStream_t st) {
     int threads = 32;
     while (threads < a.dh && threads < 512) threads <<= 1;
     const size_t esz = a.dtype == HCSA_BF16 ? sizeof(float) : sizeof(double);
-    const size_t smem = esz * ((size_t)ns + threads) + sizeof(int) * (size_t)ns;
+    const size_t smem = esz * (size_t)ns + sizeof(int) * (size_t)ns;
     if (a.dtype == HCSA_BF16) {
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -39,6 +39,7 @@ constexpr int kKT = 128;          // keys per tile (MMA M)
 constexpr int kMaxTiles = 5;
 constexpr int kNS = 6;            // key/value ring stages (even: P V pairs sit in adjacent stages)
 constexpr int kStage = 16384;     // 128 rows x 64 bf16
+constexpr int kGatherDepth = 4;   // gathered chunks in flight per producer thread
 constexpr int kQStage = kH * 128; // 64 heads x 64 bf16
 constexpr int kPBytes = kMaxTiles * kKT * 128;
 constexpr int kProdThreads = 64;      // warps 0-1
@@ -180,6 +181,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
             const Unit x = unit_of(a, u);
             if (x.nt <= 0) continue;
+            if (a.decode && pt == 0) {
+                // decode: the whole query (8 chunks of 64 dims) lands in the P region at once; P of the
+                // previous unit must have been consumed by its P V first
+                if (iu >= 1) ok &= tc::mbar_wait(&bars->o_full, (iu - 1) & 1, a.status);
+                tc::mbar_arrive_expect_tx(&bars->qf[0], 8 * kQStage);
+                for (int dc = 0; dc < 8; ++dc)
+                    tc::tma_load_3d(P + dc * kQStage, &tm_q, dc * 64, 0, (int)x.q, &bars->qf[0]);
+                tma_use[kNS] = (int32_t)iu;
+            }
             const __nv_bfloat16 **rp = rowptr + (iu & 1) * (kMaxTiles * kKT);
             {
                 // all selection indices of the unit are loaded before any is used (independent loads in flight)
@@ -239,6 +249,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                        p != nullptr);
                     }
                     tc::cp_async_arrive_noinc(&bars->rf[s]);
+                    // At most kGatherDepth chunks of this thread in flight: a thread whose copies cannot be
+                    // accepted waits here instead of holding up the shared load/store queue that the softmax
+                    // warps' shuffles, shared-memory accesses and barrier polls also go through.
+                    tc::cp_async_commit();
+                    tc::cp_async_wait<kGatherDepth - 1>();
                 }
                 ++ic;
             };
@@ -254,12 +269,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             };
             const int n1 = x.nt < 4 ? x.nt : 4;
             for (int dc = 0; dc < 8; ++dc) {          // S phase 1: tiles 0..3
-                load_q(dc);
+                if (!a.decode) load_q(dc);
                 for (int t = 0; t < n1; ++t) load_chunk(t, dc * 64);
             }
             if (x.nt == 5)
                 for (int dc = 0; dc < 8; ++dc) {      // S phase 2: tile 4
-                    load_q(dc);
+                    if (!a.decode) load_q(dc);
                     load_chunk(4, dc * 64);
                 }
             for (int t = 0; t < x.nt; ++t)            // P V: value halves, 64-dh chunks in pairs
@@ -281,9 +296,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (x.nt <= 0) continue;
                 const int n1 = x.nt < 4 ? x.nt : 4;
                 if (iu >= 1) ok &= tc::mbar_wait(&bars->s_free, (iu - 1) & 1, a.status);
+                if (a.decode) ok &= tc::mbar_wait(&bars->qf[0], iu & 1, a.status);   // whole query in P
                 for (int dc = 0; dc < 8; ++dc) {
                     const int qb = iq & 1;
-                    ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                    if (!a.decode) ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                    const uint32_t qsm = a.decode ? P + dc * kQStage : Qs + qb * kQStage;
                     for (int t = 0; t < n1; ++t, ++ic) {
                         const int s = ic % kNS;
                         ok &= tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
@@ -292,28 +309,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
                             tc::mma_bf16(tmem + s_col(t), tc::sdesc_sw128(ring + s * kStage + 32 * k, 16, 1024),
-                                         tc::sdesc_sw128(Qs + qb * kQStage + 32 * k, 16, 1024), kIdescS,
-                                         (dc | k) != 0);
+                                         tc::sdesc_sw128(qsm + 32 * k, 16, 1024), kIdescS, (dc | k) != 0);
                         tc::mma_commit(&bars->re[s]);
                     }
-                    tc::mma_commit(&bars->qe[qb]);
-                    ++iq;
+                    if (!a.decode) {
+                        tc::mma_commit(&bars->qe[qb]);
+                        ++iq;
+                    }
                 }
                 if (x.nt == 5) {
                     if (iu >= 1) ok &= tc::mbar_wait(&bars->o_free, (iu - 1) & 1, a.status);
-                    for (int dc = 0; dc < 8; ++dc, ++ic, ++iq) {
+                    for (int dc = 0; dc < 8; ++dc, ++ic) {
                         const int qb = iq & 1, s = ic % kNS;
-                        ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                        if (!a.decode) ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                        const uint32_t qsm = a.decode ? P + dc * kQStage : Qs + qb * kQStage;
                         ok &= tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
                         tc::fence_async_smem();
                         tc::tc_fence_after();
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
                             tc::mma_bf16(tmem + kColB, tc::sdesc_sw128(ring + s * kStage + 32 * k, 16, 1024),
-                                         tc::sdesc_sw128(Qs + qb * kQStage + 32 * k, 16, 1024), kIdescS,
-                                         (dc | k) != 0);
+                                         tc::sdesc_sw128(qsm + 32 * k, 16, 1024), kIdescS, (dc | k) != 0);
                         tc::mma_commit(&bars->re[s]);
-                        tc::mma_commit(&bars->qe[qb]);
+                        if (!a.decode) {
+                            tc::mma_commit(&bars->qe[qb]);
+                            ++iq;
+                        }
                     }
                 }
                 tc::mma_commit(&bars->s_full);
