@@ -13,7 +13,7 @@
 //     128-byte swizzled K-major layout (64 bf16 = one swizzle row);
 //   * 4 MMAs (K = 16 each) per key tile into one of two 256-column TMEM
 //     accumulators, so the epilogue of tile i overlaps the MMAs of tile i + 1;
-//   * 8 epilogue warps (two per TMEM lane quadrant, each owning half of the
+//   * 16 epilogue warps (four per TMEM lane quadrant, each owning a quarter of the
 //     columns) read the accumulator, apply ReLU, weight by w and sum the heads in
 //     registers -- no cross-lane traffic -- and store fp32 scores coalesced.
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, warps 2..9 = epilogue.
@@ -38,8 +38,10 @@ constexpr int kNSDec = 12;           // decode: more tiles in flight (the keys s
 constexpr int kATile = 128 * 128;    // 128 keys x 64 bf16
 constexpr int kBTile = 256 * 128;    // up to 256 (token, head) rows x 64 bf16
 constexpr int kBTileDec = 64 * 128;  // decode: one token, Hi <= 64 heads
-constexpr int kThreads = 320;        // 10 warps
-constexpr int kEpiThreads = 256;
+// epilogue warps: prefill 16 (four per TMEM lane quadrant, 64 columns each: the ReLU-weighted head sum
+// is the busy part), decode 8 (two groups taking alternate accumulators)
+__host__ __device__ constexpr int epi_warps(bool dec) { return dec ? 8 : 16; }
+__host__ __device__ constexpr int cta_threads(bool dec) { return 64 + 32 * epi_warps(dec); }
 
 struct Args {
     int64_t rows;        // prefill: T; decode: B
@@ -119,11 +121,12 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
 }
 
 template <int HI, bool DEC>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(cta_threads(DEC), 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
                        Args a) {
     // decode: key tiles that share one 128-column TMEM accumulator (Hi columns each)
     constexpr int kTPB = 128 / HI < 4 ? 128 / HI : 4;
+    constexpr int kEpiWarps = epi_warps(DEC), kEpiThreads = 32 * kEpiWarps, kGroups = kEpiWarps / 4;
     constexpr int NS = DEC ? kNSDec : kNS;
     constexpr int BT = DEC ? kBTileDec : kBTile;
     extern __shared__ uint8_t smem_raw[];
@@ -237,9 +240,9 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
     } else if (DEC) {
         // ------------------------------------------------ decode epilogue: one token, Hi columns per tile
         // The two warp groups take alternate accumulators; each holds up to kTPB key tiles.
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int quad = warp & 3, grp = (warp - 2) >> 2;   // group grp takes accumulators iacc % kGroups == grp
         const int row = quad * 32 + lane;
-        const int et = threadIdx.x - 64;              // 0..255
+        const int et = threadIdx.x - 64;              // 0..kEpiThreads-1
         const bool hist = a.hist != nullptr;
         if (hist)
             for (int i = et; i < 4096; i += kEpiThreads) shist[i] = 0;
@@ -256,7 +259,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
             float *srow = a.scores + x.b * a.N;
             const int nbat = (x.kt1 - x.kt0 + kTPB - 1) / kTPB;
             for (int bi = 0; bi < nbat && ok; ++bi, ++iacc) {
-                if ((int)(iacc & 1) != half) continue;
+                if ((int)(iacc % kGroups) != grp) continue;
                 const int ab = iacc % a.nbuf;
                 ok &= tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
                 tc::tc_fence_after();
@@ -278,7 +281,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 }
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive_cnt(&acc_empty[ab], 2);
+                if (lane == 0) tc::mbar_arrive_cnt(&acc_empty[ab], kGroups);
 #pragma unroll
                 for (int t = 0; t < kTPB; ++t) {
                     const int64_t j = (int64_t)(kt0 + t) * 128 + row;
@@ -302,13 +305,13 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
         }
     } else {
         // ------------------------------------------------ epilogue: ReLU, head weights, head sum
-        // The two warp groups split the 256 columns of every tile.
-        const int et = threadIdx.x - 64;              // 0..255
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        // The four warp groups split the 256 columns of every tile (64 each).
+        const int et = threadIdx.x - 64;              // 0..kEpiThreads-1
+        const int quad = warp & 3, grp = (warp - 2) >> 2;
         const int row = quad * 32 + lane;             // key within the tile (TMEM lane)
-        constexpr int TPH = 128 / HI > 0 ? 128 / HI : 1;   // tokens per 128 columns
-        const int tok_base = half * TPH;
-        const int col_base = half * 128;
+        constexpr int TPH = 64 / HI > 0 ? 64 / HI : 1;      // tokens per 64 columns
+        const int tok_base = grp * TPH;
+        const int col_base = grp * 64;
         uint32_t iacc = 0, iu = 0;
         Unit x;
         for (Iter it = iter_begin(a); iter_next(a, it, x);) {
@@ -335,17 +338,26 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
 #pragma unroll
                 for (int i = 0; i < TPH; ++i) s[i] = 0.f;
                 const uint32_t tl = tmem + ab * a.stride + ((uint32_t)(quad * 32) << 16);
+                // the head weights are read as float4 (the same address in every lane: a broadcast)
+                constexpr int LB = 1;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int col0 = col_base + cc * 32;
-                    if (col0 < a.ncols) {
-                        float v[32];
-                        tc::tmem_ld32(tl + col0, v);
-                        tc::tmem_ld_wait();
+                for (int c0 = 0; c0 < 2; c0 += LB) {
+                    float v[LB][32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int c = cc * 32 + i;                // column within this group's 128
-                            s[c / HI < TPH ? c / HI : TPH - 1] += w_s[col0 + i] * fmaxf(v[i], 0.f);
+                    for (int l = 0; l < LB; ++l) tc::tmem_ld32(tl + col_base + (c0 + l) * 32, v[l]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int l = 0; l < LB; ++l) {
+                        const float4 *wv = reinterpret_cast<const float4 *>(w_s + col_base + (c0 + l) * 32);
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 wq = wv[i4];
+                            const float wl[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int c = (c0 + l) * 32 + i4 * 4 + e;   // column within this group's 64
+                                s[c / HI < TPH ? c / HI : TPH - 1] += wl[e] * fmaxf(v[l][i4 * 4 + e], 0.f);
+                            }
                         }
                     }
                 }
@@ -546,7 +558,7 @@ static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, con
     }
     const int64_t grid = a.n_units < num_sms() ? a.n_units : num_sms();
     if (grid <= 0) return HCSA_OK;
-    index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, kThreads, smem, st>>>(tk, tq, a);
+    index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
     count_launch();
     return check_launch();
 }
