@@ -381,30 +381,45 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
 
 // ------------------------------------------------------------------ register-resident top-k
 constexpr int kTkThreads = 512;
+constexpr int kRankCap = 1024;   // threshold buckets up to this size are ranked directly
 
 
 template <int VPT>   // float4 vectors per thread: row capacity = 2048 * VPT
-__global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__restrict__ scores, int64_t N,
-                                                               int m, const int32_t *__restrict__ pos, int topk,
-                                                               int32_t *__restrict__ sel) {
+__global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel(const float *__restrict__ scores, int64_t rows,
+                                                               int64_t N, int m, const int32_t *__restrict__ pos,
+                                                               int topk, int32_t *__restrict__ sel) {
     using Scan = cub::BlockScan<int, kTkThreads>;
     __shared__ typename Scan::TempStorage scan_tmp;
     __shared__ int hist[4096];
     __shared__ uint32_t bitmap[1024];   // rows of up to 32768 entries
     __shared__ uint32_t eq_idx[64];
+    __shared__ uint64_t cand[kRankCap];  // (key << 32 | ~index) of the keys in the threshold bucket
     __shared__ uint32_t s_prefix;
-    __shared__ int s_rem, s_eq_total;
+    __shared__ int s_rem, s_eq_total, s_bcount, s_cnt;
     const int tid = threadIdx.x;
-    const int64_t r = blockIdx.x;
-    int64_t p = pos ? (int64_t)pos[r] : r;
-    int64_t n = p < 0 ? 0 : (p / m < N ? p / m : N);
+    const bool vec_ok = (N & 3) == 0 && ((uintptr_t)scores & 15) == 0;   // rows start 16-byte aligned
+    auto visible_of = [&](int64_t rr) -> int64_t {
+        const int64_t pp = pos ? (int64_t)pos[rr] : rr;
+        return pp < 0 ? 0 : (pp / m < N ? pp / m : N);
+    };
+    // Persistent CTAs walk the rows round-robin (every CTA sees short and long rows).  While a row is
+    // ranked, the CTA's next row is prefetched into L2: loading a row is otherwise a bare HBM round trip
+    // with nothing else to do.
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    if (tid == 0 && vec_ok && r + gridDim.x < rows) {
+        const int64_t nn = visible_of(r + gridDim.x);
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(scores + (r + gridDim.x) * N);
+        const uint32_t bytes = (uint32_t)(((nn + 3) & ~int64_t(3)) * sizeof(float));
+        for (uint32_t off = 0; off < bytes; off += 65536u)
+            tc::bulk_prefetch_l2(src + off, bytes - off < 65536u ? bytes - off : 65536u);
+    }
+    const int64_t n = visible_of(r);
     int32_t *out = sel + r * topk;
     if (n <= topk) {
         for (int i = tid; i < topk; i += kTkThreads) out[i] = i < n ? i : -1;
-        return;
+        continue;
     }
     const float *row = scores + r * N;
-    const bool vec_ok = (N & 3) == 0;   // rows start 16-byte aligned
     uint32_t key[VPT * 4];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
@@ -418,9 +433,12 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
             for (int e = 0; e < 4; ++e) key[4 * i + e] = (j0 + e < n) ? score_order_key(row[j0 + e]) : 0u;
         }
     }
-    // three histogram passes: bits [20,32), [10,20), [0,10)
+    // Histogram passes over bits [20,32), then [10,20) and [0,10) inside the threshold bucket.  Usually
+    // the first pass leaves a small bucket: its keys are then ranked directly instead (the two later
+    // passes cost more in barriers than in work).
     uint32_t prefix = 0, mask = 0;
     int rem = topk;
+    bool ranked = false;
     const int shifts[3] = {20, 10, 0};
     const int widths[3] = {12, 10, 10};
 #pragma unroll
@@ -446,6 +464,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
                 if (cum + c >= rem) {
                     s_prefix = prefix | ((uint32_t)(b0 + i) << sh);
                     s_rem = rem - cum;
+                    s_bcount = c;
                     break;
                 }
                 cum += c;
@@ -455,14 +474,52 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
         prefix = s_prefix;
         rem = s_rem;
         mask |= (uint32_t)(nb - 1) << sh;
+        const bool small = s_bcount <= kRankCap;
         __syncthreads();
+        if (pass == 0 && small) {
+            ranked = true;
+            break;
+        }
     }
-    // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first).
-    // Mark the chosen indices in a bitmap of the row, then emit them in ascending order with one scan.
     const int nw = (int)((n + 31) / 32);
     for (int i = tid; i < nw; i += kTkThreads) bitmap[i] = 0;
-    if (tid == 0) s_eq_total = 0;
+    if (tid == 0) {
+        s_eq_total = 0;
+        s_cnt = 0;
+    }
     __syncthreads();
+    if (ranked) {
+        // prefix = threshold bucket << 20: keys in higher buckets are taken; the `rem` best keys of the
+        // bucket (larger key first, then lower index) are found by ranking the bucket's keys
+        const uint32_t bucket = prefix >> 20;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t kv = key[4 * i + e];
+                const int64_t j = 4 * ((int64_t)tid + (int64_t)kTkThreads * i) + e;
+                if ((kv >> 20) > bucket) {
+                    atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                } else if ((kv >> 20) == bucket && kv != 0u) {
+                    const int q = atomicAdd(&s_cnt, 1);
+                    if (q < kRankCap) cand[q] = ((uint64_t)kv << 32) | (0xFFFFFFFFu - (uint32_t)j);
+                }
+            }
+        }
+        __syncthreads();
+        const int mb = s_cnt < kRankCap ? s_cnt : kRankCap;
+        for (int c = tid; c < mb; c += kTkThreads) {
+            const uint64_t v = cand[c];
+            int rk = 0;
+            for (int d = 0; d < mb; ++d) rk += cand[d] > v ? 1 : 0;
+            if (rk < rem) {
+                const uint32_t j = 0xFFFFFFFFu - (uint32_t)v;
+                atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+            }
+        }
+    } else {
+    // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first).
+    // Mark the chosen indices in a bitmap of the row, then emit them in ascending order with one scan.
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
 #pragma unroll
@@ -503,6 +560,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
             atomicOr(&bitmap[eq_idx[t] >> 5], 1u << (eq_idx[t] & 31));
         }
     }
+    }
     __syncthreads();
     const int per = (nw + kTkThreads - 1) / kTkThreads;
     const int w0 = tid * per;
@@ -518,6 +576,8 @@ __global__ void __launch_bounds__(kTkThreads) topk_regs_kernel(const float *__re
             if (slot < topk) out[slot] = w * 32 + bpos;
             ++slot;
         }
+    }
+    __syncthreads();   // shared state is reused by the next row
     }
 }
 
@@ -613,12 +673,17 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
     }
     if (s != HCSA_OK) return s;
     // top-k over the materialised scores
+    if (ia.rows <= 0) return HCSA_OK;
     if (ia.N <= 32768) {
         const float *sc = (const float *)ia.ws;
-        if (ia.N <= 8192)
-            topk_regs_kernel<4><<<(unsigned)ia.rows, kTkThreads, 0, st>>>(sc, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
-        else
-            topk_regs_kernel<16><<<(unsigned)ia.rows, kTkThreads, 0, st>>>(sc, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+        // persistent: as many CTAs as fit at once (one per SM at 16 vectors per thread, two at 4)
+        if (ia.N <= 8192) {
+            const int64_t g = ia.rows < 2 * num_sms() ? ia.rows : 2 * num_sms();
+            topk_regs_kernel<4><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.rows, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+        } else {
+            const int64_t g = ia.rows < num_sms() ? ia.rows : num_sms();
+            topk_regs_kernel<16><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.rows, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+        }
         count_launch();
         return check_launch();
     }
