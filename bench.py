@@ -93,7 +93,31 @@ def decode_bytes(spec, B, N):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """SM clock and clock-event reasons of this process's GPU, sampled while the timed region runs.
+
+    NVML is polled every 2 ms from a thread (a decode step is well under a millisecond, so the timed
+    region can be shorter than nvidia-smi's sampling period); nvidia-smi -lms 200 is the fallback."""
+
+    _REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
+
     def __init__(self, dev_index):
+        self.samples, self.p, self.thread = [], None, None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv, self.h = pynvml, self._handle(pynvml, dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.get_reasons = get
+            import threading
+            self.stop_ev = threading.Event()
+            self._sample()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -104,7 +128,42 @@ class ClockSampler:
         except Exception:
             self.p = None
 
+    @staticmethod
+    def _handle(nv, dev_index):
+        """NVML handle of torch's device `dev_index` (by UUID, so CUDA_VISIBLE_DEVICES remapping is honoured)."""
+        try:
+            u = str(torch.cuda.get_device_properties(dev_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        except Exception:
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ent = vis.split(",")[dev_index].strip() if vis else str(dev_index)
+        if ent.startswith("GPU-"):
+            return nv.nvmlDeviceGetHandleByUUID(ent)
+        return nv.nvmlDeviceGetHandleByIndex(int(ent))
+
+    def _sample(self):
+        sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        self.samples.append((float(sm), int(self.get_reasons(self.h))))
+
+    def _run(self):
+        while not self.stop_ev.wait(0.002):
+            try:
+                self._sample()
+            except Exception:
+                return
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_ev.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            sm = [x[0] for x in self.samples]
+            reasons = sorted({name for x in self.samples for bit, name in self._REASONS.items() if x[1] & bit})
+            loaded = sorted(sm)[len(sm) // 4:] or sm
+            return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": float(self.max_mhz), "reasons": reasons,
+                    "samples": len(sm), "source": "nvml"}
         if self.p is None:
             return None
         self.p.terminate()
@@ -132,7 +191,7 @@ class ClockSampler:
                     reasons.add(n)
         loaded = sorted(sm)[len(sm) // 4:] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi"}
 
 
 # ------------------------------------------------------------------ distributed plumbing

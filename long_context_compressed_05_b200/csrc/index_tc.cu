@@ -13,18 +13,25 @@
 //     128-byte swizzled K-major layout (64 bf16 = one swizzle row);
 //   * 4 MMAs (K = 16 each) per key tile into one of two 256-column TMEM
 //     accumulators, so the epilogue of tile i overlaps the MMAs of tile i + 1;
-//   * 16 epilogue warps (four per TMEM lane quadrant, each owning a quarter of the
-//     columns) read the accumulator, apply ReLU, weight by w and sum the heads in
-//     registers -- no cross-lane traffic -- and store fp32 scores coalesced.
-// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, warps 2..9 = epilogue.
-// Persistent CTAs walk a list of work units (prefill: one query tile each, the
-// heaviest causal tiles first; decode: (sequence, 8 key tiles)).
+//   * prefill: 16 epilogue warps (four per TMEM lane quadrant, each owning 64 of the
+//     256 columns) read the accumulator, apply ReLU, weight by w and sum the heads in
+//     registers -- no cross-lane traffic -- and store fp32 scores coalesced;
+//   * decode (one token, Hi columns): four key tiles share a 128-column accumulator,
+//     8 epilogue warps in two groups take alternate accumulators and also count the
+//     row's 12-bit key histogram for the multi-CTA top-k; a tile's four MMAs form a
+//     dependent chain whose latency sets the pace, so the K steps of two tiles are
+//     issued interleaved.
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, the rest = epilogue.
+// Persistent CTAs: prefill walks query tiles (heaviest causal tiles first); decode
+// gives every CTA an equal contiguous share of the (sequence, key tile) pairs.
 //
-// Top-k kernel.  One CTA of 512 threads per query row keeps the row's scores in
-// registers (<= 32768), and finds the k-th largest order-preserving key with three
-// histogram passes (12 + 10 + 10 bits) over the registers; the chosen indices are
-// marked in a shared-memory bitmap of the row (ties at the k-th value: lowest j) and
-// emitted in ascending order with one block scan over the bitmap words.
+// Top-k kernel.  One 512-thread CTA per query row at a time (persistent, prefetching
+// its next row into L2) keeps the row's scores in registers (<= 32768) and finds the
+// bucket of the k-th largest order-preserving key with a 12-bit histogram pass; a
+// bucket of <= 1024 keys is ranked directly (key desc, index asc), a larger one takes
+// two more 10-bit passes and an equal-key scan.  The chosen indices are marked in a
+// shared-memory bitmap of the row and emitted in ascending order with one block scan
+// over the bitmap words.
 #include <cub/block/block_scan.cuh>
 
 #include "tc_common.cuh"

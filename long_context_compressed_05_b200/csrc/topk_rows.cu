@@ -273,25 +273,26 @@ __global__ void __launch_bounds__(kThreads) rows_finish_kernel(RowArgs a) {
         }
     }
     __syncthreads();
-    // ascending emission: thread t owns words [32 t, 32 t + 32) (nw <= 32 x 256), read into registers
-    // without bank conflicts; one block scan of the threads' bit counts gives the output positions
-    uint32_t wd[32];
+    // ascending emission: thread t owns words [32 t, 32 t + 32) (nw <= 32 x 256; the padded layout puts
+    // them in 32 different banks across a warp); one block scan of the threads' bit counts gives the
+    // output positions.  The loops stay rolled: this code runs once per launch, from a cold
+    // instruction cache.
     uint32_t local = 0;
-#pragma unroll
+#pragma unroll 1
     for (int i = 0; i < 32; ++i) {
         const int w = tid * 32 + i;
-        wd[i] = w < nw ? bitmap[bw(w)] : 0u;
-        local += __popc(wd[i]);
+        local += w < nw ? __popc(bitmap[bw(w)]) : 0u;
     }
     uint32_t total;
     int q = (int)(block_incl_scan(local, warp_sums, &total) - local);
-#pragma unroll
+#pragma unroll 1
     for (int i = 0; i < 32; ++i) {
-        uint32_t bits = wd[i];
+        const int w = tid * 32 + i;
+        uint32_t bits = w < nw ? bitmap[bw(w)] : 0u;
         while (bits) {
             const int b = __ffs(bits) - 1;
             bits &= bits - 1;
-            if (q < a.topk) out[q] = (tid * 32 + i) * 32 + b;
+            if (q < a.topk) out[q] = w * 32 + b;
             ++q;
         }
     }
