@@ -211,6 +211,13 @@ hcsa_status csa_decode_index_topk_noalloc(const hcsa_params *p, const hcsa_cache
  * (HCSA_OK, HCSA_ERR_TIMEOUT or HCSA_ERR_DEVICE), or HCSA_ERR_CUDA if the wait itself failed. */
 hcsa_status hcsa_get_device_status(void *stream);
 
+/* Self-test of the failure path (not part of the method; the pages have no counterpart): enqueues one
+ * kernel whose bounded wait on a barrier that nothing completes gives up after its limit (about a
+ * second), records HCSA_ERR_TIMEOUT in the device status word and returns.  A following
+ * hcsa_get_device_status(stream) then returns HCSA_ERR_TIMEOUT (and clears it); the context stays
+ * usable.  Returns HCSA_ERR_CUDA if the launch fails. */
+hcsa_status hcsa_selftest_wait_timeout(void *stream);
+
 /* Number of kernels this library enqueued on the calling host thread since the last reset
  * (library GEMM kernels not included).  For launch accounting in benchmarks. */
 int64_t hcsa_launch_count(int32_t reset);

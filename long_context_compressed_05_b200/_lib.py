@@ -27,7 +27,7 @@ STATUS = {0: "HCSA_OK", 1: "HCSA_ERR_NULL", 2: "HCSA_ERR_SHAPE", 3: "HCSA_ERR_DT
 EXPORTS = ["hcsa_version", "hcsa_status_string", "hcsa_workspace_bytes", "hcsa_proj_cols", "hcsa_project",
            "csa_compress", "hca_compress", "csa_index_topk", "csa_attend", "hca_attend", "hcsa_cache_append",
            "csa_decode_index_topk", "csa_decode_attend", "hca_decode_attend", "csa_decode_index_topk_noalloc",
-           "hcsa_get_device_status",
+           "hcsa_get_device_status", "hcsa_selftest_wait_timeout",
            "hcsa_launch_count"]
 
 
@@ -78,6 +78,7 @@ def load():
         "hca_decode_attend": (I32, [P, CP, V, V, I64, V, V, SZ, V]),
         "csa_decode_index_topk_noalloc": (I32, [P, CP, V, V, I64, V, I64, V, V]),
         "hcsa_get_device_status": (I32, [V]),
+        "hcsa_selftest_wait_timeout": (I32, [V]),
         "hcsa_launch_count": (I64, [I32]),
     }
     for name, (res, args) in sig.items():
@@ -205,6 +206,11 @@ def csa_decode_index_topk_noalloc(p, cache: Cache, pos, qi, w, sel, stream=None)
 
 def hcsa_get_device_status(stream=None) -> int:
     return int(load().hcsa_get_device_status(_stream(stream)))
+
+
+def hcsa_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the bounded-wait self-test kernel (see include/hca_csa.h)."""
+    _check("hcsa_selftest_wait_timeout", load().hcsa_selftest_wait_timeout(_stream(stream)))
 
 
 def hcsa_launch_count(reset: bool = False) -> int:

@@ -96,7 +96,7 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 tc::tma_load_3d(Qs + dc * kChunk, &tm_q, dc * 64, 0, (int)t0, &bars->q_full);
             for (int i = 0; i < n_tiles && ok; ++i) {
                 const int s = i % kNS;
-                if (i >= kNS) ok &= tc::mbar_wait(&bars->kv_empty[s], ((i / kNS) - 1) & 1, a.status);
+                if (i >= kNS) ok = ok && tc::mbar_wait(&bars->kv_empty[s], ((i / kNS) - 1) & 1, a.status);
                 tc::mbar_arrive_expect_tx(&bars->kv_full[s], kStage);
                 const bool ent = i < n_ent_tiles;
                 const int row0 = ent ? i * kKT : (int)(t0 - (kKT - 1) + (int64_t)(i - n_ent_tiles) * kKT);
@@ -107,10 +107,10 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            ok &= tc::mbar_wait(&bars->q_full, 0, a.status);
+            ok = ok && tc::mbar_wait(&bars->q_full, 0, a.status);
             auto issue_pv = [&](int i) {
                 const int s = i % kNS;
-                ok &= tc::mbar_wait(&bars->p_full, i & 1, a.status);
+                ok = ok && tc::mbar_wait(&bars->p_full, i & 1, a.status);
                 tc::fence_async_smem();
                 tc::tc_fence_after();
                 const uint32_t v = KV + s * kStage + 2 * kChunk;
@@ -123,8 +123,8 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             };
             for (int i = 0; i < n_tiles && ok; ++i) {
                 const int s = i % kNS, sb = i & 1;
-                ok &= tc::mbar_wait(&bars->kv_full[s], (i / kNS) & 1, a.status);
-                if (i >= 2) ok &= tc::mbar_wait(&bars->s_free[sb], ((i >> 1) - 1) & 1, a.status);
+                ok = ok && tc::mbar_wait(&bars->kv_full[s], (i / kNS) & 1, a.status);
+                if (i >= 2) ok = ok && tc::mbar_wait(&bars->s_free[sb], ((i >> 1) - 1) & 1, a.status);
                 tc::tc_fence_after();
                 const uint32_t k0 = KV + s * kStage;
 #pragma unroll
@@ -148,7 +148,7 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         float m_used = -INFINITY, l = 0.f;
         for (int i = 0; i < n_tiles && ok; ++i) {
             const int sb = i & 1;
-            ok &= tc::mbar_wait(&bars->s_full[sb], (i >> 1) & 1, a.status);
+            ok = ok && tc::mbar_wait(&bars->s_full[sb], (i >> 1) & 1, a.status);
             tc::tc_fence_after();
             float sv[kKT];
 #pragma unroll
@@ -174,7 +174,7 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const float factor = need ? ex2(m_used - m_new) : 1.f;   // m_used = -inf -> 0
             if (i >= 1) {
                 // P of the previous tile must have been consumed (and O updated) before P and O change
-                ok &= tc::mbar_wait(&bars->o_done, (i - 1) & 1, a.status);
+                ok = ok && tc::mbar_wait(&bars->o_done, (i - 1) & 1, a.status);
                 tc::tc_fence_after();
                 if (__any_sync(0xffffffffu, need)) {
                     for (int c = 0; c < 4; ++c) {
@@ -214,7 +214,7 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (lane == 0) tc::mbar_arrive(&bars->p_full);
         }
         // output: O / l
-        if (ok) ok &= tc::mbar_wait(&bars->o_done, (n_tiles - 1) & 1, a.status);
+        if (ok) ok = ok && tc::mbar_wait(&bars->o_done, (n_tiles - 1) & 1, a.status);
         tc::tc_fence_after();
         const float li = l > 0.f ? 1.f / l : 0.f;
         for (int c = 0; c < 4; ++c) {

@@ -178,17 +178,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t ic = 0, iq = 0, iu = 0;
         int32_t tma_use[kNS + 2];                        // thread 0: last use index of a stage filled by TMA
         for (int i = 0; i < kNS + 2; ++i) tma_use[i] = -1;
-        for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+        // After a failed wait no producer issues another copy; the producers leave the loop together at
+        // the next per-unit barrier (an AND of their flags), so none is left waiting there.
+        for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
             const Unit x = unit_of(a, u);
             if (x.nt <= 0) continue;
-            if (a.decode && pt == 0) {
+            if (a.decode && pt == 0 && ok) {
                 // decode: the whole query (8 chunks of 64 dims) lands in the P region at once; P of the
                 // previous unit must have been consumed by its P V first
-                if (iu >= 1) ok &= tc::mbar_wait(&bars->o_full, (iu - 1) & 1, a.status);
-                tc::mbar_arrive_expect_tx(&bars->qf[0], 8 * kQStage);
-                for (int dc = 0; dc < 8; ++dc)
-                    tc::tma_load_3d(P + dc * kQStage, &tm_q, dc * 64, 0, (int)x.q, &bars->qf[0]);
-                tma_use[kNS] = (int32_t)iu;
+                if (iu >= 1) ok = ok && tc::mbar_wait(&bars->o_full, (iu - 1) & 1, a.status);
+                if (ok) {
+                    tc::mbar_arrive_expect_tx(&bars->qf[0], 8 * kQStage);
+                    for (int dc = 0; dc < 8; ++dc)
+                        tc::tma_load_3d(P + dc * kQStage, &tm_q, dc * 64, 0, (int)x.q, &bars->qf[0]);
+                    tma_use[kNS] = (int32_t)iu;
+                }
             }
             const __nv_bfloat16 **rp = rowptr + (iu & 1) * (kMaxTiles * kKT);
             {
@@ -217,11 +221,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     rp[loc] = ptr;
                 }
             }
-            tc::named_bar_sync(2, kProdThreads);
+            ok = tc::named_bar_and(2, kProdThreads, ok);
+            if (!ok) break;
             ++iu;
             auto load_chunk = [&](int t, int col) {
                 const int s = ic % kNS;
-                if (ic >= kNS) ok &= tc::mbar_wait(&bars->re[s], ((ic / kNS) - 1) & 1, a.status);
+                if (ic >= kNS) ok = ok && tc::mbar_wait(&bars->re[s], ((ic / kNS) - 1) & 1, a.status);
+                if (!ok) {
+                    ++ic;
+                    return;
+                }
                 const int kt = x.t0 + t;
                 // 128 consecutive rows: the prefill window, or a dense (HCA) entry tile inside the visible range
                 const bool win_tile = !a.decode && kt * kKT >= x.E;
@@ -259,11 +268,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             };
             auto load_q = [&](int dc) {
                 const int qb = iq & 1;
-                if (pt == 0) {
-                    if (iq >= 2) ok &= tc::mbar_wait(&bars->qe[qb], ((iq >> 1) - 1) & 1, a.status);
-                    tc::mbar_arrive_expect_tx(&bars->qf[qb], kQStage);
-                    tc::tma_load_3d(Qs + qb * kQStage, &tm_q, dc * 64, 0, (int)x.q, &bars->qf[qb]);
-                    tma_use[kNS + qb] = (int32_t)(iq >> 1);
+                if (pt == 0 && ok) {
+                    if (iq >= 2) ok = ok && tc::mbar_wait(&bars->qe[qb], ((iq >> 1) - 1) & 1, a.status);
+                    if (ok) {
+                        tc::mbar_arrive_expect_tx(&bars->qf[qb], kQStage);
+                        tc::tma_load_3d(Qs + qb * kQStage, &tm_q, dc * 64, 0, (int)x.q, &bars->qf[qb]);
+                        tma_use[kNS + qb] = (int32_t)(iq >> 1);
+                    }
                 }
                 ++iq;
             };
@@ -295,15 +306,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const Unit x = unit_of(a, u);
                 if (x.nt <= 0) continue;
                 const int n1 = x.nt < 4 ? x.nt : 4;
-                if (iu >= 1) ok &= tc::mbar_wait(&bars->s_free, (iu - 1) & 1, a.status);
-                if (a.decode) ok &= tc::mbar_wait(&bars->qf[0], iu & 1, a.status);   // whole query in P
+                if (iu >= 1) ok = ok && tc::mbar_wait(&bars->s_free, (iu - 1) & 1, a.status);
+                if (a.decode) ok = ok && tc::mbar_wait(&bars->qf[0], iu & 1, a.status);   // whole query in P
                 for (int dc = 0; dc < 8; ++dc) {
                     const int qb = iq & 1;
-                    if (!a.decode) ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                    if (!a.decode) ok = ok && tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
                     const uint32_t qsm = a.decode ? P + dc * kQStage : Qs + qb * kQStage;
                     for (int t = 0; t < n1; ++t, ++ic) {
                         const int s = ic % kNS;
-                        ok &= tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
+                        ok = ok && tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
                         tc::fence_async_smem();   // cp.async data (generic proxy) -> MMA (async proxy)
                         tc::tc_fence_after();
 #pragma unroll
@@ -318,12 +329,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
                 if (x.nt == 5) {
-                    if (iu >= 1) ok &= tc::mbar_wait(&bars->o_free, (iu - 1) & 1, a.status);
+                    if (iu >= 1) ok = ok && tc::mbar_wait(&bars->o_free, (iu - 1) & 1, a.status);
                     for (int dc = 0; dc < 8; ++dc, ++ic) {
                         const int qb = iq & 1, s = ic % kNS;
-                        if (!a.decode) ok &= tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
+                        if (!a.decode) ok = ok && tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
                         const uint32_t qsm = a.decode ? P + dc * kQStage : Qs + qb * kQStage;
-                        ok &= tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
+                        ok = ok && tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
                         tc::fence_async_smem();
                         tc::tc_fence_after();
 #pragma unroll
@@ -338,13 +349,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
                 tc::mma_commit(&bars->s_full);
-                ok &= tc::mbar_wait(&bars->p_full, iu & 1, a.status);
+                ok = ok && tc::mbar_wait(&bars->p_full, iu & 1, a.status);
                 tc::tc_fence_after();
                 for (int t = 0; t < x.nt; ++t)
                     for (int dp = 0; dp < 4; ++dp, ic += 2) {
                         const int s0 = ic % kNS, s1 = (ic + 1) % kNS;
-                        ok &= tc::mbar_wait(&bars->rf[s0], (ic / kNS) & 1, a.status);
-                        ok &= tc::mbar_wait(&bars->rf[s1], ((ic + 1) / kNS) & 1, a.status);
+                        ok = ok && tc::mbar_wait(&bars->rf[s0], (ic / kNS) & 1, a.status);
+                        ok = ok && tc::mbar_wait(&bars->rf[s1], ((ic + 1) / kNS) & 1, a.status);
                         tc::fence_async_smem();
                         tc::tc_fence_after();
                         const uint32_t av = ring + s0 * kStage, bp = P + t * kKT * 128;
@@ -369,7 +380,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int r = quad * 32 + lane;                  // key row in a tile; dh row in an output block
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         uint32_t iu = 0;
-        for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
+        for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
+            // the softmax warps meet at named barriers within a unit: they leave the loop together
+            ok = tc::named_bar_and(1, kSoftThreads, ok);
+            if (!ok) break;
             const Unit x = unit_of(a, u);
             const int64_t slot = x.q * a.nseg + x.seg;
             if (x.nt <= 0) {
@@ -403,7 +417,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     valid[t] = v;
                 }
             }
-            ok &= tc::mbar_wait(&bars->s_full, iu & 1, a.status);
+            ok = ok && tc::mbar_wait(&bars->s_full, iu & 1, a.status);
             tc::tc_fence_after();
             float v[32];
 #pragma unroll
@@ -469,7 +483,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tc::named_bar_sync(1, kSoftThreads);
             if (lane == 0) tc::mbar_arrive(&bars->p_full);
             // ---- output
-            ok &= tc::mbar_wait(&bars->o_full, iu & 1, a.status);
+            ok = ok && tc::mbar_wait(&bars->o_full, iu & 1, a.status);
             tc::tc_fence_after();
             for (int dp = 0; dp < 4; ++dp) {
                 float o[32];

@@ -168,13 +168,13 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
             Unit x;
             for (Iter it = iter_begin(a); ok && iter_next(a, it, x);) {
                 const int bb = ib & 1;
-                if (ib >= 2) ok &= tc::mbar_wait(&b_empty[bb], ((ib >> 1) - 1) & 1, a.status);
+                if (ib >= 2) ok = ok && tc::mbar_wait(&b_empty[bb], ((ib >> 1) - 1) & 1, a.status);
                 tc::mbar_arrive_expect_tx(&b_full[bb], a.ncols * 128);
                 tc::tma_load_3d(tc::smem_u32(sB + bb * BT), &tm_qi, 0, 0, (int)x.r0, &b_full[bb]);
                 ++ib;
                 for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
                     const int s = ia % NS;
-                    if (ia >= NS) ok &= tc::mbar_wait(&a_empty[s], ((ia / NS) - 1) & 1, a.status);
+                    if (ia >= NS) ok = ok && tc::mbar_wait(&a_empty[s], ((ia / NS) - 1) & 1, a.status);
                     tc::mbar_arrive_expect_tx(&a_full[s], kATile);
                     tc::tma_load_3d(tc::smem_u32(sA + s * kATile), &tm_keys, 0, kt * 128, (int)x.b, &a_full[s]);
                 }
@@ -188,7 +188,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
             Unit x;
             for (Iter it = iter_begin(a); ok && iter_next(a, it, x);) {
                 const int bb = ib & 1;
-                ok &= tc::mbar_wait(&b_full[bb], (ib >> 1) & 1, a.status);
+                ok = ok && tc::mbar_wait(&b_full[bb], (ib >> 1) & 1, a.status);
                 const uint32_t bsm = tc::smem_u32(sB + bb * BT);
                 if (DEC) {
                     // Decode: kTPB consecutive tiles share one accumulator (HI columns each).  Every tile is a
@@ -198,10 +198,10 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                         const int slot = (kt - x.kt0) % kTPB;
                         const bool two = kt + 1 < x.kt1;   // pairs start at even slots: both in one accumulator
                         const int s0 = ia % NS, s1 = (ia + 1) % NS, ab = iacc % a.nbuf;
-                        ok &= tc::mbar_wait(&a_full[s0], (ia / NS) & 1, a.status);
-                        if (two) ok &= tc::mbar_wait(&a_full[s1], ((ia + 1) / NS) & 1, a.status);
+                        ok = ok && tc::mbar_wait(&a_full[s0], (ia / NS) & 1, a.status);
+                        if (two) ok = ok && tc::mbar_wait(&a_full[s1], ((ia + 1) / NS) & 1, a.status);
                         if (slot == 0 && iacc >= (uint32_t)a.nbuf)
-                            ok &= tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
+                            ok = ok && tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
                         tc::tc_fence_after();
                         const uint32_t a0 = tc::smem_u32(sA + s0 * kATile), a1 = tc::smem_u32(sA + s1 * kATile);
                         const uint32_t d0 = tmem + ab * a.stride + slot * HI;
@@ -227,9 +227,9 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 }
                 for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
                     const int s = ia % NS, ab = iacc % a.nbuf;
-                    ok &= tc::mbar_wait(&a_full[s], (ia / NS) & 1, a.status);
+                    ok = ok && tc::mbar_wait(&a_full[s], (ia / NS) & 1, a.status);
                     if (iacc >= (uint32_t)a.nbuf)
-                        ok &= tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
+                        ok = ok && tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
                     tc::tc_fence_after();
                     const uint32_t asm_ = tc::smem_u32(sA + s * kATile);
 #pragma unroll
@@ -268,7 +268,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
             for (int bi = 0; bi < nbat && ok; ++bi, ++iacc) {
                 if ((int)(iacc % kGroups) != grp) continue;
                 const int ab = iacc % a.nbuf;
-                ok &= tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
+                ok = ok && tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
                 tc::tc_fence_after();
                 const int kt0 = x.kt0 + bi * kTPB;
                 const int nt = min(kTPB, x.kt1 - kt0);
@@ -339,7 +339,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
             }
             for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++iacc) {
                 const int ab = iacc % a.nbuf;
-                ok &= tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
+                ok = ok && tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
                 tc::tc_fence_after();
                 float s[TPH];
 #pragma unroll
