@@ -21,11 +21,12 @@
 // Q is streamed in 64-dim chunks next to the key chunks, so the scores of the next unit
 // (columns [0, 256)) accumulate while this unit's P V runs and its output drains.
 //
-// Warp roles (persistent CTAs, 11 warps): warps 0-1 load (gathered entry rows and the decode
-// window ring with 16-byte cp.async whose completion arrives on the stage's mbarrier by itself;
-// Q chunks and the prefill window tile -- 128 consecutive raw rows -- with TMA box loads), warp 2 issues the MMAs, warps 3..10 run the softmax and the output
-// epilogue (two warps per TMEM lane quadrant, 32 heads each).  Gathered 128-byte row segments
-// are what bounds this kernel: the gather rate per SM, not the tensor core, sets its speed.
+// Warp roles (persistent CTAs, 16 warps): warps 0-6 load (gathered entry rows and the decode window
+// ring with 16-byte cp.async whose completion arrives on the stage's mbarrier by itself; Q chunks and
+// the prefill window tile -- 128 consecutive raw rows -- with TMA box loads), warp 7 issues the MMAs,
+// warps 8..15 run the softmax and the output epilogue (two warps per TMEM lane quadrant, 32 heads
+// each).  Gathered 128-byte row segments are what bounds this kernel: the gather rate per SM, not the
+// tensor core, sets its speed, and that rate grows with the number of warps issuing the copies.
 #include "tc_common.cuh"
 
 namespace hcsa {
@@ -42,10 +43,13 @@ constexpr int kStage = 16384;     // 128 rows x 64 bf16
 constexpr int kGatherDepth = 4;   // gathered chunks in flight per producer thread
 constexpr int kQStage = kH * 128; // 64 heads x 64 bf16
 constexpr int kPBytes = kMaxTiles * kKT * 128;
-constexpr int kProdThreads = 64;      // warps 0-1
-constexpr int kMmaWarp = 2;
-constexpr int kSoftWarp0 = 3;         // warps 3..10
-constexpr int kThreads = 352;
+// The gather rate of cp.async grows with the number of warps issuing it, so most of the CTA's warps are
+// producers (the warps take 128 registers each either way).
+constexpr int kProdWarps = 7;
+constexpr int kProdThreads = 32 * kProdWarps;
+constexpr int kMmaWarp = kProdWarps;
+constexpr int kSoftWarp0 = kProdWarps + 1;   // 8 softmax/epilogue warps
+constexpr int kThreads = 32 * (kProdWarps + 9);
 constexpr int kSoftThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColB = 256;
@@ -197,7 +201,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const __nv_bfloat16 **rp = rowptr + (iu & 1) * (kMaxTiles * kKT);
             {
                 // all selection indices of the unit are loaded before any is used (independent loads in flight)
-                constexpr int kPer = kMaxTiles * kKT / kProdThreads;   // 10
+                constexpr int kPer = (kMaxTiles * kKT + kProdThreads - 1) / kProdThreads;
                 int32_t jsel[kPer];
 #pragma unroll
                 for (int i = 0; i < kPer; ++i) {
@@ -251,8 +255,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int g = pt & 7;
                     const __nv_bfloat16 *const *rows = rp + t * kKT;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int row = i * 8 + (pt >> 3);
+                    for (int i = 0; i < (kKT * 8 + kProdThreads - 1) / kProdThreads; ++i) {
+                        const int row = i * (kProdThreads / 8) + (pt >> 3);
+                        if ((kKT * 8) % kProdThreads != 0 && row >= kKT) break;
                         const __nv_bfloat16 *p = rows[row];
                         tc::cp_async16(ring + s * kStage + tc::sw128_offset(row, g), p ? p + col + g * 8 : a.ent,
                                        p != nullptr);
