@@ -580,12 +580,14 @@ int attend_tc_segments(const AttendArgs &a) {
 }
 
 hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
-    static bool configured = false;
-    if (!configured) {
+    static bool configured[64] = {};   // kernel attributes are set per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
+    if (!configured[dev]) {
         if (cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
             cudaSuccess)
             return HCSA_ERR_CUDA;
-        configured = true;
+        configured[dev] = true;
     }
     const bool decode = a.pos != nullptr;
     CUtensorMap tq, te, tr;

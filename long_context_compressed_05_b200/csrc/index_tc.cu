@@ -616,12 +616,14 @@ static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, con
     constexpr size_t smem = 1024 + NS * kATile + 2 * (DEC ? kBTileDec : kBTile) + (DEC ? 0 : 512 * sizeof(float)) +
                             (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 0);
     static_assert(smem <= 232448, "shared memory per CTA");
-    static bool configured = false;
-    if (!configured) {
+    static bool configured[64] = {};   // kernel attributes are set per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
+    if (!configured[dev]) {
         if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return HCSA_ERR_CUDA;
-        configured = true;
+        configured[dev] = true;
     }
     const int64_t grid = a.n_units < num_sms() ? a.n_units : num_sms();
     if (grid <= 0) return HCSA_OK;
