@@ -532,9 +532,21 @@ def main():
                     vals.append(v)
             unit, hib = "us/step", False
         v = statistics.mean(vals)
-        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": 1,
-                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": hib,
-                          "dtype": "f64", "data": "synthetic", "config": {"workload": args.workload},
+        if kind == "prefill":
+            ms = spec.T / v * 1e3
+            config = {"workload": f"{spec.kind}_prefill_bf16_T{spec.T}_D{spec.D}", "T": spec.T, "D": spec.D,
+                      "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh,
+                      "parallelism": "CPU oracle on rank 0"}
+        else:
+            ms = v / 1e3
+            config = {"workload": name, "B": d.B, "P": d.P, "layers": len(d.layers),
+                      "parallelism": "CPU oracle on rank 0"}
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": ws,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": hib,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic (seeded, the same inputs as the CUDA path; bounded sample, "
+                                  "extrapolated)",
+                          "config": config, "gpu_launches": 0,
                           "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
                                            "sample": sample},
                           "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
