@@ -16,11 +16,11 @@
 //   * prefill: 16 epilogue warps (four per TMEM lane quadrant, each owning 64 of the
 //     256 columns) read the accumulator, apply ReLU, weight by w and sum the heads in
 //     registers -- no cross-lane traffic -- and store fp32 scores coalesced;
-//   * decode (one token, Hi columns): four key tiles share a 128-column accumulator,
-//     8 epilogue warps in two groups take alternate accumulators and also count the
-//     row's 12-bit key histogram for the multi-CTA top-k; a tile's four MMAs form a
-//     dependent chain whose latency sets the pace, so the K steps of two tiles are
-//     issued interleaved.
+//   * decode (one token, Hi columns): two CTAs per SM; four key tiles share a
+//     128-column accumulator, 8 epilogue warps in two groups each own one of the CTA's
+//     two accumulators and also count the row's 12-bit key histogram for the
+//     multi-CTA top-k; a tile's four MMAs form a dependent chain whose latency sets
+//     the pace, so the K steps of two tiles are issued interleaved.
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, the rest = epilogue.
 // Persistent CTAs: prefill walks query tiles (heaviest causal tiles first); decode
 // gives every CTA an equal contiguous share of the (sequence, key tile) pairs.
@@ -41,7 +41,11 @@ namespace hcsa {
 namespace {
 
 constexpr int kNS = 8;               // key-tile ring stages (prefill)
-constexpr int kNSDec = 12;           // decode: more tiles in flight (the keys stream from HBM)
+// Decode runs two CTAs per SM (two independent TMA / MMA pipelines: a tile's dependent MMA chain and
+// the single producer thread each pace one pipeline), each with 4 stages and 2 accumulators of 128
+// TMEM columns.
+constexpr int kNSDec = 4;
+constexpr int kDecCtasPerSm = 2;
 constexpr int kATile = 128 * 128;    // 128 keys x 64 bf16
 constexpr int kBTile = 256 * 128;    // up to 256 (token, head) rows x 64 bf16
 constexpr int kBTileDec = 64 * 128;  // decode: one token, Hi <= 64 heads
@@ -128,7 +132,7 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
 }
 
 template <int HI, bool DEC>
-__global__ void __launch_bounds__(cta_threads(DEC), 1)
+__global__ void __launch_bounds__(cta_threads(DEC), DEC ? kDecCtasPerSm : 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
                        Args a) {
     // decode: key tiles that share one 128-column TMEM accumulator (Hi columns each)
@@ -154,7 +158,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
         for (int i = 0; i < 4; ++i) { tc::mbar_init(&acc_full[i], 1); tc::mbar_init(&acc_empty[i], kEpiThreads / 32); }
         tc::fence_mbar_init();
     }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
+    constexpr uint32_t kTmemCols = DEC ? 256 : 512;
+    if (warp == 0) tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -382,7 +387,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_free(tmem, 512);
+        tc::tmem_free(tmem, kTmemCols);
     }
 }
 
@@ -625,7 +630,8 @@ static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, con
             return HCSA_ERR_CUDA;
         configured[dev] = true;
     }
-    const int64_t grid = a.n_units < num_sms() ? a.n_units : num_sms();
+    const int64_t slots = (int64_t)num_sms() * (DEC ? kDecCtasPerSm : 1);
+    const int64_t grid = a.n_units < slots ? a.n_units : slots;
     if (grid <= 0) return HCSA_OK;
     index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
     count_launch();
@@ -645,7 +651,7 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         return HCSA_ERR_CUDA;
     Args a{};
     a.rows = ia.rows; a.N = ia.N; a.m = ia.m; a.tq = tq; a.ncols = tq * ia.Hi; a.decode = decode; a.pos = ia.pos;
-    a.nbuf = a.ncols <= 128 ? 4 : 2;
+    a.nbuf = 2;                                   // prefill: 2 x 256 columns; decode: 2 x 128 columns
     a.stride = a.ncols <= 128 ? 128 : 256;
     a.w = (const __nv_bfloat16 *)ia.w; a.ld_w = ia.ld_w; a.scores = (float *)ia.ws; a.status = device_status_ptr();
     // long decode rows: multi-CTA select, whose histogram the scores kernel fills; scratch after the scores
