@@ -9,17 +9,18 @@
 //
 // Work unit = (query, segment of its key list).  The key list is the entry part, padded to a
 // multiple of 128 keys, followed by one 128-key window tile.  A unit holds at most 5 tiles
-// (640 keys): prefill CSA is one unit per token (top-k 512 + window), decode splits every
-// sequence into one-tile units whose partial (accumulator, max, sum) are merged by the
-// log-sum-exp combine kernel.
+// (640 keys): prefill CSA is one unit per token (top-k 512 + window); decode splits every
+// sequence into units of equal tile counts (the fewest that still fill one wave over the SMs)
+// whose partials (accumulator, max, sum) are merged by the log-sum-exp combine kernel.
 //
 // Per unit, with 128 keys on the TMEM lanes and the 64 heads as the MMA's N:
 //   S^T[key, head] = K . Q^T   tiles 0..3 in TMEM columns [0, 256), tile 4 in [256, 320)
 //   exact softmax over all keys of the unit (per-head max / sum across lanes)
 //   P^T (bf16) -> shared memory as an MN-major operand
 //   O^T[dh, head] = V^T . P^T  4 blocks of 128 dh in columns [256, 512)
-// Q is streamed in 64-dim chunks next to the key chunks, so the scores of the next unit
-// (columns [0, 256)) accumulate while this unit's P V runs and its output drains.
+// Prefill streams Q in 64-dim chunks next to the key chunks, so the scores of the next unit
+// (columns [0, 256)) accumulate while this unit's P V runs and its output drains; decode loads a
+// unit's whole query at once into the P region, which is free until the softmax writes P.
 //
 // Warp roles (persistent CTAs, 16 warps): warps 0-6 load (gathered entry rows and the decode window
 // ring with 16-byte cp.async whose completion arrives on the stage's mbarrier by itself; Q chunks and
