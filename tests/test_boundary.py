@@ -94,3 +94,16 @@ def test_workspace_sizes(h):
     assert h.hcsa_workspace_bytes(pd, h.OP_CSA_DECODE_INDEX_TOPK) >= 32 * 65536 * 4
     assert h.hcsa_proj_cols(p, h.KIND_CSA) == 36960
     assert h.hcsa_proj_cols(p, h.KIND_HCA) == 2048 + 32768
+
+
+def test_noalloc_refuses_requests_beyond_its_scratch(h):
+    """The allocation-free decode indexer checks its fixed 8 MiB scratch before any launch: 32 sequences of
+    65536 entries need 8 MiB of scores alone (plus the multi-block select's scratch)."""
+    lib = h.load()
+    V = ctypes.c_void_p
+    p = _params(h, B=32, n_cap=65536)
+    assert h.hcsa_workspace_bytes(p, h.OP_CSA_DECODE_INDEX_TOPK) > 8 << 20
+    cache = h.make_cache(None, None, None)
+    cache.entries = cache.win_kv = cache.ring_g = cache.idx_keys = cache.ring_ki = FAKE
+    assert lib.csa_decode_index_topk_noalloc(ctypes.byref(p), ctypes.byref(cache), V(FAKE), V(FAKE), 2048,
+                                             V(FAKE), 32, V(FAKE), None) == 5
