@@ -52,7 +52,12 @@ def _load():
         lib.orc_index_scores.argtypes = [I, I, I, V, V, V, I64, V, V]
         lib.orc_topk.argtypes = [I, V, I64, V, I, V, V, V]
         lib.orc_attend.argtypes = [I, I, I, ctypes.c_double, V, I64, V, I, V, I, V, V, I64, V, I, V, I]
-        for f in ("orc_round", "orc_compress", "orc_pool_rows", "orc_index_scores", "orc_topk", "orc_attend"):
+        lib.orc_round_e4m3.argtypes = [V, I64]
+        lib.orc_round_e2m1.argtypes = [V, I64]
+        lib.orc_store_fp8_rows.argtypes = [V, I64, I, I, V]
+        lib.orc_store_fp4_rows.argtypes = [V, I64, I, I, V]
+        for f in ("orc_round", "orc_compress", "orc_pool_rows", "orc_index_scores", "orc_topk", "orc_attend",
+                  "orc_round_e4m3", "orc_round_e2m1", "orc_store_fp8_rows", "orc_store_fp4_rows"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -77,6 +82,40 @@ def round_to(a: np.ndarray, st: int) -> np.ndarray:
     a = np.ascontiguousarray(a, dtype=np.float64).copy()
     _load().orc_round(a.ctypes.data, a.size, st)
     return a
+
+
+def round_e4m3(a: np.ndarray) -> np.ndarray:
+    """Nearest OCP E4M3 value of each element (ties to even), saturating at +-448."""
+    a = np.ascontiguousarray(a, dtype=np.float64).copy()
+    _load().orc_round_e4m3(a.ctypes.data, a.size)
+    return a
+
+
+def round_e2m1(a: np.ndarray) -> np.ndarray:
+    """Nearest OCP E2M1 value of each element (ties to the even mantissa), saturating at +-6."""
+    a = np.ascontiguousarray(a, dtype=np.float64).copy()
+    _load().orc_round_e2m1(a.ctypes.data, a.size)
+    return a
+
+
+def store_fp8_rows(a: np.ndarray, block: int = 64):
+    """FP8 (E4M3) storage of the rows of a 2-D array in blocks of `block` channels, one fp32 scale
+    amax / 448 per block.  Returns (stored values, scales [rows, blocks])."""
+    a = np.ascontiguousarray(a, dtype=np.float64).copy()
+    rows, cols = a.shape
+    scales = np.empty((rows, -(-cols // block)), np.float64)
+    _load().orc_store_fp8_rows(a.ctypes.data, rows, cols, block, scales.ctypes.data)
+    return a, scales
+
+
+def store_fp4_rows(a: np.ndarray, block: int = 32):
+    """FP4 (E2M1) storage of the rows of a 2-D array in blocks of `block` channels, one power-of-two
+    scale 2^e per block (e smallest with amax / 2^e <= 6).  Returns (stored values, exponents)."""
+    a = np.ascontiguousarray(a, dtype=np.float64).copy()
+    rows, cols = a.shape
+    exps = np.empty((rows, -(-cols // block)), np.int32)
+    _load().orc_store_fp4_rows(a.ctypes.data, rows, cols, block, exps.ctypes.data)
+    return a, exps
 
 
 # ---------------------------------------------------------------- building blocks
@@ -174,12 +213,15 @@ def _col_slices(spec):
     return cols
 
 
-def prefill(spec, inp, rows=None, chunk=8192):
+def prefill(spec, inp, rows=None, chunk=8192, lowprec=False):
     """Run the whole layer on the oracle.
 
     inp: storage arrays x[T,D], W_cat[D,ncat], B[width,C] (as produced by synth).
     rows: query positions to evaluate (default: all).  Entries are always built
-    for the whole sequence.  Returns a dict of float64 arrays."""
+    for the whole sequence.  lowprec: store the compressed entries as FP8 (blocks of
+    64 channels) and the indexer keys as FP4 (blocks of 32), see store_fp8_rows /
+    store_fp4_rows; everything downstream reads the stored values.  Returns a dict of
+    float64 arrays."""
     st = storage_code(spec.dtype)
     T, C, m = spec.T, spec.C, spec.m
     cols = _col_slices(spec)
@@ -196,6 +238,10 @@ def prefill(spec, inp, rows=None, chunk=8192):
     ki_ptr = base + 8 * cols["ki"].start if csa else None
     entries, idx = compress(T, C, m, spec.width, base, ld, base + 8 * C, ld, B, ki_ptr, ld,
                             spec.di if csa else 0, st)
+    if lowprec:
+        entries = store_fp8_rows(entries, 64)[0]
+        if csa:
+            idx = store_fp4_rows(idx, 32)[0]
     rows = np.arange(T, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
     W_q = np.ascontiguousarray(W[:, pool_end:])
     yq = project(to_f64(inp["x"][rows]), W_q, st)

@@ -58,6 +58,96 @@ void orc_round(double *a, int64_t n, int st) {
     for (int64_t i = 0; i < n; ++i) a[i] = store(a[i], st);
 }
 
+/* ---------------------------------------------------------------------------------------------
+ * Low-precision cache storage (page "DeepSeek-V4 ... KV cache ...", section "FP8 y FP4": most of
+ * each compressed entry in FP8, the indexer keys in FP4).  The pages fix neither the formats' flavour
+ * nor the scaling; the readings taken:
+ *   FP8 entries: OCP E4M3 (bias 7, no infinities, largest 448, subnormals down to 2^-9).  Every entry
+ *     row is cut into blocks of `block` channels; a block's scale is s = fp32(amax / 448) and a value
+ *     x is stored as the E4M3 value nearest to x / s (ties to even), times s.
+ *   FP4 indexer keys: OCP E2M1 (0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives).  A block of `block`
+ *     channels shares a power-of-two scale 2^e, e the smallest integer with amax / 2^e <= 6 (no value
+ *     is clipped); x is stored as the E2M1 value nearest to x / 2^e (ties to the even mantissa), times 2^e.
+ * These functions return the stored values (dequantized) in place of the inputs.
+ * --------------------------------------------------------------------------------------------- */
+
+/* nearest E4M3 value (ties to even), saturating at +-448 */
+static double round_e4m3(double v) {
+    if (v == 0.0 || isnan(v)) return v;
+    const double a = fabs(v);
+    double ulp;
+    if (a < ldexp(1.0, -6)) {
+        ulp = ldexp(1.0, -9);                 /* subnormals: m / 8 * 2^-6 */
+    } else {
+        int e;
+        frexp(a, &e);                         /* a in [2^(e-1), 2^e) */
+        ulp = ldexp(1.0, e - 1 - 3);          /* 3 mantissa bits */
+    }
+    double q = nearbyint(a / ulp) * ulp;
+    if (q > 448.0) q = 448.0;
+    return v < 0 ? -q : q;
+}
+
+/* nearest E2M1 value (ties to the even mantissa), saturating at +-6 */
+static double round_e2m1(double v) {
+    if (v == 0.0 || isnan(v)) return v;
+    const double a = fabs(v);
+    const double ulp = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);
+    double q = nearbyint(a / ulp) * ulp;
+    if (q > 6.0) q = 6.0;
+    return v < 0 ? -q : q;
+}
+
+void orc_round_e4m3(double *a, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) a[i] = round_e4m3(a[i]);
+}
+
+void orc_round_e2m1(double *a, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) a[i] = round_e2m1(a[i]);
+}
+
+/* FP8 (E4M3) storage of rows [rows, cols] (row-major, leading dimension cols) in blocks of `block`
+ * channels; scales[rows][cols / block] receives the block scales (may be NULL). */
+void orc_store_fp8_rows(double *a, int64_t rows, int cols, int block, double *scales) {
+    const int nb = (cols + block - 1) / block;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int b = 0; b < nb; ++b) {
+            double *x = a + r * cols + (int64_t)b * block;
+            const int n = (b + 1) * block <= cols ? block : cols - b * block;
+            double amax = 0.0;
+            for (int i = 0; i < n; ++i) amax = fmax(amax, fabs(x[i]));
+            const double s = (double)(float)(amax / 448.0);
+            if (scales) scales[r * nb + b] = s;
+            for (int i = 0; i < n; ++i) x[i] = s > 0.0 ? round_e4m3(x[i] / s) * s : 0.0;
+        }
+    }
+}
+
+/* FP4 (E2M1) storage of rows [rows, cols] in blocks of `block` channels with power-of-two scales;
+ * exps[rows][cols / block] receives the scale exponents (may be NULL). */
+void orc_store_fp4_rows(double *a, int64_t rows, int cols, int block, int32_t *exps) {
+    const int nb = (cols + block - 1) / block;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int b = 0; b < nb; ++b) {
+            double *x = a + r * cols + (int64_t)b * block;
+            const int n = (b + 1) * block <= cols ? block : cols - b * block;
+            double amax = 0.0;
+            for (int i = 0; i < n; ++i) amax = fmax(amax, fabs(x[i]));
+            int e = 0;
+            if (amax > 0.0) {
+                e = (int)ceil(log2(amax / 6.0));
+                while (amax / ldexp(1.0, e) > 6.0) ++e;          /* guard log2 rounding */
+                while (amax / ldexp(1.0, e - 1) <= 6.0) --e;
+            }
+            if (exps) exps[r * nb + b] = e;
+            const double s = ldexp(1.0, e);
+            for (int i = 0; i < n; ++i) x[i] = amax > 0.0 ? round_e2m1(x[i] / s) * s : 0.0;
+        }
+    }
+}
+
 /* One gated-softmax pool over n tokens for channels [0, nch): the learned
  * compressor of "CSA: compresion 4x mas recuperacion dispersa" (learned pool,
  * overlapping windows) and "HCA: compresion 128x" (m'=128), per channel.
