@@ -271,13 +271,16 @@ def attend_rows(spec, res, q, sel):
     return attend(q, spec.H, spec.dh, spec.scale, res["entries"], sel, res["n_vis"], ypool, win, st)
 
 
-def decode_step(spec, inp, P, seqs=None):
+def decode_step(spec, inp, P, seqs=None, lowprec=False):
     """One decode step of one layer.
 
     inp: storage arrays as produced by synth.decode_inputs: W_cat, B, x[Ball, D] and the cache
     entries[Ball,N,C], idx_keys[Ball,N,di], win_kv[Ball,win,C], ring_g[Ball,width,C], ring_ki[Ball,width,di].
     P: position of the new token, one int or one per batch row.  seqs: the batch rows to evaluate
-    (default all).  Returns per-evaluated-row results (float64), in the order of seqs."""
+    (default all).  lowprec: the cache holds its entries in FP8 and its indexer keys in FP4 (the
+    given values are stored in those formats first, and an entry formed by this step is stored so too);
+    the window ring stays in the layer's storage format.  Returns per-evaluated-row results (float64),
+    in the order of seqs."""
     st = storage_code(spec.dtype)
     csa = spec.kind == "csa"
     m, Wd, win, C = spec.m, spec.width, spec.window, spec.C
@@ -298,6 +301,10 @@ def decode_step(spec, inp, P, seqs=None):
         ring_g = to_f64(inp["ring_g"][b]).copy()
         ent_b = to_f64(inp["entries"][b])
         idx_b = to_f64(inp["idx_keys"][b]) if csa else None
+        if lowprec:
+            ent_b = store_fp8_rows(ent_b, 64)[0]
+            if csa:
+                idx_b = store_fp4_rows(idx_b, 32)[0]
         ring_ki = to_f64(inp["ring_ki"][b]).copy() if csa else None
         Ncap = ent_b.shape[0]
         # append: the new token enters the rings
@@ -314,9 +321,13 @@ def decode_step(spec, inp, P, seqs=None):
             g_t = np.stack([ring_g[i % Wd] for i in toks])
             b_t = np.stack([Bm[i - lo] for i in toks])
             new = {"j": j, "entry": pool_rows(kv_t, g_t, b_t, C, st)}
+            if lowprec:
+                new["entry"] = store_fp8_rows(new["entry"][None], 64)[0][0]
             if csa:
                 ki_t = np.stack([ring_ki[i % Wd] for i in toks])
                 new["idx_key"] = pool_rows(ki_t, g_t, b_t, spec.di, st)
+                if lowprec:
+                    new["idx_key"] = store_fp4_rows(new["idx_key"][None], 32)[0][0]
             if j < Ncap:
                 ent_b = ent_b.copy()
                 ent_b[j] = new["entry"]

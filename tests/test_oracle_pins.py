@@ -314,10 +314,12 @@ def test_csa_layer_small_against_masked_sdpa(orc):
 
 # ------------------------------------------------------------------ decode
 
+@pytest.mark.parametrize("lowprec", [False, True])
 @pytest.mark.parametrize("kind", ["csa", "hca"])
-def test_decode_steps_match_prefill(orc, kind):
+def test_decode_steps_match_prefill(orc, kind, lowprec):
     """Decode at positions P..P+n-1 over a cache built from a prefill of P tokens reproduces the
-    prefill of P+n tokens (outputs, selections and newly completed entries)."""
+    prefill of P+n tokens (outputs, selections and newly completed entries) -- also with FP8 entries and
+    FP4 indexer keys in the cache (storing already stored values changes nothing)."""
     import synth
     if kind == "csa":
         spec = _small_csa(T=0, dtype="f32")
@@ -328,8 +330,9 @@ def test_decode_steps_match_prefill(orc, kind):
         P0, n = 29, 5
     full = spec.replace(T=P0 + n)
     inp = synth.prefill_inputs(full)
-    ref = orc.prefill(full, inp)
+    ref = orc.prefill(full, inp, lowprec=lowprec)
     cols = orc._col_slices(spec)
+    cdt = np.float64 if lowprec else np.float32   # stored FP8 / FP4 values are not all fp32 numbers
     m, W, win = spec.m, spec.width, spec.window
     ypool = ref["y_pool"]
     for step in range(n):
@@ -337,7 +340,7 @@ def test_decode_steps_match_prefill(orc, kind):
         nc = P // m
         ncap = nc + 2
         cache = {"W_cat": inp["W_cat"], "B": inp["B"], "x": inp["x"][P:P + 1]}
-        ent = np.zeros((1, ncap, spec.C), np.float32)
+        ent = np.zeros((1, ncap, spec.C), cdt)
         ent[0, :nc] = ref["entries"][:nc]
         cache["entries"] = ent
         wk = np.zeros((1, win, spec.C), np.float32)
@@ -348,13 +351,13 @@ def test_decode_steps_match_prefill(orc, kind):
             rg[0, p % W] = ypool[p, cols["g"]]
         cache["win_kv"], cache["ring_g"] = wk, rg
         if kind == "csa":
-            ik = np.zeros((1, ncap, spec.di), np.float32)
+            ik = np.zeros((1, ncap, spec.di), cdt)
             ik[0, :nc] = ref["idx_keys"][:nc]
             rk = np.zeros((1, W, spec.di), np.float32)
             for p in range(max(0, P - W), P):
                 rk[0, p % W] = ypool[p, cols["ki"]]
             cache["idx_keys"], cache["ring_ki"] = ik, rk
-        d = orc.decode_step(spec, cache, P)
+        d = orc.decode_step(spec, cache, P, lowprec=lowprec)
         np.testing.assert_allclose(d["out"][0], ref["out"][P], rtol=0, atol=1e-6)
         if kind == "csa":
             np.testing.assert_array_equal(d["sel"][0], ref["sel"][P])
