@@ -61,7 +61,7 @@ typedef enum {
     HCSA_ERR_WORKSPACE = 5,
     HCSA_ERR_CUDA = 6,
     HCSA_ERR_TIMEOUT = 7,      /* a bounded device-side wait gave up */
-    HCSA_ERR_UNSUPPORTED = 8,  /* valid request this build does not implement */
+    HCSA_ERR_UNSUPPORTED = 8,  /* valid request the library does not implement */
     HCSA_ERR_DEVICE = 9        /* a kernel's own bounds check fired */
 } hcsa_status;
 

@@ -93,7 +93,7 @@ const char *hcsa_status_string(hcsa_status s) {
         case HCSA_ERR_WORKSPACE: return "workspace too small";
         case HCSA_ERR_CUDA: return "CUDA launch or runtime error";
         case HCSA_ERR_TIMEOUT: return "a bounded device-side wait gave up";
-        case HCSA_ERR_UNSUPPORTED: return "configuration not supported by this build";
+        case HCSA_ERR_UNSUPPORTED: return "configuration not supported by the library";
         case HCSA_ERR_DEVICE: return "device-side bounds check failed";
     }
     return "unknown status";
