@@ -259,8 +259,8 @@ static int by_index(const void *pa, const void *pb) {
     return (a > b) - (a < b);
 }
 
-/* Top-k selection ("selecciona los bloques top-k mas relevantes"), exact, via a
- * library sort on (score descending, index ascending).
+/* Top-k selection (page "DeepSeek-V4 ... KV cache ...", section "CSA": the indexer's best-scoring
+ * compressed entries are kept), exact, via a library sort on (score descending, index ascending).
  * sel[q, 0..k) = the min(k, n_vis) best entries in ascending j, -1 padded.
  * kth_gap[q] (may be NULL) receives (s_(k) - s_(k+1)) / |s_(k)| (INFINITY when n_vis <= k). */
 void orc_topk(int nq, const double *scores, int64_t N, const int64_t *n_vis, int k, int32_t *sel,
