@@ -6,7 +6,8 @@ its own independent sequence: weak scaling, no collective on the data path).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-Other workloads (--workload): hca_prefill_T65536, csa_decode_B32_P262144, hybrid_decode_B4_P1048576.
+Other workloads (--workload): hca_prefill_T65536, csa_decode_B32_P262144, hybrid_decode_B4_P1048576,
+v4_decode_B4_P1048576 (two HCA layers, then CSA/HCA alternating, chained through the residual stream).
 """
 from __future__ import annotations
 
@@ -33,6 +34,7 @@ WORKLOADS = {
     "hca_prefill_T65536": ("prefill", "hca_bf16_t65536"),
     "csa_decode_B32_P262144": ("decode", "csa_decode_b32_p262144"),
     "hybrid_decode_B4_P1048576": ("decode", "hybrid_decode_b4_p1048576"),
+    "v4_decode_B4_P1048576": ("decode", "v4_decode_b4_p1048576"),
 }
 
 
@@ -76,8 +78,9 @@ def prefill_work(spec):
     return w
 
 
-def decode_bytes(spec, B, N):
-    """Algorithmic HBM bytes of one decode step of one layer (weights + cache reads + writes)."""
+def decode_bytes(spec, B, N, residual=False):
+    """Algorithmic HBM bytes of one decode step of one layer (weights + cache reads + writes; with the
+    residual chain also the output projection and the hidden state read and written)."""
     bpe = 2
     ncols = 2 * spec.C + spec.H * spec.dh + (spec.di + spec.Hi * spec.di + spec.Hi if spec.kind == "csa" else 0)
     b = spec.D * ncols * bpe                                   # weights
@@ -87,6 +90,8 @@ def decode_bytes(spec, B, N):
     else:
         b += B * (N + spec.window) * spec.C * bpe              # all entries + window
     b += B * spec.H * spec.dh * bpe * 2                        # q in, out
+    if residual:
+        b += spec.H * spec.dh * spec.D * bpe + B * spec.D * bpe * 2   # W_o, x in and out
     return float(b)
 
 
@@ -416,8 +421,7 @@ def run_decode(args, spec_name, ws, rank):
     if args.batch:
         import dataclasses
         d = dataclasses.replace(d, B=args.batch)
-    layers, Ws, Bs, xs = [], [], [], None
-    shared = {}
+    layers, Ws, Bs, Wos, xs = [], [], [], [], None
     for li, spec in enumerate(d.layers):
         inp = synth.decode_inputs(d, li)
         cache = {k: dev(inp[k]) for k in ("entries", "win_kv", "ring_g", "idx_keys", "ring_ki") if k in inp}
@@ -425,15 +429,23 @@ def run_decode(args, spec_name, ws, rank):
         layers.append(h.DecodeLayer(spec, d.B, n_cap, cache))
         Ws.append(dev(inp["W_cat"]))
         Bs.append(dev(inp["B"]))
+        Wos.append(dev(inp["W_o"]) if d.residual else None)
         if xs is None:
             xs = dev(inp["x"])
         del inp
     pos = torch.full((d.B,), d.P, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
+    xw = torch.empty_like(xs)   # the residual stream of a chained stack (restarts from xs every step)
 
     def step():
-        for L, W, B in zip(layers, Ws, Bs):
-            L.step(xs, W, B, pos)   # each layer reads the same hidden state; pos is not advanced (idempotent)
+        if d.residual:
+            xw.copy_(xs)
+            for L, W, B, Wo in zip(layers, Ws, Bs, Wos):
+                L.step(xw, W, B, pos)
+                L.out_project(xw, Wo)
+        else:
+            for L, W, B in zip(layers, Ws, Bs):
+                L.step(xs, W, B, pos)   # each layer reads the same hidden state
 
     for _ in range(args.warmup):
         step()
@@ -463,20 +475,21 @@ def run_decode(args, spec_name, ws, rank):
     torch.cuda.synchronize()
     launches = h.hcsa_launch_count() * args.steps
     hbm, tc, tc_sus, src = peaks()
-    total_bytes = sum(decode_bytes(L.spec, d.B, L.p.n_cap) for L in layers)
+    total_bytes = sum(decode_bytes(L.spec, d.B, L.p.n_cap, d.residual) for L in layers)
     ach = total_bytes / (us / 1e6) / 1e9
     roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
             "kernel": "whole decode step (CUDA graph)", "peak_kind": f"{src} hbm"}
     xh = torch.empty(xs.shape, dtype=xs.dtype, pin_memory=True)
     xh.copy_(xs)
-    oh = torch.empty(layers[-1].out.shape, dtype=layers[-1].out.dtype, pin_memory=True)
+    result = xw if d.residual else layers[-1].out   # the step's result: hidden state or last layer's output
+    oh = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
     torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record(stream)
     for _ in range(args.steps):
         xs.copy_(xh, non_blocking=True)
         g.replay()
-        oh.copy_(layers[-1].out, non_blocking=True)
+        oh.copy_(result, non_blocking=True)
     a1.record(stream)
     torch.cuda.synchronize()
     eus = max_over_ranks(a0.elapsed_time(a1), ws) / args.steps * 1e3
@@ -484,7 +497,7 @@ def run_decode(args, spec_name, ws, rank):
     line = {"metric": METRIC, "value": us, "unit": "us/step", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
-            "config": {"workload": spec_name, "B": d.B, "P": d.P, "layers": len(d.layers),
+            "config": {"workload": spec_name, "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
                        "parallelism": f"replicas x{ws}", "l2": "working set larger than L2",
                        "bytes_per_step": total_bytes},
             "roofline": roof,

@@ -136,6 +136,17 @@ int64_t hcsa_proj_cols(const hcsa_params *p, int32_t kind);
 hcsa_status hcsa_project(const hcsa_params *p, int32_t kind, int64_t rows, const void *x, const void *W_cat,
                          void *y, void *ws, size_t ws_bytes, void *stream);
 
+/* Output projection with the residual stream, for stacks whose layers are chained (the V4-style
+ * schedule: two HCA layers, then CSA and HCA alternating).  The pages define no output projection
+ * or normalisation; the reading is x_{l+1} = x_l + out_l W_o,l.
+ *   out [rows, ld_out]   the layer's attention output (H*dh columns used)
+ *   W_o [H*dh, D]        row-major
+ *   x   [rows, ld_x]     the hidden state, updated in place: x += out W_o, fp32 accumulate, one
+ *                        rounding to bf16 (cuBLAS GEMM with beta = 1)
+ * bf16 storage only (HCSA_ERR_UNSUPPORTED otherwise).  ws as for hcsa_project (may be NULL). */
+hcsa_status hcsa_out_project(const hcsa_params *p, int64_t rows, const void *out, int64_t ld_out, const void *W_o,
+                             void *x, int64_t ld_x, void *ws, size_t ws_bytes, void *stream);
+
 /* CSA compressor (m, width = 8 overlapping pools), prefill of one sequence of p->T tokens.
  *   kv [T, ld_kv] (C used), g [T, ld_g] (C used), ki [T, ld_ki] (di used), bias [width, C]
  *   entries [N, C], idx_keys [N, di] with N = ceil(T / m) (edge pools are truncated to [0, T)). */

@@ -25,6 +25,7 @@ STATUS = {0: "HCSA_OK", 1: "HCSA_ERR_NULL", 2: "HCSA_ERR_SHAPE", 3: "HCSA_ERR_DT
 
 # every entry point the header declares (checked by the CPU export test)
 EXPORTS = ["hcsa_version", "hcsa_status_string", "hcsa_workspace_bytes", "hcsa_proj_cols", "hcsa_project",
+           "hcsa_out_project",
            "csa_compress", "hca_compress", "csa_index_topk", "csa_attend", "hca_attend", "hcsa_cache_append",
            "csa_decode_index_topk", "csa_decode_attend", "hca_decode_attend", "csa_decode_index_topk_noalloc",
            "hcsa_get_device_status", "hcsa_selftest_wait_timeout",
@@ -67,6 +68,7 @@ def load():
         "hcsa_workspace_bytes": (SZ, [P, I32]),
         "hcsa_proj_cols": (I64, [P, I32]),
         "hcsa_project": (I32, [P, I32, I64, V, V, V, V, SZ, V]),
+        "hcsa_out_project": (I32, [P, I64, V, I64, V, V, I64, V, SZ, V]),
         "csa_compress": (I32, [P, V, I64, V, I64, V, I64, V, V, V, V]),
         "hca_compress": (I32, [P, V, I64, V, I64, V, V, V]),
         "csa_index_topk": (I32, [P, V, I64, V, I64, V, V, V, SZ, V]),
@@ -141,6 +143,12 @@ def hcsa_project(p, kind, x, W_cat, y, ws=None, stream=None):
     _check("hcsa_project", load().hcsa_project(ctypes.byref(p), kind, x.shape[0], _ptr(x), _ptr(W_cat), _ptr(y),
                                                _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                                _stream(stream)))
+
+
+def hcsa_out_project(p, out, W_o, x, ws=None, stream=None):
+    """x += out W_o in place (the residual update of a chained stack; bf16)."""
+    _check("hcsa_out_project", load().hcsa_out_project(ctypes.byref(p), x.shape[0], _ptr(out), _ld(out), _ptr(W_o),
+                                                       _ptr(x), _ld(x), _ptr(ws), _wsz(ws), _stream(stream)))
 
 
 def csa_compress(p, kv, g, ki, bias, entries, idx_keys, stream=None):

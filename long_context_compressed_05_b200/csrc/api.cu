@@ -142,6 +142,20 @@ hcsa_status hcsa_project(const hcsa_params *p, int32_t kind, int64_t rows, const
     return launch_project(p->dtype, rows, p->D, nc, x, W_cat, y, ws, ws_bytes, (cudaStream_t)stream);
 }
 
+hcsa_status hcsa_out_project(const hcsa_params *p, int64_t rows, const void *out, int64_t ld_out, const void *W_o,
+                             void *x, int64_t ld_x, void *ws, size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_common(p));
+    if (p->dtype != HCSA_BF16) return HCSA_ERR_UNSUPPORTED;
+    if (!out || !W_o || !x) return HCSA_ERR_NULL;
+    if (rows < 0 || p->D < 1) return HCSA_ERR_SHAPE;
+    const int64_t hd = (int64_t)p->H * p->dh;
+    if (!aligned(out) || !aligned(W_o) || !aligned(x)) return HCSA_ERR_ALIGN;
+    if (!ld_ok(p->dtype, ld_out, hd) || !ld_ok(p->dtype, ld_x, p->D) || (p->D * esize(p->dtype)) % 16)
+        return HCSA_ERR_ALIGN;
+    if (ws && ws_bytes < project_ws_bytes(p->dtype)) return HCSA_ERR_WORKSPACE;
+    return launch_out_project(rows, hd, p->D, out, ld_out, W_o, x, ld_x, ws, ws_bytes, (cudaStream_t)stream);
+}
+
 hcsa_status csa_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
                          const void *ki, int64_t ld_ki, const void *bias, void *entries, void *idx_keys,
                          void *stream) {

@@ -139,5 +139,8 @@ hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st);
 size_t project_ws_bytes(int dtype);
 hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const void *x, const void *W, void *y,
                            void *ws, size_t ws_bytes, cudaStream_t st);
+// x[rows, D] += out[rows, HD] W_o[HD, D] (bf16)
+hcsa_status launch_out_project(int64_t rows, int64_t HD, int D, const void *out, int64_t ld_out, const void *W_o,
+                               void *x, int64_t ld_x, void *ws, size_t ws_bytes, cudaStream_t st);
 
 }  // namespace hcsa

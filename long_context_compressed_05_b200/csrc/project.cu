@@ -93,4 +93,22 @@ hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const 
     return s == CUBLAS_STATUS_SUCCESS ? check_launch() : HCSA_ERR_CUDA;
 }
 
+// Output projection with the residual: x[rows, D] += out[rows, HD] W_o[HD, D] (bf16 storage, fp32
+// accumulate, one rounding: cuBLAS with beta = 1 reads x as C).
+hcsa_status launch_out_project(int64_t rows, int64_t HD, int D, const void *out, int64_t ld_out, const void *W_o,
+                               void *x, int64_t ld_x, void *ws, size_t ws_bytes, cudaStream_t st) {
+    if (rows == 0) return HCSA_OK;
+    if (rows > INT32_MAX || HD > INT32_MAX || ld_out > INT32_MAX || ld_x > INT32_MAX) return HCSA_ERR_UNSUPPORTED;
+    cublasHandle_t h = handle_for_device();
+    if (!h) return HCSA_ERR_CUDA;
+    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
+    if (ws && ws_bytes && cublasSetWorkspace(h, ws, ws_bytes) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
+    const float alpha = 1.0f, beta = 1.0f;
+    // row-major x[rows, D] += out[rows, HD] W_o[HD, D]  <=>  column-major x^T += W_o^T out^T
+    cublasStatus_t s = cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, D, (int)rows, (int)HD, &alpha, W_o, CUDA_R_16BF, D,
+                                    out, CUDA_R_16BF, (int)ld_out, &beta, x, CUDA_R_16BF, (int)ld_x,
+                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+    return s == CUBLAS_STATUS_SUCCESS ? check_launch() : HCSA_ERR_CUDA;
+}
+
 }  // namespace hcsa

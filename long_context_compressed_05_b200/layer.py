@@ -139,3 +139,8 @@ class DecodeLayer:
         else:
             L.hca_decode_attend(self.p, self.cache, pos, self.view("q"), self.out, self.ws_attend)
         return self.out
+
+    def out_project(self, x, W_o):
+        """Residual update of a chained stack: x += out W_o, in place."""
+        L.hcsa_out_project(self.p, self.out, W_o, x, self.ws_proj)
+        return x

@@ -361,6 +361,28 @@ def decode_step(spec, inp, P, seqs=None, lowprec=False):
     return res
 
 
+def decode_stack(specs, layer_inputs, P, residual=True, lowprec=False):
+    """Decode steps of a stack of layers for one batch.
+
+    Layer l reads the hidden state x_l (x_0 = layer_inputs[0]["x"]).  With residual, the layers chain
+    through the residual stream: x_{l+1} = x_l + out_l W_o,l, rounded once to the storage format (the
+    pages define neither an output projection nor a normalisation; this is the reading taken for the
+    V4-style schedule).  Without residual every layer reads x_0.  layer_inputs[l]: as for decode_step,
+    plus W_o [H*dh, D] when residual.  Returns (the hidden state after the last layer, per-layer
+    results of decode_step)."""
+    x0 = to_f64(layer_inputs[0]["x"])
+    x = x0
+    results = []
+    for spec, inp in zip(specs, layer_inputs):
+        li = dict(inp)
+        li["x"] = x
+        r = decode_step(spec, li, P, lowprec=lowprec)
+        results.append(r)
+        if residual:
+            x = round_to(x + r["out"] @ to_f64(inp["W_o"]), storage_code(spec.dtype))
+    return x, results
+
+
 def decode_attend_with_sel(spec, res, i, sel_row):
     """Recompute the i-th evaluated row of a decode_step result on a given selection (e.g. the GPU's)."""
     st = storage_code(spec.dtype)

@@ -10,6 +10,7 @@ decode caches ~ N(0,1).
 Tensor ids (the generator's stream selector) are fixed per layer:
   0 x | 1 W_kv | 2 W_g | 3 W_ki | 4 W_qi | 5 W_w | 6 W_q | 7 B
   8 entries cache | 9 indexer-key cache | 10 window ring | 11 gate ring | 12 indexer-key ring
+  13 W_o (output projection of a residual-chained stack)
 Layer L of a multi-layer stack adds 16*L to every id except x (id 0), which
 all layers share.
 """
@@ -56,6 +57,7 @@ class DecodeSpec:
     B: int               # sequences
     P: int               # position of the new token (= prefix length)
     seed: int = 0
+    residual: bool = False   # chain the layers: x_{l+1} = x_l + out_l W_o,l (W_o ~ N(0, 1/(H dh)))
 
     def n_cache_entries(self, layer: LayerSpec) -> int:
         # entries fully formed by the prefix [0, P): entry j is complete once token m*j+m-1 < P
@@ -101,6 +103,12 @@ DECODE = {
         layers=tuple(LayerSpec(T=0, seed=4, **dict(_CSA_BIG, topk=1024)) if i % 2 == 0
                      else LayerSpec(T=0, seed=4, **_HCA_BIG) for i in range(8)),
         B=4, P=1048576, seed=4),
+    # V4-style schedule: two HCA layers, then CSA and HCA alternating, chained through the residual
+    # stream by an output projection per layer; 4 sequences at 1M context
+    "v4_decode_b4_p1048576": DecodeSpec(
+        layers=tuple(LayerSpec(T=0, seed=5, **_HCA_BIG) if (i < 2 or i % 2 == 1)
+                     else LayerSpec(T=0, seed=5, **dict(_CSA_BIG, topk=1024)) for i in range(8)),
+        B=4, P=1048576, seed=5, residual=True),
 }
 
 
@@ -145,6 +153,8 @@ def decode_inputs(d: DecodeSpec, layer_index: int, with_cache: bool = True, seqs
     out = _weights(s, d.seed, base, kind)
     out["W_cat"] = w_cat(s, out)
     out["x"] = normal(d.seed, 0, (d.B, s.D), 1.0, kind)
+    if d.residual:
+        out["W_o"] = normal(d.seed, base + 13, (s.H * s.dh, s.D), 1.0 / math.sqrt(s.H * s.dh), kind)
     if with_cache:
         N = d.n_cache_entries(s) if n_cap is None else n_cap
         seqs = list(range(d.B)) if seqs is None else list(seqs)

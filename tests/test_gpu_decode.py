@@ -164,3 +164,30 @@ def test_decode_long_rows_select():
         want = np.full(spec.topk, -1, dtype=np.int64)
         want[: len(order)] = np.sort(order)
         np.testing.assert_array_equal(sel[b], want)
+
+
+def test_decode_residual_stack():
+    """A V4-style stack (two HCA layers, then a CSA layer) chained through the residual stream: every layer's
+    output against the oracle on the GPU's own hidden state, and every residual update x += out W_o against
+    the fp64 update of the GPU's own output, rounded once to bf16."""
+    from long_context_compressed_05_b200 import DecodeLayer, hcsa_get_device_status
+    d = synth.DecodeSpec(layers=(HCA_D.replace(seed=41), HCA_D.replace(seed=41), CSA_D.replace(seed=41)), B=3,
+                         P=1000, seed=41, residual=True)
+    pos = torch.full((d.B,), d.P, dtype=torch.int32, device="cuda")
+    x = None
+    for li, spec in enumerate(d.layers):
+        inp = synth.decode_inputs(d, li)
+        if x is None:
+            x = dev(inp["x"])
+        cache = {k: dev(inp[k]) for k in ("entries", "win_kv", "ring_g", "idx_keys", "ring_ki") if k in inp}
+        layer = DecodeLayer(spec, d.B, inp["entries"].shape[1], cache)
+        x_in = host64(x)
+        layer.step(x, dev(inp["W_cat"]), dev(inp["B"]), pos)
+        torch.cuda.synchronize()
+        assert hcsa_get_device_status() == 0
+        compare_step(spec, dict(inp, x=x_in), layer, cache, np.full(d.B, d.P), list(range(d.B)))
+        out = host64(layer.out)
+        layer.out_project(x, dev(inp["W_o"]))
+        torch.cuda.synchronize()
+        want = oracle.round_to(x_in + out @ oracle.to_f64(inp["W_o"]), oracle.ST_BF16)
+        np.testing.assert_allclose(host64(x), want, rtol=2 ** -7, atol=2 ** -10)

@@ -366,3 +366,31 @@ def test_decode_steps_match_prefill(orc, kind, lowprec):
             np.testing.assert_allclose(d["new_entry"][0]["entry"], ref["entries"][j], rtol=0, atol=1e-6)
         else:
             assert d["new_entry"][0] is None
+
+
+def test_decode_stack_residual_chain_brute_force(orc):
+    """A residual-chained decode stack: each layer reads the previous layer's hidden state, and the update
+    x + out W_o (checked by explicit sums on a tiny case) is rounded once; with W_o = 0 the stack is the
+    same step repeated on the same input."""
+    import synth
+    hca = synth.LayerSpec(kind="hca", T=0, D=16, m=8, width=8, C=16, window=8, H=2, dh=8, scale=8 ** -0.5,
+                          dtype="bf16", seed=21)
+    csa = synth.LayerSpec(kind="csa", T=0, D=16, m=4, width=8, C=16, di=8, Hi=2, topk=4, window=8, H=2, dh=8,
+                          scale=8 ** -0.5, dtype="bf16", seed=21)
+    d = synth.DecodeSpec(layers=(hca, hca, csa), B=2, P=45, seed=21, residual=True)
+    inps = [synth.decode_inputs(d, i) for i in range(3)]
+    x_end, res = orc.decode_stack(d.layers, inps, d.P)
+    x = orc.to_f64(inps[0]["x"])
+    for li, (spec, inp) in enumerate(zip(d.layers, inps)):
+        step = orc.decode_step(spec, dict(inp, x=x), d.P)
+        np.testing.assert_array_equal(step["out"], res[li]["out"])
+        Wo = orc.to_f64(inp["W_o"])
+        upd = np.array([[x[b, c] + sum(step["out"][b, k] * Wo[k, c] for k in range(Wo.shape[0]))
+                         for c in range(spec.D)] for b in range(d.B)])
+        x = orc.round_to(upd, orc.ST_BF16)
+    np.testing.assert_allclose(x_end, x, rtol=0, atol=0)
+    # zero output projection: every layer sees the input hidden state
+    zero = [dict(inp, W_o=np.zeros_like(inp["W_o"])) for inp in inps]
+    x_same, res0 = orc.decode_stack(d.layers, zero, d.P)
+    np.testing.assert_array_equal(x_same, orc.to_f64(inps[0]["x"]))
+    np.testing.assert_array_equal(res0[1]["out"], orc.decode_step(hca, dict(inps[1]), d.P)["out"])
