@@ -552,7 +552,7 @@ def main():
                       "parallelism": "CPU oracle on rank 0"}
         else:
             ms = v / 1e3
-            config = {"workload": name, "B": d.B, "P": d.P, "layers": len(d.layers),
+            config = {"workload": name, "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
                       "parallelism": "CPU oracle on rank 0"}
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": ws,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": hib,
