@@ -64,3 +64,22 @@ def test_oracle_regression_snapshot(orc):
     ref = np.load(os.path.join(GOLD, "oracle_csa_tiny.npz"))
     for k in ref.files:
         np.testing.assert_array_equal(got[k], ref[k])
+
+
+def test_v4_schedule_workload():
+    """The residual-chained 1M-context workload: two HCA layers, then CSA and HCA alternating; every layer has
+    its own output projection W_o ~ N(0, 1/(H dh)) drawn from a stream of its own."""
+    import synth
+    d = synth.DECODE["v4_decode_b4_p1048576"]
+    assert d.residual and [s.kind for s in d.layers] == ["hca", "hca", "csa", "hca", "csa", "hca", "csa", "hca"]
+    small = synth.DecodeSpec(layers=tuple(s.replace(D=64, C=32, H=2, dh=16, di=16, Hi=2, topk=8, window=8,
+                                                    width=8 if s.kind == "csa" else 128) for s in d.layers[:3]),
+                             B=2, P=300, seed=d.seed, residual=True)
+    wo = [synth.decode_inputs(small, i, with_cache=False)["W_o"] for i in range(3)]
+    from oracle import to_f64
+    w0 = to_f64(wo[0])
+    assert w0.shape == (32, 64)
+    assert abs(w0.std() * (32 ** 0.5) - 1.0) < 0.1 and abs(w0.mean()) < 0.03
+    assert not np.array_equal(wo[0], wo[1])          # per-layer streams
+    plain = synth.DecodeSpec(layers=small.layers, B=2, P=300, seed=d.seed)
+    assert "W_o" not in synth.decode_inputs(plain, 0, with_cache=False)
