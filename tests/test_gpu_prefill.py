@@ -82,7 +82,8 @@ def compare(spec, inp, layer, rows, ref):
         np.testing.assert_allclose(host64(layer.idx_keys), idx_iso, rtol=rt_iso, atol=1e-6)
         np.testing.assert_allclose(host64(layer.idx_keys), ref["idx_keys"], rtol=rt, atol=at)
         sel = layer.sel.cpu().numpy()[rows]
-        check_selection(sel, ref["sel"], ref["gap"], ref["scores"], ref["n_vis"], spec.topk, exact=f32)
+        check_selection(sel, ref["sel"], ref["gap"], ref["scores"], ref["n_vis"], spec.topk, exact=f32,
+                        label=f"{spec.kind} T={spec.T} k={spec.topk}")
         ref_out = oracle.attend_rows(spec, ref, ref["q"], sel)     # oracle on the GPU's own selection
     else:
         ref_out = ref["out"]

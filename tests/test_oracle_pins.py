@@ -394,3 +394,31 @@ def test_decode_stack_residual_chain_brute_force(orc):
     x_same, res0 = orc.decode_stack(d.layers, zero, d.P)
     np.testing.assert_array_equal(x_same, orc.to_f64(inps[0]["x"]))
     np.testing.assert_array_equal(res0[1]["out"], orc.decode_step(hca, dict(inps[1]), d.P)["out"])
+
+
+# ------------------------------------------------------------------ visibility (pinned from both sides)
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 7, 128])
+def test_prefill_visibility_matches_brute_force_count(orc, m):
+    # entry j is visible to query t iff m j + m <= t (its last pooled token m j + m - 1 lies before t);
+    # counting those j directly pins the cut from above and from below
+    T = 300 if m == 128 else 64
+    N = -(-T // m)
+    t = np.arange(T)
+    want = np.array([sum(1 for j in range(N) if m * j + m <= tt) for tt in t])
+    np.testing.assert_array_equal(orc.prefill_n_vis(t, m, N), want)
+
+
+def test_selection_with_k_at_least_visible_is_exactly_the_visible_set(orc):
+    # with top-k >= every visible count the selection is the visible set itself: at t = m j + m the
+    # entry j (just completed) is selected, entry j + 1 is not
+    import synth
+    spec = _small_csa(T=64, topk=64)
+    inp = synth.prefill_inputs(spec)
+    res = orc.prefill(spec, inp)
+    for t in range(spec.T):
+        want = [j for j in range(-(-spec.T // spec.m)) if spec.m * j + spec.m <= t]
+        got = [int(j) for j in res["sel"][t] if j >= 0]
+        assert got == want, t
+        if t % spec.m == 0 and t >= spec.m:
+            assert t // spec.m - 1 in got and t // spec.m not in got
