@@ -79,6 +79,21 @@ int64_t n_entries(const hcsa_params *p) { return ((int64_t)p->T + p->m - 1) / p-
 
 }  // namespace
 
+namespace hcsa {
+
+hcsa_status check_decode_index_topk_args(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                         const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
+                                         const int32_t *sel) {
+    HCSA_TRY(check_csa(p));
+    HCSA_TRY(check_decode(p, cache, pos, true));
+    if (!qi || !w || !sel) return HCSA_ERR_NULL;
+    if (!aligned(qi) || !aligned(w) || !aligned(sel)) return HCSA_ERR_ALIGN;
+    if (ld_qi < (int64_t)p->Hi * p->di || ld_w < p->Hi) return HCSA_ERR_SHAPE;
+    return HCSA_OK;
+}
+
+}  // namespace hcsa
+
 extern "C" {
 
 int32_t hcsa_version(void) { return 100; }
@@ -240,11 +255,7 @@ hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, con
 hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
                                   const void *qi, int64_t ld_qi, const void *w, int64_t ld_w, int32_t *sel,
                                   void *ws, size_t ws_bytes, void *stream) {
-    HCSA_TRY(check_csa(p));
-    HCSA_TRY(check_decode(p, cache, pos, true));
-    if (!qi || !w || !sel) return HCSA_ERR_NULL;
-    if (!aligned(qi) || !aligned(w) || !aligned(sel)) return HCSA_ERR_ALIGN;
-    if (ld_qi < (int64_t)p->Hi * p->di || ld_w < p->Hi) return HCSA_ERR_SHAPE;
+    HCSA_TRY(hcsa::check_decode_index_topk_args(p, cache, pos, qi, ld_qi, w, ld_w, sel));
     if (!ws || ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
     IndexArgs a{p->dtype, p->B, p->Hi, p->di, p->topk, p->m, p->n_cap, qi, ld_qi, w, ld_w, cache->idx_keys,
                 pos, sel, ws, ws_bytes, nullptr};

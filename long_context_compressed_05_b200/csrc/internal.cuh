@@ -57,6 +57,10 @@ __device__ __forceinline__ void report(int *status, int code) {
 
 // ---------------------------------------------------------------- host side helpers
 int *device_status_ptr();           // lazily resolved per device; nullptr on failure
+// host-side argument checks of csa_decode_index_topk (everything but the workspace)
+hcsa_status check_decode_index_topk_args(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                         const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
+                                         const int32_t *sel);
 void count_launch(int n = 1);
 hcsa_status check_launch();         // maps cudaGetLastError() to a status
 

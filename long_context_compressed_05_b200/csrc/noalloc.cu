@@ -50,9 +50,9 @@ using namespace hcsa;
 extern "C" hcsa_status csa_decode_index_topk_noalloc(const hcsa_params *p, const hcsa_cache *cache,
                                                      const int32_t *pos, const void *qi, int64_t ld_qi,
                                                      const void *w, int64_t ld_w, int32_t *sel, void *stream) {
-    if (!p) return HCSA_ERR_NULL;
-    if (p->dtype != HCSA_BF16 && p->dtype != HCSA_F32) return HCSA_ERR_DTYPE;
-    if (p->B < 1 || p->n_cap < 1) return HCSA_ERR_SHAPE;
+    // malformed requests get the same answer as from csa_decode_index_topk, whatever their size
+    const hcsa_status v = check_decode_index_topk_args(p, cache, pos, qi, ld_qi, w, ld_w, sel);
+    if (v != HCSA_OK) return v;
     // the scores of all B sequences must fit the fixed scratch array
     const size_t need = hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK);
     if (need > sizeof(g_noalloc_scores)) return HCSA_ERR_WORKSPACE;

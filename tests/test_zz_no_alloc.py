@@ -12,7 +12,10 @@ from tests._helpers import dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("Hi,P,n_cap", [(32, [4000, 4093, 2047], 1100), (8, [517, 1023, 300], 300)])
+# the last case has rows longer than 32768 entries: the multi-block selection keeps its histograms,
+# counters and candidates after the scores inside the fixed array
+@pytest.mark.parametrize("Hi,P,n_cap", [(32, [4000, 4093, 2047], 1100), (8, [517, 1023, 300], 300),
+                                        (32, [262000, 200003], 65536)])
 def test_noalloc_matches_workspace_entry_point(Hi, P, n_cap):
     import long_context_compressed_05_b200 as h
     spec = synth.LayerSpec(kind="csa", T=0, D=256, m=4, width=8, C=256, di=64, Hi=Hi, topk=128, window=128, H=4,
@@ -45,8 +48,23 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     spec = synth.LayerSpec(kind="csa", T=0, D=256, m=4, width=8, C=256, di=64, Hi=32, topk=128, window=128, H=4,
                            dh=128, scale=0.1, dtype="bf16")
     p = h.params_for(spec, T=0, B=3, n_cap=1 << 20)       # 3 Mi scores > 2 Mi
-    cache = h.make_cache(None, None, None)
-    dummy = torch.empty(16, dtype=torch.int32, device="cuda")
+    dummy = torch.zeros(64, dtype=torch.int32, device="cuda")
+    pos = torch.zeros(3, dtype=torch.int32, device="cuda")
+    qi = torch.zeros((3, spec.Hi * spec.di), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((3, spec.Hi), dtype=torch.bfloat16, device="cuda")
+    sel = torch.zeros((3, spec.topk), dtype=torch.int32, device="cuda")
+    # well-formed arguments: the request is refused for its size alone, before anything is launched
+    cache = h.make_cache(dummy, dummy, dummy, dummy, dummy)
     with pytest.raises(h.HcsaError) as e:
-        h.csa_decode_index_topk_noalloc(p, cache, dummy, dummy, dummy, dummy)
+        h.csa_decode_index_topk_noalloc(p, cache, pos, qi, w, sel)
     assert e.value.code == 5
+    # a malformed request is refused for what is wrong with it, whatever its size
+    with pytest.raises(h.HcsaError) as e:
+        h.csa_decode_index_topk_noalloc(p, h.make_cache(None, None, None), pos, qi, w, sel)
+    assert e.value.code == 1
+    with pytest.raises(h.HcsaError) as e:
+        narrow = torch.zeros((3, 64), dtype=torch.bfloat16, device="cuda")   # rows narrower than Hi * di
+        h.csa_decode_index_topk_noalloc(p, cache, pos, narrow, w, sel)
+    assert e.value.code == 2
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dummy) == 0 and torch.count_nonzero(sel) == 0
