@@ -20,12 +20,18 @@ constexpr int kHeadsPerCta = 8;
 constexpr int kMaxEpl = 16;          // dh <= 512
 constexpr int kDecodeSplit = 128;    // keys per split (decode)
 
+// Key row kk of query r: entries first (the selection, or every visible entry), then the raw window.
+// A selected index that is neither the -1 padding nor a visible entry is skipped and reported.
 template <typename S>
-__device__ __forceinline__ const S *key_row(const AttendArgs &a, int64_t r, int64_t p, int64_t ne, int64_t kk) {
+__device__ __forceinline__ const S *key_row(const AttendArgs &a, int64_t r, int64_t p, int64_t ne, int64_t nvis,
+                                            int64_t kk, int *status) {
     const S *ent = reinterpret_cast<const S *>(a.entries) + (a.pos ? r * a.N * a.C : 0);
     if (kk < ne) {
         int64_t j = a.dense ? kk : (int64_t)a.sel[r * a.topk + kk];
-        if (j < 0 || j >= a.N) return nullptr;
+        if (j < 0 || j >= nvis) {
+            if (j != -1) report(status, kStatusBounds);
+            return nullptr;
+        }
         return ent + j * a.C;
     }
     int64_t pp = p - a.window + 1 + (kk - ne);
@@ -35,7 +41,7 @@ __device__ __forceinline__ const S *key_row(const AttendArgs &a, int64_t r, int6
 }
 
 template <typename S>
-__global__ void __launch_bounds__(kHeadsPerCta * 32) attend_kernel(AttendArgs a, int nsplit) {
+__global__ void __launch_bounds__(kHeadsPerCta * 32) attend_kernel(AttendArgs a, int nsplit, int *status) {
     using A = typename Traits<S>::A;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int h = blockIdx.y * kHeadsPerCta + warp;
@@ -60,7 +66,7 @@ __global__ void __launch_bounds__(kHeadsPerCta * 32) attend_kernel(AttendArgs a,
     A mx = -INFINITY, z = A(0);
     const A scale = (A)a.scale;
     for (int64_t kk = k0; kk < k1; ++kk) {
-        const S *row = key_row<S>(a, r, p, ne, kk);
+        const S *row = key_row<S>(a, r, p, ne, nvis, kk, status);
         if (!row) continue;
         A dot = A(0);
 #pragma unroll
@@ -220,8 +226,9 @@ hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st) {
         return HCSA_ERR_WORKSPACE;
     if (ns > 65535) return HCSA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)a.rows, (a.H + kHeadsPerCta - 1) / kHeadsPerCta, ns);
-    if (a.dtype == HCSA_BF16) attend_kernel<__nv_bfloat16><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns);
-    else attend_kernel<float><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns);
+    int *status = device_status_ptr();
+    if (a.dtype == HCSA_BF16) attend_kernel<__nv_bfloat16><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns, status);
+    else attend_kernel<float><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns, status);
     if (ns > 1) launch_combine(a, ns, st);
     count_launch(ns > 1 ? 2 : 1);
     return check_launch();

@@ -219,6 +219,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (kk < x.E) {
                         const int64_t j = a.dense ? (int64_t)kk : (int64_t)jsel[i];
                         if (j >= 0 && j < x.nvis) ptr = a.ent + ((a.decode ? x.q * a.N : 0) + j) * (int64_t)kC;
+                        else if (j != -1) report(a.status, kStatusBounds);   // not padding, not visible: skipped
                     } else {
                         const int64_t pp = x.p - (kKT - 1) + (kk - x.E);
                         if (pp >= 0) ptr = a.raw + (a.decode ? x.q * kKT + pp % kKT : pp) * a.ld_raw;

@@ -35,3 +35,39 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert h.hcsa_get_device_status() == 0
     assert torch.isfinite(out.float()).all()
     assert np.abs(out.float().cpu().numpy()).max() > 0
+
+
+HCSA_ERR_DEVICE = 9
+
+
+@pytest.mark.parametrize("H,dh,C", [(8, 128, 256), (64, 512, 1024)])   # generic and tensor-core attention
+def test_selection_outside_the_visible_range_is_skipped_and_reported(H, dh, C):
+    """A caller-provided selection index that is neither -1 padding nor a visible entry (here: one entry
+    past the visible range, and one far beyond the sequence) is not read: the kernel checks the index
+    before the access, skips that key, and records HCSA_ERR_DEVICE.  The output equals the one computed
+    with those indices replaced by -1."""
+    import long_context_compressed_05_b200 as h
+    from long_context_compressed_05_b200 import PrefillLayer
+    spec = synth.LayerSpec(kind="csa", T=900, D=256, m=4, width=8, C=C, di=64, Hi=8, topk=128, window=128, H=H,
+                           dh=dh, scale=dh ** -0.5, dtype="bf16", seed=92)
+    inp = synth.prefill_inputs(spec)
+    layer = PrefillLayer(spec)
+    layer.forward(dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"]))
+    torch.cuda.synchronize()
+    assert h.hcsa_get_device_status() == 0
+    t = 801                                          # 200 visible entries, 128 selected
+    bad = layer.sel.clone()
+    bad[t, 5] = t // spec.m                          # first entry that is not yet visible
+    bad[t, 9] = 1 << 30                              # far beyond the sequence
+    good = bad.clone()
+    good[t, 5] = -1
+    good[t, 9] = -1
+    layer.attend(sel=good)
+    torch.cuda.synchronize()
+    assert h.hcsa_get_device_status() == 0
+    want = layer.out.clone()
+    layer.attend(sel=bad)
+    torch.cuda.synchronize()
+    assert h.hcsa_get_device_status() == HCSA_ERR_DEVICE
+    assert h.hcsa_get_device_status() == 0
+    assert torch.equal(layer.out, want)
