@@ -1,17 +1,23 @@
 """Benchmark of the hybrid compressed attention path on B200.
 
-Default workload: one CSA layer prefill, bf16, T=131072, D=2048 (projection + compressor + lightning
-indexer/top-k + attention), inputs resident in HBM.  `value` is tokens/s over all ranks (each rank runs
-its own independent sequence: weak scaling, no collective on the data path).
+Default run: the headline workload, one CSA layer prefill, bf16, T=131072, D=2048 (projection +
+compressor + lightning indexer/top-k + attention), inputs resident in HBM; `value` is tokens/s over all
+ranks (each rank runs its own independent sequence: weak scaling, no collective on the data path).
+Then the other workloads, each measured the same way and nested in the same JSON line under
+"workloads": HCA prefill T=65536, CSA decode B=32 at a 262144-token prefix, the 8-layer CSA/HCA decode
+stack B=4 at 1M context, and the V4-style stack (two HCA layers, then CSA/HCA alternating, chained
+through the residual stream).  Every workload carries its roofline, end-to-end and CPU-oracle figures.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference] [--no-extra]
 
-Other workloads (--workload): hca_prefill_T65536, csa_decode_B32_P262144, hybrid_decode_B4_P1048576,
-v4_decode_B4_P1048576 (two HCA layers, then CSA/HCA alternating, chained through the residual stream).
+--workload NAME runs one workload alone (hca_prefill_T65536, csa_decode_B32_P262144,
+hybrid_decode_B4_P1048576, v4_decode_B4_P1048576, csa_prefill_T131072).
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
+import gc
 import json
 import math
 import os
@@ -235,83 +241,63 @@ def max_over_ranks(x: float, ws: int) -> float:
 
 # ------------------------------------------------------------------ CPU oracle timing (bounded sample)
 
-def oracle_prefill_rate(spec, inp, budget_rows=8):
-    """Oracle throughput (tokens/s) extrapolated from a bounded sample of the whole layer:
-    projection of 256 rows, the compressor over 1024 tokens, and index/top-k/attention for
-    `budget_rows` queries spread uniformly over the sequence."""
+def _host_cores():
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_prefill_rate(spec, inp, n_rows=1024, offset=0.5, entries=None):
+    """Oracle throughput (tokens/s) of the whole layer, from a bounded sample of the workload's own inputs.
+
+    The sequence-wide half (projections of the pooled columns and the compressor over all T tokens) is
+    timed in full, unless `entries` = (result, seconds) of an earlier timing is passed.  The per-query half
+    (query projections, indexer, top-k, attention over the real entries) is timed on n_rows query
+    positions spread evenly over the sequence -- row i at (i + offset) T / n_rows, so the sample has the
+    sequence's mix of visible counts -- and scaled by T / n_rows.  Returns (tokens/s, sample description,
+    (result, seconds) of the sequence-wide half)."""
     import oracle
-    st = oracle.storage_code(spec.dtype)
     T = spec.T
-    W = oracle.to_f64(inp["W_cat"])
-    cols = oracle._col_slices(spec)
+    if entries is None:
+        t0 = time.perf_counter()
+        res = oracle.prefill_entries(spec, inp)
+        entries = (res, time.perf_counter() - t0)
+    res, t_fixed = entries
+    n_rows = min(n_rows, T)
+    rows = np.unique(((np.arange(n_rows) + offset) * T / n_rows).astype(np.int64))
     t0 = time.perf_counter()
-    nr = min(256, T)
-    y = oracle.project(oracle.to_f64(inp["x"][:nr]), W, st)
-    t_proj = (time.perf_counter() - t0) * T / nr
-    nt = min(1024, T)
-    t0 = time.perf_counter()
-    csa = spec.kind == "csa"
-    yp = np.ascontiguousarray(np.concatenate([y] * (-(-nt // nr)))[:nt])
-    base = yp.ctypes.data
-    oracle.compress(nt, spec.C, spec.m, spec.width, base, yp.shape[1], base + 8 * spec.C, yp.shape[1],
-                    oracle.to_f64(inp["B"]), base + 8 * cols["ki"].start if csa else None, yp.shape[1],
-                    spec.di if csa else 0, st)
-    t_comp = (time.perf_counter() - t0) * T / nt
-    # per-query work at uniformly spread positions, on synthetic stand-in rows of the right sizes
-    rows = ((np.arange(budget_rows) + 0.5) * T / budget_rows).astype(np.int64)
-    N = -(-T // spec.m)
-    rng = np.random.default_rng(0)
-    entries = rng.standard_normal((N, spec.C))
-    kvraw = rng.standard_normal((T, spec.C))
-    q = rng.standard_normal((budget_rows, spec.H * spec.dh))
-    nvis = np.minimum(rows // spec.m, N)
-    t0 = time.perf_counter()
-    if csa:
-        keys = rng.standard_normal((N, spec.di))
-        qi = rng.standard_normal((budget_rows, spec.Hi * spec.di))
-        w = rng.standard_normal((budget_rows, spec.Hi))
-        s = oracle.index_scores(qi, w, keys, nvis, spec.Hi, spec.di)
-        sel, _, _ = oracle.topk(s, nvis, spec.topk)
-    else:
-        sel = None
-    oracle.attend(q, spec.H, spec.dh, spec.scale, entries, sel, nvis, kvraw,
-                  oracle.prefill_window_rows(rows, spec.window), st)
-    t_q = (time.perf_counter() - t0) * T / budget_rows
-    total = t_proj + t_comp + t_q
-    sample = (f"projection of {nr} rows, compressor over {nt} tokens, indexer/top-k/attention for "
-              f"{budget_rows} queries spread over T={T}; whole-layer time extrapolated ({total:.1f} s)")
-    return T / total, sample
+    oracle.prefill_queries(spec, inp, res, rows)
+    t_q = time.perf_counter() - t0
+    total = t_fixed + t_q * T / len(rows)
+    sample = (f"projections + compressor over all T={T} tokens ({t_fixed:.1f} s), then query projections + "
+              f"indexer + top-k + attention for {len(rows)} evenly spread query rows ({t_q:.1f} s) scaled by "
+              f"T/{len(rows)}; {oracle.num_threads()} OpenMP threads on {_host_cores()} host cores; "
+              f"whole-layer time {total:.1f} s")
+    return T / total, sample, entries
 
 
-def oracle_decode_rate(layers, B, N_list, P):
-    """Oracle µs/step from one sequence of each distinct layer shape, scaled to B sequences."""
+def oracle_decode_rate(d, seq=0):
+    """Oracle µs per decode step, timed on one sequence of the workload's own inputs (its cache, weights
+    and new token) through every layer in order -- with the residual chain, each layer's output
+    projection and residual update included -- and scaled to the batch of B independent sequences.
+    Returns (µs/step, sample description)."""
     import oracle
-    rng = np.random.default_rng(0)
-    total = 0.0
-    for spec, N in zip(layers, N_list):
-        st = oracle.storage_code(spec.dtype)
-        ncols = 2 * spec.C + spec.H * spec.dh + (spec.di + spec.Hi * spec.di + spec.Hi if spec.kind == "csa" else 0)
-        W = rng.standard_normal((spec.D, ncols))
-        x = rng.standard_normal((1, spec.D))
+    import synth
+    x = None
+    elapsed = 0.0
+    for li, spec in enumerate(d.layers):
+        inp = synth.decode_inputs(d, li, seqs=[seq])
+        inp["x"] = inp["x"][seq:seq + 1] if x is None else x
         t0 = time.perf_counter()
-        y = oracle.project(x, W, st)
-        t_proj = time.perf_counter() - t0
-        entries = rng.standard_normal((N, spec.C))
-        win = rng.standard_normal((spec.window, spec.C))
-        nv = np.array([N], np.int64)
-        t0 = time.perf_counter()
-        if spec.kind == "csa":
-            keys = rng.standard_normal((N, spec.di))
-            s = oracle.index_scores(y[:, 2 * spec.C + spec.di:2 * spec.C + spec.di + spec.Hi * spec.di],
-                                    rng.standard_normal((1, spec.Hi)), keys, nv, spec.Hi, spec.di)
-            sel, _, _ = oracle.topk(s, nv, spec.topk)
-        else:
-            sel = None
-        wrows = (np.arange(spec.window, dtype=np.int64) % spec.window)[None]
-        oracle.attend(rng.standard_normal((1, spec.H * spec.dh)), spec.H, spec.dh, spec.scale, entries, sel, nv,
-                      win, wrows, st)
-        total += t_proj + (time.perf_counter() - t0) * B
-    return total * 1e6, f"one sequence per layer shape, N={N_list[0]} entries, scaled to B={B}"
+        x, _ = oracle.decode_stack([spec], [inp], d.P, residual=d.residual)
+        elapsed += time.perf_counter() - t0
+        if not d.residual:
+            x = None
+        del inp
+    us = elapsed * d.B * 1e6
+    sample = (f"sequence {seq} of {d.B} through all {len(d.layers)} layers (append, indexer, top-k, attention"
+              f"{', output projection + residual' if d.residual else ''}) on its own cache at P={d.P} "
+              f"({elapsed:.1f} s), scaled by B={d.B}; {oracle.num_threads()} OpenMP threads on "
+              f"{_host_cores()} host cores")
+    return us, sample
 
 
 # ------------------------------------------------------------------ our arm
@@ -319,7 +305,7 @@ def oracle_decode_rate(layers, B, N_list, P):
 def run_prefill(args, spec_name, ws, rank):
     import long_context_compressed_05_b200 as h
     import synth
-    from tests._helpers import dev
+    from long_context_compressed_05_b200.host import to_device as dev
     spec = synth.PREFILL[spec_name]
     if args.tokens:
         spec = spec.replace(T=args.tokens)
@@ -416,7 +402,7 @@ def run_prefill(args, spec_name, ws, rank):
 def run_decode(args, spec_name, ws, rank):
     import long_context_compressed_05_b200 as h
     import synth
-    from tests._helpers import dev
+    from long_context_compressed_05_b200.host import to_device as dev
     d = synth.DECODE[spec_name]
     if args.batch:
         import dataclasses
@@ -507,82 +493,111 @@ def run_decode(args, spec_name, ws, rank):
     return line, (d, None)
 
 
+DEFAULT_WORKLOAD = "csa_prefill_T131072"
+# measured after the headline in the default run and nested in its line under "workloads"
+EXTRA_WORKLOADS = ["hca_prefill_T65536", "csa_decode_B32_P262144", "hybrid_decode_B4_P1048576",
+                   "v4_decode_B4_P1048576"]
+NESTED_KEYS = ["value", "unit", "higher_is_better", "steps", "warmup", "ms_per_step", "config", "phase_ms",
+               "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"]
+
+
+def run_workload(args, wl, ws, rank):
+    """One workload on our arm: its JSON line, with the CPU oracle baseline (rank 0, one GPU)."""
+    kind, name = WORKLOADS[wl]
+    if kind == "prefill":
+        line, (spec, inp) = run_prefill(args, name, ws, rank)
+    else:
+        line, (d, _) = run_decode(args, name, ws, rank)
+    line["cpu_baseline"] = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
+        if kind == "prefill":
+            v, sample, _ = oracle_prefill_rate(spec, inp)
+            unit = "tokens/s"
+        else:
+            v, sample = oracle_decode_rate(d)
+            unit = "us/step"
+        line["cpu_baseline"] = {"value": v, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": sample}
+    gc.collect()
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_reference(args, wl, ws, rank):
+    """The reference arm: the CPU oracle as it stands, timed on the host cores on bounded samples of the
+    same workload (rank 0 only)."""
+    import oracle
+    import synth
+    kind, name = WORKLOADS[wl]
+    vals = []
+    n = args.warmup + args.steps
+    if kind == "prefill":
+        spec = synth.PREFILL[name]
+        inp = synth.prefill_inputs(spec)
+        entries = None
+        for i in range(n):
+            # the sequence-wide half is timed once (first step) and reused; every step times the per-query
+            # half on 64 evenly spread rows, shifted from step to step
+            v, sample, entries = oracle_prefill_rate(spec, inp, n_rows=64, offset=(i + 0.5) / n, entries=entries)
+            if i >= args.warmup:
+                vals.append(v)
+        sample += f"; per step: 64 query rows shifted by (step + 0.5)/{n} of a stratum, mean over {args.steps} steps"
+        unit, hib = "tokens/s", True
+        ms = spec.T / statistics.mean(vals) * 1e3
+        config = {"workload": f"{spec.kind}_prefill_bf16_T{spec.T}_D{spec.D}", "T": spec.T, "D": spec.D,
+                  "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh, "parallelism": "CPU oracle on rank 0"}
+    else:
+        d = synth.DECODE[name]
+        for i in range(n):
+            v, sample = oracle_decode_rate(d, seq=i % d.B)
+            if i >= args.warmup:
+                vals.append(v)
+        unit, hib = "us/step", False
+        ms = statistics.mean(vals) / 1e3
+        config = {"workload": name, "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
+                  "parallelism": "CPU oracle on rank 0"}
+    v = statistics.mean(vals)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": hib, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, the same inputs as the CUDA path; bounded sample, scaled to the workload)",
+            "config": config, "gpu_launches": 0,
+            "cpu_baseline": {"value": v, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="csa_prefill_T131072", choices=list(WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=list(WORKLOADS),
+                    help="run this workload alone (default: the CSA prefill headline, then the other workloads "
+                         "nested in its line)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="default run without the nested workloads")
     ap.add_argument("--tokens", type=int, default=0, help="override T of a prefill workload (profiling small cases)")
     ap.add_argument("--batch", type=int, default=0, help="override B of a decode workload (profiling small cases)")
     args = ap.parse_args()
-    kind, name = WORKLOADS[args.workload]
     ws, rank, local = dist_setup()
+    wl = args.workload or DEFAULT_WORKLOAD
 
     if args.impl == "reference":
-        if rank != 0:
-            return
-        import synth
-        cores = len(os.sched_getaffinity(0))
-        vals = []
-        if kind == "prefill":
-            spec = synth.PREFILL[name]
-            inp = synth.prefill_inputs(spec)
-            for i in range(args.warmup + args.steps):
-                v, sample = oracle_prefill_rate(spec, inp, budget_rows=4)
-                if i >= args.warmup:
-                    vals.append(v)
-            unit, hib = "tokens/s", True
-        else:
-            d = synth.DECODE[name]
-            Ns = [d.n_cache_entries(s) for s in d.layers]
-            for i in range(args.warmup + args.steps):
-                v, sample = oracle_decode_rate(list(d.layers), d.B, Ns, d.P)
-                if i >= args.warmup:
-                    vals.append(v)
-            unit, hib = "us/step", False
-        v = statistics.mean(vals)
-        if kind == "prefill":
-            ms = spec.T / v * 1e3
-            config = {"workload": f"{spec.kind}_prefill_bf16_T{spec.T}_D{spec.D}", "T": spec.T, "D": spec.D,
-                      "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh,
-                      "parallelism": "CPU oracle on rank 0"}
-        else:
-            ms = v / 1e3
-            config = {"workload": name, "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
-                      "parallelism": "CPU oracle on rank 0"}
-        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": ws,
-                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": hib,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                          "data": "synthetic (seeded, the same inputs as the CUDA path; bounded sample, "
-                                  "extrapolated)",
-                          "config": config, "gpu_launches": 0,
-                          "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
-                                           "sample": sample},
-                          "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl, ws, rank)))
         return
 
-    if kind == "prefill":
-        line, (spec, inp) = run_prefill(args, name, ws, rank)
-    else:
-        line, (d, _) = run_decode(args, name, ws, rank)
+    line = run_workload(args, wl, ws, rank)
+    if args.workload is None and not args.no_extra and not args.tokens and not args.batch:
+        line["workloads"] = {}
+        for x in EXTRA_WORKLOADS:
+            sub = run_workload(args, x, ws, rank)
+            line["workloads"][x] = {k: sub.get(k) for k in NESTED_KEYS}
     if rank == 0:
-        if not args.no_cpu_baseline and ws == 1:
-            cores = len(os.sched_getaffinity(0))
-            if kind == "prefill":
-                v, sample = oracle_prefill_rate(spec, inp)
-                line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                        "sample": sample}
-            else:
-                Ns = [d.n_cache_entries(s) for s in d.layers]
-                v, sample = oracle_decode_rate(list(d.layers), d.B, Ns, d.P)
-                line["cpu_baseline"] = {"value": v, "unit": "us/step", "cores": cores, "kind": "oracle",
-                                        "sample": sample}
-        else:
-            line["cpu_baseline"] = None
         print(json.dumps(line))
     if ws > 1:
         import torch.distributed as dist

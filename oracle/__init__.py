@@ -56,6 +56,8 @@ def _load():
         lib.orc_round_e2m1.argtypes = [V, I64]
         lib.orc_store_fp8_rows.argtypes = [V, I64, I, I, V]
         lib.orc_store_fp4_rows.argtypes = [V, I64, I, I, V]
+        lib.orc_num_threads.argtypes = []
+        lib.orc_num_threads.restype = ctypes.c_int
         for f in ("orc_round", "orc_compress", "orc_pool_rows", "orc_index_scores", "orc_topk", "orc_attend",
                   "orc_round_e4m3", "orc_round_e2m1", "orc_store_fp8_rows", "orc_store_fp4_rows"):
             getattr(lib, f).restype = None
@@ -222,6 +224,13 @@ def prefill(spec, inp, rows=None, chunk=8192, lowprec=False):
     64 channels) and the indexer keys as FP4 (blocks of 32), see store_fp8_rows /
     store_fp4_rows; everything downstream reads the stored values.  Returns a dict of
     float64 arrays."""
+    res = prefill_entries(spec, inp, chunk=chunk, lowprec=lowprec)
+    return prefill_queries(spec, inp, res, rows)
+
+
+def prefill_entries(spec, inp, chunk=8192, lowprec=False):
+    """The sequence-wide half of prefill(): projections of the pooled columns (kv, g, ki) of every
+    token, then the compressor (entries and indexer keys of the whole sequence)."""
     st = storage_code(spec.dtype)
     T, C, m = spec.T, spec.C, spec.m
     cols = _col_slices(spec)
@@ -242,17 +251,29 @@ def prefill(spec, inp, rows=None, chunk=8192, lowprec=False):
         entries = store_fp8_rows(entries, 64)[0]
         if csa:
             idx = store_fp4_rows(idx, 32)[0]
-    rows = np.arange(T, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
-    W_q = np.ascontiguousarray(W[:, pool_end:])
-    yq = project(to_f64(inp["x"][rows]), W_q, st)
-    off = pool_end
+    return {"y_pool": ypool, "entries": entries, "idx_keys": idx, "W_q": np.ascontiguousarray(W[:, pool_end:]),
+            "pool_end": pool_end}
+
+
+def prefill_queries(spec, inp, ent, rows=None):
+    """The per-query half of prefill() for the positions `rows` (default all), over the sequence-wide
+    results `ent` of prefill_entries(): query projections (qi, w, q), indexer scores, top-k and
+    attention.  Returns the dict prefill() documents."""
+    st = storage_code(spec.dtype)
+    m = spec.m
+    cols = _col_slices(spec)
+    csa = spec.kind == "csa"
+    rows = np.arange(spec.T, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    yq = project(to_f64(inp["x"][rows]), ent["W_q"], st)
+    off = ent["pool_end"]
     qcols = {n: slice(s.start - off, s.stop - off) for n, s in cols.items() if s.start >= off}
-    res = {"y_pool": ypool, "entries": entries, "idx_keys": idx, "rows": rows, "y_q": yq}
-    N = entries.shape[0]
+    res = {"y_pool": ent["y_pool"], "entries": ent["entries"], "idx_keys": ent["idx_keys"], "rows": rows,
+           "y_q": yq}
+    N = ent["entries"].shape[0]
     n_vis = prefill_n_vis(rows, m, N)
     res["n_vis"] = n_vis
     if csa:
-        scores = index_scores(yq[:, qcols["qi"]], yq[:, qcols["w"]], idx, n_vis, spec.Hi, spec.di)
+        scores = index_scores(yq[:, qcols["qi"]], yq[:, qcols["w"]], ent["idx_keys"], n_vis, spec.Hi, spec.di)
         sel, gap, kth = topk(scores, n_vis, spec.topk)
         res.update(scores=scores, sel=sel, gap=gap, kth=kth)
     else:
@@ -260,6 +281,11 @@ def prefill(spec, inp, rows=None, chunk=8192, lowprec=False):
     res["out"] = attend_rows(spec, res, yq[:, qcols["q"]], sel)
     res["q"] = yq[:, qcols["q"]]
     return res
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle's loops use."""
+    return int(_load().orc_num_threads())
 
 
 def attend_rows(spec, res, q, sel):

@@ -32,6 +32,7 @@
  * force); nothing here is unpinned.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -52,6 +53,9 @@ static double store(double v, int st) {
     }
     return v;
 }
+
+/* threads the OpenMP loops below use (reported next to the oracle's timings) */
+int orc_num_threads(void) { return omp_get_max_threads(); }
 
 void orc_round(double *a, int64_t n, int st) {
     #pragma omp parallel for schedule(static)
