@@ -24,9 +24,9 @@
  *
  * Conventions for every call
  *   - All tensors are row-major and live in device memory owned by the caller.
- *     The library allocates nothing (an internal cuBLAS handle per device is
- *     the one exception, made on the first bf16 projection) and keeps one
- *     device status word per device.
+ *     The library allocates nothing and keeps one device status word per
+ *     device (plus the fixed scratch array of the allocation-free entry
+ *     point below).
  *   - Storage type is p->dtype: HCSA_F32 (fp32 storage; the kernels compute in
  *     fp64) or HCSA_BF16 (bf16 storage; fp32 accumulation, tensor cores).
  *   - Pointers must be 16-byte aligned; every leading dimension `ld_*` (in
@@ -128,55 +128,75 @@ size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op);
  * CSA: C (kv) + C (g) + di (ki) + Hi*di (qi) + Hi (w) + H*dh (q);  HCA: C + C + H*dh. */
 int64_t hcsa_proj_cols(const hcsa_params *p, int32_t kind);
 
-/* Token projections (the "projection" step of the layer; a plain GEMM).
+/* Token projections: every per-token input of the layer in one GEMM -- the compressor's kv and gate
+ * logits, the indexer's "lower-dimensional projection" keys, queries and head weights, and the
+ * attention queries (page "DeepSeek-V4: interleaved compressed attention ...", TL;DR and "The HCA-CSA
+ * pair"; the weight list of the CSA workload definition).
  *   x     [rows, D]           (ld = D)
  *   W_cat [D, ncols]          the concatenation [W_kv | W_g | W_ki | W_qi | W_w | W_q] (HCA: [W_kv | W_g | W_q])
- *   y     [rows, ncols]       y = x W_cat rounded to the storage type; ncols = hcsa_proj_cols(p, kind)
- * bf16: cuBLAS GEMM, fp32 accumulate; f32: fp64 accumulate.  ws may be NULL for f32. */
+ *   y     [rows, ncols]       y = x W_cat rounded once to the storage type; ncols = hcsa_proj_cols(p, kind)
+ * bf16: tcgen05 tensor-core GEMM, fp32 accumulate.  ws (hcsa_workspace_bytes(p, HCSA_OP_PROJECT)
+ * bytes) is optional: with it, outputs with too few column tiles to fill the GPU split the contraction
+ * over CTAs; with NULL every tile is one CTA (same result up to fp32 summation order).
+ * f32: CUDA cores, fp64 accumulate, ws unused.  Requires D and ncols to keep rows 16-byte aligned. */
 hcsa_status hcsa_project(const hcsa_params *p, int32_t kind, int64_t rows, const void *x, const void *W_cat,
                          void *y, void *ws, size_t ws_bytes, void *stream);
 
 /* Output projection with the residual stream, for stacks whose layers are chained (the V4-style
- * schedule: two HCA layers, then CSA and HCA alternating).  The pages define no output projection
- * or normalisation; the reading is x_{l+1} = x_l + out_l W_o,l.
- *   out [rows, ld_out]   the layer's attention output (H*dh columns used)
- *   W_o [H*dh, D]        row-major
- *   x   [rows, ld_x]     the hidden state, updated in place: x += out W_o, fp32 accumulate, one
- *                        rounding to bf16 (cuBLAS GEMM with beta = 1)
+ * schedule of page "DeepSeek-V4 ... KV cache ... atencion comprimida", section "Pila hibrida de
+ * capas": two HCA layers, then CSA and HCA alternating).  The pages define no output projection or
+ * normalisation; the reading is x_{l+1} = x_l + out_l W_o,l.
+ *   out [rows, ld_out]   the layer's attention output (H*dh columns used); must hold rows * ld_out elements
+ *   W_o [H*dh, D]        row-major, H*dh * D elements
+ *   x   [rows, ld_x]     the hidden state, updated in place: x = round(x + out W_o), fp32 accumulate,
+ *                        one rounding to bf16 (the tcgen05 GEMM of hcsa_project with the residual added
+ *                        in its epilogue); must hold rows * ld_x elements
+ * Decode parameters (p->T == 0) allow at most p->B rows (HCSA_ERR_SHAPE otherwise).
  * bf16 storage only (HCSA_ERR_UNSUPPORTED otherwise).  ws as for hcsa_project (may be NULL). */
 hcsa_status hcsa_out_project(const hcsa_params *p, int64_t rows, const void *out, int64_t ld_out, const void *W_o,
                              void *x, int64_t ld_x, void *ws, size_t ws_bytes, void *stream);
 
-/* CSA compressor (m, width = 8 overlapping pools), prefill of one sequence of p->T tokens.
+/* CSA compressor: the learned compression pool over overlapping windows (page "DeepSeek-V4 ... KV
+ * cache ... atencion comprimida", section "CSA: compresion 4x mas recuperacion dispersa"; the pool
+ * formula of the CSA workload definition), m = 4 with width 8, prefill of one sequence of p->T tokens.
  *   kv [T, ld_kv] (C used), g [T, ld_g] (C used), ki [T, ld_ki] (di used), bias [width, C]
  *   entries [N, C], idx_keys [N, di] with N = ceil(T / m) (edge pools are truncated to [0, T)). */
 hcsa_status csa_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
                          const void *ki, int64_t ld_ki, const void *bias, void *entries, void *idx_keys,
                          void *stream);
 
-/* HCA compressor (width = m, non-overlapping pools); as csa_compress without indexer keys. */
+/* HCA compressor: 128 tokens into one entry (same page, section "HCA: compresion 128x mas atencion
+ * densa"; the HCA prefill workload definition), width = m, non-overlapping pools; as csa_compress
+ * without indexer keys. */
 hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
                          const void *bias, void *entries, void *stream);
 
-/* CSA lightning indexer + top-k, causal prefill.
+/* CSA lightning indexer + top-k, causal prefill (section "CSA: compresion 4x mas recuperacion
+ * dispersa": the indexer scores the compressed entries, the query keeps the most relevant ones; the
+ * score, visibility and tie rule of the CSA workload definition).
  *   qi [T, ld_qi] (Hi*di used, head-major), w [T, ld_w] (Hi used), idx_keys [N, di]
  *   sel [T, topk] int32: for query t the min(topk, t / m) best visible entries, ascending, -1 padded.
  * ws: hcsa_workspace_bytes(p, HCSA_OP_CSA_INDEX_TOPK) bytes (materialised scores). */
 hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
                            const void *idx_keys, int32_t *sel, void *ws, size_t ws_bytes, void *stream);
 
-/* CSA attention, causal prefill.
+/* CSA attention, causal prefill: one softmax over the selected entries and the uncompressed recent
+ * window (sections "CSA: ..." and "Ventana deslizante: el contexto reciente conserva detalle"; MQA,
+ * key / value halves and scale as in the CSA workload definition).
  *   q [T, ld_q] (H*dh used, head-major), kv [T, ld_kv] raw window rows (C used), entries [N, C], sel [T, topk]
  *   out [T, H*dh]: softmax over selected entries and raw tokens (t - window, t]. */
 hcsa_status csa_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
                        const void *entries, const int32_t *sel, void *out, void *ws, size_t ws_bytes,
                        void *stream);
 
-/* HCA attention, causal prefill: every visible entry (j < t / m) plus the raw window. */
+/* HCA attention, causal prefill: every visible entry (j < t / m) plus the raw window (sections "HCA:
+ * compresion 128x mas atencion densa" and "Ventana deslizante"). */
 hcsa_status hca_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
                        const void *entries, void *out, void *ws, size_t ws_bytes, void *stream);
 
-/* Decode: append one new token per sequence to the cache.
+/* Decode: append one new token per sequence to the cache.  Each decode step reads the past keys and
+ * values (page "DeepSeek-V4 ... KV cache ... atencion comprimida", opening section); the cache holds the
+ * compressed entries plus the uncompressed window (sections "CSA", "HCA", "Ventana deslizante").
  *   pos [B] int32 (device): position of the new token of each sequence (not modified)
  *   kv/g/ki [B, ld] the new token's projections (ki NULL for HCA), bias [width, C]
  * Writes the rings; when pos[b] = m j + m - 1 the entry j is formed from the rings
@@ -229,8 +249,8 @@ hcsa_status hcsa_get_device_status(void *stream);
  * usable.  Returns HCSA_ERR_CUDA if the launch fails. */
 hcsa_status hcsa_selftest_wait_timeout(void *stream);
 
-/* Number of kernels this library enqueued on the calling host thread since the last reset
- * (library GEMM kernels not included).  For launch accounting in benchmarks. */
+/* Number of kernels this library enqueued on the calling host thread since the last reset.
+ * For launch accounting in benchmarks. */
 int64_t hcsa_launch_count(int32_t reset);
 
 #ifdef __cplusplus

@@ -125,7 +125,10 @@ size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op) {
     if (!p) return 0;
     switch (op) {
         case HCSA_OP_PROJECT: return project_ws_bytes(p->dtype);
-        case HCSA_OP_CSA_INDEX_TOPK: return index_topk_ws_bytes(p->dtype, p->T, n_entries(p));
+        case HCSA_OP_CSA_INDEX_TOPK:
+            if (index_fused_supported(p->dtype, p->Hi, p->di, p->topk, n_entries(p)) && p->T > 0)
+                return index_fused_ws_bytes();
+            return index_topk_ws_bytes(p->dtype, p->T, n_entries(p));
         case HCSA_OP_CSA_ATTEND: return attend_ws_bytes(p->dtype, false, false, p->T, p->H, p->dh, p->topk,
                                                         p->window, n_entries(p));
         case HCSA_OP_HCA_ATTEND: return attend_ws_bytes(p->dtype, false, true, p->T, p->H, p->dh, 0, p->window,
@@ -163,6 +166,7 @@ hcsa_status hcsa_out_project(const hcsa_params *p, int64_t rows, const void *out
     if (p->dtype != HCSA_BF16) return HCSA_ERR_UNSUPPORTED;
     if (!out || !W_o || !x) return HCSA_ERR_NULL;
     if (rows < 0 || p->D < 1) return HCSA_ERR_SHAPE;
+    if (p->T == 0 && rows > p->B) return HCSA_ERR_SHAPE;   // decode: one row per sequence of the batch
     const int64_t hd = (int64_t)p->H * p->dh;
     if (!aligned(out) || !aligned(W_o) || !aligned(x)) return HCSA_ERR_ALIGN;
     if (!ld_ok(p->dtype, ld_out, hd) || !ld_ok(p->dtype, ld_x, p->D) || (p->D * esize(p->dtype)) % 16)

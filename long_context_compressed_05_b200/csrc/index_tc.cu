@@ -41,6 +41,7 @@ namespace hcsa {
 namespace {
 
 constexpr int kNS = 8;               // key-tile ring stages (prefill)
+constexpr int kNSFuse = 6;           // prefill with the fused top-k (its row state takes shared memory)
 // Decode runs two CTAs per SM (two independent TMA / MMA pipelines: a tile's dependent MMA chain and
 // the single producer thread each pace one pipeline), each with 4 stages and 2 accumulators of 128
 // TMEM columns.
@@ -68,7 +69,197 @@ struct Args {
     int64_t n_units, n_qtiles;   // prefill: query tiles; decode: (sequence, key tile) pairs
     int64_t tps;         // decode: key tiles per sequence (ceil(N / 128))
     int *status;
+    // fused top-k (prefill): per CTA and token of a unit, a candidate buffer of `cap` (order key << 32 | j)
+    uint64_t *cand;
+    int cap, trig, topk; // compaction when a buffer holds more than trig = cap - topk - 128 candidates
+    int32_t *sel;        // [rows, topk]
 };
+
+// Row state of the fused top-k, one per epilogue group (four warps, 128 threads: the tokens
+// [grp * TPH, grp * TPH + TPH) of a unit).
+struct GroupTopk {
+    uint32_t hist[256];
+    uint32_t bitmap[1024];   // rows of up to 32768 visible entries
+    uint32_t cnt[8], thr[8]; // per token: candidates held, order key a new score must exceed
+    uint32_t wsum[8];        // group_sum partials (two alternating sets)
+    uint32_t xsum[4];        // group_excl_scan partials
+    uint32_t out;
+};
+
+// Group-wide sum of one value per thread (128 threads of a group, named barrier `bar`).  `slot` alternates
+// between two sets of partial sums so that consecutive calls need one barrier each.
+__device__ __forceinline__ uint32_t group_sum(uint32_t v, GroupTopk &g, int gt, int bar, int &slot) {
+    v = __reduce_add_sync(0xffffffffu, v);
+    uint32_t *ws = slot ? g.wsum + 4 : g.wsum;
+    slot ^= 1;
+    if ((gt & 31) == 0) ws[gt >> 5] = v;
+    tc::named_bar_sync(bar, 128);
+    return ws[0] + ws[1] + ws[2] + ws[3];
+}
+
+// Exclusive prefix sum over the 128 threads of a group (gt = quadrant * 32 + lane).
+__device__ __forceinline__ uint32_t group_excl_scan(uint32_t v, GroupTopk &g, int gt, int bar) {
+    const int lane = gt & 31, w = gt >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) g.xsum[w] = incl;
+    tc::named_bar_sync(bar, 128);
+    uint32_t base = 0;
+    for (int i = 0; i < w; ++i) base += g.xsum[i];
+    return base + incl - v;
+}
+
+// The k best of the n candidates cand[0..n) of one row (order key << 32 | entry index; PER per thread:
+// candidate gt + 128 i), by the 128 threads of a group.  tau = the k-th largest order key is found bit by
+// bit from the top (a bit stays set when at least k keys reach the prefix with it); every key above tau
+// is taken, and the lowest entry indices among the keys equal to tau complete the k.
+//   out == nullptr: compaction -- the k best are moved to cand[0..k), *cnt = k; returns tau, the row's new
+//                   threshold.
+//   out != nullptr: emission -- the k best entry indices are written to out[0..k) in ascending order
+//                   (through a bitmap of the row's nw words).
+template <int PER>
+__device__ uint32_t compact_or_emit(uint64_t *cand, uint32_t n, uint32_t k, GroupTopk &g, int gt, int bar,
+                                    uint32_t *cnt, int32_t *out, int nw) {
+    static_assert(PER <= 32, "one bit per held candidate");
+    const int lane = gt & 31;
+    int slot = 0;
+    uint32_t key[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const uint32_t c = gt + 128 * i;
+        key[i] = c < n ? (uint32_t)(__ldcg(&cand[c]) >> 32) : 0u;   // 0: no candidate (real order keys are > 0)
+    }
+    uint32_t takem = 0, tau = 0;   // bit i: candidate gt + 128 i is among the k best
+    uint32_t thr_out = 0;          // compaction: later scores must exceed this order key to matter
+    if (n <= k) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) takem |= (gt + 128u * i < n ? 1u : 0u) << i;
+    } else {
+        // the bits above the highest one in which the largest and the smallest key differ are common to
+        // every candidate, so the search starts below them; it stops as soon as exactly k keys reach the
+        // prefix (then those k are the set), else it ends with tau = the k-th largest key
+        uint32_t kmax = 0, kmin = 0xffffffffu;
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+            if (key[i]) { kmax = max(kmax, key[i]); kmin = min(kmin, key[i]); }
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        if ((gt & 31) == 0) { g.wsum[gt >> 5] = kmax; g.wsum[4 + (gt >> 5)] = kmin; }
+        tc::named_bar_sync(bar, 128);
+        kmax = max(max(g.wsum[0], g.wsum[1]), max(g.wsum[2], g.wsum[3]));
+        kmin = min(min(g.wsum[4], g.wsum[5]), min(g.wsum[6], g.wsum[7]));
+        tc::named_bar_sync(bar, 128);
+        const int top = kmax == kmin ? -1 : 31 - __clz(kmax ^ kmin);
+        uint32_t prefix = top < 0 ? kmax : top >= 31 ? 0u : kmax & ~((2u << top) - 1u);
+        bool exact = false;
+#pragma unroll 1
+        for (int b = top; b >= 0; --b) {
+            const uint32_t cut = prefix | (1u << b);
+            uint32_t c = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) c += key[i] >= cut ? 1u : 0u;
+            const uint32_t tot = group_sum(c, g, gt, bar, slot);
+            if (tot >= k) prefix = cut;
+            if (tot == k) { exact = true; break; }
+        }
+        tau = prefix;
+        thr_out = tau;               // tau = the k-th largest key: a later score must exceed it
+        if (exact) {
+            // exactly k keys reach the prefix: they are the set; a later score must reach the prefix
+#pragma unroll
+            for (int i = 0; i < PER; ++i) takem |= (key[i] >= tau ? 1u : 0u) << i;
+            thr_out = tau - 1u;
+            tau = 0;
+        }
+        uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            gtm |= (key[i] > tau ? 1u : 0u) << i;
+            eqm |= (key[i] == tau ? 1u : 0u) << i;
+        }
+        const uint32_t n_gt = exact ? k : group_sum(__popc(gtm), g, gt, bar, slot);
+        const uint32_t n_eq = exact ? 0 : group_sum(__popc(eqm), g, gt, bar, slot);
+        const uint32_t rem = k - n_gt;   // keys equal to tau that complete the k, lowest entry index first
+        uint32_t tm = eqm;
+        if (n_eq > rem) {
+            // rank the ties by entry index (< 32768): the rem largest values of 32767 - j, found bit by bit
+#pragma unroll
+            for (int i = 0; i < PER; ++i)
+                key[i] = (eqm >> i & 1u) ? 32768u + 32767u - ((uint32_t)__ldcg(&cand[gt + 128 * i]) & 32767u) : 0u;
+            uint32_t pj = 32768u;
+#pragma unroll 1
+            for (int b = 14; b >= 0; --b) {
+                const uint32_t cut = pj | (1u << b);
+                uint32_t c = 0;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) c += key[i] >= cut ? 1u : 0u;
+                if (group_sum(c, g, gt, bar, slot) >= rem) pj = cut;
+            }
+            tm = 0;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) tm |= (key[i] >= pj ? 1u : 0u) << i;
+        }
+        if (!exact) takem = gtm | tm;
+    }
+    if (out)
+        for (int w = gt; w < nw; w += 128) g.bitmap[w] = 0;
+    else if (gt == 0)
+        g.out = 0;
+    tc::named_bar_sync(bar, 128);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const uint32_t c = gt + 128 * i;
+        const bool take = (takem >> i) & 1u;
+        const uint64_t v = take ? __ldcg(&cand[c]) : 0ull;
+        if (out) {
+            if (take) atomicOr(&g.bitmap[(uint32_t)v >> 5], 1u << ((uint32_t)v & 31));
+        } else {
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            if (bal) {
+                uint32_t base = 0;
+                if (lane == 0) base = atomicAdd(&g.out, (uint32_t)__popc(bal));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (take) cand[n + base + __popc(bal & ((1u << lane) - 1u))] = v;
+            }
+        }
+    }
+    tc::named_bar_sync(bar, 128);
+    if (!out) {
+        for (uint32_t c = gt; c < k; c += 128) cand[c] = __ldcg(&cand[n + c]);
+        if (gt == 0) *cnt = k;
+        tc::named_bar_sync(bar, 128);
+        return thr_out;
+    }
+    const int per = (nw + 127) / 128, w0 = gt * per;
+    uint32_t local = 0;
+    for (int w = w0; w < w0 + per && w < nw; ++w) local += __popc(g.bitmap[w]);
+    uint32_t pos = group_excl_scan(local, g, gt, bar);
+    for (int w = w0; w < w0 + per && w < nw; ++w) {
+        uint32_t bits = g.bitmap[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (pos < k) out[pos] = w * 32 + b;
+            ++pos;
+        }
+    }
+    tc::named_bar_sync(bar, 128);   // bitmap and partial sums are reused by the next row
+    return thr_out;
+}
+
+// compact_or_emit with the register array sized to the candidates actually held (PER, PER/2, ... >= 8)
+template <int PER>
+__device__ __noinline__ uint32_t select_k(uint64_t *cand, uint32_t n, uint32_t k, GroupTopk &g, int gt, int bar,
+                                          uint32_t *cnt, int32_t *out, int nw) {
+    if constexpr (PER > 8) {
+        if (n <= 128u * (PER / 2)) return select_k<PER / 2>(cand, n, k, g, gt, bar, cnt, out, nw);
+    }
+    return compact_or_emit<PER>(cand, n, k, g, gt, bar, cnt, out, nw);
+}
 
 struct Unit {
     int64_t b, r0;       // sequence, first query row
@@ -113,7 +304,7 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
         while (it.u < a.n_units) {
             x = unit_of(a, it.u);
             it.u += gridDim.x;
-            if (x.kt0 < x.kt1) return true;
+            if (x.kt0 < x.kt1 || a.cand) return true;   // the fused top-k also writes rows that see no entry
         }
         return false;
     }
@@ -131,14 +322,15 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
     return false;
 }
 
-template <int HI, bool DEC>
+template <int HI, bool DEC, bool FUSE>
 __global__ void __launch_bounds__(cta_threads(DEC), DEC ? kDecCtasPerSm : 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
                        Args a) {
     // decode: key tiles that share one 128-column TMEM accumulator (Hi columns each)
     constexpr int kTPB = 128 / HI < 4 ? 128 / HI : 4;
     constexpr int kEpiWarps = epi_warps(DEC), kEpiThreads = 32 * kEpiWarps, kGroups = kEpiWarps / 4;
-    constexpr int NS = DEC ? kNSDec : kNS;
+    constexpr int NS = DEC ? kNSDec : FUSE ? kNSFuse : kNS;
+    constexpr int kPer = HI < 32 ? HI : 32;   // fused top-k: candidates per thread (capacity 128 kPer per token)
     constexpr int BT = DEC ? kBTileDec : kBTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,6 +342,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
     uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 4);
     uint32_t *shist = tmem_slot + 4;          // decode: [4096] key-bit histogram of the current unit
+    GroupTopk *gtk = reinterpret_cast<GroupTopk *>(tmem_slot + 4);   // fused top-k: [4] group row states
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -342,6 +535,15 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 const int64_t r = x.r0 + tok_base + i;
                 vis[i] = (tok_base + i < ntok && r < a.rows) ? visible(a, r) : 0;
             }
+            // fused top-k: this group's rows start empty, accepting every score (order keys are > 0)
+            const int gt = quad * 32 + lane, gbar = 2 + grp;
+            GroupTopk &g = gtk[FUSE ? grp : 0];
+            uint32_t thr[TPH];
+#pragma unroll
+            for (int i = 0; i < TPH; ++i) thr[i] = 0;
+            if (FUSE && gt < TPH) g.cnt[gt] = 0;
+            if (FUSE) tc::named_bar_sync(gbar, 128);
+            uint64_t *cand = FUSE ? a.cand + ((size_t)blockIdx.x * a.tq + tok_base) * a.cap : nullptr;
             for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++iacc) {
                 const int ab = iacc % a.nbuf;
                 ok = ok && tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
@@ -377,9 +579,56 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
                 const int64_t j = (int64_t)kt * 128 + row;
+                if constexpr (!FUSE) {
 #pragma unroll
-                for (int i = 0; i < TPH; ++i)
-                    if (j < vis[i]) a.scores[(x.r0 + tok_base + i) * a.N + j] = s[i];
+                    for (int i = 0; i < TPH; ++i)
+                        if (j < vis[i]) a.scores[(x.r0 + tok_base + i) * a.N + j] = s[i];
+                } else {
+                    // threshold filter: only scores that can still be among the row's k best are kept
+                    // (warp-aggregated appends: one shared-memory atomic per warp and token)
+#pragma unroll
+                    for (int i = 0; i < TPH; ++i) {
+                        const uint32_t key = score_order_key(s[i]);
+                        const bool keep = ok && vis[i] > a.topk && j < vis[i] && key > thr[i];
+                        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+                        if (bal) {
+                            uint32_t base0 = 0;
+                            if (lane == 0) base0 = atomicAdd(&g.cnt[i], (uint32_t)__popc(bal));
+                            base0 = __shfl_sync(0xffffffffu, base0, 0);
+                            if (keep)
+                                cand[(size_t)i * a.cap + base0 + __popc(bal & ((1u << lane) - 1u))] =
+                                    ((uint64_t)key << 32) | (uint32_t)j;
+                        }
+                    }
+                    ok = tc::named_bar_and(gbar, 128, ok);   // the group's four warps leave together
+                    if (!ok) break;
+                    // compaction: a buffer near its capacity keeps exactly its k best (the order key of the
+                    // k-th becomes the row's new threshold; later entries have larger indices, so a later
+                    // score equal to it can never displace a kept one)
+#pragma unroll
+                    for (int i = 0; i < TPH; ++i) {   // unrolled: thr[] stays in registers
+                        const uint32_t n = g.cnt[i];
+                        if (n <= (uint32_t)a.trig) continue;
+                        uint64_t *ci = cand + (size_t)i * a.cap;
+                        thr[i] = select_k<kPer>(ci, n, (uint32_t)a.topk, g, gt, gbar, &g.cnt[i], nullptr, 0);
+                    }
+                }
+            }
+            if constexpr (FUSE) {
+                // the k best of each row, emitted in ascending entry order
+#pragma unroll 1
+                for (int i = 0; i < TPH && ok; ++i) {
+                    const int64_t r = x.r0 + tok_base + i;
+                    if (tok_base + i >= ntok || r >= a.rows) continue;
+                    int32_t *out = a.sel + r * a.topk;
+                    const int64_t nv = vis[i];
+                    if (nv <= a.topk) {
+                        for (int c = gt; c < a.topk; c += 128) out[c] = c < nv ? c : -1;
+                        continue;
+                    }
+                    select_k<kPer>(cand + (size_t)i * a.cap, g.cnt[i], (uint32_t)a.topk, g, gt, gbar, nullptr, out,
+                                   (int)((nv + 31) / 32));
+                }
             }
         }
     }
@@ -595,15 +844,7 @@ __global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel
 
 }  // namespace
 
-bool index_tc_supported(const IndexArgs &a) {
-    if (a.dtype != HCSA_BF16 || a.di != 64) return false;
-    if (!(a.Hi == 8 || a.Hi == 16 || a.Hi == 32 || a.Hi == 64)) return false;
-    if (a.pos && a.Hi < 16) return false;          // decode MMA N = Hi must be >= 16
-    if (((uintptr_t)a.qi & 15) || ((uintptr_t)a.keys & 15) || (a.ld_qi * 2) % 16) return false;
-    return a.N <= INT32_MAX && a.rows <= INT32_MAX;
-}
-
-static int num_sms() {
+int num_sms_host() {
     static int n = 0;
     if (!n) {
         int dev = 0;
@@ -614,26 +855,54 @@ static int num_sms() {
     return n;
 }
 
-template <int HI, bool DEC>
+// Fused prefill top-k: a row may hold up to 32768 visible entries (the emission bitmap) and every token of
+// a unit gets 32768 / tq = 128 Hi candidates, which must leave room for k and a tile above a compaction.
+constexpr size_t kFuseBytesPerCta = 32768 * sizeof(uint64_t);
+
+static int fuse_cap(int Hi) { return 128 * (Hi < 32 ? Hi : 32); }
+
+bool index_fused_supported(int dtype, int Hi, int di, int topk, int64_t N) {
+    if (dtype != HCSA_BF16 || di != 64 || !(Hi == 8 || Hi == 16 || Hi == 32 || Hi == 64)) return false;
+    return N <= 32768 && topk >= 1 && 2 * (int64_t)topk + 256 <= fuse_cap(Hi);
+}
+
+size_t index_fused_ws_bytes() { return (size_t)num_sms_host() * kFuseBytesPerCta; }
+
+bool index_tc_supported(const IndexArgs &a) {
+    if (a.dtype != HCSA_BF16 || a.di != 64) return false;
+    if (!(a.Hi == 8 || a.Hi == 16 || a.Hi == 32 || a.Hi == 64)) return false;
+    if (a.pos && a.Hi < 16) return false;          // decode MMA N = Hi must be >= 16
+    if (((uintptr_t)a.qi & 15) || ((uintptr_t)a.keys & 15) || (a.ld_qi * 2) % 16) return false;
+    return a.N <= INT32_MAX && a.rows <= INT32_MAX;
+}
+
+
+template <int HI, bool DEC, bool FUSE>
 static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, const CUtensorMap &tq, Args a,
                                  cudaStream_t st) {
-    constexpr int NS = DEC ? kNSDec : kNS;
+    constexpr int NS = DEC ? kNSDec : FUSE ? kNSFuse : kNS;
+    constexpr int kPer = HI < 32 ? HI : 32;   // fused top-k: candidates per thread (capacity 128 kPer per token)
     constexpr size_t smem = 1024 + NS * kATile + 2 * (DEC ? kBTileDec : kBTile) + (DEC ? 0 : 512 * sizeof(float)) +
-                            (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 0);
+                            (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 0) +
+                            (FUSE ? 4 * sizeof(GroupTopk) : 0);
     static_assert(smem <= 232448, "shared memory per CTA");
     static bool configured[64] = {};   // kernel attributes are set per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return HCSA_ERR_CUDA;
         configured[dev] = true;
     }
-    const int64_t slots = (int64_t)num_sms() * (DEC ? kDecCtasPerSm : 1);
-    const int64_t grid = a.n_units < slots ? a.n_units : slots;
-    if (grid <= 0) return HCSA_OK;
-    index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
+    const int64_t slots = (int64_t)num_sms_host() * (DEC ? kDecCtasPerSm : 1);
+    int64_t grid = a.n_units < slots ? a.n_units : slots;
+    if (FUSE) {   // one candidate region per CTA in the workspace
+        const int64_t fit = (int64_t)(ia.ws_bytes / kFuseBytesPerCta);
+        grid = grid < fit ? grid : fit;
+    }
+    if (grid <= 0) return a.n_units > 0 ? HCSA_ERR_WORKSPACE : HCSA_OK;
+    index_scores_tc_kernel<HI, DEC, FUSE><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
     count_launch();
     return check_launch();
 }
@@ -672,18 +941,36 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         a.tps = 0;
     }
     hcsa_status s;
+    const bool fuse = !decode && index_fused_supported(ia.dtype, ia.Hi, ia.di, ia.topk, ia.N);
+    if (fuse) {
+        // top-k inside the indexer's epilogue: candidates per CTA and token in the workspace, no scores
+        a.scores = nullptr;
+        a.cand = (uint64_t *)ia.ws;
+        a.cap = fuse_cap(ia.Hi);
+        a.trig = a.cap - ia.topk - 128;
+        a.topk = ia.topk;
+        a.sel = ia.sel;
+    }
     if (decode) {
         switch (ia.Hi) {
-            case 16: s = launch_scores<16, true>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, true>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, true>(ia, tk, tq_map, a, st); break;
+            case 16: s = launch_scores<16, true, false>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, true, false>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, true, false>(ia, tk, tq_map, a, st); break;
         }
+    } else if (fuse) {
+        switch (ia.Hi) {
+            case 8: s = launch_scores<8, false, true>(ia, tk, tq_map, a, st); break;
+            case 16: s = launch_scores<16, false, true>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, false, true>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, false, true>(ia, tk, tq_map, a, st); break;
+        }
+        return s;
     } else {
         switch (ia.Hi) {
-            case 8: s = launch_scores<8, false>(ia, tk, tq_map, a, st); break;
-            case 16: s = launch_scores<16, false>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, false>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, false>(ia, tk, tq_map, a, st); break;
+            case 8: s = launch_scores<8, false, false>(ia, tk, tq_map, a, st); break;
+            case 16: s = launch_scores<16, false, false>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, false, false>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, false, false>(ia, tk, tq_map, a, st); break;
         }
     }
     if (s != HCSA_OK) return s;
@@ -693,10 +980,10 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         const float *sc = (const float *)ia.ws;
         // persistent: as many CTAs as fit at once (one per SM at 16 vectors per thread, two at 4)
         if (ia.N <= 8192) {
-            const int64_t g = ia.rows < 2 * num_sms() ? ia.rows : 2 * num_sms();
+            const int64_t g = ia.rows < 2 * num_sms_host() ? ia.rows : 2 * num_sms_host();
             topk_regs_kernel<4><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.rows, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
         } else {
-            const int64_t g = ia.rows < num_sms() ? ia.rows : num_sms();
+            const int64_t g = ia.rows < num_sms_host() ? ia.rows : num_sms_host();
             topk_regs_kernel<16><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.rows, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
         }
         count_launch();

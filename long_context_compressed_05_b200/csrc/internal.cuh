@@ -110,6 +110,10 @@ hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st);
 // tensor-core indexer scores (bf16, di = 64) + register-resident top-k
 bool index_tc_supported(const IndexArgs &a);
 hcsa_status launch_index_tc(const IndexArgs &a, cudaStream_t st);
+// prefill indexer with the top-k fused into its epilogue (no materialised scores); workspace per launch
+bool index_fused_supported(int dtype, int Hi, int di, int topk, int64_t N);
+size_t index_fused_ws_bytes();
+int num_sms_host();
 
 // attention.  Prefill (pos == nullptr): query t of one sequence, window rows kv[t-window+1 .. t].
 // Decode: query b at position pos[b], entries of sequence b, window ring win_kv[b].
@@ -139,6 +143,13 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st);
 bool hca_attend_tc_supported(const AttendArgs &a);
 hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st);
 
+// tcgen05 GEMM y[M, N] = x[M, K] W[K, N] (+ res), bf16 (gemm_tc.cu); ws (optional) enables split-K
+size_t gemm_tc_ws_bytes();
+bool gemm_tc_supported(int64_t M, int N, int K, const void *x, int64_t ld_x, const void *W, int64_t ld_w,
+                       const void *y, int64_t ld_y);
+hcsa_status launch_gemm_tc(int64_t M, int N, int K, const void *x, int64_t ld_x, const void *W, int64_t ld_w,
+                           void *y, int64_t ld_y, const void *res, int64_t ld_res, void *ws, size_t ws_bytes,
+                           cudaStream_t st);
 // projection y[rows, ncols] = x[rows, D] W[D, ncols]
 size_t project_ws_bytes(int dtype);
 hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const void *x, const void *W, void *y,

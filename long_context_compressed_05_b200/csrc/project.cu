@@ -1,11 +1,10 @@
 // Token projections y = x W_cat (the layer's "low-dimensional projection"
 // inputs: kv, gate, indexer key / query / head weight and query columns).
 //
-// A plain dense GEMM.  bf16 storage runs it through cuBLAS (bf16 tensor
-// cores, fp32 accumulate, bf16 output); fp32 storage uses a tiled CUDA-core
-// kernel that accumulates in fp64 and rounds once to fp32.
-#include <cublas_v2.h>
-
+// A plain dense GEMM.  bf16 storage runs the tcgen05 kernel of gemm_tc.cu
+// (bf16 tensor cores, fp32 accumulate, one rounding to bf16); fp32 storage
+// uses a tiled CUDA-core kernel that accumulates in fp64 and rounds once to
+// fp32.
 #include "internal.cuh"
 
 namespace hcsa {
@@ -55,20 +54,7 @@ __global__ void __launch_bounds__(256) project_f64acc_kernel(int64_t rows, int D
     }
 }
 
-static cublasHandle_t g_handles[64];
-
-static cublasHandle_t handle_for_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!g_handles[dev]) {
-        cublasHandle_t h;
-        if (cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) return nullptr;
-        g_handles[dev] = h;
-    }
-    return g_handles[dev];
-}
-
-size_t project_ws_bytes(int dtype) { return dtype == HCSA_BF16 ? (size_t)32 << 20 : 0; }
+size_t project_ws_bytes(int dtype) { return dtype == HCSA_BF16 ? gemm_tc_ws_bytes() : 0; }
 
 hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const void *x, const void *W, void *y,
                            void *ws, size_t ws_bytes, cudaStream_t st) {
@@ -80,35 +66,19 @@ hcsa_status launch_project(int dtype, int64_t rows, int D, int64_t ncols, const 
         count_launch();
         return check_launch();
     }
-    if (rows > INT32_MAX || ncols > INT32_MAX) return HCSA_ERR_UNSUPPORTED;
-    cublasHandle_t h = handle_for_device();
-    if (!h) return HCSA_ERR_CUDA;
-    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
-    if (ws && ws_bytes && cublasSetWorkspace(h, ws, ws_bytes) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
-    const float alpha = 1.0f, beta = 0.0f;
-    // row-major y[rows, ncols] = x[rows, D] W[D, ncols]  <=>  column-major y^T = W^T x^T
-    cublasStatus_t s = cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, (int)ncols, (int)rows, D, &alpha, W, CUDA_R_16BF,
-                                    (int)ncols, x, CUDA_R_16BF, D, &beta, y, CUDA_R_16BF, (int)ncols,
-                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-    return s == CUBLAS_STATUS_SUCCESS ? check_launch() : HCSA_ERR_CUDA;
+    if (ncols > INT32_MAX || !gemm_tc_supported(rows, (int)ncols, D, x, D, W, ncols, y, ncols))
+        return HCSA_ERR_UNSUPPORTED;
+    return launch_gemm_tc(rows, (int)ncols, D, x, D, W, ncols, y, ncols, nullptr, 0, ws, ws_bytes, st);
 }
 
 // Output projection with the residual: x[rows, D] += out[rows, HD] W_o[HD, D] (bf16 storage, fp32
-// accumulate, one rounding: cuBLAS with beta = 1 reads x as C).
+// accumulate, one rounding of x + out W_o).
 hcsa_status launch_out_project(int64_t rows, int64_t HD, int D, const void *out, int64_t ld_out, const void *W_o,
                                void *x, int64_t ld_x, void *ws, size_t ws_bytes, cudaStream_t st) {
     if (rows == 0) return HCSA_OK;
-    if (rows > INT32_MAX || HD > INT32_MAX || ld_out > INT32_MAX || ld_x > INT32_MAX) return HCSA_ERR_UNSUPPORTED;
-    cublasHandle_t h = handle_for_device();
-    if (!h) return HCSA_ERR_CUDA;
-    if (cublasSetStream(h, st) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
-    if (ws && ws_bytes && cublasSetWorkspace(h, ws, ws_bytes) != CUBLAS_STATUS_SUCCESS) return HCSA_ERR_CUDA;
-    const float alpha = 1.0f, beta = 1.0f;
-    // row-major x[rows, D] += out[rows, HD] W_o[HD, D]  <=>  column-major x^T += W_o^T out^T
-    cublasStatus_t s = cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, D, (int)rows, (int)HD, &alpha, W_o, CUDA_R_16BF, D,
-                                    out, CUDA_R_16BF, (int)ld_out, &beta, x, CUDA_R_16BF, (int)ld_x,
-                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-    return s == CUBLAS_STATUS_SUCCESS ? check_launch() : HCSA_ERR_CUDA;
+    if (HD > INT32_MAX || !gemm_tc_supported(rows, D, (int)HD, out, ld_out, W_o, D, x, ld_x))
+        return HCSA_ERR_UNSUPPORTED;
+    return launch_gemm_tc(rows, D, (int)HD, out, ld_out, W_o, D, x, ld_x, x, ld_x, ws, ws_bytes, st);
 }
 
 }  // namespace hcsa
