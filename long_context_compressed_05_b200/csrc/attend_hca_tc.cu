@@ -7,13 +7,18 @@
 //
 // HCA entries are visible to whole runs of consecutive tokens, so the kernel is flash-style over
 // query blocks: 128 / H consecutive tokens x H heads = 128 query rows (the MMA's M, one row per TMEM
-// lane).  Key tiles of 128 rows (entries 0 .. visible, then the raw rows t0 - 127 .. t0 + TB) are
+// lane).  Key tiles of 128 rows (entries 0 .. visible, then the raw rows t0 - 127 .. t0 + 128) are
 // loaded by TMA boxes; per-row masks select what each token may see.
 //   S = Q K^T          [128 rows x 128 keys] fp32 in TMEM, two buffers
-//   online softmax     one thread per row; the running reference max is raised only when a row's
-//                      max grows by more than 2^8 in exp2 units, and only then is that row's O rescaled
-//   O += P V           P (bf16) in shared memory as the A operand, V as an MN-major B operand
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 softmax + output epilogue.
+//   online softmax     two threads per row (8 warps, each a TMEM lane quadrant and 64 of the 128 key
+//                      columns); the running reference max is raised only when a row's max grows by
+//                      more than 2^8 in exp2 units, and only then is that row's O rescaled
+//   O += P V           P (bf16) as the A operand, written over the tile's K half in shared memory (the
+//                      S MMAs are its only readers and have completed), V as an MN-major B operand;
+//                      three K/V stages, so the softmax of tile i overlaps the MMAs of its neighbours
+// Persistent CTAs walk the query blocks heaviest first; the next block's Q is loaded as soon as the
+// current block's last S MMA has read its Q.  Warp roles: warp 0 TMA producer, warp 1 MMA issuer,
+// warps 2..9 softmax + output epilogue.
 #include "tc_common.cuh"
 
 namespace hcsa {
@@ -22,13 +27,14 @@ namespace {
 
 constexpr int kDh = 128;
 constexpr int kC = 256;
-constexpr int kKT = 128;          // keys per tile
-constexpr int kRows = 128;        // query rows per block
-constexpr int kNS = 2;            // K/V stages
-constexpr int kChunk = 16384;     // 128 rows x 64 bf16
+constexpr int kKT = 128;             // keys per tile
+constexpr int kRows = 128;           // query rows per block
+constexpr int kNS = 3;               // K/V stages (the K half of a stage then holds the tile's P)
+constexpr int kChunk = 16384;        // 128 rows x 64 bf16
 constexpr int kStage = 4 * kChunk;   // K (2 chunks) + V (2 chunks)
-constexpr int kThreads = 192;
-constexpr uint32_t kColO = 256;   // S buffers at columns 0 and 128, O at 256
+constexpr int kSoftWarps = 8;
+constexpr int kThreads = 64 + 32 * kSoftWarps;
+constexpr uint32_t kColO = 256;      // S buffers at columns 0 and 128, O at 256
 constexpr float kRescaleLog2 = 8.f;
 
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, 128, false, false);
@@ -37,13 +43,19 @@ constexpr uint32_t kIdescPV = tc::idesc_bf16(128, 128, false, true);
 struct Params {
     int64_t T, N;
     int H, m, tb;            // heads, compression ratio, tokens per block (128 / H)
+    int64_t n_blocks;
     float scale_log2;
     __nv_bfloat16 *out;
     int *status;
 };
 
 struct Bars {
-    uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_free[2], p_full, o_done, q_full;
+    uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_free[2], p_full[2], o_done[2], q_full, q_empty;
+};
+
+// exchange between the two softmax threads of a row: tile max, then (at the end) row sum
+struct Xchg {
+    float v[2][kRows];       // [half][row]
 };
 
 __device__ __forceinline__ int64_t vis_of(const Params &a, int64_t t) {
@@ -57,28 +69,44 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+struct Block {
+    int64_t t0;
+    int n_ent_tiles, n_tiles;
+};
+
+__device__ __forceinline__ Block block_of(const Params &a, int64_t u) {
+    Block b;
+    b.t0 = (a.n_blocks - 1 - u) * a.tb;   // heaviest (latest) blocks first
+    const int64_t t_last = b.t0 + a.tb - 1 < a.T ? b.t0 + a.tb - 1 : a.T - 1;
+    b.n_ent_tiles = (int)((vis_of(a, t_last) + kKT - 1) / kKT);
+    b.n_tiles = b.n_ent_tiles + 2;   // + raw rows t0 - 127 .. t0 + 128
+    return b;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ent,
                      const __grid_constant__ CUtensorMap tm_raw, Params a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // small state first, then the 1024-byte aligned tiles (the alignment gap follows the small state)
+    Bars *bars = reinterpret_cast<Bars *>(smem_raw);
+    Xchg *xc = reinterpret_cast<Xchg *>(bars + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xc + 1);
+    uint8_t *base =
+        reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = base;                       // 2 chunks
-    uint8_t *sKV = sQ + 2 * kChunk;           // kNS stages
-    uint8_t *sP = sKV + kNS * kStage;         // 2 chunks
-    Bars *bars = reinterpret_cast<Bars *>(sP + 2 * kChunk);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
+    uint8_t *sKV = sQ + 2 * kChunk;           // kNS stages: K (later P) | V
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t0 = (int64_t)blockIdx.x * a.tb;
-    const int64_t t_last = t0 + a.tb - 1 < a.T ? t0 + a.tb - 1 : a.T - 1;
-    const int n_ent_tiles = (int)((vis_of(a, t_last) + kKT - 1) / kKT);
-    const int n_tiles = n_ent_tiles + 2;      // + raw rows t0 - 127 .. t0 + 128
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNS; ++i) { tc::mbar_init(&bars->kv_full[i], 1); tc::mbar_init(&bars->kv_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(&bars->s_full[i], 1); tc::mbar_init(&bars->s_free[i], 4); }
-        tc::mbar_init(&bars->p_full, 4);
-        tc::mbar_init(&bars->o_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&bars->s_full[i], 1);
+            tc::mbar_init(&bars->s_free[i], kSoftWarps);
+            tc::mbar_init(&bars->p_full[i], kSoftWarps);
+            tc::mbar_init(&bars->o_done[i], 1);
+        }
         tc::mbar_init(&bars->q_full, 1);
+        tc::mbar_init(&bars->q_empty, 1);
         tc::fence_mbar_init();
     }
     if (warp == 0) tc::tmem_alloc(tmem_slot, 512);
@@ -86,152 +114,195 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t Qs = tc::smem_u32(sQ), KV = tc::smem_u32(sKV), Ps = tc::smem_u32(sP);
+    const uint32_t Qs = tc::smem_u32(sQ), KV = tc::smem_u32(sKV);
     bool ok = true;
 
     if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
-            tc::mbar_arrive_expect_tx(&bars->q_full, 2 * kChunk);
-            for (int dc = 0; dc < 2; ++dc)
-                tc::tma_load_3d(Qs + dc * kChunk, &tm_q, dc * 64, 0, (int)t0, &bars->q_full);
-            for (int i = 0; i < n_tiles && ok; ++i) {
-                const int s = i % kNS;
-                if (i >= kNS) ok = ok && tc::mbar_wait(&bars->kv_empty[s], ((i / kNS) - 1) & 1, a.status);
-                tc::mbar_arrive_expect_tx(&bars->kv_full[s], kStage);
-                const bool ent = i < n_ent_tiles;
-                const int row0 = ent ? i * kKT : (int)(t0 - (kKT - 1) + (int64_t)(i - n_ent_tiles) * kKT);
-                for (int c = 0; c < 4; ++c)
-                    tc::tma_load_2d(KV + s * kStage + c * kChunk, ent ? &tm_ent : &tm_raw, c * 64, row0,
-                                    &bars->kv_full[s]);
+            uint32_t it = 0, nb = 0;
+            for (int64_t u = blockIdx.x; u < a.n_blocks && ok; u += gridDim.x, ++nb) {
+                const Block b = block_of(a, u);
+                if (nb >= 1) ok = ok && tc::mbar_wait(&bars->q_empty, (nb - 1) & 1, a.status);
+                if (!ok) break;
+                tc::mbar_arrive_expect_tx(&bars->q_full, 2 * kChunk);
+                for (int dc = 0; dc < 2; ++dc)
+                    tc::tma_load_3d(Qs + dc * kChunk, &tm_q, dc * 64, 0, (int)b.t0, &bars->q_full);
+                for (int i = 0; i < b.n_tiles && ok; ++i, ++it) {
+                    const int s = it % kNS;
+                    if (it >= kNS) ok = ok && tc::mbar_wait(&bars->kv_empty[s], ((it / kNS) - 1) & 1, a.status);
+                    if (!ok) break;
+                    tc::mbar_arrive_expect_tx(&bars->kv_full[s], kStage);
+                    const bool ent = i < b.n_ent_tiles;
+                    const int row0 = ent ? i * kKT : (int)(b.t0 - (kKT - 1) + (int64_t)(i - b.n_ent_tiles) * kKT);
+                    for (int c = 0; c < 4; ++c)
+                        tc::tma_load_2d(KV + s * kStage + c * kChunk, ent ? &tm_ent : &tm_raw, c * 64, row0,
+                                        &bars->kv_full[s]);
+                }
             }
         }
     } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            ok = ok && tc::mbar_wait(&bars->q_full, 0, a.status);
-            auto issue_pv = [&](int i) {
-                const int s = i % kNS;
-                ok = ok && tc::mbar_wait(&bars->p_full, i & 1, a.status);
-                tc::fence_async_smem();
+            uint32_t it = 0, is = 0, ip = 0, nb = 0;
+            // O += P V for the tile that used K/V stage s; first tile of a block overwrites O
+            auto issue_pv = [&](int s, bool first) {
+                const int pb = ip & 1;
+                ok = ok && tc::mbar_wait(&bars->p_full[pb], (ip >> 1) & 1, a.status);
+                if (!ok) return;
                 tc::tc_fence_after();
                 const uint32_t v = KV + s * kStage + 2 * kChunk;
+                const uint32_t p = KV + s * kStage;   // P over the K half of the stage
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    tc::mma_bf16(tmem + kColO, tc::sdesc_sw128(Ps + (k >> 2) * kChunk + 32 * (k & 3), 16, 1024),
-                                 tc::sdesc_sw128(v + 2048 * k, kChunk, 1024), kIdescPV, (i | k) != 0);
+                    tc::mma_bf16(tmem + kColO, tc::sdesc_sw128(p + (k >> 2) * kChunk + 32 * (k & 3), 16, 1024),
+                                 tc::sdesc_sw128(v + 2048 * k, kChunk, 1024), kIdescPV, (!first || k != 0) ? 1u : 0u);
                 tc::mma_commit(&bars->kv_empty[s]);
-                tc::mma_commit(&bars->o_done);
+                tc::mma_commit(&bars->o_done[pb]);
+                ++ip;
             };
-            for (int i = 0; i < n_tiles && ok; ++i) {
-                const int s = i % kNS, sb = i & 1;
-                ok = ok && tc::mbar_wait(&bars->kv_full[s], (i / kNS) & 1, a.status);
-                if (i >= 2) ok = ok && tc::mbar_wait(&bars->s_free[sb], ((i >> 1) - 1) & 1, a.status);
-                tc::tc_fence_after();
-                const uint32_t k0 = KV + s * kStage;
+            for (int64_t u = blockIdx.x; u < a.n_blocks && ok; u += gridDim.x, ++nb) {
+                const Block b = block_of(a, u);
+                ok = ok && tc::mbar_wait(&bars->q_full, nb & 1, a.status);
+                int prev_s = -1;
+                for (int i = 0; i < b.n_tiles && ok; ++i, ++it, ++is) {
+                    const int s = it % kNS, sb = is & 1;
+                    ok = ok && tc::mbar_wait(&bars->kv_full[s], (it / kNS) & 1, a.status);
+                    if (is >= 2) ok = ok && tc::mbar_wait(&bars->s_free[sb], ((is >> 1) - 1) & 1, a.status);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    const uint32_t k0 = KV + s * kStage;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc::mma_bf16(tmem + sb * 128, tc::sdesc_sw128(Qs + (k >> 2) * kChunk + 32 * (k & 3), 16, 1024),
-                                 tc::sdesc_sw128(k0 + (k >> 2) * kChunk + 32 * (k & 3), 16, 1024), kIdescS, k != 0);
-                tc::mma_commit(&bars->s_full[sb]);
-                if (i >= 1) issue_pv(i - 1);
+                    for (int k = 0; k < 8; ++k)
+                        tc::mma_bf16(tmem + sb * 128, tc::sdesc_sw128(Qs + (k >> 2) * kChunk + 32 * (k & 3), 16, 1024),
+                                     tc::sdesc_sw128(k0 + (k >> 2) * kChunk + 32 * (k & 3), 16, 1024), kIdescS,
+                                     k != 0 ? 1u : 0u);
+                    tc::mma_commit(&bars->s_full[sb]);
+                    if (i == b.n_tiles - 1) tc::mma_commit(&bars->q_empty);   // Q free once these S MMAs complete
+                    if (prev_s >= 0) issue_pv(prev_s, i == 1);
+                    prev_s = s;
+                }
+                if (ok && prev_s >= 0) issue_pv(prev_s, b.n_tiles == 1);
             }
-            if (ok) issue_pv(n_tiles - 1);
         }
     } else {
-        // ---------------------------------------------------------- softmax + epilogue (4 warps, one row each)
-        const int quad = warp & 3;
+        // ---------------------------------------------------------- softmax + output epilogue (8 warps)
+        const int quad = warp & 3, half = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
         const int tl = r / a.H, h = r % a.H;
-        const int64_t t = t0 + tl;
-        const bool row_ok = t < a.T;
-        const int64_t vis = row_ok ? vis_of(a, t) : 0;
         const uint32_t tl_addr = tmem + ((uint32_t)(quad * 32) << 16);
-        float m_used = -INFINITY, l = 0.f;
-        for (int i = 0; i < n_tiles && ok; ++i) {
-            const int sb = i & 1;
-            ok = ok && tc::mbar_wait(&bars->s_full[sb], (i >> 1) & 1, a.status);
-            tc::tc_fence_after();
-            float sv[kKT];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tl_addr + sb * 128 + c * 32, sv + c * 32);
-            tc::tmem_ld_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->s_free[sb]);
-            // mask: which keys of this tile the row's token may see
-            const bool ent = i < n_ent_tiles;
-            const int64_t key0 = ent ? (int64_t)i * kKT : t0 - (kKT - 1) + (int64_t)(i - n_ent_tiles) * kKT;
-            float mt = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kKT; ++c) {
-                const int64_t key = key0 + c;
-                const bool v = row_ok && (ent ? key < vis : (key >= 0 && key <= t && key > t - kKT));
-                sv[c] = v ? sv[c] * a.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, sv[c]);
-            }
-            // lazy rescale of the reference max (exp2 units)
-            const bool need = mt > m_used + kRescaleLog2;
-            const float m_new = need ? mt : m_used;
-            const float factor = need ? ex2(m_used - m_new) : 1.f;   // m_used = -inf -> 0
-            if (i >= 1) {
-                // P of the previous tile must have been consumed (and O updated) before P and O change
-                ok = ok && tc::mbar_wait(&bars->o_done, (i - 1) & 1, a.status);
+        const int pbar = 2 + quad;   // the two warps of this lane quadrant
+        uint32_t is = 0;
+        for (int64_t u = blockIdx.x; u < a.n_blocks && ok; u += gridDim.x) {
+            const Block b = block_of(a, u);
+            const int64_t t = b.t0 + tl;
+            const bool row_ok = t < a.T;
+            const int64_t vis = row_ok ? vis_of(a, t) : 0;
+            float m_used = -INFINITY, l = 0.f;
+            for (int i = 0; i < b.n_tiles; ++i, ++is) {
+                const int sb = is & 1;
+                ok = ok && tc::mbar_wait(&bars->s_full[sb], (is >> 1) & 1, a.status);
                 tc::tc_fence_after();
-                if (__any_sync(0xffffffffu, need)) {
-                    for (int c = 0; c < 4; ++c) {
+                float sv[64];
+                tc::tmem_ld32(tl_addr + sb * 128 + half * 64, sv);
+                tc::tmem_ld32(tl_addr + sb * 128 + half * 64 + 32, sv + 32);
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars->s_free[sb]);
+                // mask: which keys of this tile the row's token may see
+                const bool ent = i < b.n_ent_tiles;
+                const int64_t key0 =
+                    (ent ? (int64_t)i * kKT : b.t0 - (kKT - 1) + (int64_t)(i - b.n_ent_tiles) * kKT) + half * 64;
+                float mt = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const int64_t key = key0 + c;
+                    const bool v = row_ok && (ent ? key < vis : (key >= 0 && key <= t && key > t - kKT));
+                    sv[c] = v ? sv[c] * a.scale_log2 : -INFINITY;
+                    mt = fmaxf(mt, sv[c]);
+                }
+                xc->v[half][r] = mt;
+                ok = tc::named_bar_and(pbar, 64, ok);   // both halves of every row leave together
+                if (!ok) break;
+                mt = fmaxf(mt, xc->v[half ^ 1][r]);
+                tc::named_bar_sync(pbar, 64);           // both have read before the slot is written again
+                // lazy rescale of the reference max (exp2 units)
+                const bool need = mt > m_used + kRescaleLog2;
+                const float m_new = need ? mt : m_used;
+                const float factor = need ? ex2(m_used - m_new) : 1.f;   // m_used = -inf -> 0
+                if (i >= 1 && __any_sync(0xffffffffu, need)) {
+                    // O must hold the previous tile's P V before it is rescaled (and before P V of this tile)
+                    const uint32_t q = is - 1;
+                    ok = ok && tc::mbar_wait(&bars->o_done[q & 1], (q >> 1) & 1, a.status);
+                    tc::tc_fence_after();
+                    for (int c = 0; c < 2; ++c) {
                         float o[32];
-                        tc::tmem_ld32(tl_addr + kColO + c * 32, o);
+                        tc::tmem_ld32(tl_addr + kColO + half * 64 + c * 32, o);
                         tc::tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] *= factor;
-                        tc::tmem_st32(tl_addr + kColO + c * 32, o);
+                        tc::tmem_st32(tl_addr + kColO + half * 64 + c * 32, o);
                     }
                     tc::tmem_st_wait();
                 }
-            }
-            l *= factor;
-            m_used = m_new;
-            // P row (bf16) into the K-major A operand: 2 chunks of 64 keys
+                l *= factor;
+                m_used = m_new;
+                // P row half (bf16) into the K-major A operand: chunk `half` (64 keys) of the K half of
+                // this tile's stage (its S MMAs, the only readers of K, have completed)
+                const uint32_t pbase = KV + (is % kNS) * kStage + half * kChunk;   // stage of tile is
 #pragma unroll
-            for (int g = 0; g < 16; ++g) {
-                uint32_t w[4];
+                for (int g = 0; g < 8; ++g) {
+                    uint32_t w[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = g * 8 + 2 * e;
-                    const float p0 = sv[c] == -INFINITY ? 0.f : ex2(sv[c] - m_used);
-                    const float p1 = sv[c + 1] == -INFINITY ? 0.f : ex2(sv[c + 1] - m_used);
-                    l += p0 + p1;
-                    __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<uint32_t *>(&pr);
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = g * 8 + 2 * e;
+                        const float p0 = sv[c] == -INFINITY ? 0.f : ex2(sv[c] - m_used);
+                        const float p1 = sv[c + 1] == -INFINITY ? 0.f : ex2(sv[c + 1] - m_used);
+                        l += p0 + p1;
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+                        w[e] = *reinterpret_cast<uint32_t *>(&pr);
+                    }
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + tc::sw128_offset(r, g)),
+                                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
                 }
-                const uint32_t addr = Ps + (g >> 3) * kChunk + tc::sw128_offset(r, g & 7);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                             "r"(w[3])
-                             : "memory");
+                tc::fence_async_smem();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bars->p_full[sb]);
             }
-            tc::fence_async_smem();
+            if (!ok) break;
+            // output: O / l (both halves' sums), 64 dims per thread
+            const uint32_t q = is - 1;
+            ok = ok && tc::mbar_wait(&bars->o_done[q & 1], (q >> 1) & 1, a.status);
+            tc::tc_fence_after();
+            xc->v[half][r] = l;
+            ok = tc::named_bar_and(pbar, 64, ok);
+            if (!ok) break;
+            l += xc->v[half ^ 1][r];
+            tc::named_bar_sync(pbar, 64);
+            const float li = l > 0.f ? 1.f / l : 0.f;
+            for (int c = 0; c < 2; ++c) {
+                float o[32];
+                tc::tmem_ld32(tl_addr + kColO + half * 64 + c * 32, o);
+                tc::tmem_ld_wait();
+                if (row_ok) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(o[2 * e] * li, o[2 * e + 1] * li);
+                        w[e] = *reinterpret_cast<uint32_t *>(&pr);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + t * (int64_t)a.H * kDh + (int64_t)h * kDh + half * 64 +
+                                                           c * 32);
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) dst[qq] = make_uint4(w[4 * qq], w[4 * qq + 1], w[4 * qq + 2], w[4 * qq + 3]);
+                }
+            }
+            // the next block's first P V overwrites O only after this block's softmax warps signal its P,
+            // which comes after these reads
             tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->p_full);
-        }
-        // output: O / l
-        if (ok) ok = ok && tc::mbar_wait(&bars->o_done, (n_tiles - 1) & 1, a.status);
-        tc::tc_fence_after();
-        const float li = l > 0.f ? 1.f / l : 0.f;
-        for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tc::tmem_ld32(tl_addr + kColO + c * 32, o);
-            tc::tmem_ld_wait();
-            if (row_ok && ok) {
-                uint32_t w[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    __nv_bfloat162 pr = __floats2bfloat162_rn(o[2 * e] * li, o[2 * e + 1] * li);
-                    w[e] = *reinterpret_cast<uint32_t *>(&pr);
-                }
-                uint4 *dst = reinterpret_cast<uint4 *>(a.out + t * (int64_t)a.H * kDh + (int64_t)h * kDh + c * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            }
         }
     }
     tc::tc_fence_before();
@@ -242,7 +313,19 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
 }
 
-constexpr size_t kSmemBytes = 1024 + 2 * kChunk + kNS * kStage + 2 * kChunk + sizeof(Bars) + 16;
+constexpr size_t kSmemBytes = sizeof(Bars) + sizeof(Xchg) + 16 + 1023 + 2 * kChunk + kNS * kStage;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
 
 }  // namespace
 
@@ -279,11 +362,12 @@ hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.H = a.H;
     p.m = a.m;
     p.tb = tb;
+    p.n_blocks = (a.rows + tb - 1) / tb;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out = (__nv_bfloat16 *)a.out;
     p.status = device_status_ptr();
-    const int64_t blocks = (a.rows + tb - 1) / tb;
-    hca_attend_tc_kernel<<<(unsigned)blocks, kThreads, kSmemBytes, st>>>(tq, te, tr, p);
+    const int64_t grid = p.n_blocks < sm_count() ? p.n_blocks : sm_count();
+    hca_attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tq, te, tr, p);
     count_launch();
     return check_launch();
 }
