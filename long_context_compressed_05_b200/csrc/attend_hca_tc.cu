@@ -10,15 +10,17 @@
 // lane).  Key tiles of 128 rows (entries 0 .. visible, then the raw rows t0 - 127 .. t0 + 128) are
 // loaded by TMA boxes; per-row masks select what each token may see.
 //   S = Q K^T          [128 rows x 128 keys] fp32 in TMEM, two buffers
-//   online softmax     two threads per row (8 warps, each a TMEM lane quadrant and 64 of the 128 key
-//                      columns); the running reference max is raised only when a row's max grows by
-//                      more than 2^8 in exp2 units, and only then is that row's O rescaled
+//   online softmax     four threads per row (16 warps, each a TMEM lane quadrant and 32 of the 128 key
+//                      columns; the mask is a column range per row; the four exchange their tile max
+//                      and final sum through spare TMEM columns of the row's lane); the running max is
+//                      raised only when a row's max grows by more than 2^8 in exp2 units, and only then
+//                      is that row's O rescaled
 //   O += P V           P (bf16) as the A operand, written over the tile's K half in shared memory (the
 //                      S MMAs are its only readers and have completed), V as an MN-major B operand;
 //                      three K/V stages, so the softmax of tile i overlaps the MMAs of its neighbours
 // Persistent CTAs walk the query blocks heaviest first; the next block's Q is loaded as soon as the
 // current block's last S MMA has read its Q.  Warp roles: warp 0 TMA producer, warp 1 MMA issuer,
-// warps 2..9 softmax + output epilogue.
+// warps 2..17 softmax + output epilogue.
 #include "tc_common.cuh"
 
 namespace hcsa {
@@ -32,9 +34,12 @@ constexpr int kRows = 128;           // query rows per block
 constexpr int kNS = 3;               // K/V stages (the K half of a stage then holds the tile's P)
 constexpr int kChunk = 16384;        // 128 rows x 64 bf16
 constexpr int kStage = 4 * kChunk;   // K (2 chunks) + V (2 chunks)
-constexpr int kSoftWarps = 8;
+constexpr int kSoftWarps = 16;
+constexpr int kParts = kSoftWarps / 4;   // threads per query row
+constexpr int kPartCols = kKT / kParts;  // key columns (and output dims) per thread
 constexpr int kThreads = 64 + 32 * kSoftWarps;
 constexpr uint32_t kColO = 256;      // S buffers at columns 0 and 128, O at 256
+constexpr uint32_t kColX = 384;      // exchange between the threads of a row: one column per part
 constexpr float kRescaleLog2 = 8.f;
 
 constexpr uint32_t kIdescS = tc::idesc_bf16(128, 128, false, false);
@@ -53,10 +58,6 @@ struct Bars {
     uint64_t kv_full[kNS], kv_empty[kNS], s_full[2], s_free[2], p_full[2], o_done[2], q_full, q_empty;
 };
 
-// exchange between the two softmax threads of a row: tile max, then (at the end) row sum
-struct Xchg {
-    float v[2][kRows];       // [half][row]
-};
 
 __device__ __forceinline__ int64_t vis_of(const Params &a, int64_t t) {
     const int64_t v = t / a.m;
@@ -89,8 +90,7 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     // small state first, then the 1024-byte aligned tiles (the alignment gap follows the small state)
     Bars *bars = reinterpret_cast<Bars *>(smem_raw);
-    Xchg *xc = reinterpret_cast<Xchg *>(bars + 1);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xc + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 1);
     uint8_t *base =
         reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tmem_slot + 4) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = base;                       // 2 chunks
@@ -186,12 +186,13 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
     } else {
-        // ---------------------------------------------------------- softmax + output epilogue (8 warps)
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        // ---------------------------------------------------------- softmax + output epilogue (16 warps)
+        static_assert(kPartCols == 32, "one 32-column TMEM load per thread and tile");
+        const int quad = warp & 3, part = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
         const int tl = r / a.H, h = r % a.H;
         const uint32_t tl_addr = tmem + ((uint32_t)(quad * 32) << 16);
-        const int pbar = 2 + quad;   // the two warps of this lane quadrant
+        const int pbar = 2 + quad;   // the four warps of this lane quadrant
         uint32_t is = 0;
         for (int64_t u = blockIdx.x; u < a.n_blocks && ok; u += gridDim.x) {
             const Block b = block_of(a, u);
@@ -203,30 +204,50 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int sb = is & 1;
                 ok = ok && tc::mbar_wait(&bars->s_full[sb], (is >> 1) & 1, a.status);
                 tc::tc_fence_after();
-                float sv[64];
-                tc::tmem_ld32(tl_addr + sb * 128 + half * 64, sv);
-                tc::tmem_ld32(tl_addr + sb * 128 + half * 64 + 32, sv + 32);
+                float sv[32];
+                tc::tmem_ld32(tl_addr + sb * 128 + part * 32, sv);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bars->s_free[sb]);
-                // mask: which keys of this tile the row's token may see
+                // visible key columns of this thread: [lo, hi) of its 32
                 const bool ent = i < b.n_ent_tiles;
-                const int64_t key0 =
-                    (ent ? (int64_t)i * kKT : b.t0 - (kKT - 1) + (int64_t)(i - b.n_ent_tiles) * kKT) + half * 64;
+                const int64_t kb =
+                    (ent ? (int64_t)i * kKT : b.t0 - (kKT - 1) + (int64_t)(i - b.n_ent_tiles) * kKT) + part * 32;
+                int64_t lo64 = 0, hi64 = 0;
+                if (row_ok) {
+                    if (ent) {
+                        hi64 = vis - kb;
+                    } else {
+                        lo64 = (t - (kKT - 1) > 0 ? t - (kKT - 1) : 0) - kb;
+                        hi64 = t + 1 - kb;
+                    }
+                }
+                const int lo = (int)(lo64 < 0 ? 0 : lo64 > 32 ? 32 : lo64);
+                const int hi = (int)(hi64 < 0 ? 0 : hi64 > 32 ? 32 : hi64);
                 float mt = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int64_t key = key0 + c;
-                    const bool v = row_ok && (ent ? key < vis : (key >= 0 && key <= t && key > t - kKT));
-                    sv[c] = v ? sv[c] * a.scale_log2 : -INFINITY;
+                for (int c = 0; c < 32; ++c) {
+                    sv[c] = (c >= lo && c < hi) ? sv[c] * a.scale_log2 : -INFINITY;
                     mt = fmaxf(mt, sv[c]);
                 }
-                xc->v[half][r] = mt;
-                ok = tc::named_bar_and(pbar, 64, ok);   // both halves of every row leave together
+                // the row's tile max over its four threads, through TMEM columns kColX .. kColX + 3 of its lane
+                tc::tmem_st1(tl_addr + kColX + part, mt);
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                ok = tc::named_bar_and(pbar, 128, ok);   // the row's four threads leave together
                 if (!ok) break;
-                mt = fmaxf(mt, xc->v[half ^ 1][r]);
-                tc::named_bar_sync(pbar, 64);           // both have read before the slot is written again
+                tc::tc_fence_after();
+                {
+                    float xv[4];
+                    tc::tmem_ld4(tl_addr + kColX, xv);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < kParts; ++q) mt = fmaxf(mt, xv[q]);
+                }
+                tc::tc_fence_before();
+                tc::named_bar_sync(pbar, 128);           // all have read before the columns are written again
+                tc::tc_fence_after();
                 // lazy rescale of the reference max (exp2 units)
                 const bool need = mt > m_used + kRescaleLog2;
                 const float m_new = need ? mt : m_used;
@@ -236,34 +257,32 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const uint32_t q = is - 1;
                     ok = ok && tc::mbar_wait(&bars->o_done[q & 1], (q >> 1) & 1, a.status);
                     tc::tc_fence_after();
-                    for (int c = 0; c < 2; ++c) {
-                        float o[32];
-                        tc::tmem_ld32(tl_addr + kColO + half * 64 + c * 32, o);
-                        tc::tmem_ld_wait();
+                    float o[32];
+                    tc::tmem_ld32(tl_addr + kColO + part * 32, o);
+                    tc::tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= factor;
-                        tc::tmem_st32(tl_addr + kColO + half * 64 + c * 32, o);
-                    }
+                    for (int e = 0; e < 32; ++e) o[e] *= factor;
+                    tc::tmem_st32(tl_addr + kColO + part * 32, o);
                     tc::tmem_st_wait();
                 }
                 l *= factor;
                 m_used = m_new;
-                // P row half (bf16) into the K-major A operand: chunk `half` (64 keys) of the K half of
-                // this tile's stage (its S MMAs, the only readers of K, have completed)
-                const uint32_t pbase = KV + (is % kNS) * kStage + half * kChunk;   // stage of tile is
+                // P (bf16) into the K-major A operand over the K half of this tile's stage (its S MMAs, the only
+                // readers of K, have completed): chunk part / 2, granules (part % 2) * 4 .. + 4 of row r
+                const uint32_t pbase = KV + (is % kNS) * kStage + (part >> 1) * kChunk;
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
+                for (int g = 0; g < 4; ++g) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c = g * 8 + 2 * e;
-                        const float p0 = sv[c] == -INFINITY ? 0.f : ex2(sv[c] - m_used);
-                        const float p1 = sv[c + 1] == -INFINITY ? 0.f : ex2(sv[c + 1] - m_used);
+                        const float p0 = ex2(sv[c] - m_used), p1 = ex2(sv[c + 1] - m_used);   // ex2(-inf) = 0
                         l += p0 + p1;
                         __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
                         w[e] = *reinterpret_cast<uint32_t *>(&pr);
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase + tc::sw128_offset(r, g)),
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pbase +
+                                                                              tc::sw128_offset(r, (part & 1) * 4 + g)),
                                  "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                                  : "memory");
                 }
@@ -273,32 +292,39 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (lane == 0) tc::mbar_arrive(&bars->p_full[sb]);
             }
             if (!ok) break;
-            // output: O / l (both halves' sums), 64 dims per thread
+            // output: O / l (the four threads' sums), 32 dims per thread
             const uint32_t q = is - 1;
             ok = ok && tc::mbar_wait(&bars->o_done[q & 1], (q >> 1) & 1, a.status);
             tc::tc_fence_after();
-            xc->v[half][r] = l;
-            ok = tc::named_bar_and(pbar, 64, ok);
+            tc::tmem_st1(tl_addr + kColX + part, l);
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            ok = tc::named_bar_and(pbar, 128, ok);
             if (!ok) break;
-            l += xc->v[half ^ 1][r];
-            tc::named_bar_sync(pbar, 64);
-            const float li = l > 0.f ? 1.f / l : 0.f;
-            for (int c = 0; c < 2; ++c) {
-                float o[32];
-                tc::tmem_ld32(tl_addr + kColO + half * 64 + c * 32, o);
+            tc::tc_fence_after();
+            {
+                float xv[4];
+                tc::tmem_ld4(tl_addr + kColX, xv);
                 tc::tmem_ld_wait();
-                if (row_ok) {
-                    uint32_t w[16];
+                l = xv[0] + xv[1] + xv[2] + xv[3];
+            }
+            tc::tc_fence_before();
+            tc::named_bar_sync(pbar, 128);
+            tc::tc_fence_after();
+            const float li = l > 0.f ? 1.f / l : 0.f;
+            float o[32];
+            tc::tmem_ld32(tl_addr + kColO + part * 32, o);
+            tc::tmem_ld_wait();
+            if (row_ok) {
+                uint32_t w[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        __nv_bfloat162 pr = __floats2bfloat162_rn(o[2 * e] * li, o[2 * e + 1] * li);
-                        w[e] = *reinterpret_cast<uint32_t *>(&pr);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + t * (int64_t)a.H * kDh + (int64_t)h * kDh + half * 64 +
-                                                           c * 32);
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) dst[qq] = make_uint4(w[4 * qq], w[4 * qq + 1], w[4 * qq + 2], w[4 * qq + 3]);
+                for (int e = 0; e < 16; ++e) {
+                    __nv_bfloat162 pr = __floats2bfloat162_rn(o[2 * e] * li, o[2 * e + 1] * li);
+                    w[e] = *reinterpret_cast<uint32_t *>(&pr);
                 }
+                uint4 *dst = reinterpret_cast<uint4 *>(a.out + t * (int64_t)a.H * kDh + (int64_t)h * kDh + part * 32);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) dst[qq] = make_uint4(w[4 * qq], w[4 * qq + 1], w[4 * qq + 2], w[4 * qq + 3]);
             }
             // the next block's first P V overwrites O only after this block's softmax warps signal its P,
             // which comes after these reads
@@ -313,7 +339,7 @@ hca_attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
 }
 
-constexpr size_t kSmemBytes = sizeof(Bars) + sizeof(Xchg) + 16 + 1023 + 2 * kChunk + kNS * kStage;
+constexpr size_t kSmemBytes = sizeof(Bars) + 16 + 1023 + 2 * kChunk + kNS * kStage;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 int sm_count() {

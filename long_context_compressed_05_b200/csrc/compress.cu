@@ -8,10 +8,13 @@
 //   c_j[c] = sum_i softmax_i(g[i,c] + B[i - m j + width - m, c]) kv[i,c];
 // the indexer key of entry j is the same pool over ki with gate channel d.
 //
-// HBM-bound: one thread owns one 16-byte channel vector of one entry and
-// streams the pool's tokens with 16-byte loads (adjacent threads read
-// adjacent vectors of the same row, so every warp load is fully coalesced).
-// The softmax is a single-pass running max per channel.
+// HBM-bound.  bf16 storage: narrow pools (CSA, width 8) take one thread per
+// 16-byte channel vector of one entry, which loads the whole pool first and
+// runs a two-pass softmax; wide pools (HCA, 128 tokens) split each pool's
+// tokens over 8 warps and merge their partial softmaxes.  Adjacent threads
+// read adjacent 16-byte vectors of the same row, so every warp load is
+// coalesced.  fp32 storage (computed in fp64) keeps the generic form, a
+// single-pass running max per channel.
 #include "internal.cuh"
 
 namespace hcsa {
@@ -83,6 +86,167 @@ __global__ void __launch_bounds__(256) compress_kernel(int64_t T, int C, int m, 
     else store_vec(entries + j * C + c0, r);
 }
 
+// ---------------------------------------------------------------- bf16 prefill, faster forms
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(e[i]);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Pools of at most WMAX tokens (CSA: width 8): one thread per 16-byte channel vector (8 channels) of one
+// entry.  Every row of the pool is loaded first (up to 3 WMAX independent 16-byte loads in flight per
+// thread, adjacent threads reading adjacent vectors of a row), then a two-pass softmax in fp32.
+template <int WMAX>
+__global__ void __launch_bounds__(256) compress_narrow_bf16_kernel(
+    int T, int C, int m, int width, const __nv_bfloat16 *__restrict__ kv, int64_t ld_kv,
+    const __nv_bfloat16 *__restrict__ g, int64_t ld_g, const __nv_bfloat16 *__restrict__ ki, int64_t ld_ki, int di,
+    const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys,
+    int N) {
+    const int slots_c = C >> 3;
+    const int slots = slots_c + (ki ? di >> 3 : 0);
+    const int gid = blockIdx.x * 256 + threadIdx.x;
+    if (gid >= N * slots) return;
+    const int j = gid / slots, s = gid - j * slots;
+    const bool is_key = s >= slots_c;
+    const int c0 = (is_key ? s - slots_c : s) * 8;   // value channel, also the gate channel
+    const __nv_bfloat16 *val = is_key ? ki : kv;
+    const int64_t ld_val = is_key ? ld_ki : ld_kv;
+    const int lo = m * j - (width - m);
+    uint4 gr[WMAX], br[WMAX], vr[WMAX];
+    uint32_t in = 0;
+#pragma unroll
+    for (int r = 0; r < WMAX; ++r) {
+        const int i = lo + r;
+        if (r < width && i >= 0 && i < T) {
+            in |= 1u << r;
+            gr[r] = __ldg(reinterpret_cast<const uint4 *>(g + (int64_t)i * ld_g + c0));
+            br[r] = __ldg(reinterpret_cast<const uint4 *>(bias + (int64_t)r * C + c0));
+            vr[r] = __ldg(reinterpret_cast<const uint4 *>(val + (int64_t)i * ld_val + c0));
+        }
+    }
+    float mx[8], z[8], acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; z[e] = 0.f; acc[e] = 0.f; }
+#pragma unroll
+    for (int r = 0; r < WMAX; ++r) {
+        if (!(in >> r & 1u)) continue;
+        float gv[8], bv[8];
+        unpack8(gr[r], gv);
+        unpack8(br[r], bv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], gv[e] + bv[e]);
+    }
+#pragma unroll
+    for (int r = 0; r < WMAX; ++r) {
+        if (!(in >> r & 1u)) continue;
+        float gv[8], bv[8], vv[8];
+        unpack8(gr[r], gv);
+        unpack8(br[r], bv);
+        unpack8(vr[r], vv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float p = ex2_fast((gv[e] + bv[e] - mx[e]) * kLog2e);
+            z[e] += p;
+            acc[e] = fmaf(p, vv[e], acc[e]);
+        }
+    }
+    uint4 o;
+    __nv_bfloat16 *oe = reinterpret_cast<__nv_bfloat16 *>(&o);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) oe[e] = __float2bfloat16_rn(acc[e] / z[e]);
+    if (is_key) *reinterpret_cast<uint4 *>(idx_keys + (int64_t)j * di + c0) = o;
+    else *reinterpret_cast<uint4 *>(entries + (int64_t)j * C + c0) = o;
+}
+
+// Wide pools (HCA: 128 tokens): a block of 8 warps per (entry, 32 channel vectors); lane = channel vector,
+// warp w takes the pool's tokens w, w + 8, ... with a running (max, sum, weighted sum) per channel, and
+// warp 0 merges the eight partial softmaxes.
+constexpr int kWideWarps = 8;
+__global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
+    int T, int C, int m, int width, const __nv_bfloat16 *__restrict__ kv, int64_t ld_kv,
+    const __nv_bfloat16 *__restrict__ g, int64_t ld_g, const __nv_bfloat16 *__restrict__ ki, int64_t ld_ki, int di,
+    const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys) {
+    __shared__ float part[kWideWarps][3][8][32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int slots_c = C >> 3;
+    const int slots = slots_c + (ki ? di >> 3 : 0);
+    const int s = blockIdx.x * 32 + lane;
+    const int j = blockIdx.y;
+    const bool active = s < slots;
+    const bool is_key = s >= slots_c;
+    const int c0 = (is_key ? s - slots_c : s) * 8;
+    const __nv_bfloat16 *val = is_key ? ki : kv;
+    const int64_t ld_val = is_key ? ld_ki : ld_kv;
+    const int lo = m * j - (width - m);
+    float mx[8], z[8], acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; z[e] = 0.f; acc[e] = 0.f; }
+    if (active) {
+        for (int r0 = w; r0 < width; r0 += 4 * kWideWarps) {
+            uint4 gr[4], br[4], vr[4];
+            uint32_t in = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = r0 + q * kWideWarps, i = lo + r;
+                if (r < width && i >= 0 && i < T) {
+                    in |= 1u << q;
+                    gr[q] = __ldg(reinterpret_cast<const uint4 *>(g + (int64_t)i * ld_g + c0));
+                    br[q] = __ldg(reinterpret_cast<const uint4 *>(bias + (int64_t)r * C + c0));
+                    vr[q] = __ldg(reinterpret_cast<const uint4 *>(val + (int64_t)i * ld_val + c0));
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (!(in >> q & 1u)) continue;
+                float gv[8], bv[8], vv[8];
+                unpack8(gr[q], gv);
+                unpack8(br[q], bv);
+                unpack8(vr[q], vv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float l = gv[e] + bv[e];
+                    const float mn = fmaxf(mx[e], l);
+                    const float sc = ex2_fast((mx[e] - mn) * kLog2e);   // mx = -inf -> 0
+                    const float p = ex2_fast((l - mn) * kLog2e);
+                    z[e] = z[e] * sc + p;
+                    acc[e] = fmaf(p, vv[e], acc[e] * sc);
+                    mx[e] = mn;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { part[w][0][e][lane] = mx[e]; part[w][1][e][lane] = z[e]; part[w][2][e][lane] = acc[e]; }
+    __syncthreads();
+    if (w != 0 || !active) return;
+    uint4 o;
+    __nv_bfloat16 *oe = reinterpret_cast<__nv_bfloat16 *>(&o);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        float M = -INFINITY;
+        for (int q = 0; q < kWideWarps; ++q) M = fmaxf(M, part[q][0][e][lane]);
+        float Z = 0.f, Acc = 0.f;
+        for (int q = 0; q < kWideWarps; ++q) {
+            const float mq = part[q][0][e][lane];
+            if (mq == -INFINITY) continue;
+            const float sc = ex2_fast((mq - M) * kLog2e);
+            Z = fmaf(part[q][1][e][lane], sc, Z);
+            Acc = fmaf(part[q][2][e][lane], sc, Acc);
+        }
+        oe[e] = __float2bfloat16_rn(Acc / Z);
+    }
+    if (is_key) *reinterpret_cast<uint4 *>(idx_keys + (int64_t)j * di + c0) = o;
+    else *reinterpret_cast<uint4 *>(entries + (int64_t)j * C + c0) = o;
+}
+
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
                             void *entries, void *idx_keys, cudaStream_t st) {
@@ -92,10 +256,22 @@ hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const
     if (dtype == HCSA_BF16) {
         using S = __nv_bfloat16;
         const int64_t slots = C / 8 + (ki ? di / 8 : 0);
-        const int64_t blocks = (N * slots + threads - 1) / threads;
-        compress_kernel<S><<<(unsigned)blocks, threads, 0, st>>>(
-            T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di, (const S *)bias,
-            (S *)entries, (S *)idx_keys, N);
+        if (width <= 8 && N * slots <= INT32_MAX && T <= INT32_MAX) {
+            const int64_t blocks = (N * slots + threads - 1) / threads;
+            compress_narrow_bf16_kernel<8><<<(unsigned)blocks, threads, 0, st>>>(
+                (int)T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di,
+                (const S *)bias, (S *)entries, (S *)idx_keys, (int)N);
+        } else if (N <= 65535 && T <= INT32_MAX && (int64_t)m * N <= INT32_MAX) {
+            dim3 grid((unsigned)((slots + 31) / 32), (unsigned)N);
+            compress_wide_bf16_kernel<<<grid, 32 * kWideWarps, 0, st>>>(
+                (int)T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di,
+                (const S *)bias, (S *)entries, (S *)idx_keys);
+        } else {
+            const int64_t blocks = (N * slots + threads - 1) / threads;
+            compress_kernel<S><<<(unsigned)blocks, threads, 0, st>>>(
+                T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di, (const S *)bias,
+                (S *)entries, (S *)idx_keys, N);
+        }
     } else {
         const int64_t slots = C / 4 + (ki ? di / 4 : 0);
         const int64_t blocks = (N * slots + threads - 1) / threads;
