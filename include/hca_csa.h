@@ -86,6 +86,17 @@ typedef struct {
     float scale;     /* softmax scale tau */
     int32_t dtype;   /* hcsa_dtype */
     int32_t n_cap;   /* decode: entry capacity per sequence of the cache arrays */
+    /* Prefill row range (both 0: the whole sequence).  The calls keep global token positions and
+     * full-length arrays, but compute only query rows [row0, row1) of the T tokens: csa_compress /
+     * hca_compress form the entries whose pools end in the range (j in [row0 / m, ceil(row1 / m))), the
+     * indexer + top-k and the attention compute those query rows.  Such a call reads no projection row
+     * outside [row0 - max(window - 1, width - m), row1) and no entry (or indexer key) at or past
+     * (row1 - 1) / m, the last one the range's last query sees; so a sequence split over ranks needs,
+     * in its arrays, only its rows with that halo and the entries it gathered from the other ranks
+     * between the compressor and the indexer.  row0 must be a multiple of 128; row1 a multiple of 128
+     * or T; otherwise the calls return HCSA_ERR_SHAPE. */
+    int32_t row0;
+    int32_t row1;
 } hcsa_params;
 
 /* Decode cache of one layer (device pointers, caller-owned).

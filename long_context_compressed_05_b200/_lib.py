@@ -41,7 +41,8 @@ class HcsaError(RuntimeError):
 class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "T", "D", "m", "width", "C", "di", "Hi", "topk", "window",
                                               "H", "dh")] + [("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-                                                             ("n_cap", ctypes.c_int32)]
+                                                             ("n_cap", ctypes.c_int32), ("row0", ctypes.c_int32),
+                                                             ("row1", ctypes.c_int32)]
 
 
 class Cache(ctypes.Structure):
@@ -111,9 +112,10 @@ def _stream(stream):
 
 
 def make_params(*, T=0, D=0, m=4, width=8, C=0, di=0, Hi=0, topk=0, window=128, H=1, dh=0, scale=1.0,
-                dtype="bf16", B=1, n_cap=0) -> Params:
+                dtype="bf16", B=1, n_cap=0, row0=0, row1=0) -> Params:
     return Params(B=B, T=T, D=D, m=m, width=width, C=C, di=di, Hi=Hi, topk=topk, window=window, H=H, dh=dh,
-                  scale=scale, dtype=HCSA_BF16 if dtype == "bf16" else HCSA_F32, n_cap=n_cap)
+                  scale=scale, dtype=HCSA_BF16 if dtype == "bf16" else HCSA_F32, n_cap=n_cap, row0=row0,
+                  row1=row1)
 
 
 def make_cache(entries, win_kv, ring_g, idx_keys=None, ring_ki=None) -> Cache:

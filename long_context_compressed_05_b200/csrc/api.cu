@@ -77,6 +77,27 @@ hcsa_status check_decode(const hcsa_params *p, const hcsa_cache *c, const int32_
 
 int64_t n_entries(const hcsa_params *p) { return ((int64_t)p->T + p->m - 1) / p->m; }
 
+// Prefill row range [r0, r1) of the T query rows (both fields 0: all rows).
+hcsa_status row_range(const hcsa_params *p, int64_t *r0, int64_t *r1) {
+    if (p->row0 == 0 && p->row1 == 0) {
+        *r0 = 0;
+        *r1 = p->T;
+        return HCSA_OK;
+    }
+    if (p->row0 < 0 || p->row1 < p->row0 || p->row1 > p->T || p->row0 % 128 != 0 ||
+        (p->row1 % 128 != 0 && p->row1 != p->T))
+        return HCSA_ERR_SHAPE;
+    *r0 = p->row0;
+    *r1 = p->row1;
+    return HCSA_OK;
+}
+
+// Entries whose pools end in rows [r0, r1): j in [r0 / m, ceil(r1 / m)) (r1 < T is a multiple of m).
+void entry_range(const hcsa_params *p, int64_t r0, int64_t r1, int64_t *j0, int64_t *j1) {
+    *j0 = r0 / p->m;
+    *j1 = r1 == p->T ? n_entries(p) : r1 / p->m;
+}
+
 }  // namespace
 
 namespace hcsa {
@@ -125,10 +146,7 @@ size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op) {
     if (!p) return 0;
     switch (op) {
         case HCSA_OP_PROJECT: return project_ws_bytes(p->dtype);
-        case HCSA_OP_CSA_INDEX_TOPK:
-            if (index_fused_supported(p->dtype, p->Hi, p->di, p->topk, n_entries(p)) && p->T > 0)
-                return index_fused_ws_bytes();
-            return index_topk_ws_bytes(p->dtype, p->T, n_entries(p));
+        case HCSA_OP_CSA_INDEX_TOPK: return index_topk_ws_bytes(p->dtype, p->T, n_entries(p));
         case HCSA_OP_CSA_ATTEND: return attend_ws_bytes(p->dtype, false, false, p->T, p->H, p->dh, p->topk,
                                                         p->window, n_entries(p));
         case HCSA_OP_HCA_ATTEND: return attend_ws_bytes(p->dtype, false, true, p->T, p->H, p->dh, 0, p->window,
@@ -185,8 +203,11 @@ hcsa_status csa_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, co
         return HCSA_ERR_ALIGN;
     if (!ld_ok(p->dtype, ld_kv, p->C) || !ld_ok(p->dtype, ld_g, p->C) || !ld_ok(p->dtype, ld_ki, p->di))
         return HCSA_ERR_ALIGN;
+    int64_t r0, r1, j0, j1;
+    HCSA_TRY(row_range(p, &r0, &r1));
+    entry_range(p, r0, r1, &j0, &j1);
     return launch_compress(p->dtype, p->T, p->C, p->m, p->width, kv, ld_kv, g, ld_g, ki, ld_ki, p->di, bias,
-                           entries, idx_keys, (cudaStream_t)stream);
+                           entries, idx_keys, j0, j1, (cudaStream_t)stream);
 }
 
 hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
@@ -196,8 +217,11 @@ hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, co
     if (p->T < 0) return HCSA_ERR_SHAPE;
     if (!aligned(kv) || !aligned(g) || !aligned(bias) || !aligned(entries)) return HCSA_ERR_ALIGN;
     if (!ld_ok(p->dtype, ld_kv, p->C) || !ld_ok(p->dtype, ld_g, p->C)) return HCSA_ERR_ALIGN;
+    int64_t r0, r1, j0, j1;
+    HCSA_TRY(row_range(p, &r0, &r1));
+    entry_range(p, r0, r1, &j0, &j1);
     return launch_compress(p->dtype, p->T, p->C, p->m, p->width, kv, ld_kv, g, ld_g, nullptr, 0, 0, bias, entries,
-                           nullptr, (cudaStream_t)stream);
+                           nullptr, j0, j1, (cudaStream_t)stream);
 }
 
 hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
@@ -209,8 +233,10 @@ hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, 
     if (ld_qi < (int64_t)p->Hi * p->di || ld_w < p->Hi) return HCSA_ERR_SHAPE;
     if (!ws && p->T > 0) return HCSA_ERR_WORKSPACE;
     if (ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
+    int64_t r0, r1;
+    HCSA_TRY(row_range(p, &r0, &r1));
     IndexArgs a{p->dtype, p->T, p->Hi, p->di, p->topk, p->m, n_entries(p), qi, ld_qi, w, ld_w, idx_keys,
-                nullptr, sel, ws, ws_bytes, nullptr};
+                nullptr, sel, ws, ws_bytes, nullptr, r0, r1};
     return launch_index_topk(a, (cudaStream_t)stream);
 }
 
@@ -221,9 +247,12 @@ static hcsa_status attend_prefill(const hcsa_params *p, bool dense, const void *
     if (p->T < 0) return HCSA_ERR_SHAPE;
     if (!aligned(q) || !aligned(kv) || !aligned(entries) || !aligned(out)) return HCSA_ERR_ALIGN;
     if (ld_q < (int64_t)p->H * p->dh || ld_kv < p->C) return HCSA_ERR_SHAPE;
+    int64_t r0, r1;
+    HCSA_TRY(row_range(p, &r0, &r1));
     AttendArgs a{};
     a.dtype = p->dtype; a.rows = p->T; a.H = p->H; a.dh = p->dh; a.C = p->C; a.window = p->window; a.m = p->m;
     a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = n_entries(p);
+    a.row0 = r0; a.row1 = r1;
     a.q = q; a.ld_q = ld_q; a.kv = kv; a.ld_kv = ld_kv; a.entries = entries; a.sel = sel; a.pos = nullptr;
     a.out = out; a.ws = ws; a.ws_bytes = ws_bytes;
     return launch_attend(a, (cudaStream_t)stream);
@@ -262,7 +291,7 @@ hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache,
     HCSA_TRY(hcsa::check_decode_index_topk_args(p, cache, pos, qi, ld_qi, w, ld_w, sel));
     if (!ws || ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
     IndexArgs a{p->dtype, p->B, p->Hi, p->di, p->topk, p->m, p->n_cap, qi, ld_qi, w, ld_w, cache->idx_keys,
-                pos, sel, ws, ws_bytes, nullptr};
+                pos, sel, ws, ws_bytes, nullptr, 0, p->B};
     return launch_index_topk(a, (cudaStream_t)stream);
 }
 
@@ -279,6 +308,7 @@ static hcsa_status attend_decode(const hcsa_params *p, bool dense, const hcsa_ca
     a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = p->n_cap;
     a.q = q; a.ld_q = ld_q; a.kv = cache->win_kv; a.ld_kv = p->C; a.entries = cache->entries; a.sel = sel;
     a.pos = pos; a.out = out; a.ws = ws; a.ws_bytes = ws_bytes;
+    a.row0 = 0; a.row1 = p->B;
     return launch_attend(a, (cudaStream_t)stream);
 }
 

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kHeadsPerCta * 32) attend_kernel(AttendArgs a,
     using A = typename Traits<S>::A;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int h = blockIdx.y * kHeadsPerCta + warp;
-    const int64_t r = blockIdx.x;
+    const int64_t r = a.row0 + blockIdx.x;
     const int split = blockIdx.z;
     if (h >= a.H) return;
     const int64_t p = a.pos ? a.pos[r] : r;
@@ -225,7 +225,8 @@ hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st) {
     if (ns > 1 && a.ws_bytes < attend_ws_bytes(a.dtype, true, a.dense, a.rows, a.H, a.dh, a.topk, a.window, a.N))
         return HCSA_ERR_WORKSPACE;
     if (ns > 65535) return HCSA_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)a.rows, (a.H + kHeadsPerCta - 1) / kHeadsPerCta, ns);
+    if (a.row1 <= a.row0) return HCSA_OK;
+    dim3 grid((unsigned)(a.row1 - a.row0), (a.H + kHeadsPerCta - 1) / kHeadsPerCta, ns);
     int *status = device_status_ptr();
     if (a.dtype == HCSA_BF16) attend_kernel<__nv_bfloat16><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns, status);
     else attend_kernel<float><<<grid, kHeadsPerCta * 32, 0, st>>>(a, ns, status);

@@ -48,7 +48,7 @@ constexpr uint32_t kIdescPV = tc::idesc_bf16(128, 128, false, true);
 struct Params {
     int64_t T, N;
     int H, m, tb;            // heads, compression ratio, tokens per block (128 / H)
-    int64_t n_blocks;
+    int64_t n_blocks, b_end;   // blocks of the row range: b_end - n_blocks .. b_end - 1
     float scale_log2;
     __nv_bfloat16 *out;
     int *status;
@@ -77,7 +77,7 @@ struct Block {
 
 __device__ __forceinline__ Block block_of(const Params &a, int64_t u) {
     Block b;
-    b.t0 = (a.n_blocks - 1 - u) * a.tb;   // heaviest (latest) blocks first
+    b.t0 = (a.b_end - 1 - u) * a.tb;   // heaviest (latest) blocks of the row range first
     const int64_t t_last = b.t0 + a.tb - 1 < a.T ? b.t0 + a.tb - 1 : a.T - 1;
     b.n_ent_tiles = (int)((vis_of(a, t_last) + kKT - 1) / kKT);
     b.n_tiles = b.n_ent_tiles + 2;   // + raw rows t0 - 127 .. t0 + 128
@@ -378,9 +378,15 @@ hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st) {
     if (!make_tmap_bf16_3d(&tq, a.q, kDh, (uint64_t)a.H, (uint64_t)a.rows, kDh * 2, (uint64_t)a.ld_q * 2, 64,
                            (uint32_t)a.H, (uint32_t)tb, true))
         return HCSA_ERR_CUDA;
-    if (!make_tmap_bf16_2d(&te, a.entries, kC, (uint64_t)(a.N > 0 ? a.N : 1), kC * 2, 64, kKT, true))
-        return HCSA_ERR_CUDA;
-    if (!make_tmap_bf16_2d(&tr, a.kv, kC, (uint64_t)a.rows, (uint64_t)a.ld_kv * 2, 64, kKT, true))
+    // entries end at the last one the range's last query sees: the last entry tile rounds up past it, and
+    // those rows read as zeros, so a row-range caller need not have gathered them
+    const int64_t last_vis = a.row1 > 0 ? (a.row1 - 1) / a.m : 0;
+    const uint64_t ent_rows = (uint64_t)std::max<int64_t>(1, std::min<int64_t>(a.N, last_vis));
+    if (!make_tmap_bf16_2d(&te, a.entries, kC, ent_rows, kC * 2, 64, kKT, true)) return HCSA_ERR_CUDA;
+    // raw rows end at the row range's end: the second window tile of a range's last block reaches one row
+    // past it, which a row-range caller need not have projected (rows past the end read as zeros and are
+    // masked like any other key a query may not see)
+    if (!make_tmap_bf16_2d(&tr, a.kv, kC, (uint64_t)a.row1, (uint64_t)a.ld_kv * 2, 64, kKT, true))
         return HCSA_ERR_CUDA;
     Params p{};
     p.T = a.rows;
@@ -388,10 +394,12 @@ hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.H = a.H;
     p.m = a.m;
     p.tb = tb;
-    p.n_blocks = (a.rows + tb - 1) / tb;
+    p.b_end = (a.row1 + tb - 1) / tb;
+    p.n_blocks = p.b_end - a.row0 / tb;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out = (__nv_bfloat16 *)a.out;
     p.status = device_status_ptr();
+    if (p.n_blocks <= 0) return HCSA_OK;
     const int64_t grid = p.n_blocks < sm_count() ? p.n_blocks : sm_count();
     hca_attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tq, te, tr, p);
     count_launch();

@@ -70,6 +70,7 @@ struct Params {
     __nv_bfloat16 *out;  // direct output [nq, H*dh] (nseg == 1)
     float *part;         // partials: acc [nq][nseg][H][dh], then (max, sum) [nq][nseg][H][2]
     int64_t n_units;
+    int64_t q0;          // first query of the row range
     int *status;
 };
 
@@ -80,7 +81,7 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_of(const Params &a, int64_t u) {
     Unit x;
-    x.q = u / a.nseg;
+    x.q = a.q0 + u / a.nseg;
     x.seg = (int)(u % a.nseg);
     x.p = a.decode ? (int64_t)a.pos[x.q] : x.q;
     x.nvis = x.p < 0 ? 0 : (x.p / a.m < a.N ? x.p / a.m : a.N);
@@ -219,7 +220,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (kk < x.E) {
                         const int64_t j = a.dense ? (int64_t)kk : (int64_t)jsel[i];
                         if (j >= 0 && j < x.nvis) ptr = a.ent + ((a.decode ? x.q * a.N : 0) + j) * (int64_t)kC;
-                        else if (j != -1) report(a.status, kStatusBounds);   // not padding, not visible: skipped
+                        else if (!a.dense && j != -1) report(a.status, kStatusBounds);   // a selected index that is
+                                                                                        // neither padding nor visible
                     } else {
                         const int64_t pp = x.p - (kKT - 1) + (kk - x.E);
                         if (pp >= 0) ptr = a.raw + (a.decode ? x.q * kKT + pp % kKT : pp) * a.ld_raw;
@@ -593,7 +595,11 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     }
     const bool decode = a.pos != nullptr;
     CUtensorMap tq, te, tr;
-    const uint64_t ent_rows = decode ? (uint64_t)a.rows * a.N : (uint64_t)a.N;
+    // prefill: entries end at the last one the range's last query sees (the dense tiles round up past it;
+    // those rows read as zeros, so a row-range caller need not have gathered them)
+    const int64_t last_vis = a.row1 > 0 ? (a.row1 - 1) / a.m : 0;
+    const uint64_t ent_rows = decode ? (uint64_t)a.rows * a.N
+                                     : (uint64_t)std::max<int64_t>(1, std::min<int64_t>(a.N, last_vis));
     if (!make_tmap_bf16_3d(&tq, a.q, kDh, kH, (uint64_t)a.rows, kDh * 2, (uint64_t)a.ld_q * 2, 64, kH, 1, true))
         return HCSA_ERR_CUDA;
     if (!make_tmap_bf16_2d(&te, a.entries, kC, ent_rows, kC * 2, 64, kKT, true)) return HCSA_ERR_CUDA;
@@ -620,8 +626,10 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out = (__nv_bfloat16 *)a.out;
     p.part = p.nseg > 1 ? (float *)a.ws : nullptr;
-    p.n_units = a.rows * p.nseg;
+    p.q0 = a.row0;
+    p.n_units = (a.row1 - a.row0) * p.nseg;
     p.status = device_status_ptr();
+    if (p.n_units <= 0) return HCSA_OK;
     const int64_t grid = p.n_units < num_sms() ? p.n_units : num_sms();
     attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tq, te, tr, p);
     count_launch();

@@ -53,15 +53,16 @@ __global__ void __launch_bounds__(256) compress_kernel(int64_t T, int C, int m, 
                                                        int64_t ld_kv, const S *__restrict__ g, int64_t ld_g,
                                                        const S *__restrict__ ki, int64_t ld_ki, int di,
                                                        const S *__restrict__ bias, S *__restrict__ entries,
-                                                       S *__restrict__ idx_keys, int64_t N) {
+                                                       S *__restrict__ idx_keys, int64_t j0, int64_t N) {
     using A = typename Traits<S>::A;
     constexpr int V = Traits<S>::VEC;
     const int slots_c = C / V;
     const int slots = slots_c + (ki ? di / V : 0);
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= N * slots) return;
-    const int64_t j = gid / slots;
-    const int s = (int)(gid - j * slots);
+    if (gid >= N * slots) return;   // entries j0 .. j0 + N - 1
+    const int64_t jl = gid / slots;
+    const int s = (int)(gid - jl * slots);
+    const int64_t j = j0 + jl;
     const bool is_key = s >= slots_c;
     const int c0 = (is_key ? s - slots_c : s) * V;   // value channel; also the gate channel
     const S *val = is_key ? ki : kv;
@@ -109,12 +110,13 @@ __global__ void __launch_bounds__(256) compress_narrow_bf16_kernel(
     int T, int C, int m, int width, const __nv_bfloat16 *__restrict__ kv, int64_t ld_kv,
     const __nv_bfloat16 *__restrict__ g, int64_t ld_g, const __nv_bfloat16 *__restrict__ ki, int64_t ld_ki, int di,
     const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys,
-    int N) {
+    int j0, int N) {
     const int slots_c = C >> 3;
     const int slots = slots_c + (ki ? di >> 3 : 0);
     const int gid = blockIdx.x * 256 + threadIdx.x;
-    if (gid >= N * slots) return;
-    const int j = gid / slots, s = gid - j * slots;
+    if (gid >= N * slots) return;   // entries j0 .. j0 + N - 1
+    const int jl = gid / slots, s = gid - jl * slots;
+    const int j = j0 + jl;
     const bool is_key = s >= slots_c;
     const int c0 = (is_key ? s - slots_c : s) * 8;   // value channel, also the gate channel
     const __nv_bfloat16 *val = is_key ? ki : kv;
@@ -173,13 +175,14 @@ constexpr int kWideWarps = 8;
 __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
     int T, int C, int m, int width, const __nv_bfloat16 *__restrict__ kv, int64_t ld_kv,
     const __nv_bfloat16 *__restrict__ g, int64_t ld_g, const __nv_bfloat16 *__restrict__ ki, int64_t ld_ki, int di,
-    const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys) {
+    const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys,
+    int j0) {
     __shared__ float part[kWideWarps][3][8][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int slots_c = C >> 3;
     const int slots = slots_c + (ki ? di >> 3 : 0);
     const int s = blockIdx.x * 32 + lane;
-    const int j = blockIdx.y;
+    const int j = j0 + blockIdx.y;
     const bool active = s < slots;
     const bool is_key = s >= slots_c;
     const int c0 = (is_key ? s - slots_c : s) * 8;
@@ -249,35 +252,35 @@ __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
 
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
-                            void *entries, void *idx_keys, cudaStream_t st) {
-    const int64_t N = (T + m - 1) / m;
-    if (N == 0) return HCSA_OK;
+                            void *entries, void *idx_keys, int64_t j0, int64_t j1, cudaStream_t st) {
+    const int64_t N = j1 - j0;   // entries j0 .. j1 - 1 of the sequence
+    if (N <= 0) return HCSA_OK;
     const int threads = 256;
     if (dtype == HCSA_BF16) {
         using S = __nv_bfloat16;
         const int64_t slots = C / 8 + (ki ? di / 8 : 0);
-        if (width <= 8 && N * slots <= INT32_MAX && T <= INT32_MAX) {
+        if (width <= 8 && j1 * slots <= INT32_MAX && T <= INT32_MAX) {
             const int64_t blocks = (N * slots + threads - 1) / threads;
             compress_narrow_bf16_kernel<8><<<(unsigned)blocks, threads, 0, st>>>(
                 (int)T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di,
-                (const S *)bias, (S *)entries, (S *)idx_keys, (int)N);
-        } else if (N <= 65535 && T <= INT32_MAX && (int64_t)m * N <= INT32_MAX) {
+                (const S *)bias, (S *)entries, (S *)idx_keys, (int)j0, (int)N);
+        } else if (N <= 65535 && T <= INT32_MAX && (int64_t)m * j1 <= INT32_MAX) {
             dim3 grid((unsigned)((slots + 31) / 32), (unsigned)N);
             compress_wide_bf16_kernel<<<grid, 32 * kWideWarps, 0, st>>>(
                 (int)T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di,
-                (const S *)bias, (S *)entries, (S *)idx_keys);
+                (const S *)bias, (S *)entries, (S *)idx_keys, (int)j0);
         } else {
             const int64_t blocks = (N * slots + threads - 1) / threads;
             compress_kernel<S><<<(unsigned)blocks, threads, 0, st>>>(
                 T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di, (const S *)bias,
-                (S *)entries, (S *)idx_keys, N);
+                (S *)entries, (S *)idx_keys, j0, N);
         }
     } else {
         const int64_t slots = C / 4 + (ki ? di / 4 : 0);
         const int64_t blocks = (N * slots + threads - 1) / threads;
         compress_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
             T, C, m, width, (const float *)kv, ld_kv, (const float *)g, ld_g, (const float *)ki, ld_ki, di,
-            (const float *)bias, (float *)entries, (float *)idx_keys, N);
+            (const float *)bias, (float *)entries, (float *)idx_keys, j0, N);
     }
     count_launch();
     return check_launch();

@@ -41,7 +41,6 @@ namespace hcsa {
 namespace {
 
 constexpr int kNS = 8;               // key-tile ring stages (prefill)
-constexpr int kNSFuse = 6;           // prefill with the fused top-k (its row state takes shared memory)
 // Decode runs two CTAs per SM (two independent TMA / MMA pipelines: a tile's dependent MMA chain and
 // the single producer thread each pace one pipeline), each with 4 stages and 2 accumulators of 128
 // TMEM columns.
@@ -69,197 +68,8 @@ struct Args {
     int64_t n_units, n_qtiles;   // prefill: query tiles; decode: (sequence, key tile) pairs
     int64_t tps;         // decode: key tiles per sequence (ceil(N / 128))
     int *status;
-    // fused top-k (prefill): per CTA and token of a unit, a candidate buffer of `cap` (order key << 32 | j)
-    uint64_t *cand;
-    int cap, trig, topk; // compaction when a buffer holds more than trig = cap - topk - 128 candidates
-    int32_t *sel;        // [rows, topk]
+    uint32_t *bound;     // prefill, or nullptr: per row a lower bound of the order key of its k-th best score
 };
-
-// Row state of the fused top-k, one per epilogue group (four warps, 128 threads: the tokens
-// [grp * TPH, grp * TPH + TPH) of a unit).
-struct GroupTopk {
-    uint32_t hist[256];
-    uint32_t bitmap[1024];   // rows of up to 32768 visible entries
-    uint32_t cnt[8], thr[8]; // per token: candidates held, order key a new score must exceed
-    uint32_t wsum[8];        // group_sum partials (two alternating sets)
-    uint32_t xsum[4];        // group_excl_scan partials
-    uint32_t out;
-};
-
-// Group-wide sum of one value per thread (128 threads of a group, named barrier `bar`).  `slot` alternates
-// between two sets of partial sums so that consecutive calls need one barrier each.
-__device__ __forceinline__ uint32_t group_sum(uint32_t v, GroupTopk &g, int gt, int bar, int &slot) {
-    v = __reduce_add_sync(0xffffffffu, v);
-    uint32_t *ws = slot ? g.wsum + 4 : g.wsum;
-    slot ^= 1;
-    if ((gt & 31) == 0) ws[gt >> 5] = v;
-    tc::named_bar_sync(bar, 128);
-    return ws[0] + ws[1] + ws[2] + ws[3];
-}
-
-// Exclusive prefix sum over the 128 threads of a group (gt = quadrant * 32 + lane).
-__device__ __forceinline__ uint32_t group_excl_scan(uint32_t v, GroupTopk &g, int gt, int bar) {
-    const int lane = gt & 31, w = gt >> 5;
-    uint32_t incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-    }
-    if (lane == 31) g.xsum[w] = incl;
-    tc::named_bar_sync(bar, 128);
-    uint32_t base = 0;
-    for (int i = 0; i < w; ++i) base += g.xsum[i];
-    return base + incl - v;
-}
-
-// The k best of the n candidates cand[0..n) of one row (order key << 32 | entry index; PER per thread:
-// candidate gt + 128 i), by the 128 threads of a group.  tau = the k-th largest order key is found bit by
-// bit from the top (a bit stays set when at least k keys reach the prefix with it); every key above tau
-// is taken, and the lowest entry indices among the keys equal to tau complete the k.
-//   out == nullptr: compaction -- the k best are moved to cand[0..k), *cnt = k; returns tau, the row's new
-//                   threshold.
-//   out != nullptr: emission -- the k best entry indices are written to out[0..k) in ascending order
-//                   (through a bitmap of the row's nw words).
-template <int PER>
-__device__ uint32_t compact_or_emit(uint64_t *cand, uint32_t n, uint32_t k, GroupTopk &g, int gt, int bar,
-                                    uint32_t *cnt, int32_t *out, int nw) {
-    static_assert(PER <= 32, "one bit per held candidate");
-    const int lane = gt & 31;
-    int slot = 0;
-    uint32_t key[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const uint32_t c = gt + 128 * i;
-        key[i] = c < n ? (uint32_t)(__ldcg(&cand[c]) >> 32) : 0u;   // 0: no candidate (real order keys are > 0)
-    }
-    uint32_t takem = 0, tau = 0;   // bit i: candidate gt + 128 i is among the k best
-    uint32_t thr_out = 0;          // compaction: later scores must exceed this order key to matter
-    if (n <= k) {
-#pragma unroll
-        for (int i = 0; i < PER; ++i) takem |= (gt + 128u * i < n ? 1u : 0u) << i;
-    } else {
-        // the bits above the highest one in which the largest and the smallest key differ are common to
-        // every candidate, so the search starts below them; it stops as soon as exactly k keys reach the
-        // prefix (then those k are the set), else it ends with tau = the k-th largest key
-        uint32_t kmax = 0, kmin = 0xffffffffu;
-#pragma unroll
-        for (int i = 0; i < PER; ++i)
-            if (key[i]) { kmax = max(kmax, key[i]); kmin = min(kmin, key[i]); }
-        kmax = __reduce_max_sync(0xffffffffu, kmax);
-        kmin = __reduce_min_sync(0xffffffffu, kmin);
-        if ((gt & 31) == 0) { g.wsum[gt >> 5] = kmax; g.wsum[4 + (gt >> 5)] = kmin; }
-        tc::named_bar_sync(bar, 128);
-        kmax = max(max(g.wsum[0], g.wsum[1]), max(g.wsum[2], g.wsum[3]));
-        kmin = min(min(g.wsum[4], g.wsum[5]), min(g.wsum[6], g.wsum[7]));
-        tc::named_bar_sync(bar, 128);
-        const int top = kmax == kmin ? -1 : 31 - __clz(kmax ^ kmin);
-        uint32_t prefix = top < 0 ? kmax : top >= 31 ? 0u : kmax & ~((2u << top) - 1u);
-        bool exact = false;
-#pragma unroll 1
-        for (int b = top; b >= 0; --b) {
-            const uint32_t cut = prefix | (1u << b);
-            uint32_t c = 0;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) c += key[i] >= cut ? 1u : 0u;
-            const uint32_t tot = group_sum(c, g, gt, bar, slot);
-            if (tot >= k) prefix = cut;
-            if (tot == k) { exact = true; break; }
-        }
-        tau = prefix;
-        thr_out = tau;               // tau = the k-th largest key: a later score must exceed it
-        if (exact) {
-            // exactly k keys reach the prefix: they are the set; a later score must reach the prefix
-#pragma unroll
-            for (int i = 0; i < PER; ++i) takem |= (key[i] >= tau ? 1u : 0u) << i;
-            thr_out = tau - 1u;
-            tau = 0;
-        }
-        uint32_t gtm = 0, eqm = 0;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            gtm |= (key[i] > tau ? 1u : 0u) << i;
-            eqm |= (key[i] == tau ? 1u : 0u) << i;
-        }
-        const uint32_t n_gt = exact ? k : group_sum(__popc(gtm), g, gt, bar, slot);
-        const uint32_t n_eq = exact ? 0 : group_sum(__popc(eqm), g, gt, bar, slot);
-        const uint32_t rem = k - n_gt;   // keys equal to tau that complete the k, lowest entry index first
-        uint32_t tm = eqm;
-        if (n_eq > rem) {
-            // rank the ties by entry index (< 32768): the rem largest values of 32767 - j, found bit by bit
-#pragma unroll
-            for (int i = 0; i < PER; ++i)
-                key[i] = (eqm >> i & 1u) ? 32768u + 32767u - ((uint32_t)__ldcg(&cand[gt + 128 * i]) & 32767u) : 0u;
-            uint32_t pj = 32768u;
-#pragma unroll 1
-            for (int b = 14; b >= 0; --b) {
-                const uint32_t cut = pj | (1u << b);
-                uint32_t c = 0;
-#pragma unroll
-                for (int i = 0; i < PER; ++i) c += key[i] >= cut ? 1u : 0u;
-                if (group_sum(c, g, gt, bar, slot) >= rem) pj = cut;
-            }
-            tm = 0;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) tm |= (key[i] >= pj ? 1u : 0u) << i;
-        }
-        if (!exact) takem = gtm | tm;
-    }
-    if (out)
-        for (int w = gt; w < nw; w += 128) g.bitmap[w] = 0;
-    else if (gt == 0)
-        g.out = 0;
-    tc::named_bar_sync(bar, 128);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const uint32_t c = gt + 128 * i;
-        const bool take = (takem >> i) & 1u;
-        const uint64_t v = take ? __ldcg(&cand[c]) : 0ull;
-        if (out) {
-            if (take) atomicOr(&g.bitmap[(uint32_t)v >> 5], 1u << ((uint32_t)v & 31));
-        } else {
-            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            if (bal) {
-                uint32_t base = 0;
-                if (lane == 0) base = atomicAdd(&g.out, (uint32_t)__popc(bal));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (take) cand[n + base + __popc(bal & ((1u << lane) - 1u))] = v;
-            }
-        }
-    }
-    tc::named_bar_sync(bar, 128);
-    if (!out) {
-        for (uint32_t c = gt; c < k; c += 128) cand[c] = __ldcg(&cand[n + c]);
-        if (gt == 0) *cnt = k;
-        tc::named_bar_sync(bar, 128);
-        return thr_out;
-    }
-    const int per = (nw + 127) / 128, w0 = gt * per;
-    uint32_t local = 0;
-    for (int w = w0; w < w0 + per && w < nw; ++w) local += __popc(g.bitmap[w]);
-    uint32_t pos = group_excl_scan(local, g, gt, bar);
-    for (int w = w0; w < w0 + per && w < nw; ++w) {
-        uint32_t bits = g.bitmap[w];
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1;
-            if (pos < k) out[pos] = w * 32 + b;
-            ++pos;
-        }
-    }
-    tc::named_bar_sync(bar, 128);   // bitmap and partial sums are reused by the next row
-    return thr_out;
-}
-
-// compact_or_emit with the register array sized to the candidates actually held (PER, PER/2, ... >= 8)
-template <int PER>
-__device__ __noinline__ uint32_t select_k(uint64_t *cand, uint32_t n, uint32_t k, GroupTopk &g, int gt, int bar,
-                                          uint32_t *cnt, int32_t *out, int nw) {
-    if constexpr (PER > 8) {
-        if (n <= 128u * (PER / 2)) return select_k<PER / 2>(cand, n, k, g, gt, bar, cnt, out, nw);
-    }
-    return compact_or_emit<PER>(cand, n, k, g, gt, bar, cnt, out, nw);
-}
 
 struct Unit {
     int64_t b, r0;       // sequence, first query row
@@ -304,7 +114,7 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
         while (it.u < a.n_units) {
             x = unit_of(a, it.u);
             it.u += gridDim.x;
-            if (x.kt0 < x.kt1 || a.cand) return true;   // the fused top-k also writes rows that see no entry
+            if (x.kt0 < x.kt1) return true;
         }
         return false;
     }
@@ -322,15 +132,14 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
     return false;
 }
 
-template <int HI, bool DEC, bool FUSE>
+template <int HI, bool DEC>
 __global__ void __launch_bounds__(cta_threads(DEC), DEC ? kDecCtasPerSm : 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
                        Args a) {
     // decode: key tiles that share one 128-column TMEM accumulator (Hi columns each)
     constexpr int kTPB = 128 / HI < 4 ? 128 / HI : 4;
     constexpr int kEpiWarps = epi_warps(DEC), kEpiThreads = 32 * kEpiWarps, kGroups = kEpiWarps / 4;
-    constexpr int NS = DEC ? kNSDec : FUSE ? kNSFuse : kNS;
-    constexpr int kPer = HI < 32 ? HI : 32;   // fused top-k: candidates per thread (capacity 128 kPer per token)
+    constexpr int NS = DEC ? kNSDec : kNS;
     constexpr int BT = DEC ? kBTileDec : kBTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -342,7 +151,6 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
     uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 4);
     uint32_t *shist = tmem_slot + 4;          // decode: [4096] key-bit histogram of the current unit
-    GroupTopk *gtk = reinterpret_cast<GroupTopk *>(tmem_slot + 4);   // fused top-k: [4] group row states
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -535,15 +343,12 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 const int64_t r = x.r0 + tok_base + i;
                 vis[i] = (tok_base + i < ntok && r < a.rows) ? visible(a, r) : 0;
             }
-            // fused top-k: this group's rows start empty, accepting every score (order keys are > 0)
-            const int gt = quad * 32 + lane, gbar = 2 + grp;
-            GroupTopk &g = gtk[FUSE ? grp : 0];
-            uint32_t thr[TPH];
+            // per token, the four largest order keys this thread sees (one key per tile: its TMEM lane)
+            uint32_t t4[TPH][4];
 #pragma unroll
-            for (int i = 0; i < TPH; ++i) thr[i] = 0;
-            if (FUSE && gt < TPH) g.cnt[gt] = 0;
-            if (FUSE) tc::named_bar_sync(gbar, 128);
-            uint64_t *cand = FUSE ? a.cand + ((size_t)blockIdx.x * a.tq + tok_base) * a.cap : nullptr;
+            for (int i = 0; i < TPH; ++i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) t4[i][q] = 0u;
             for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++iacc) {
                 const int ab = iacc % a.nbuf;
                 ok = ok && tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
@@ -579,55 +384,37 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
                 const int64_t j = (int64_t)kt * 128 + row;
-                if constexpr (!FUSE) {
 #pragma unroll
-                    for (int i = 0; i < TPH; ++i)
-                        if (j < vis[i]) a.scores[(x.r0 + tok_base + i) * a.N + j] = s[i];
-                } else {
-                    // threshold filter: only scores that can still be among the row's k best are kept
-                    // (warp-aggregated appends: one shared-memory atomic per warp and token)
+                for (int i = 0; i < TPH; ++i)
+                    if (j < vis[i]) {
+                        a.scores[(x.r0 + tok_base + i) * a.N + j] = s[i];
+                        uint32_t key = score_order_key(s[i]);
+                        if (key > t4[i][3]) {   // insert into the descending top four
 #pragma unroll
-                    for (int i = 0; i < TPH; ++i) {
-                        const uint32_t key = score_order_key(s[i]);
-                        const bool keep = ok && vis[i] > a.topk && j < vis[i] && key > thr[i];
-                        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-                        if (bal) {
-                            uint32_t base0 = 0;
-                            if (lane == 0) base0 = atomicAdd(&g.cnt[i], (uint32_t)__popc(bal));
-                            base0 = __shfl_sync(0xffffffffu, base0, 0);
-                            if (keep)
-                                cand[(size_t)i * a.cap + base0 + __popc(bal & ((1u << lane) - 1u))] =
-                                    ((uint64_t)key << 32) | (uint32_t)j;
+                            for (int q = 0; q < 4; ++q) {
+                                const uint32_t hi = max(t4[i][q], key), lo = min(t4[i][q], key);
+                                t4[i][q] = hi;
+                                key = lo;
+                            }
                         }
                     }
-                    ok = tc::named_bar_and(gbar, 128, ok);   // the group's four warps leave together
-                    if (!ok) break;
-                    // compaction: a buffer near its capacity keeps exactly its k best (the order key of the
-                    // k-th becomes the row's new threshold; later entries have larger indices, so a later
-                    // score equal to it can never displace a kept one)
-#pragma unroll
-                    for (int i = 0; i < TPH; ++i) {   // unrolled: thr[] stays in registers
-                        const uint32_t n = g.cnt[i];
-                        if (n <= (uint32_t)a.trig) continue;
-                        uint64_t *ci = cand + (size_t)i * a.cap;
-                        thr[i] = select_k<kPer>(ci, n, (uint32_t)a.topk, g, gt, gbar, &g.cnt[i], nullptr, 0);
-                    }
-                }
             }
-            if constexpr (FUSE) {
-                // the k best of each row, emitted in ascending entry order
-#pragma unroll 1
-                for (int i = 0; i < TPH && ok; ++i) {
-                    const int64_t r = x.r0 + tok_base + i;
-                    if (tok_base + i >= ntok || r >= a.rows) continue;
-                    int32_t *out = a.sel + r * a.topk;
-                    const int64_t nv = vis[i];
-                    if (nv <= a.topk) {
-                        for (int c = gt; c < a.topk; c += 128) out[c] = c < nv ? c : -1;
-                        continue;
+            if (a.bound) {
+                // The 128 threads of this group saw every score of its tokens, four best each: at least 512
+                // scores reach the smallest of their fourth-best keys, a lower bound of the k-th best (k <= 512).
+                uint32_t *gmin = reinterpret_cast<uint32_t *>(tmem_slot + 4) + grp * 32;   // [token][quadrant]
+#pragma unroll
+                for (int i = 0; i < TPH; ++i) {
+                    const uint32_t wm = __reduce_min_sync(0xffffffffu, t4[i][3]);
+                    if (lane == 0) gmin[i * 4 + quad] = wm;
+                }
+                tc::named_bar_sync(2 + grp, 128);
+                if (quad == 0 && lane < TPH) {
+                    const int64_t r = x.r0 + tok_base + lane;
+                    if (tok_base + lane < ntok && r < a.rows) {
+                        const uint32_t *gm = gmin + lane * 4;
+                        a.bound[r] = min(min(gm[0], gm[1]), min(gm[2], gm[3]));
                     }
-                    select_k<kPer>(cand + (size_t)i * a.cap, g.cnt[i], (uint32_t)a.topk, g, gt, gbar, nullptr, out,
-                                   (int)((nv + 31) / 32));
                 }
             }
         }
@@ -643,18 +430,27 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
 // ------------------------------------------------------------------ register-resident top-k
 constexpr int kTkThreads = 512;
 constexpr int kRankCap = 1024;   // threshold buckets up to this size are ranked directly
+constexpr int kCandCap = 4096;   // bound path: candidates of a row held in shared memory
 
 
 template <int VPT>   // float4 vectors per thread: row capacity = 2048 * VPT
-__global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel(const float *__restrict__ scores, int64_t rows,
+__global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel(const float *__restrict__ scores, int64_t row0,
+                                                               int64_t rows,
                                                                int64_t N, int m, const int32_t *__restrict__ pos,
-                                                               int topk, int32_t *__restrict__ sel) {
+                                                               int topk, int32_t *__restrict__ sel,
+                                                               const int32_t *__restrict__ flags) {
     using Scan = cub::BlockScan<int, kTkThreads>;
     __shared__ typename Scan::TempStorage scan_tmp;
-    __shared__ int hist[4096];
+    // histogram path: hist[4096] and cand[kRankCap]; bound path: the same bytes hold ckey[kCandCap] and
+    // cj[kCandCap] (a row takes one path or the other)
+    __shared__ __align__(16) uint8_t pool[4096 * sizeof(int) + kRankCap * sizeof(uint64_t)];
+    int *hist = reinterpret_cast<int *>(pool);
+    uint64_t *cand = reinterpret_cast<uint64_t *>(pool + 4096 * sizeof(int));  // (key << 32 | ~index)
+    uint32_t *ckey = reinterpret_cast<uint32_t *>(pool);
+    uint16_t *cj = reinterpret_cast<uint16_t *>(pool + kCandCap * sizeof(uint32_t));
     __shared__ uint32_t bitmap[1024];   // rows of up to 32768 entries
     __shared__ uint32_t eq_idx[64];
-    __shared__ uint64_t cand[kRankCap];  // (key << 32 | ~index) of the keys in the threshold bucket
+    __shared__ uint32_t s_red[64];      // per-warp partials (two alternating sets of 16, then min / max)
     __shared__ uint32_t s_prefix;
     __shared__ int s_rem, s_eq_total, s_bcount, s_cnt;
     const int tid = threadIdx.x;
@@ -666,8 +462,9 @@ __global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel
     // Persistent CTAs walk the rows round-robin (every CTA sees short and long rows).  While a row is
     // ranked, the CTA's next row is prefetched into L2: loading a row is otherwise a bare HBM round trip
     // with nothing else to do.
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    if (tid == 0 && vec_ok && r + gridDim.x < rows) {
+    for (int64_t r = row0 + blockIdx.x; r < rows; r += gridDim.x) {
+    if (flags && flags[r] == 0) continue;   // only the rows the warp kernel left to this one
+    if (tid == 0 && vec_ok && !flags && r + gridDim.x < rows) {
         const int64_t nn = visible_of(r + gridDim.x);
         const uint8_t *src = reinterpret_cast<const uint8_t *>(scores + (r + gridDim.x) * N);
         const uint32_t bytes = (uint32_t)(((nn + 3) & ~int64_t(3)) * sizeof(float));
@@ -694,133 +491,248 @@ __global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel
             for (int e = 0; e < 4; ++e) key[4 * i + e] = (j0 + e < n) ? score_order_key(row[j0 + e]) : 0u;
         }
     }
-    // Histogram passes over bits [20,32), then [10,20) and [0,10) inside the threshold bucket.  Usually
-    // the first pass leaves a small bucket: its keys are then ranked directly instead (the two later
-    // passes cost more in barriers than in work).
-    uint32_t prefix = 0, mask = 0;
-    int rem = topk;
-    bool ranked = false;
-    const int shifts[3] = {20, 10, 0};
-    const int widths[3] = {12, 10, 10};
+    const int nw = (int)((n + 31) / 32);
+    const int lane = tid & 31, warp = tid >> 5;
+    bool marked = false;
+    // Bound path.  Every thread's largest key is at least tau0, the smallest of those maxima, so at least
+    // kTkThreads >= k keys reach tau0 and the k best lie among the keys >= tau0 (a few per thread for random
+    // scores).  They are gathered in shared memory and selected exactly: the k-th largest key bit by bit
+    // from the top (a bit stays set while at least k candidates reach the prefix; the search stops when
+    // exactly k do), then the lowest entry indices among the keys equal to it.
+    if (topk <= kTkThreads && n >= 4 * kTkThreads) {   // k <= threads, and every thread holds a visible key
+        uint32_t mymax = 0;
 #pragma unroll
-    for (int pass = 0; pass < 3; ++pass) {
-        const int sh = shifts[pass], nb = 1 << widths[pass];
-        for (int i = tid; i < nb; i += kTkThreads) hist[i] = 0;
+        for (int i = 0; i < VPT * 4; ++i) mymax = max(mymax, key[i]);
+        const uint32_t wmin = __reduce_min_sync(0xffffffffu, mymax), wmax = __reduce_max_sync(0xffffffffu, mymax);
+        if (lane == 0) { s_red[32 + warp] = wmin; s_red[48 + warp] = wmax; }
         __syncthreads();
+        uint32_t tau0 = s_red[32], kmax = s_red[48];
 #pragma unroll
-        for (int i = 0; i < VPT * 4; ++i)
-            if ((key[i] & mask) == prefix && key[i] != 0u) atomicAdd(&hist[(key[i] >> sh) & (nb - 1)], 1);
-        __syncthreads();
-        // suffix scan: thread tid owns bins [(nb/512) * (511 - tid), ...) so thread 0 holds the highest bins
-        const int per = nb / kTkThreads;
-        const int b0 = per * (kTkThreads - 1 - tid);
-        int local = 0;
-        for (int i = 0; i < per; ++i) local += hist[b0 + i];
-        int above, total;
-        Scan(scan_tmp).ExclusiveSum(local, above, total);
-        if (above < rem && above + local >= rem) {
-            int cum = above;
-            for (int i = per - 1; i >= 0; --i) {
-                const int c = hist[b0 + i];
-                if (cum + c >= rem) {
-                    s_prefix = prefix | ((uint32_t)(b0 + i) << sh);
-                    s_rem = rem - cum;
-                    s_bcount = c;
-                    break;
+        for (int w = 1; w < kTkThreads / 32; ++w) { tau0 = min(tau0, s_red[32 + w]); kmax = max(kmax, s_red[48 + w]); }
+        int c = 0;
+#pragma unroll
+        for (int i = 0; i < VPT * 4; ++i) c += key[i] >= tau0 ? 1 : 0;
+        int off, total;
+        Scan(scan_tmp).ExclusiveSum(c, off, total);
+        if (total <= kCandCap) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (key[4 * i + e] >= tau0) {
+                        ckey[off] = key[4 * i + e];
+                        cj[off] = (uint16_t)(4 * (tid + kTkThreads * i) + e);
+                        ++off;
+                    }
+            __syncthreads();
+            constexpr int CPT = kCandCap / kTkThreads;   // candidates per thread
+            uint32_t ck[CPT];
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int q = tid + kTkThreads * i;
+                ck[i] = q < total ? ckey[q] : 0u;
+            }
+            int sset = 0;
+            auto block_sum = [&](uint32_t v) -> uint32_t {
+                v = __reduce_add_sync(0xffffffffu, v);
+                if (lane == 0) s_red[sset * 16 + warp] = v;
+                __syncthreads();
+                uint32_t t = 0;
+#pragma unroll
+                for (int w = 0; w < kTkThreads / 32; ++w) t += s_red[sset * 16 + w];
+                sset ^= 1;
+                return t;
+            };
+            const uint32_t k = (uint32_t)topk;
+            const int top = kmax == tau0 ? -1 : 31 - __clz(kmax ^ tau0);
+            uint32_t prefix = top < 0 ? kmax : top >= 31 ? 0u : kmax & ~((2u << top) - 1u);
+            bool exact = false;
+            for (int bb = top; bb >= 0; --bb) {
+                const uint32_t cut = prefix | (1u << bb);
+                uint32_t cc = 0;
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) cc += ck[i] >= cut ? 1u : 0u;
+                const uint32_t tot = block_sum(cc);
+                if (tot >= k) prefix = cut;
+                if (tot == k) { exact = true; break; }
+            }
+            const uint32_t tau = prefix;
+            uint32_t takem = 0;   // bit i: candidate tid + kTkThreads i is taken
+            if (exact) {
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) takem |= (ck[i] >= tau ? 1u : 0u) << i;
+            } else {
+                uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    gtm |= (ck[i] > tau ? 1u : 0u) << i;
+                    eqm |= (ck[i] == tau ? 1u : 0u) << i;
                 }
-                cum += c;
+                const uint32_t n_gt = block_sum(__popc(gtm));
+                const uint32_t n_eq = block_sum(__popc(eqm));
+                const uint32_t rem = k - n_gt;
+                uint32_t tm = eqm;
+                if (n_eq > rem) {
+                    // the rem lowest entry indices among the ties: the rem largest 32767 - j, bit by bit
+                    uint32_t rk[CPT];
+#pragma unroll
+                    for (int i = 0; i < CPT; ++i)
+                        rk[i] = (eqm >> i & 1u) ? 32768u + 32767u - (uint32_t)cj[tid + kTkThreads * i] : 0u;
+                    uint32_t pj = 32768u;
+                    for (int bb = 14; bb >= 0; --bb) {
+                        const uint32_t cut = pj | (1u << bb);
+                        uint32_t cc = 0;
+#pragma unroll
+                        for (int i = 0; i < CPT; ++i) cc += rk[i] >= cut ? 1u : 0u;
+                        if (block_sum(cc) >= rem) pj = cut;
+                    }
+                    tm = 0;
+#pragma unroll
+                    for (int i = 0; i < CPT; ++i) tm |= (rk[i] >= pj ? 1u : 0u) << i;
+                }
+                takem = gtm | tm;
+            }
+            for (int i = tid; i < nw; i += kTkThreads) bitmap[i] = 0;
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < CPT; ++i)
+                if (takem >> i & 1u) {
+                    const uint32_t j = cj[tid + kTkThreads * i];
+                    atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                }
+            marked = true;
+        } else {
+            __syncthreads();   // the scan storage is used again below
+        }
+    }
+    if (!marked) {
+        // Histogram passes over bits [20,32), then [10,20) and [0,10) inside the threshold bucket.  Usually
+        // the first pass leaves a small bucket: its keys are then ranked directly instead (the two later
+        // passes cost more in barriers than in work).
+        uint32_t prefix = 0, mask = 0;
+        int rem = topk;
+        bool ranked = false;
+        const int shifts[3] = {20, 10, 0};
+        const int widths[3] = {12, 10, 10};
+    #pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {
+            const int sh = shifts[pass], nb = 1 << widths[pass];
+            for (int i = tid; i < nb; i += kTkThreads) hist[i] = 0;
+            __syncthreads();
+    #pragma unroll
+            for (int i = 0; i < VPT * 4; ++i)
+                if ((key[i] & mask) == prefix && key[i] != 0u) atomicAdd(&hist[(key[i] >> sh) & (nb - 1)], 1);
+            __syncthreads();
+            // suffix scan: thread tid owns bins [(nb/512) * (511 - tid), ...) so thread 0 holds the highest bins
+            const int per = nb / kTkThreads;
+            const int b0 = per * (kTkThreads - 1 - tid);
+            int local = 0;
+            for (int i = 0; i < per; ++i) local += hist[b0 + i];
+            int above, total;
+            Scan(scan_tmp).ExclusiveSum(local, above, total);
+            if (above < rem && above + local >= rem) {
+                int cum = above;
+                for (int i = per - 1; i >= 0; --i) {
+                    const int c = hist[b0 + i];
+                    if (cum + c >= rem) {
+                        s_prefix = prefix | ((uint32_t)(b0 + i) << sh);
+                        s_rem = rem - cum;
+                        s_bcount = c;
+                        break;
+                    }
+                    cum += c;
+                }
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            rem = s_rem;
+            mask |= (uint32_t)(nb - 1) << sh;
+            const bool small = s_bcount <= kRankCap;
+            __syncthreads();
+            if (pass == 0 && small) {
+                ranked = true;
+                break;
             }
         }
-        __syncthreads();
-        prefix = s_prefix;
-        rem = s_rem;
-        mask |= (uint32_t)(nb - 1) << sh;
-        const bool small = s_bcount <= kRankCap;
-        __syncthreads();
-        if (pass == 0 && small) {
-            ranked = true;
-            break;
+        for (int i = tid; i < nw; i += kTkThreads) bitmap[i] = 0;
+        if (tid == 0) {
+            s_eq_total = 0;
+            s_cnt = 0;
         }
-    }
-    const int nw = (int)((n + 31) / 32);
-    for (int i = tid; i < nw; i += kTkThreads) bitmap[i] = 0;
-    if (tid == 0) {
-        s_eq_total = 0;
-        s_cnt = 0;
-    }
-    __syncthreads();
-    if (ranked) {
-        // prefix = threshold bucket << 20: keys in higher buckets are taken; the `rem` best keys of the
-        // bucket (larger key first, then lower index) are found by ranking the bucket's keys
-        const uint32_t bucket = prefix >> 20;
-#pragma unroll
+        __syncthreads();
+        if (ranked) {
+            // prefix = threshold bucket << 20: keys in higher buckets are taken; the `rem` best keys of the
+            // bucket (larger key first, then lower index) are found by ranking the bucket's keys
+            const uint32_t bucket = prefix >> 20;
+    #pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t kv = key[4 * i + e];
+                    const int64_t j = 4 * ((int64_t)tid + (int64_t)kTkThreads * i) + e;
+                    if ((kv >> 20) > bucket) {
+                        atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                    } else if ((kv >> 20) == bucket && kv != 0u) {
+                        const int q = atomicAdd(&s_cnt, 1);
+                        if (q < kRankCap) cand[q] = ((uint64_t)kv << 32) | (0xFFFFFFFFu - (uint32_t)j);
+                    }
+                }
+            }
+            __syncthreads();
+            const int mb = s_cnt < kRankCap ? s_cnt : kRankCap;
+            for (int c = tid; c < mb; c += kTkThreads) {
+                const uint64_t v = cand[c];
+                int rk = 0;
+                for (int d = 0; d < mb; ++d) rk += cand[d] > v ? 1 : 0;
+                if (rk < rem) {
+                    const uint32_t j = 0xFFFFFFFFu - (uint32_t)v;
+                    atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                }
+            }
+        } else {
+        // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first).
+        // Mark the chosen indices in a bitmap of the row, then emit them in ascending order with one scan.
+    #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-#pragma unroll
+    #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const uint32_t kv = key[4 * i + e];
                 const int64_t j = 4 * ((int64_t)tid + (int64_t)kTkThreads * i) + e;
-                if ((kv >> 20) > bucket) {
-                    atomicOr(&bitmap[j >> 5], 1u << (j & 31));
-                } else if ((kv >> 20) == bucket && kv != 0u) {
-                    const int q = atomicAdd(&s_cnt, 1);
-                    if (q < kRankCap) cand[q] = ((uint64_t)kv << 32) | (0xFFFFFFFFu - (uint32_t)j);
+                if (kv > prefix) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                else if (kv == prefix && kv != 0u) {
+                    const int q = atomicAdd(&s_eq_total, 1);
+                    if (q < 64) eq_idx[q] = (uint32_t)j;
                 }
             }
         }
         __syncthreads();
-        const int mb = s_cnt < kRankCap ? s_cnt : kRankCap;
-        for (int c = tid; c < mb; c += kTkThreads) {
-            const uint64_t v = cand[c];
-            int rk = 0;
-            for (int d = 0; d < mb; ++d) rk += cand[d] > v ? 1 : 0;
-            if (rk < rem) {
-                const uint32_t j = 0xFFFFFFFFu - (uint32_t)v;
-                atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+        if (s_eq_total > 64) {
+            // many equal keys at the threshold: mark the lowest `rem` of them by scanning the row in order
+            if (tid < 32) {
+                int taken = 0;
+                for (int64_t base = 0; base < n && taken < rem; base += 32) {
+                    const int64_t j = base + tid;
+                    bool eq = false;
+                    if (j < n) eq = score_order_key(row[j]) == prefix;
+                    const uint32_t m = __ballot_sync(0xffffffffu, eq);
+                    const int before = __popc(m & ((1u << tid) - 1u));
+                    if (eq && taken + before < rem) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
+                    taken += __popc(m);
+                }
+            }
+        } else if (tid == 0) {
+            const int ne = s_eq_total;
+            for (int t = 0; t < rem && t < ne; ++t) {   // repeated minimum over the few equal keys
+                int best = t;
+                for (int q = t + 1; q < ne; ++q)
+                    if (eq_idx[q] < eq_idx[best]) best = q;
+                const uint32_t tmp = eq_idx[t];
+                eq_idx[t] = eq_idx[best];
+                eq_idx[best] = tmp;
+                atomicOr(&bitmap[eq_idx[t] >> 5], 1u << (eq_idx[t] & 31));
             }
         }
-    } else {
-    // prefix = k-th largest key; rem = keys equal to it that are taken (lowest j first).
-    // Mark the chosen indices in a bitmap of the row, then emit them in ascending order with one scan.
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const uint32_t kv = key[4 * i + e];
-            const int64_t j = 4 * ((int64_t)tid + (int64_t)kTkThreads * i) + e;
-            if (kv > prefix) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
-            else if (kv == prefix && kv != 0u) {
-                const int q = atomicAdd(&s_eq_total, 1);
-                if (q < 64) eq_idx[q] = (uint32_t)j;
-            }
         }
-    }
-    __syncthreads();
-    if (s_eq_total > 64) {
-        // many equal keys at the threshold: mark the lowest `rem` of them by scanning the row in order
-        if (tid < 32) {
-            int taken = 0;
-            for (int64_t base = 0; base < n && taken < rem; base += 32) {
-                const int64_t j = base + tid;
-                bool eq = false;
-                if (j < n) eq = score_order_key(row[j]) == prefix;
-                const uint32_t m = __ballot_sync(0xffffffffu, eq);
-                const int before = __popc(m & ((1u << tid) - 1u));
-                if (eq && taken + before < rem) atomicOr(&bitmap[j >> 5], 1u << (j & 31));
-                taken += __popc(m);
-            }
-        }
-    } else if (tid == 0) {
-        const int ne = s_eq_total;
-        for (int t = 0; t < rem && t < ne; ++t) {   // repeated minimum over the few equal keys
-            int best = t;
-            for (int q = t + 1; q < ne; ++q)
-                if (eq_idx[q] < eq_idx[best]) best = q;
-            const uint32_t tmp = eq_idx[t];
-            eq_idx[t] = eq_idx[best];
-            eq_idx[best] = tmp;
-            atomicOr(&bitmap[eq_idx[t] >> 5], 1u << (eq_idx[t] & 31));
-        }
-    }
     }
     __syncthreads();
     const int per = (nw + kTkThreads - 1) / kTkThreads;
@@ -842,9 +754,184 @@ __global__ void __launch_bounds__(kTkThreads, VPT <= 4 ? 2 : 1) topk_regs_kernel
     }
 }
 
+// ------------------------------------------------------------------ warp-per-row top-k over a bounded row
+// Prefill rows whose scores' lower bound (indexer epilogue) is known: one warp per row reads the row
+// once and keeps the keys at or above the bound (a few percent of the row) in shared memory, then
+// selects the k best exactly: the k-th largest key bit by bit from the top (the search stops when exactly
+// k candidates reach the prefix), ties to the lowest entry indices, which are emitted in ascending order
+// through a bitmap of the row.  A row with more than kWCap candidates is flagged for the block kernel.
+constexpr int kWCap = 2048;          // candidates per row
+constexpr int kWarpsPerCta = 12;
+struct WarpTopk {
+    uint32_t key[kWCap];
+    uint16_t j[kWCap];
+    uint32_t bitmap[1024];           // rows of up to 32768 entries
+};
+constexpr size_t kWarpTopkSmem = kWarpsPerCta * sizeof(WarpTopk);
+
+__global__ void __launch_bounds__(32 * kWarpsPerCta) topk_warp_kernel(const float *__restrict__ scores, int64_t row0,
+                                                                     int64_t rows, int64_t N, int m, int topk,
+                                                                     const uint32_t *__restrict__ bound,
+                                                                     int32_t *__restrict__ flags,
+                                                                     int32_t *__restrict__ sel) {
+    extern __shared__ __align__(16) uint8_t wsm[];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    WarpTopk &S = reinterpret_cast<WarpTopk *>(wsm)[w];
+    const bool vec_ok = (N & 3) == 0 && ((uintptr_t)scores & 15) == 0;
+    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    const uint32_t k = (uint32_t)topk;
+    for (int64_t r = row0 + (int64_t)blockIdx.x * kWarpsPerCta + w; r < rows; r += nwarps) {
+        const int64_t n = r / m < N ? r / m : N;
+        int32_t *out = sel + r * topk;
+        if (n <= topk) {
+            for (int c = lane; c < topk; c += 32) out[c] = c < n ? c : -1;
+            if (lane == 0) flags[r] = 0;
+            continue;
+        }
+        const uint32_t b = bound[r];
+        const float *row = scores + r * N;
+        uint32_t cnt = 0;
+        // one pass over the row, 8 vectors of 4 scores per lane in flight
+        for (int64_t base = 0; base < n; base += 32 * 4 * 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t j0 = base + 4 * (lane + 32 * u);
+                if (vec_ok && j0 + 3 < n) {
+                    v[u] = __ldcs(reinterpret_cast<const float4 *>(row + j0));
+                } else {
+                    v[u].x = j0 < n ? row[j0] : 0.f;
+                    v[u].y = j0 + 1 < n ? row[j0 + 1] : 0.f;
+                    v[u].z = j0 + 2 < n ? row[j0 + 2] : 0.f;
+                    v[u].w = j0 + 3 < n ? row[j0 + 3] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t j0 = base + 4 * (lane + 32 * u);
+                const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = score_order_key(f[e]);
+                    const bool take = j0 + e < n && key >= b;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+                    const uint32_t q = cnt + __popc(bal & ((1u << lane) - 1u));
+                    if (take && q < kWCap) {
+                        S.key[q] = key;
+                        S.j[q] = (uint16_t)(j0 + e);
+                    }
+                    cnt += __popc(bal);
+                }
+            }
+        }
+        if (cnt > kWCap || cnt < k) {   // too many candidates (or a bound that does not hold): block kernel
+            if (lane == 0) flags[r] = 1;
+            continue;
+        }
+        __syncwarp();
+        constexpr int CPL = kWCap / 32;   // candidates per lane: c = lane + 32 i
+        uint32_t ck[CPL];
+        uint32_t kmax = 0;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const uint32_t c = lane + 32 * i;
+            ck[i] = c < cnt ? S.key[c] : 0u;
+            kmax = max(kmax, ck[i]);
+        }
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        const int top = kmax == b ? -1 : 31 - __clz(kmax ^ b);   // every candidate lies in [b, kmax]
+        uint32_t prefix = top < 0 ? kmax : top >= 31 ? 0u : kmax & ~((2u << top) - 1u);
+        bool exact = false;
+        for (int bb = top; bb >= 0; --bb) {
+            const uint32_t cut = prefix | (1u << bb);
+            uint32_t cc = 0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) cc += ck[i] >= cut ? 1u : 0u;
+            const uint32_t tot = __reduce_add_sync(0xffffffffu, cc);
+            if (tot >= k) prefix = cut;
+            if (tot == k) { exact = true; break; }
+        }
+        const uint32_t tau = prefix;
+        uint64_t takem = 0;   // bit i: candidate lane + 32 i is among the k best
+        if (exact) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) takem |= (uint64_t)(ck[i] >= tau ? 1u : 0u) << i;
+        } else {
+            uint64_t gtm = 0, eqm = 0;
+            uint32_t ng = 0, ne = 0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                gtm |= (uint64_t)(ck[i] > tau ? 1u : 0u) << i;
+                eqm |= (uint64_t)(ck[i] == tau ? 1u : 0u) << i;
+            }
+            ng = __reduce_add_sync(0xffffffffu, (uint32_t)__popcll(gtm));
+            ne = __reduce_add_sync(0xffffffffu, (uint32_t)__popcll(eqm));
+            const uint32_t rem = k - ng;
+            uint64_t tm = eqm;
+            if (ne > rem) {
+                // the rem lowest entry indices among the ties: the rem largest 32767 - j, bit by bit
+#pragma unroll
+                for (int i = 0; i < CPL; ++i)
+                    ck[i] = (eqm >> i & 1ull) ? 32768u + 32767u - (uint32_t)S.j[lane + 32 * i] : 0u;
+                uint32_t pj = 32768u;
+                for (int bb = 14; bb >= 0; --bb) {
+                    const uint32_t cut = pj | (1u << bb);
+                    uint32_t cc = 0;
+#pragma unroll
+                    for (int i = 0; i < CPL; ++i) cc += ck[i] >= cut ? 1u : 0u;
+                    if (__reduce_add_sync(0xffffffffu, cc) >= rem) pj = cut;
+                }
+                tm = 0;
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) tm |= (uint64_t)(ck[i] >= pj ? 1u : 0u) << i;
+            }
+            takem = gtm | tm;
+        }
+        const int nw = (int)((n + 31) / 32);
+        for (int i = lane; i < nw; i += 32) S.bitmap[i] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < CPL; ++i)
+            if (takem >> i & 1ull) {
+                const uint32_t jj = S.j[lane + 32 * i];
+                atomicOr(&S.bitmap[jj >> 5], 1u << (jj & 31));
+            }
+        __syncwarp();
+        const int per = (nw + 31) / 32, w0 = lane * per;
+        uint32_t local = 0;
+        for (int i = w0; i < w0 + per && i < nw; ++i) local += __popc(S.bitmap[i]);
+        uint32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        uint32_t pos = incl - local;
+        for (int i = w0; i < w0 + per && i < nw; ++i) {
+            uint32_t bits = S.bitmap[i];
+            while (bits) {
+                const int bp = __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (pos < k) out[pos] = i * 32 + bp;
+                ++pos;
+            }
+        }
+        if (lane == 0) flags[r] = 0;
+        __syncwarp();   // the warp's candidate list and bitmap are reused by its next row
+    }
+}
+
 }  // namespace
 
-int num_sms_host() {
+bool index_tc_supported(const IndexArgs &a) {
+    if (a.dtype != HCSA_BF16 || a.di != 64) return false;
+    if (!(a.Hi == 8 || a.Hi == 16 || a.Hi == 32 || a.Hi == 64)) return false;
+    if (a.pos && a.Hi < 16) return false;          // decode MMA N = Hi must be >= 16
+    if (((uintptr_t)a.qi & 15) || ((uintptr_t)a.keys & 15) || (a.ld_qi * 2) % 16) return false;
+    return a.N <= INT32_MAX && a.rows <= INT32_MAX;
+}
+
+static int num_sms() {
     static int n = 0;
     if (!n) {
         int dev = 0;
@@ -855,54 +942,26 @@ int num_sms_host() {
     return n;
 }
 
-// Fused prefill top-k: a row may hold up to 32768 visible entries (the emission bitmap) and every token of
-// a unit gets 32768 / tq = 128 Hi candidates, which must leave room for k and a tile above a compaction.
-constexpr size_t kFuseBytesPerCta = 32768 * sizeof(uint64_t);
-
-static int fuse_cap(int Hi) { return 128 * (Hi < 32 ? Hi : 32); }
-
-bool index_fused_supported(int dtype, int Hi, int di, int topk, int64_t N) {
-    if (dtype != HCSA_BF16 || di != 64 || !(Hi == 8 || Hi == 16 || Hi == 32 || Hi == 64)) return false;
-    return N <= 32768 && topk >= 1 && 2 * (int64_t)topk + 256 <= fuse_cap(Hi);
-}
-
-size_t index_fused_ws_bytes() { return (size_t)num_sms_host() * kFuseBytesPerCta; }
-
-bool index_tc_supported(const IndexArgs &a) {
-    if (a.dtype != HCSA_BF16 || a.di != 64) return false;
-    if (!(a.Hi == 8 || a.Hi == 16 || a.Hi == 32 || a.Hi == 64)) return false;
-    if (a.pos && a.Hi < 16) return false;          // decode MMA N = Hi must be >= 16
-    if (((uintptr_t)a.qi & 15) || ((uintptr_t)a.keys & 15) || (a.ld_qi * 2) % 16) return false;
-    return a.N <= INT32_MAX && a.rows <= INT32_MAX;
-}
-
-
-template <int HI, bool DEC, bool FUSE>
+template <int HI, bool DEC>
 static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, const CUtensorMap &tq, Args a,
                                  cudaStream_t st) {
-    constexpr int NS = DEC ? kNSDec : FUSE ? kNSFuse : kNS;
-    constexpr int kPer = HI < 32 ? HI : 32;   // fused top-k: candidates per thread (capacity 128 kPer per token)
+    constexpr int NS = DEC ? kNSDec : kNS;
     constexpr size_t smem = 1024 + NS * kATile + 2 * (DEC ? kBTileDec : kBTile) + (DEC ? 0 : 512 * sizeof(float)) +
-                            (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 0) +
-                            (FUSE ? 4 * sizeof(GroupTopk) : 0);
+                            (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 128 * sizeof(uint32_t));
     static_assert(smem <= 232448, "shared memory per CTA");
     static bool configured[64] = {};   // kernel attributes are set per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return HCSA_ERR_CUDA;
         configured[dev] = true;
     }
-    const int64_t slots = (int64_t)num_sms_host() * (DEC ? kDecCtasPerSm : 1);
-    int64_t grid = a.n_units < slots ? a.n_units : slots;
-    if (FUSE) {   // one candidate region per CTA in the workspace
-        const int64_t fit = (int64_t)(ia.ws_bytes / kFuseBytesPerCta);
-        grid = grid < fit ? grid : fit;
-    }
-    if (grid <= 0) return a.n_units > 0 ? HCSA_ERR_WORKSPACE : HCSA_OK;
-    index_scores_tc_kernel<HI, DEC, FUSE><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
+    const int64_t slots = (int64_t)num_sms() * (DEC ? kDecCtasPerSm : 1);
+    const int64_t grid = a.n_units < slots ? a.n_units : slots;
+    if (grid <= 0) return HCSA_OK;
+    index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
     count_launch();
     return check_launch();
 }
@@ -912,7 +971,11 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
     const int64_t nseq = decode ? ia.rows : 1;
     const int tq = decode ? 1 : 256 / ia.Hi;
     CUtensorMap tk, tq_map;
-    if (!make_tmap_bf16_3d(&tk, ia.keys, 64, (uint64_t)ia.N, (uint64_t)nseq, 128, (uint64_t)ia.N * 128, 64, 128, 1,
+    // prefill: keys end at the last entry the range's last query sees (the key tiles round up past it; those
+    // rows read as zeros, so a row-range caller need not have gathered them)
+    const int64_t last_vis = ia.row1 > 0 ? (ia.row1 - 1) / ia.m : 0;
+    const uint64_t key_rows = decode ? (uint64_t)ia.N : (uint64_t)std::max<int64_t>(1, std::min<int64_t>(ia.N, last_vis));
+    if (!make_tmap_bf16_3d(&tk, ia.keys, 64, key_rows, (uint64_t)nseq, 128, (uint64_t)ia.N * 128, 64, 128, 1,
                            true))
         return HCSA_ERR_CUDA;
     if (!make_tmap_bf16_3d(&tq_map, ia.qi, 64, (uint64_t)ia.Hi, (uint64_t)ia.rows, 128, (uint64_t)ia.ld_qi * 2, 64,
@@ -927,6 +990,10 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
     const bool rows_path = ia.N > 32768 && topk_rows_supported(ia);
     uint8_t *scratch = (uint8_t *)ia.ws + (((size_t)ia.rows * ia.N * sizeof(float) + 255) & ~(size_t)255);
     a.hist = nullptr;
+    a.bound = nullptr;
+    if (!decode && ia.topk <= 512 && ia.N <= 32768 &&
+        ia.ws_bytes >= index_topk_ws_bytes(ia.dtype, ia.rows, ia.N))   // bound + flags after the scores
+        a.bound = reinterpret_cast<uint32_t *>(scratch);
     if (rows_path) {
         if (topk_rows_begin(ia, scratch, st) != HCSA_OK) return HCSA_ERR_CUDA;
         a.hist = reinterpret_cast<uint32_t *>(scratch);
@@ -936,55 +1003,62 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         a.n_units = ia.rows * a.tps;
         a.n_qtiles = 0;
     } else {
-        a.n_qtiles = (ia.rows + tq - 1) / tq;
-        a.n_units = a.n_qtiles;
+        // query tiles of the row range [row0, row1): tiles row0 / tq .. n_qtiles - 1, heaviest first
+        a.n_qtiles = (ia.row1 + tq - 1) / tq;
+        a.n_units = a.n_qtiles - ia.row0 / tq;
         a.tps = 0;
     }
     hcsa_status s;
-    const bool fuse = !decode && index_fused_supported(ia.dtype, ia.Hi, ia.di, ia.topk, ia.N);
-    if (fuse) {
-        // top-k inside the indexer's epilogue: candidates per CTA and token in the workspace, no scores
-        a.scores = nullptr;
-        a.cand = (uint64_t *)ia.ws;
-        a.cap = fuse_cap(ia.Hi);
-        a.trig = a.cap - ia.topk - 128;
-        a.topk = ia.topk;
-        a.sel = ia.sel;
-    }
     if (decode) {
         switch (ia.Hi) {
-            case 16: s = launch_scores<16, true, false>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, true, false>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, true, false>(ia, tk, tq_map, a, st); break;
+            case 16: s = launch_scores<16, true>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, true>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, true>(ia, tk, tq_map, a, st); break;
         }
-    } else if (fuse) {
-        switch (ia.Hi) {
-            case 8: s = launch_scores<8, false, true>(ia, tk, tq_map, a, st); break;
-            case 16: s = launch_scores<16, false, true>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, false, true>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, false, true>(ia, tk, tq_map, a, st); break;
-        }
-        return s;
     } else {
         switch (ia.Hi) {
-            case 8: s = launch_scores<8, false, false>(ia, tk, tq_map, a, st); break;
-            case 16: s = launch_scores<16, false, false>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, false, false>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, false, false>(ia, tk, tq_map, a, st); break;
+            case 8: s = launch_scores<8, false>(ia, tk, tq_map, a, st); break;
+            case 16: s = launch_scores<16, false>(ia, tk, tq_map, a, st); break;
+            case 32: s = launch_scores<32, false>(ia, tk, tq_map, a, st); break;
+            default: s = launch_scores<64, false>(ia, tk, tq_map, a, st); break;
         }
     }
     if (s != HCSA_OK) return s;
     // top-k over the materialised scores
-    if (ia.rows <= 0) return HCSA_OK;
+    const int64_t nrows = ia.row1 - ia.row0;
+    if (nrows <= 0) return HCSA_OK;
     if (ia.N <= 32768) {
         const float *sc = (const float *)ia.ws;
+        const int32_t *flags = nullptr;
+        if (a.bound) {
+            // warp per row over the bounded rows; the block kernel below takes only the rows it flags
+            static bool configured_w[64] = {};
+            int dev = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
+            if (!configured_w[dev]) {
+                if (cudaFuncSetAttribute(topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kWarpTopkSmem) != cudaSuccess)
+                    return HCSA_ERR_CUDA;
+                configured_w[dev] = true;
+            }
+            int32_t *fl = reinterpret_cast<int32_t *>(a.bound + ia.rows);
+            const int64_t need = (nrows + kWarpsPerCta - 1) / kWarpsPerCta;
+            const int64_t g = need < num_sms() ? need : num_sms();
+            topk_warp_kernel<<<(unsigned)g, 32 * kWarpsPerCta, kWarpTopkSmem, st>>>(sc, ia.row0, ia.row1, ia.N, ia.m,
+                                                                                    ia.topk, a.bound, fl, ia.sel);
+            count_launch();
+            if (check_launch() != HCSA_OK) return HCSA_ERR_CUDA;
+            flags = fl;
+        }
         // persistent: as many CTAs as fit at once (one per SM at 16 vectors per thread, two at 4)
         if (ia.N <= 8192) {
-            const int64_t g = ia.rows < 2 * num_sms_host() ? ia.rows : 2 * num_sms_host();
-            topk_regs_kernel<4><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.rows, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+            const int64_t g = nrows < 2 * num_sms() ? nrows : 2 * num_sms();
+            topk_regs_kernel<4><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.row0, ia.row1, ia.N, ia.m, ia.pos, ia.topk,
+                                                                   ia.sel, flags);
         } else {
-            const int64_t g = ia.rows < num_sms_host() ? ia.rows : num_sms_host();
-            topk_regs_kernel<16><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.rows, ia.N, ia.m, ia.pos, ia.topk, ia.sel);
+            const int64_t g = nrows < num_sms() ? nrows : num_sms();
+            topk_regs_kernel<16><<<(unsigned)g, kTkThreads, 0, st>>>(sc, ia.row0, ia.row1, ia.N, ia.m, ia.pos, ia.topk,
+                                                                    ia.sel, flags);
         }
         count_launch();
         return check_launch();

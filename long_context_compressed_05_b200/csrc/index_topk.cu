@@ -30,10 +30,10 @@ __global__ void __launch_bounds__(256) index_scores_kernel(IndexArgs a, int qt) 
     A *sw = sq + qt * a.Hi * a.di;                       // [qt][Hi]
     A *sk = sw + qt * a.Hi;                              // [kJT][di + 1]
     const int hd = a.Hi * a.di;
-    const int64_t r0 = (int64_t)blockIdx.y * qt;
+    const int64_t r0 = a.row0 + (int64_t)blockIdx.y * qt;   // query tile of the row range
     const int64_t j0 = (int64_t)blockIdx.x * kJT;
     // visible entries of the last query in the tile bound the whole tile
-    int64_t last = r0 + qt - 1 < a.rows ? r0 + qt - 1 : a.rows - 1;
+    int64_t last = r0 + qt - 1 < a.row1 ? r0 + qt - 1 : a.row1 - 1;
     int64_t pmax = a.pos ? a.pos[last] : last;
     int64_t nv_max = pmax / a.m < a.N ? pmax / a.m : a.N;
     if (a.pos) {   // decode: qt == 1, one sequence per row
@@ -46,11 +46,11 @@ __global__ void __launch_bounds__(256) index_scores_kernel(IndexArgs a, int qt) 
     const S *keys = reinterpret_cast<const S *>(a.keys) + (a.pos ? r0 * a.N * a.di : 0);
     for (int i = threadIdx.x; i < qt * hd; i += blockDim.x) {
         int64_t r = r0 + i / hd;
-        sq[i] = r < a.rows ? to_acc(qi[r * a.ld_qi + i % hd], A()) : A(0);
+        sq[i] = r < a.row1 ? to_acc(qi[r * a.ld_qi + i % hd], A()) : A(0);
     }
     for (int i = threadIdx.x; i < qt * a.Hi; i += blockDim.x) {
         int64_t r = r0 + i / a.Hi;
-        sw[i] = r < a.rows ? to_acc(w[r * a.ld_w + i % a.Hi], A()) : A(0);
+        sw[i] = r < a.row1 ? to_acc(w[r * a.ld_w + i % a.Hi], A()) : A(0);
     }
     for (int i = threadIdx.x; i < kJT * a.di; i += blockDim.x) {
         int64_t j = j0 + i / a.di;
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) index_scores_kernel(IndexArgs a, int qt) 
     const int64_t j = j0 + jl;
     for (int ql = threadIdx.x / kJT; ql < qt; ql += blockDim.x / kJT) {
         const int64_t r = r0 + ql;
-        if (r >= a.rows) break;
+        if (r >= a.row1) break;
         const int64_t p = a.pos ? a.pos[r] : r;
         const int64_t nv = p < 0 ? 0 : (p / a.m < a.N ? p / a.m : a.N);
         if (j >= nv) continue;
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
     __shared__ int s_digit, s_rem;
     __shared__ int s_base_eq, s_base_out;
 
-    const int64_t r = blockIdx.x;
+    const int64_t r = a.row0 + blockIdx.x;
     if (a.only_rows && a.only_rows[4 * r + 3] == 0) return;
     const int64_t p = a.pos ? a.pos[r] : r;
     const int64_t n = p < 0 ? 0 : (p / a.m < a.N ? p / a.m : a.N);
@@ -171,12 +171,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(IndexArgs a) {
 }
 
 size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N) {
-    return (size_t)rows * (size_t)N * (dtype == HCSA_BF16 ? sizeof(float) : sizeof(double));
+    const size_t scores = (size_t)rows * (size_t)N * (dtype == HCSA_BF16 ? sizeof(float) : sizeof(double));
+    if (dtype != HCSA_BF16) return scores;
+    // bf16 (tensor-core indexer): after the scores, 256-byte aligned, a per-row key bound and a per-row flag
+    return ((scores + 255) & ~(size_t)255) + (size_t)rows * 2 * sizeof(uint32_t);
 }
 
 hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st) {
-    if (a.dtype == HCSA_BF16) topk_kernel<float><<<(unsigned)a.rows, kTopkThreads, 0, st>>>(a);
-    else topk_kernel<double><<<(unsigned)a.rows, kTopkThreads, 0, st>>>(a);
+    const unsigned nrows = (unsigned)(a.row1 - a.row0);
+    if (nrows == 0) return HCSA_OK;
+    if (a.dtype == HCSA_BF16) topk_kernel<float><<<nrows, kTopkThreads, 0, st>>>(a);
+    else topk_kernel<double><<<nrows, kTopkThreads, 0, st>>>(a);
     count_launch();
     return check_launch();
 }
@@ -190,7 +195,7 @@ hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st) {
     const size_t esz = a.dtype == HCSA_BF16 ? sizeof(float) : sizeof(double);
     const size_t smem = esz * ((size_t)qt * a.Hi * a.di + (size_t)qt * a.Hi + (size_t)kJT * (a.di + 1));
     if (smem > 200 * 1024) return HCSA_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)((a.N + kJT - 1) / kJT), (unsigned)((a.rows + qt - 1) / qt));
+    dim3 grid((unsigned)((a.N + kJT - 1) / kJT), (unsigned)((a.row1 - a.row0 + qt - 1) / qt));
     if (grid.y > 65535 || a.rows > INT32_MAX) return HCSA_ERR_UNSUPPORTED;
     if (a.N > 0) {
         if (a.dtype == HCSA_BF16) {

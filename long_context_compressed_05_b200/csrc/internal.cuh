@@ -65,10 +65,11 @@ void count_launch(int n = 1);
 hcsa_status check_launch();         // maps cudaGetLastError() to a status
 
 // ---------------------------------------------------------------- launchers
-// compressor (prefill): entries [N, C] (+ idx_keys [N, di] when ki != nullptr)
+// compressor (prefill): entries j0 .. j1 - 1 of [N, C] (+ idx_keys [N, di] when ki != nullptr); the pools
+// are truncated to the sequence [0, T) and read kv / g / ki by global token index
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
-                            void *entries, void *idx_keys, cudaStream_t st);
+                            void *entries, void *idx_keys, int64_t j0, int64_t j1, cudaStream_t st);
 
 hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cache &c, const int32_t *pos,
                                 const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
@@ -88,6 +89,7 @@ struct IndexArgs {
     int32_t *sel;
     void *ws; size_t ws_bytes;
     const int32_t *only_rows;   // if set: the generic select handles only rows r with only_rows[4 r + 3] != 0
+    int64_t row0, row1;         // query rows computed (prefill row range; decode: 0, rows)
 };
 size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N);
 // multi-CTA exact top-k for long decode rows (N > 32768); scratch after the scores.  The scratch starts
@@ -110,10 +112,7 @@ hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st);
 // tensor-core indexer scores (bf16, di = 64) + register-resident top-k
 bool index_tc_supported(const IndexArgs &a);
 hcsa_status launch_index_tc(const IndexArgs &a, cudaStream_t st);
-// prefill indexer with the top-k fused into its epilogue (no materialised scores); workspace per launch
-bool index_fused_supported(int dtype, int Hi, int di, int topk, int64_t N);
-size_t index_fused_ws_bytes();
-int num_sms_host();
+
 
 // attention.  Prefill (pos == nullptr): query t of one sequence, window rows kv[t-window+1 .. t].
 // Decode: query b at position pos[b], entries of sequence b, window ring win_kv[b].
@@ -131,6 +130,7 @@ struct AttendArgs {
     const int32_t *pos;              // decode positions or nullptr
     void *out;
     void *ws; size_t ws_bytes;
+    int64_t row0, row1;              // query rows computed (prefill row range; decode: 0, rows)
 };
 size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, int dh, int topk, int window,
                        int64_t N);

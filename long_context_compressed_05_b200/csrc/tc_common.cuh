@@ -115,8 +115,11 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t g) { retur
 
 // ---------------------------------------------------------------- TMEM loads
 // 32 lanes x 32 bits, 32 consecutive columns: thread i of the warp gets lane (base lane + i).
+// The tcgen05.ld / tcgen05.st / bar forms below are .aligned: every thread of the warp must execute the
+// same instruction, so each helper first reconverges the warp (call sites may follow divergent code).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     uint32_t r[32];
+    __syncwarp();
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -132,6 +135,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 // 32 lanes x 32 bits, 16 consecutive columns.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
     uint32_t r[16];
+    __syncwarp();
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -141,10 +145,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld_wait() {
+    __syncwarp();
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 
 // 32 lanes x 32 bits, 32 consecutive columns, written from registers.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
+    __syncwarp();
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -164,18 +172,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
 }
 // One 32-bit column per lane (thread i of the warp -> lane base + i).
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+    __syncwarp();
     asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
 }
 // Four consecutive 32-bit columns per lane.
 __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float *v) {
     uint32_t r[4];
+    __syncwarp();
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(taddr));
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() {
+    __syncwarp();
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- cp.async
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
@@ -241,6 +254,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    __syncwarp();   // bar.sync is .aligned: the whole warp arrives with one instruction
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
@@ -248,6 +262,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // result, so loops that leave on a failed wait leave together (nobody is left at a later barrier).
 __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
     uint32_t r;
+    __syncwarp();
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"

@@ -107,3 +107,15 @@ def test_noalloc_refuses_requests_beyond_its_scratch(h):
     cache.entries = cache.win_kv = cache.ring_g = cache.idx_keys = cache.ring_ki = FAKE
     assert lib.csa_decode_index_topk_noalloc(ctypes.byref(p), ctypes.byref(cache), V(FAKE), V(FAKE), 2048,
                                              V(FAKE), 32, V(FAKE), None) == 5
+
+
+def test_row_range_is_checked_before_launch(h):
+    """Prefill row ranges: row0 a multiple of 128, row1 a multiple of 128 or T, row0 <= row1 <= T."""
+    lib = h.load()
+    V = ctypes.c_void_p
+    for r0, r1 in [(64, 256), (0, 200), (256, 128), (0, 131072 + 128), (-128, 0)]:
+        p = _params(h, row0=r0, row1=r1)
+        assert lib.csa_compress(ctypes.byref(p), V(FAKE), 36960, V(FAKE), 36960, V(FAKE), 36960, V(FAKE),
+                                V(FAKE), V(FAKE), None) == 2, (r0, r1)
+        assert lib.hca_attend(ctypes.byref(p), V(FAKE), 36960, V(FAKE), 36960, V(FAKE), V(FAKE), None, 0,
+                              None) == 2, (r0, r1)

@@ -1,14 +1,14 @@
-"""The prefill indexer's fused top-k on score patterns that random data rarely produces, through the C ABI,
+"""The prefill indexer + top-k on score patterns that random data rarely produces, through the C ABI,
 against the oracle's top-k (a stable sort on (-score, j)).
 
 The indexer keys, queries and head weights are chosen so that every score is a bf16 value computed exactly
 in fp32 (one head, one channel: s[t, j] = 1 * ReLU(1 * key_j), key_j >= 1), and the selections must
 therefore be bit-exact:
-  * scores that grow with j: every key tile beats everything kept so far, so the candidate buffers fill
-    and are compacted again and again;
-  * plateaus of equal scores that grow with j: compactions and the final selection cut through runs of
-    ties, which must go to the lowest j;
-  * a permuted pattern with many ties: the general case.
+  * scores that grow with j: the k best are the last visible entries of every row;
+  * plateaus of equal scores that grow with j: the threshold cuts through a run of ties, which must go to
+    the lowest j;
+  * a permuted pattern with many ties: about N / 101 keys share each value, so the threshold bucket holds
+    hundreds of equal keys.
 """
 import numpy as np
 import pytest
