@@ -100,14 +100,14 @@ def round_e2m1(a: np.ndarray) -> np.ndarray:
     return a
 
 
-def store_fp8_rows(a: np.ndarray, block: int = 64):
-    """FP8 (E4M3) storage of the rows of a 2-D array in blocks of `block` channels, one fp32 scale
-    amax / 448 per block.  Returns (stored values, scales [rows, blocks])."""
+def store_fp8_rows(a: np.ndarray, block: int = 32):
+    """FP8 (E4M3) storage of the rows of a 2-D array in blocks of `block` channels, one power-of-two
+    scale 2^e per block (e smallest with amax / 2^e <= 448).  Returns (stored values, exponents)."""
     a = np.ascontiguousarray(a, dtype=np.float64).copy()
     rows, cols = a.shape
-    scales = np.empty((rows, -(-cols // block)), np.float64)
-    _load().orc_store_fp8_rows(a.ctypes.data, rows, cols, block, scales.ctypes.data)
-    return a, scales
+    exps = np.empty((rows, -(-cols // block)), np.int32)
+    _load().orc_store_fp8_rows(a.ctypes.data, rows, cols, block, exps.ctypes.data)
+    return a, exps
 
 
 def store_fp4_rows(a: np.ndarray, block: int = 32):
@@ -221,7 +221,7 @@ def prefill(spec, inp, rows=None, chunk=8192, lowprec=False):
     inp: storage arrays x[T,D], W_cat[D,ncat], B[width,C] (as produced by synth).
     rows: query positions to evaluate (default: all).  Entries are always built
     for the whole sequence.  lowprec: store the compressed entries as FP8 (blocks of
-    64 channels) and the indexer keys as FP4 (blocks of 32), see store_fp8_rows /
+    32 channels) and the indexer keys as FP4 (blocks of 32), see store_fp8_rows /
     store_fp4_rows; everything downstream reads the stored values.  Returns a dict of
     float64 arrays."""
     res = prefill_entries(spec, inp, chunk=chunk, lowprec=lowprec)
@@ -248,7 +248,7 @@ def prefill_entries(spec, inp, chunk=8192, lowprec=False):
     entries, idx = compress(T, C, m, spec.width, base, ld, base + 8 * C, ld, B, ki_ptr, ld,
                             spec.di if csa else 0, st)
     if lowprec:
-        entries = store_fp8_rows(entries, 64)[0]
+        entries = store_fp8_rows(entries, 32)[0]
         if csa:
             idx = store_fp4_rows(idx, 32)[0]
     return {"y_pool": ypool, "entries": entries, "idx_keys": idx, "W_q": np.ascontiguousarray(W[:, pool_end:]),
@@ -328,7 +328,7 @@ def decode_step(spec, inp, P, seqs=None, lowprec=False):
         ent_b = to_f64(inp["entries"][b])
         idx_b = to_f64(inp["idx_keys"][b]) if csa else None
         if lowprec:
-            ent_b = store_fp8_rows(ent_b, 64)[0]
+            ent_b = store_fp8_rows(ent_b, 32)[0]
             if csa:
                 idx_b = store_fp4_rows(idx_b, 32)[0]
         ring_ki = to_f64(inp["ring_ki"][b]).copy() if csa else None
@@ -348,7 +348,7 @@ def decode_step(spec, inp, P, seqs=None, lowprec=False):
             b_t = np.stack([Bm[i - lo] for i in toks])
             new = {"j": j, "entry": pool_rows(kv_t, g_t, b_t, C, st)}
             if lowprec:
-                new["entry"] = store_fp8_rows(new["entry"][None], 64)[0][0]
+                new["entry"] = store_fp8_rows(new["entry"][None], 32)[0][0]
             if csa:
                 ki_t = np.stack([ring_ki[i % Wd] for i in toks])
                 new["idx_key"] = pool_rows(ki_t, g_t, b_t, spec.di, st)

@@ -67,8 +67,10 @@ void orc_round(double *a, int64_t n, int st) {
  * each compressed entry in FP8, the indexer keys in FP4).  The pages fix neither the formats' flavour
  * nor the scaling; the readings taken:
  *   FP8 entries: OCP E4M3 (bias 7, no infinities, largest 448, subnormals down to 2^-9).  Every entry
- *     row is cut into blocks of `block` channels; a block's scale is s = fp32(amax / 448) and a value
- *     x is stored as the E4M3 value nearest to x / s (ties to even), times s.
+ *     row is cut into blocks of `block` (32) channels sharing a power-of-two scale 2^e, e the smallest
+ *     integer with amax / 2^e <= 448 (no value is clipped); x is stored as the E4M3 value nearest to
+ *     x / 2^e (ties to even), times 2^e.  Power-of-two block scales over 32 elements are the shared
+ *     scales of the OCP Microscaling formats; a stored value is then exactly a bf16 number.
  *   FP4 indexer keys: OCP E2M1 (0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives).  A block of `block`
  *     channels shares a power-of-two scale 2^e, e the smallest integer with amax / 2^e <= 6 (no value
  *     is clipped); x is stored as the E2M1 value nearest to x / 2^e (ties to the even mantissa), times 2^e.
@@ -110,9 +112,17 @@ void orc_round_e2m1(double *a, int64_t n) {
     for (int64_t i = 0; i < n; ++i) a[i] = round_e2m1(a[i]);
 }
 
+/* smallest e with amax / 2^e <= top (amax > 0) */
+static int block_exponent(double amax, double top) {
+    int e = (int)ceil(log2(amax / top));
+    while (amax / ldexp(1.0, e) > top) ++e;          /* guard log2 rounding */
+    while (amax / ldexp(1.0, e - 1) <= top) --e;
+    return e;
+}
+
 /* FP8 (E4M3) storage of rows [rows, cols] (row-major, leading dimension cols) in blocks of `block`
- * channels; scales[rows][cols / block] receives the block scales (may be NULL). */
-void orc_store_fp8_rows(double *a, int64_t rows, int cols, int block, double *scales) {
+ * channels with power-of-two scales; exps[rows][cols / block] receives the scale exponents (may be NULL). */
+void orc_store_fp8_rows(double *a, int64_t rows, int cols, int block, int32_t *exps) {
     const int nb = (cols + block - 1) / block;
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
@@ -121,9 +131,10 @@ void orc_store_fp8_rows(double *a, int64_t rows, int cols, int block, double *sc
             const int n = (b + 1) * block <= cols ? block : cols - b * block;
             double amax = 0.0;
             for (int i = 0; i < n; ++i) amax = fmax(amax, fabs(x[i]));
-            const double s = (double)(float)(amax / 448.0);
-            if (scales) scales[r * nb + b] = s;
-            for (int i = 0; i < n; ++i) x[i] = s > 0.0 ? round_e4m3(x[i] / s) * s : 0.0;
+            const int e = amax > 0.0 ? block_exponent(amax, 448.0) : 0;
+            if (exps) exps[r * nb + b] = e;
+            const double s = ldexp(1.0, e);
+            for (int i = 0; i < n; ++i) x[i] = amax > 0.0 ? round_e4m3(x[i] / s) * s : 0.0;
         }
     }
 }
@@ -139,12 +150,7 @@ void orc_store_fp4_rows(double *a, int64_t rows, int cols, int block, int32_t *e
             const int n = (b + 1) * block <= cols ? block : cols - b * block;
             double amax = 0.0;
             for (int i = 0; i < n; ++i) amax = fmax(amax, fabs(x[i]));
-            int e = 0;
-            if (amax > 0.0) {
-                e = (int)ceil(log2(amax / 6.0));
-                while (amax / ldexp(1.0, e) > 6.0) ++e;          /* guard log2 rounding */
-                while (amax / ldexp(1.0, e - 1) <= 6.0) --e;
-            }
+            const int e = amax > 0.0 ? block_exponent(amax, 6.0) : 0;
             if (exps) exps[r * nb + b] = e;
             const double s = ldexp(1.0, e);
             for (int i = 0; i < n; ++i) x[i] = amax > 0.0 ? round_e2m1(x[i] / s) * s : 0.0;

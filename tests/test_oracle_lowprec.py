@@ -53,22 +53,38 @@ def test_e2m1_rounding_matches_brute_force():
 def test_fp8_block_storage_invariants():
     rng = np.random.default_rng(3)
     a = rng.standard_normal((64, 1024)) * np.exp(rng.uniform(-6, 6, (64, 1)))   # rows of very different scales
-    a[5, :64] = 0.0                                                              # an all-zero block
-    q, s = oracle.store_fp8_rows(a, 64)
-    blocks = a.reshape(64, 16, 64)
+    a[5, :32] = 0.0                                                              # an all-zero block
+    q, e = oracle.store_fp8_rows(a, 32)
+    blocks = a.reshape(64, 32, 32)
     amax = np.abs(blocks).max(axis=2)
-    np.testing.assert_array_equal(s, (amax / 448.0).astype(np.float32).astype(np.float64))
-    qb = q.reshape(64, 16, 64)
-    with np.errstate(invalid="ignore", divide="ignore"):
-        codes = np.where(s[..., None] > 0, qb / s[..., None], 0.0)
-    # every stored value is scale x (an E4M3 value), the block maximum lands on +-448
+    scale = np.ldexp(1.0, e)
+    nz = amax > 0
+    r = amax[nz] / scale[nz]
+    assert np.all(r <= 448.0) and np.all(r > 224.0)     # the smallest power of two that clips nothing
+    assert np.all(e[~nz] == 0)
+    codes = q.reshape(64, 32, 32) / scale[..., None]
+    # every stored value is 2^e x (an E4M3 value): exact in the E4M3 grid (the rounding itself is pinned
+    # against torch's cast above), and the nearest one to x / 2^e (checked against torch on fp32-exact inputs)
     np.testing.assert_array_equal(oracle.round_e4m3(codes.ravel()).reshape(codes.shape), codes)
-    nz = s > 0
-    assert np.all(np.abs(codes).max(axis=2)[nz] == 448.0)
-    assert np.all(qb[5, 0] == 0.0)
+    assert np.all(q.reshape(64, 32, 32)[5, 0] == 0.0)
     # error: half a unit in the last place of E4M3 (3 mantissa bits) in the normal range
-    rel = np.abs(qb - blocks)[nz] / np.maximum(np.abs(blocks)[nz], 2.0 ** -6 * s[nz][:, None])
-    assert rel.max() <= 2.0 ** -4 + 1e-12
+    with np.errstate(invalid="ignore", divide="ignore"):
+        rel = np.abs(codes * scale[..., None] - blocks) / np.maximum(np.abs(blocks), 2.0 ** -6 * scale[..., None])
+    assert np.nanmax(rel[nz]) <= 2.0 ** -4 + 1e-12
+    # a stored value is a bf16 number (4 significant bits times a power of two)
+    q32 = torch.from_numpy(q).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(q32, q)
+
+
+def test_fp8_block_rounding_against_torch_on_exact_inputs():
+    rng = np.random.default_rng(6)
+    # bf16 inputs (the storage type the entries arrive in): x / 2^e is exact in fp32, so torch's cast is an
+    # independent reference for the element rounding of a whole block
+    a = torch.from_numpy(rng.standard_normal((16, 256)) * 3.0).to(torch.bfloat16).to(torch.float64).numpy()
+    q, e = oracle.store_fp8_rows(a, 32)
+    scale = np.repeat(np.ldexp(1.0, e), 32, axis=1)
+    want = torch.from_numpy((a / scale).astype(np.float32)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(q / scale, want)
 
 
 def test_fp4_block_storage_invariants():
@@ -92,6 +108,6 @@ def test_lowprec_prefill_reads_the_stored_entries():
     inp = synth.prefill_inputs(spec)
     ref = oracle.prefill(spec, inp)
     low = oracle.prefill(spec, inp, lowprec=True)
-    np.testing.assert_array_equal(low["entries"], oracle.store_fp8_rows(ref["entries"], 64)[0])
+    np.testing.assert_array_equal(low["entries"], oracle.store_fp8_rows(ref["entries"], 32)[0])
     np.testing.assert_array_equal(low["idx_keys"], oracle.store_fp4_rows(ref["idx_keys"], 32)[0])
     assert not np.array_equal(low["out"], ref["out"])
