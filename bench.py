@@ -36,11 +36,15 @@ import torch  # noqa: E402
 METRIC = "CSA/HCA prefill tokens/s and decode µs/step at 128K-1M ctx; % of HBM/TC roofline"
 
 WORKLOADS = {
-    "csa_prefill_T131072": ("prefill", "csa_bf16_t131072"),
-    "hca_prefill_T65536": ("prefill", "hca_bf16_t65536"),
-    "csa_decode_B32_P262144": ("decode", "csa_decode_b32_p262144"),
-    "hybrid_decode_B4_P1048576": ("decode", "hybrid_decode_b4_p1048576"),
-    "v4_decode_B4_P1048576": ("decode", "v4_decode_b4_p1048576"),
+    "csa_prefill_T131072": ("prefill", "csa_bf16_t131072", False),
+    "hca_prefill_T65536": ("prefill", "hca_bf16_t65536", False),
+    "csa_decode_B32_P262144": ("decode", "csa_decode_b32_p262144", False),
+    "hybrid_decode_B4_P1048576": ("decode", "hybrid_decode_b4_p1048576", False),
+    "v4_decode_B4_P1048576": ("decode", "v4_decode_b4_p1048576", False),
+    # the same layers with FP8 entries and FP4 indexer keys (block-scaled storage; bf16 arithmetic)
+    "csa_prefill_fp8fp4_T131072": ("prefill", "csa_bf16_t131072", True),
+    "csa_decode_fp8fp4_B32_P262144": ("decode", "csa_decode_b32_p262144", True),
+    "hybrid_decode_fp8fp4_B4_P1048576": ("decode", "hybrid_decode_b4_p1048576", True),
 }
 
 
@@ -84,17 +88,20 @@ def prefill_work(spec):
     return w
 
 
-def decode_bytes(spec, B, N, residual=False):
+def decode_bytes(spec, B, N, residual=False, lowprec=False):
     """Algorithmic HBM bytes of one decode step of one layer (weights + cache reads + writes; with the
-    residual chain also the output projection and the hidden state read and written)."""
+    residual chain also the output projection and the hidden state read and written).  lowprec: entries
+    of C + C/32 bytes (FP8 codes + exponents), indexer keys of di/2 + di/32 bytes (FP4)."""
     bpe = 2
+    ent = spec.C + spec.C // 32 if lowprec else spec.C * bpe
     ncols = 2 * spec.C + spec.H * spec.dh + (spec.di + spec.Hi * spec.di + spec.Hi if spec.kind == "csa" else 0)
     b = spec.D * ncols * bpe                                   # weights
     if spec.kind == "csa":
-        b += B * N * spec.di * bpe                             # indexer key scan
-        b += B * (spec.topk + spec.window) * spec.C * bpe      # selected rows + window
+        key = spec.di // 2 + spec.di // 32 if lowprec else spec.di * bpe
+        b += B * N * key                                       # indexer key scan
+        b += B * spec.topk * ent + B * spec.window * spec.C * bpe   # selected rows + window
     else:
-        b += B * (N + spec.window) * spec.C * bpe              # all entries + window
+        b += B * N * ent + B * spec.window * spec.C * bpe      # all entries + window
     b += B * spec.H * spec.dh * bpe * 2                        # q in, out
     if residual:
         b += spec.H * spec.dh * spec.D * bpe + B * spec.D * bpe * 2   # W_o, x in and out
@@ -245,7 +252,7 @@ def _host_cores():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_prefill_rate(spec, inp, n_rows=1024, offset=0.5, entries=None):
+def oracle_prefill_rate(spec, inp, n_rows=1024, offset=0.5, entries=None, lowprec=False):
     """Oracle throughput (tokens/s) of the whole layer, from a bounded sample of the workload's own inputs.
 
     The sequence-wide half (projections of the pooled columns and the compressor over all T tokens) is
@@ -258,7 +265,7 @@ def oracle_prefill_rate(spec, inp, n_rows=1024, offset=0.5, entries=None):
     T = spec.T
     if entries is None:
         t0 = time.perf_counter()
-        res = oracle.prefill_entries(spec, inp)
+        res = oracle.prefill_entries(spec, inp, lowprec=lowprec)
         entries = (res, time.perf_counter() - t0)
     res, t_fixed = entries
     n_rows = min(n_rows, T)
@@ -274,7 +281,7 @@ def oracle_prefill_rate(spec, inp, n_rows=1024, offset=0.5, entries=None):
     return T / total, sample, entries
 
 
-def oracle_decode_rate(d, seq=0):
+def oracle_decode_rate(d, seq=0, lowprec=False):
     """Oracle µs per decode step, timed on one sequence of the workload's own inputs (its cache, weights
     and new token) through every layer in order -- with the residual chain, each layer's output
     projection and residual update included -- and scaled to the batch of B independent sequences.
@@ -287,7 +294,7 @@ def oracle_decode_rate(d, seq=0):
         inp = synth.decode_inputs(d, li, seqs=[seq])
         inp["x"] = inp["x"][seq:seq + 1] if x is None else x
         t0 = time.perf_counter()
-        x, _ = oracle.decode_stack([spec], [inp], d.P, residual=d.residual)
+        x, _ = oracle.decode_stack([spec], [inp], d.P, residual=d.residual, lowprec=lowprec)
         elapsed += time.perf_counter() - t0
         if not d.residual:
             x = None
@@ -302,7 +309,7 @@ def oracle_decode_rate(d, seq=0):
 
 # ------------------------------------------------------------------ our arm
 
-def run_prefill(args, spec_name, ws, rank):
+def run_prefill(args, spec_name, ws, rank, lowprec=False):
     import long_context_compressed_05_b200 as h
     import synth
     from long_context_compressed_05_b200.host import to_device as dev
@@ -313,7 +320,7 @@ def run_prefill(args, spec_name, ws, rank):
         spec = spec.replace(seed=spec.seed + 1000 * rank)   # independent sequence per rank
     inp = synth.prefill_inputs(spec)
     x, W, B = dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"])
-    layer = h.PrefillLayer(spec)
+    layer = h.PrefillLayer(spec, lowprec=lowprec)
     stream = torch.cuda.current_stream()
     calls = ["hcsa_project", "compress"] + (["csa_index_topk"] if spec.kind == "csa" else []) + ["attend"]
 
@@ -359,7 +366,7 @@ def run_prefill(args, spec_name, ws, rank):
     if "flops" in wk:
         ach = wk["flops"] / (ours[dom] / 1e3) / 1e12
         traffic = None
-        if dom == "attend" and spec.kind == "csa" and spec.H == 64 and spec.dh == 512:
+        if dom == "attend" and spec.kind == "csa" and spec.H == 64 and spec.dh == 512 and not lowprec:
             traffic = ATTEND_TC_DRAM_BYTES_PER_TOKEN * spec.T
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_sus, "unit": "TFLOP/s", "frac": ach / tc_sus,
                 "traffic": traffic, "kernel": dom, "peak_kind": f"{src} bf16 sustained"}
@@ -391,15 +398,17 @@ def run_prefill(args, spec_name, ws, rank):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, N(0,1/D) weights)",
-            "config": {"workload": f"{spec.kind}_prefill_bf16_T{spec.T}_D{spec.D}", "T": spec.T, "D": spec.D,
-                       "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh,
+            "config": {"workload": f"{spec.kind}_prefill_{'fp8fp4' if lowprec else 'bf16'}_T{spec.T}_D{spec.D}",
+                       "T": spec.T, "D": spec.D, "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh,
+                       "storage": ("entries FP8 E4M3, indexer keys FP4 E2M1, power-of-two scale per 32 channels"
+                                   if lowprec else "bf16"),
                        "parallelism": f"replicas x{ws} (one sequence per GPU)",
                        "l2": "inputs larger than L2 (x 0.5 GB, projections 9.7 GB)"},
             "phase_ms": phase_ms, "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
     return line, (spec, inp)
 
 
-def run_decode(args, spec_name, ws, rank):
+def run_decode(args, spec_name, ws, rank, lowprec=False):
     import long_context_compressed_05_b200 as h
     import synth
     from long_context_compressed_05_b200.host import to_device as dev
@@ -412,7 +421,17 @@ def run_decode(args, spec_name, ws, rank):
         inp = synth.decode_inputs(d, li)
         cache = {k: dev(inp[k]) for k in ("entries", "win_kv", "ring_g", "idx_keys", "ring_ki") if k in inp}
         n_cap = inp["entries"].shape[1]
-        layers.append(h.DecodeLayer(spec, d.B, n_cap, cache))
+        if lowprec:   # the same cache stored as FP8 entries / FP4 indexer keys (library quantizer)
+            p = h.params_for(spec, T=0, B=d.B, n_cap=n_cap, lowprec=True)
+            rows = d.B * n_cap
+            for key, what, nbytes in (("entries", h.STORE_ENTRIES, h.hcsa_entry_bytes(p, rows)),
+                                      ("idx_keys", h.STORE_KEYS, h.hcsa_key_bytes(p, rows))):
+                if key in cache:
+                    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+                    h.hcsa_quantize_rows(p, what, cache[key].reshape(rows, -1), buf)
+                    cache[key] = buf
+            torch.cuda.synchronize()
+        layers.append(h.DecodeLayer(spec, d.B, n_cap, cache, lowprec=lowprec))
         Ws.append(dev(inp["W_cat"]))
         Bs.append(dev(inp["B"]))
         Wos.append(dev(inp["W_o"]) if d.residual else None)
@@ -461,7 +480,7 @@ def run_decode(args, spec_name, ws, rank):
     torch.cuda.synchronize()
     launches = h.hcsa_launch_count() * args.steps
     hbm, tc, tc_sus, src = peaks()
-    total_bytes = sum(decode_bytes(L.spec, d.B, L.p.n_cap, d.residual) for L in layers)
+    total_bytes = sum(decode_bytes(L.spec, d.B, L.p.n_cap, d.residual, lowprec) for L in layers)
     ach = total_bytes / (us / 1e6) / 1e9
     roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
             "kernel": "whole decode step (CUDA graph)", "peak_kind": f"{src} hbm"}
@@ -483,7 +502,10 @@ def run_decode(args, spec_name, ws, rank):
     line = {"metric": METRIC, "value": us, "unit": "us/step", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
-            "config": {"workload": spec_name, "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
+            "config": {"workload": spec_name.replace("_b", "_fp8fp4_b", 1) if lowprec else spec_name,
+                       "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
+                       "storage": ("entries FP8 E4M3, indexer keys FP4 E2M1, power-of-two scale per 32 channels"
+                                   if lowprec else "bf16"),
                        "parallelism": f"replicas x{ws}", "l2": "working set larger than L2",
                        "bytes_per_step": total_bytes},
             "roofline": roof,
@@ -503,19 +525,19 @@ NESTED_KEYS = ["value", "unit", "higher_is_better", "steps", "warmup", "ms_per_s
 
 def run_workload(args, wl, ws, rank):
     """One workload on our arm: its JSON line, with the CPU oracle baseline (rank 0, one GPU)."""
-    kind, name = WORKLOADS[wl]
+    kind, name, lowprec = WORKLOADS[wl]
     if kind == "prefill":
-        line, (spec, inp) = run_prefill(args, name, ws, rank)
+        line, (spec, inp) = run_prefill(args, name, ws, rank, lowprec)
     else:
-        line, (d, _) = run_decode(args, name, ws, rank)
+        line, (d, _) = run_decode(args, name, ws, rank, lowprec)
     line["cpu_baseline"] = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle
         if kind == "prefill":
-            v, sample, _ = oracle_prefill_rate(spec, inp)
+            v, sample, _ = oracle_prefill_rate(spec, inp, lowprec=lowprec)
             unit = "tokens/s"
         else:
-            v, sample = oracle_decode_rate(d)
+            v, sample = oracle_decode_rate(d, lowprec=lowprec)
             unit = "us/step"
         line["cpu_baseline"] = {"value": v, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
                                 "sample": sample}
@@ -529,7 +551,7 @@ def run_reference(args, wl, ws, rank):
     same workload (rank 0 only)."""
     import oracle
     import synth
-    kind, name = WORKLOADS[wl]
+    kind, name, lowprec = WORKLOADS[wl]
     vals = []
     n = args.warmup + args.steps
     if kind == "prefill":
@@ -539,24 +561,26 @@ def run_reference(args, wl, ws, rank):
         for i in range(n):
             # the sequence-wide half is timed once (first step) and reused; every step times the per-query
             # half on 64 evenly spread rows, shifted from step to step
-            v, sample, entries = oracle_prefill_rate(spec, inp, n_rows=64, offset=(i + 0.5) / n, entries=entries)
+            v, sample, entries = oracle_prefill_rate(spec, inp, n_rows=64, offset=(i + 0.5) / n, entries=entries,
+                                                     lowprec=lowprec)
             if i >= args.warmup:
                 vals.append(v)
         sample += f"; per step: 64 query rows shifted by (step + 0.5)/{n} of a stratum, mean over {args.steps} steps"
         unit, hib = "tokens/s", True
         ms = spec.T / statistics.mean(vals) * 1e3
-        config = {"workload": f"{spec.kind}_prefill_bf16_T{spec.T}_D{spec.D}", "T": spec.T, "D": spec.D,
-                  "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh, "parallelism": "CPU oracle on rank 0"}
+        config = {"workload": f"{spec.kind}_prefill_{'fp8fp4' if lowprec else 'bf16'}_T{spec.T}_D{spec.D}",
+                  "T": spec.T, "D": spec.D, "C": spec.C, "topk": spec.topk, "H": spec.H, "dh": spec.dh,
+                  "parallelism": "CPU oracle on rank 0"}
     else:
         d = synth.DECODE[name]
         for i in range(n):
-            v, sample = oracle_decode_rate(d, seq=i % d.B)
+            v, sample = oracle_decode_rate(d, seq=i % d.B, lowprec=lowprec)
             if i >= args.warmup:
                 vals.append(v)
         unit, hib = "us/step", False
         ms = statistics.mean(vals) / 1e3
-        config = {"workload": name, "B": d.B, "P": d.P, "layers": len(d.layers), "residual": d.residual,
-                  "parallelism": "CPU oracle on rank 0"}
+        config = {"workload": name.replace("_b", "_fp8fp4_b", 1) if lowprec else name, "B": d.B, "P": d.P,
+                  "layers": len(d.layers), "residual": d.residual, "parallelism": "CPU oracle on rank 0"}
     v = statistics.mean(vals)
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": hib, "scaling": "weak",

@@ -97,6 +97,21 @@ typedef struct {
      * or T; otherwise the calls return HCSA_ERR_SHAPE. */
     int32_t row0;
     int32_t row1;
+    /* Storage of the compressed entries and the indexer keys ("DeepSeek-V4 ... KV cache ...", section
+     * "FP8 y FP4": most of each entry in FP8, the indexer keys in FP4).  0: the layer's dtype.
+     * 1 (bf16 layers, C and di multiples of 32): block-scaled FP8 / FP4, every 32 channels of a row
+     * sharing a power-of-two scale 2^e, e the smallest integer that clips nothing:
+     *   entries   rows x C bytes of OCP E4M3 codes, then rows x C/32 int8 exponents e
+     *             (stored value = E4M3(code) x 2^e; |value| / 2^e <= 448)
+     *   idx_keys  rows x di/2 bytes of OCP E2M1 code pairs (channel 2i in the low nibble, 2i + 1 in
+     *             the high one), then rows x di/32 int8 exponents (|value| / 2^e <= 6)
+     * rows = ceil(T / m) for prefill arrays, B * n_cap for a decode cache (row b * n_cap + j);
+     * hcsa_entry_bytes / hcsa_key_bytes give the sizes.  Codes round to nearest, ties to even.
+     * Every stored value is a bf16 number, so the kernels dequantize exactly and compute as in the bf16
+     * path.  Supported: compressors, cache append, the CSA calls (prefill and decode, tensor-core
+     * shapes: di = 64; H = 64, dh = 512 for the attention) and hca_decode_attend (same shape);
+     * hca_attend and the fp32 / CUDA-core paths return HCSA_ERR_UNSUPPORTED. */
+    int32_t lowprec;
 } hcsa_params;
 
 /* Decode cache of one layer (device pointers, caller-owned).
@@ -138,6 +153,22 @@ size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op);
 /* Number of projected columns for a layer of `kind`:
  * CSA: C (kv) + C (g) + di (ki) + Hi*di (qi) + Hi (w) + H*dh (q);  HCA: C + C + H*dh. */
 int64_t hcsa_proj_cols(const hcsa_params *p, int32_t kind);
+
+/* Bytes of an entries array (hcsa_entry_bytes) or an indexer-key array (hcsa_key_bytes) of `rows`
+ * rows in the storage p selects (dtype, lowprec); 0 for a NULL p or negative rows. */
+size_t hcsa_entry_bytes(const hcsa_params *p, int64_t rows);
+size_t hcsa_key_bytes(const hcsa_params *p, int64_t rows);
+
+/* hcsa_quantize_rows: store bf16 rows in the block-scaled formats of p->lowprec = 1 (the FP8 / FP4 of
+ * the "FP8 y FP4" section, layout as documented at hcsa_params.lowprec), e.g. to convert a bf16 cache.
+ *   what  HCSA_STORE_ENTRIES: src [rows, C] bf16 -> dst of hcsa_entry_bytes(p, rows) bytes (E4M3)
+ *         HCSA_STORE_KEYS:    src [rows, di] bf16 -> dst of hcsa_key_bytes(p, rows) bytes (E2M1)
+ * The same rounding as the compressor and the cache append.  Errors: HCSA_ERR_UNSUPPORTED when
+ * p->lowprec is 0 or the shape has no low-precision form; the usual checks otherwise. */
+#define HCSA_STORE_ENTRIES 0
+#define HCSA_STORE_KEYS 1
+hcsa_status hcsa_quantize_rows(const hcsa_params *p, int32_t what, const void *src, int64_t rows, void *dst,
+                               void *stream);
 
 /* Token projections: every per-token input of the layer in one GEMM -- the compressor's kv and gate
  * logits, the indexer's "lower-dimensional projection" keys, queries and head weights, and the

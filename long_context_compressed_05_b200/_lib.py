@@ -29,7 +29,8 @@ EXPORTS = ["hcsa_version", "hcsa_status_string", "hcsa_workspace_bytes", "hcsa_p
            "csa_compress", "hca_compress", "csa_index_topk", "csa_attend", "hca_attend", "hcsa_cache_append",
            "csa_decode_index_topk", "csa_decode_attend", "hca_decode_attend", "csa_decode_index_topk_noalloc",
            "hcsa_get_device_status", "hcsa_selftest_wait_timeout",
-           "hcsa_launch_count"]
+           "hcsa_launch_count", "hcsa_entry_bytes", "hcsa_key_bytes", "hcsa_quantize_rows"]
+STORE_ENTRIES, STORE_KEYS = 0, 1
 
 
 class HcsaError(RuntimeError):
@@ -42,7 +43,7 @@ class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "T", "D", "m", "width", "C", "di", "Hi", "topk", "window",
                                               "H", "dh")] + [("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
                                                              ("n_cap", ctypes.c_int32), ("row0", ctypes.c_int32),
-                                                             ("row1", ctypes.c_int32)]
+                                                             ("row1", ctypes.c_int32), ("lowprec", ctypes.c_int32)]
 
 
 class Cache(ctypes.Structure):
@@ -83,6 +84,9 @@ def load():
         "hcsa_get_device_status": (I32, [V]),
         "hcsa_selftest_wait_timeout": (I32, [V]),
         "hcsa_launch_count": (I64, [I32]),
+        "hcsa_entry_bytes": (SZ, [P, I64]),
+        "hcsa_key_bytes": (SZ, [P, I64]),
+        "hcsa_quantize_rows": (I32, [P, I32, V, I64, V, V]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -112,10 +116,10 @@ def _stream(stream):
 
 
 def make_params(*, T=0, D=0, m=4, width=8, C=0, di=0, Hi=0, topk=0, window=128, H=1, dh=0, scale=1.0,
-                dtype="bf16", B=1, n_cap=0, row0=0, row1=0) -> Params:
+                dtype="bf16", B=1, n_cap=0, row0=0, row1=0, lowprec=0) -> Params:
     return Params(B=B, T=T, D=D, m=m, width=width, C=C, di=di, Hi=Hi, topk=topk, window=window, H=H, dh=dh,
                   scale=scale, dtype=HCSA_BF16 if dtype == "bf16" else HCSA_F32, n_cap=n_cap, row0=row0,
-                  row1=row1)
+                  row1=row1, lowprec=int(lowprec))
 
 
 def make_cache(entries, win_kv, ring_g, idx_keys=None, ring_ki=None) -> Cache:
@@ -221,6 +225,20 @@ def hcsa_get_device_status(stream=None) -> int:
 def hcsa_selftest_wait_timeout(stream=None) -> None:
     """Enqueue the bounded-wait self-test kernel (see include/hca_csa.h)."""
     _check("hcsa_selftest_wait_timeout", load().hcsa_selftest_wait_timeout(_stream(stream)))
+
+
+def hcsa_entry_bytes(p: Params, rows: int) -> int:
+    return int(load().hcsa_entry_bytes(ctypes.byref(p), rows))
+
+
+def hcsa_key_bytes(p: Params, rows: int) -> int:
+    return int(load().hcsa_key_bytes(ctypes.byref(p), rows))
+
+
+def hcsa_quantize_rows(p, what, src, dst, stream=None):
+    """src: [rows, C] (entries) or [rows, di] (keys) bf16; dst: a byte buffer of the matching size."""
+    _check("hcsa_quantize_rows", load().hcsa_quantize_rows(ctypes.byref(p), what, _ptr(src), src.shape[0],
+                                                           _ptr(dst), _stream(stream)))
 
 
 def hcsa_launch_count(reset: bool = False) -> int:

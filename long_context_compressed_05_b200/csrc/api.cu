@@ -56,6 +56,8 @@ hcsa_status check_common(const hcsa_params *p) {
     const int V = vec(p->dtype);
     if (p->m < 1 || p->width < p->m || p->width > 512 || p->C < 2 || p->C % (2 * V) != 0) return HCSA_ERR_SHAPE;
     if (p->H < 1 || p->dh != p->C / 2 || p->window < 1) return HCSA_ERR_SHAPE;
+    if (p->lowprec != 0 && p->lowprec != 1) return HCSA_ERR_SHAPE;
+    if (p->lowprec && (p->dtype != HCSA_BF16 || p->C % 32 != 0)) return HCSA_ERR_UNSUPPORTED;
     return HCSA_OK;
 }
 
@@ -63,6 +65,7 @@ hcsa_status check_csa(const hcsa_params *p) {
     HCSA_TRY(check_common(p));
     if (p->di < 1 || p->di > p->C || p->di % vec(p->dtype) != 0 || p->Hi < 1 || p->topk < 1)
         return HCSA_ERR_SHAPE;
+    if (p->lowprec && p->di % 32 != 0) return HCSA_ERR_UNSUPPORTED;
     return HCSA_OK;
 }
 
@@ -142,6 +145,18 @@ int64_t hcsa_proj_cols(const hcsa_params *p, int32_t kind) {
     return c;
 }
 
+size_t hcsa_entry_bytes(const hcsa_params *p, int64_t rows) {
+    if (!p || rows < 0) return 0;
+    if (p->lowprec) return (size_t)rows * (p->C + p->C / 32);
+    return (size_t)rows * p->C * esize(p->dtype);
+}
+
+size_t hcsa_key_bytes(const hcsa_params *p, int64_t rows) {
+    if (!p || rows < 0) return 0;
+    if (p->lowprec) return (size_t)rows * (p->di / 2 + p->di / 32);
+    return (size_t)rows * p->di * esize(p->dtype);
+}
+
 size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op) {
     if (!p) return 0;
     switch (op) {
@@ -207,7 +222,7 @@ hcsa_status csa_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, co
     HCSA_TRY(row_range(p, &r0, &r1));
     entry_range(p, r0, r1, &j0, &j1);
     return launch_compress(p->dtype, p->T, p->C, p->m, p->width, kv, ld_kv, g, ld_g, ki, ld_ki, p->di, bias,
-                           entries, idx_keys, j0, j1, (cudaStream_t)stream);
+                           entries, idx_keys, j0, j1, p->lowprec != 0, n_entries(p), (cudaStream_t)stream);
 }
 
 hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, const void *g, int64_t ld_g,
@@ -221,7 +236,7 @@ hcsa_status hca_compress(const hcsa_params *p, const void *kv, int64_t ld_kv, co
     HCSA_TRY(row_range(p, &r0, &r1));
     entry_range(p, r0, r1, &j0, &j1);
     return launch_compress(p->dtype, p->T, p->C, p->m, p->width, kv, ld_kv, g, ld_g, nullptr, 0, 0, bias, entries,
-                           nullptr, j0, j1, (cudaStream_t)stream);
+                           nullptr, j0, j1, p->lowprec != 0, n_entries(p), (cudaStream_t)stream);
 }
 
 hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, const void *w, int64_t ld_w,
@@ -236,7 +251,7 @@ hcsa_status csa_index_topk(const hcsa_params *p, const void *qi, int64_t ld_qi, 
     int64_t r0, r1;
     HCSA_TRY(row_range(p, &r0, &r1));
     IndexArgs a{p->dtype, p->T, p->Hi, p->di, p->topk, p->m, n_entries(p), qi, ld_qi, w, ld_w, idx_keys,
-                nullptr, sel, ws, ws_bytes, nullptr, r0, r1};
+                nullptr, sel, ws, ws_bytes, nullptr, r0, r1, p->lowprec != 0};
     return launch_index_topk(a, (cudaStream_t)stream);
 }
 
@@ -252,7 +267,7 @@ static hcsa_status attend_prefill(const hcsa_params *p, bool dense, const void *
     AttendArgs a{};
     a.dtype = p->dtype; a.rows = p->T; a.H = p->H; a.dh = p->dh; a.C = p->C; a.window = p->window; a.m = p->m;
     a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = n_entries(p);
-    a.row0 = r0; a.row1 = r1;
+    a.row0 = r0; a.row1 = r1; a.lowprec = p->lowprec != 0;
     a.q = q; a.ld_q = ld_q; a.kv = kv; a.ld_kv = ld_kv; a.entries = entries; a.sel = sel; a.pos = nullptr;
     a.out = out; a.ws = ws; a.ws_bytes = ws_bytes;
     return launch_attend(a, (cudaStream_t)stream);
@@ -268,6 +283,7 @@ hcsa_status csa_attend(const hcsa_params *p, const void *q, int64_t ld_q, const 
 hcsa_status hca_attend(const hcsa_params *p, const void *q, int64_t ld_q, const void *kv, int64_t ld_kv,
                        const void *entries, void *out, void *ws, size_t ws_bytes, void *stream) {
     HCSA_TRY(check_common(p));
+    if (p->lowprec) return HCSA_ERR_UNSUPPORTED;
     return attend_prefill(p, true, q, ld_q, kv, ld_kv, entries, nullptr, out, ws, ws_bytes, stream);
 }
 
@@ -291,7 +307,7 @@ hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache,
     HCSA_TRY(hcsa::check_decode_index_topk_args(p, cache, pos, qi, ld_qi, w, ld_w, sel));
     if (!ws || ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK)) return HCSA_ERR_WORKSPACE;
     IndexArgs a{p->dtype, p->B, p->Hi, p->di, p->topk, p->m, p->n_cap, qi, ld_qi, w, ld_w, cache->idx_keys,
-                pos, sel, ws, ws_bytes, nullptr, 0, p->B};
+                pos, sel, ws, ws_bytes, nullptr, 0, p->B, p->lowprec != 0};
     return launch_index_topk(a, (cudaStream_t)stream);
 }
 
@@ -308,7 +324,7 @@ static hcsa_status attend_decode(const hcsa_params *p, bool dense, const hcsa_ca
     a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = p->n_cap;
     a.q = q; a.ld_q = ld_q; a.kv = cache->win_kv; a.ld_kv = p->C; a.entries = cache->entries; a.sel = sel;
     a.pos = pos; a.out = out; a.ws = ws; a.ws_bytes = ws_bytes;
-    a.row0 = 0; a.row1 = p->B;
+    a.row0 = 0; a.row1 = p->B; a.lowprec = p->lowprec != 0;
     return launch_attend(a, (cudaStream_t)stream);
 }
 
@@ -325,6 +341,19 @@ hcsa_status hca_decode_attend(const hcsa_params *p, const hcsa_cache *cache, con
     HCSA_TRY(check_common(p));
     HCSA_TRY(check_decode(p, cache, pos, false));
     return attend_decode(p, true, cache, pos, q, ld_q, nullptr, out, ws, ws_bytes, stream);
+}
+
+hcsa_status hcsa_quantize_rows(const hcsa_params *p, int32_t what, const void *src, int64_t rows, void *dst,
+                               void *stream) {
+    if (!p) return HCSA_ERR_NULL;
+    if (what != HCSA_STORE_ENTRIES && what != HCSA_STORE_KEYS) return HCSA_ERR_SHAPE;
+    const bool keys = what == HCSA_STORE_KEYS;
+    HCSA_TRY(keys ? check_csa(p) : check_common(p));
+    if (!p->lowprec) return HCSA_ERR_UNSUPPORTED;
+    if (!src || !dst) return HCSA_ERR_NULL;
+    if (rows < 0) return HCSA_ERR_SHAPE;
+    if (!aligned(src) || !aligned(dst)) return HCSA_ERR_ALIGN;
+    return launch_quantize_rows(src, rows, keys ? p->di : p->C, keys, dst, (cudaStream_t)stream);
 }
 
 hcsa_status hcsa_get_device_status(void *stream) {

@@ -208,7 +208,8 @@ size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, 
 
 hcsa_status launch_attend(const AttendArgs &a, cudaStream_t st) {
     if (a.rows == 0) return HCSA_OK;
-    if (hca_attend_tc_supported(a)) return launch_hca_attend_tc(a, st);
+    if (a.lowprec && !attend_tc_supported(a)) return HCSA_ERR_UNSUPPORTED;   // FP8 entries: tensor-core shapes only
+    if (!a.lowprec && hca_attend_tc_supported(a)) return launch_hca_attend_tc(a, st);
     if (attend_tc_supported(a)) {
         const int ns = attend_tc_segments(a);
         if (ns > 1 &&

@@ -28,6 +28,7 @@
 // warps 8..15 run the softmax and the output epilogue (two warps per TMEM lane quadrant, 32 heads
 // each).  Gathered 128-byte row segments are what bounds this kernel: the gather rate per SM, not the
 // tensor core, sets its speed, and that rate grows with the number of warps issuing the copies.
+#include "lowprec.cuh"
 #include "tc_common.cuh"
 
 namespace hcsa {
@@ -60,7 +61,10 @@ constexpr uint32_t kIdescPV = tc::idesc_bf16(128, kH, true, true);    // O^T = V
 
 struct Params {
     bool decode, dense;
+    bool lowprec;                     // entries: E4M3 codes (ld C bytes), then int8 exponents (ld C / 32)
     const __nv_bfloat16 *ent, *raw;   // entry rows (ld C) and raw window rows
+    const uint8_t *ent8;              // lowprec: code rows
+    const int8_t *ent_exp;            // lowprec: exponent rows
     int64_t ld_raw;
     int64_t nq;          // queries (prefill T, decode B)
     int64_t N;           // entries per sequence (prefill ceil(T/m), decode n_cap)
@@ -219,7 +223,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const __nv_bfloat16 *ptr = nullptr;
                     if (kk < x.E) {
                         const int64_t j = a.dense ? (int64_t)kk : (int64_t)jsel[i];
-                        if (j >= 0 && j < x.nvis) ptr = a.ent + ((a.decode ? x.q * a.N : 0) + j) * (int64_t)kC;
+                        if (j >= 0 && j < x.nvis) {
+                            const int64_t R = (a.decode ? x.q * a.N : 0) + j;
+                            ptr = a.lowprec ? reinterpret_cast<const __nv_bfloat16 *>(a.ent8 + R * kC)
+                                            : a.ent + R * (int64_t)kC;
+                        }
                         else if (!a.dense && j != -1) report(a.status, kStatusBounds);   // a selected index that is
                                                                                         // neither padding nor visible
                     } else {
@@ -234,15 +242,53 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ++iu;
             auto load_chunk = [&](int t, int col) {
                 const int s = ic % kNS;
+                const int kt = x.t0 + t;
+                if (a.lowprec && kt * kKT < x.E) {
+                    // FP8 entry rows: 8 codes (one 16-byte bf16 chunk) and their block exponent per thread, loaded
+                    // into registers before the stage is free, then rebuilt as bf16 (exact) in the swizzled stage
+                    constexpr int kIt = (kKT * 8 + kProdThreads - 1) / kProdThreads;
+                    const int g = pt & 7;
+                    const __nv_bfloat16 *const *rows = rp + t * kKT;
+                    uint2 cv[kIt];
+                    int ev[kIt];
+#pragma unroll
+                    for (int i = 0; i < kIt; ++i) {
+                        const int row = i * (kProdThreads / 8) + (pt >> 3);
+                        cv[i] = make_uint2(0u, 0u);
+                        ev[i] = 0;
+                        if ((kKT * 8) % kProdThreads != 0 && row >= kKT) break;
+                        const uint8_t *p = reinterpret_cast<const uint8_t *>(rows[row]);
+                        if (p) {
+                            const int ch = col + g * 8;
+                            cv[i] = __ldg(reinterpret_cast<const uint2 *>(p + ch));
+                            ev[i] = __ldg(a.ent_exp + ((p - a.ent8) + ch) / lp::kBlock);
+                        }
+                    }
+                    if (ic >= kNS) ok = ok && tc::mbar_wait(&bars->re[s], ((ic / kNS) - 1) & 1, a.status);
+                    if (!ok) {
+                        ++ic;
+                        return;
+                    }
+#pragma unroll
+                    for (int i = 0; i < kIt; ++i) {
+                        const int row = i * (kProdThreads / 8) + (pt >> 3);
+                        if ((kKT * 8) % kProdThreads != 0 && row >= kKT) break;
+                        const uint4 v = lp::fp8x8_to_bf16x8(cv[i], lp::pow2f(ev[i]));
+                        *reinterpret_cast<uint4 *>(sRing + s * kStage + tc::sw128_offset(row, g)) = v;
+                    }
+                    tc::fence_async_smem();   // generic-proxy stores -> the MMA's async proxy
+                    tc::mbar_arrive(&bars->rf[s]);
+                    ++ic;
+                    return;
+                }
                 if (ic >= kNS) ok = ok && tc::mbar_wait(&bars->re[s], ((ic / kNS) - 1) & 1, a.status);
                 if (!ok) {
                     ++ic;
                     return;
                 }
-                const int kt = x.t0 + t;
                 // 128 consecutive rows: the prefill window, or a dense (HCA) entry tile inside the visible range
                 const bool win_tile = !a.decode && kt * kKT >= x.E;
-                const bool ent_tile = a.dense && (int64_t)(kt + 1) * kKT <= x.nvis;
+                const bool ent_tile = a.dense && !a.lowprec && (int64_t)(kt + 1) * kKT <= x.nvis;
                 if (win_tile || ent_tile) {
                     if (pt == 0) {
                         tc::mbar_arrive_expect_tx(&bars->rf[s], kStage);
@@ -610,6 +656,12 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     }
     Params p{};
     p.ent = (const __nv_bfloat16 *)a.entries;
+    p.lowprec = a.lowprec;
+    if (a.lowprec) {   // code rows [ent_rows][C], then exponent rows [ent_rows][C / 32]
+        const int64_t rows_all = decode ? a.rows * a.N : a.N;
+        p.ent8 = (const uint8_t *)a.entries;
+        p.ent_exp = (const int8_t *)(p.ent8 + rows_all * kC);
+    }
     p.raw = (const __nv_bfloat16 *)a.kv;
     p.ld_raw = decode ? kC : a.ld_kv;
     p.decode = decode;

@@ -16,8 +16,41 @@
 // coalesced.  fp32 storage (computed in fp64) keeps the generic form, a
 // single-pass running max per channel.
 #include "internal.cuh"
+#include "lowprec.cuh"
 
 namespace hcsa {
+
+// Store one 8-channel vector (c0 .. c0 + 7) of entry row `row`: in the storage dtype, or (lp.on) rounded to
+// bf16 and then as block-scaled FP8 (entries) / FP4 (indexer keys); the 4 lanes of a 32-channel block call
+// this together.
+struct LowPrecOut {
+    bool on;
+    int64_t rows;   // rows of the whole array: the exponents follow rows x ch code bytes
+};
+
+__device__ __forceinline__ void store_row_vec(const float *r, bool is_key, int64_t row, int C, int di, int c0,
+                                              __nv_bfloat16 *entries, __nv_bfloat16 *idx_keys, LowPrecOut lp) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(__float2bfloat16_rn(r[e]));
+    if (lp.on) {
+        if (is_key) {
+            uint8_t *codes = reinterpret_cast<uint8_t *>(idx_keys);
+            lp::store_fp4x8(v, codes, reinterpret_cast<int8_t *>(codes + lp.rows * (di / 2)), row, di, c0);
+        } else {
+            uint8_t *codes = reinterpret_cast<uint8_t *>(entries);
+            lp::store_fp8x8(v, codes, reinterpret_cast<int8_t *>(codes + lp.rows * C), row, C, c0);
+        }
+        return;
+    }
+    uint4 o;
+    __nv_bfloat16 *oe = reinterpret_cast<__nv_bfloat16 *>(&o);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) oe[e] = __float2bfloat16_rn(v[e]);
+    if (is_key) *reinterpret_cast<uint4 *>(idx_keys + row * di + c0) = o;
+    else *reinterpret_cast<uint4 *>(entries + row * C + c0) = o;
+}
+
 
 template <typename A, int V>
 struct PoolAcc {
@@ -53,7 +86,8 @@ __global__ void __launch_bounds__(256) compress_kernel(int64_t T, int C, int m, 
                                                        int64_t ld_kv, const S *__restrict__ g, int64_t ld_g,
                                                        const S *__restrict__ ki, int64_t ld_ki, int di,
                                                        const S *__restrict__ bias, S *__restrict__ entries,
-                                                       S *__restrict__ idx_keys, int64_t j0, int64_t N) {
+                                                       S *__restrict__ idx_keys, int64_t j0, int64_t N,
+                                                       LowPrecOut lp) {
     using A = typename Traits<S>::A;
     constexpr int V = Traits<S>::VEC;
     const int slots_c = C / V;
@@ -83,9 +117,17 @@ __global__ void __launch_bounds__(256) compress_kernel(int64_t T, int C, int m, 
     }
     A r[V];
     pa.result(r);
+    if constexpr (V == 8) {   // bf16 storage
+        if (lp.on) {
+            store_row_vec(r, is_key, j, C, di, c0, reinterpret_cast<__nv_bfloat16 *>(entries),
+                          reinterpret_cast<__nv_bfloat16 *>(idx_keys), lp);
+            return;
+        }
+    }
     if (is_key) store_vec(idx_keys + j * di + c0, r);
     else store_vec(entries + j * C + c0, r);
 }
+
 
 // ---------------------------------------------------------------- bf16 prefill, faster forms
 __device__ __forceinline__ float ex2_fast(float x) {
@@ -110,7 +152,7 @@ __global__ void __launch_bounds__(256) compress_narrow_bf16_kernel(
     int T, int C, int m, int width, const __nv_bfloat16 *__restrict__ kv, int64_t ld_kv,
     const __nv_bfloat16 *__restrict__ g, int64_t ld_g, const __nv_bfloat16 *__restrict__ ki, int64_t ld_ki, int di,
     const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys,
-    int j0, int N) {
+    int j0, int N, LowPrecOut lp) {
     const int slots_c = C >> 3;
     const int slots = slots_c + (ki ? di >> 3 : 0);
     const int gid = blockIdx.x * 256 + threadIdx.x;
@@ -160,12 +202,10 @@ __global__ void __launch_bounds__(256) compress_narrow_bf16_kernel(
             acc[e] = fmaf(p, vv[e], acc[e]);
         }
     }
-    uint4 o;
-    __nv_bfloat16 *oe = reinterpret_cast<__nv_bfloat16 *>(&o);
+    float r[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) oe[e] = __float2bfloat16_rn(acc[e] / z[e]);
-    if (is_key) *reinterpret_cast<uint4 *>(idx_keys + (int64_t)j * di + c0) = o;
-    else *reinterpret_cast<uint4 *>(entries + (int64_t)j * C + c0) = o;
+    for (int e = 0; e < 8; ++e) r[e] = acc[e] / z[e];
+    store_row_vec(r, is_key, j, C, di, c0, entries, idx_keys, lp);
 }
 
 // Wide pools (HCA: 128 tokens): a block of 8 warps per (entry, 32 channel vectors); lane = channel vector,
@@ -176,7 +216,7 @@ __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
     int T, int C, int m, int width, const __nv_bfloat16 *__restrict__ kv, int64_t ld_kv,
     const __nv_bfloat16 *__restrict__ g, int64_t ld_g, const __nv_bfloat16 *__restrict__ ki, int64_t ld_ki, int di,
     const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ entries, __nv_bfloat16 *__restrict__ idx_keys,
-    int j0) {
+    int j0, LowPrecOut lp) {
     __shared__ float part[kWideWarps][3][8][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int slots_c = C >> 3;
@@ -230,8 +270,7 @@ __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
     for (int e = 0; e < 8; ++e) { part[w][0][e][lane] = mx[e]; part[w][1][e][lane] = z[e]; part[w][2][e][lane] = acc[e]; }
     __syncthreads();
     if (w != 0 || !active) return;
-    uint4 o;
-    __nv_bfloat16 *oe = reinterpret_cast<__nv_bfloat16 *>(&o);
+    float res[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         float M = -INFINITY;
@@ -244,17 +283,18 @@ __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
             Z = fmaf(part[q][1][e][lane], sc, Z);
             Acc = fmaf(part[q][2][e][lane], sc, Acc);
         }
-        oe[e] = __float2bfloat16_rn(Acc / Z);
+        res[e] = Acc / Z;
     }
-    if (is_key) *reinterpret_cast<uint4 *>(idx_keys + (int64_t)j * di + c0) = o;
-    else *reinterpret_cast<uint4 *>(entries + (int64_t)j * C + c0) = o;
+    store_row_vec(res, is_key, j, C, di, c0, entries, idx_keys, lp);
 }
 
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
-                            void *entries, void *idx_keys, int64_t j0, int64_t j1, cudaStream_t st) {
+                            void *entries, void *idx_keys, int64_t j0, int64_t j1, bool lowprec, int64_t rows,
+                            cudaStream_t st) {
     const int64_t N = j1 - j0;   // entries j0 .. j1 - 1 of the sequence
     if (N <= 0) return HCSA_OK;
+    const LowPrecOut lp{lowprec, rows};
     const int threads = 256;
     if (dtype == HCSA_BF16) {
         using S = __nv_bfloat16;
@@ -263,25 +303,52 @@ hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const
             const int64_t blocks = (N * slots + threads - 1) / threads;
             compress_narrow_bf16_kernel<8><<<(unsigned)blocks, threads, 0, st>>>(
                 (int)T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di,
-                (const S *)bias, (S *)entries, (S *)idx_keys, (int)j0, (int)N);
+                (const S *)bias, (S *)entries, (S *)idx_keys, (int)j0, (int)N, lp);
         } else if (N <= 65535 && T <= INT32_MAX && (int64_t)m * j1 <= INT32_MAX) {
             dim3 grid((unsigned)((slots + 31) / 32), (unsigned)N);
             compress_wide_bf16_kernel<<<grid, 32 * kWideWarps, 0, st>>>(
                 (int)T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di,
-                (const S *)bias, (S *)entries, (S *)idx_keys, (int)j0);
+                (const S *)bias, (S *)entries, (S *)idx_keys, (int)j0, lp);
         } else {
             const int64_t blocks = (N * slots + threads - 1) / threads;
             compress_kernel<S><<<(unsigned)blocks, threads, 0, st>>>(
                 T, C, m, width, (const S *)kv, ld_kv, (const S *)g, ld_g, (const S *)ki, ld_ki, di, (const S *)bias,
-                (S *)entries, (S *)idx_keys, j0, N);
+                (S *)entries, (S *)idx_keys, j0, N, lp);
         }
     } else {
         const int64_t slots = C / 4 + (ki ? di / 4 : 0);
         const int64_t blocks = (N * slots + threads - 1) / threads;
         compress_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
             T, C, m, width, (const float *)kv, ld_kv, (const float *)g, ld_g, (const float *)ki, ld_ki, di,
-            (const float *)bias, (float *)entries, (float *)idx_keys, j0, N);
+            (const float *)bias, (float *)entries, (float *)idx_keys, j0, N, LowPrecOut{false, 0});
     }
+    count_launch();
+    return check_launch();
+}
+
+// ---------------------------------------------------------------- bf16 rows -> FP8 / FP4 storage
+// One thread per 8-channel vector of a row (the 4 lanes of a 32-channel block are adjacent threads).
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, int64_t rows,
+                                                            int ch, bool keys, uint8_t *dst) {
+    const int vpr = ch / 8;
+    const int64_t gid = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    if (gid >= rows * vpr) return;   // rows x vpr is a multiple of 4: blocks are whole
+    const int64_t r = gid / vpr;
+    const int c0 = (int)(gid - r * vpr) * 8;
+    const uint4 u = *reinterpret_cast<const uint4 *>(src + r * ch + c0);
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(e[i]);
+    if (keys) lp::store_fp4x8(v, dst, reinterpret_cast<int8_t *>(dst + rows * (ch / 2)), r, ch, c0);
+    else lp::store_fp8x8(v, dst, reinterpret_cast<int8_t *>(dst + rows * ch), r, ch, c0);
+}
+
+hcsa_status launch_quantize_rows(const void *src, int64_t rows, int ch, bool keys, void *dst, cudaStream_t st) {
+    if (rows <= 0) return HCSA_OK;
+    const int64_t n = rows * (ch / 8);
+    quantize_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((const __nv_bfloat16 *)src, rows, ch, keys,
+                                                                        (uint8_t *)dst);
     count_launch();
     return check_launch();
 }
@@ -295,7 +362,7 @@ __global__ void __launch_bounds__(128) cache_append_kernel(
     int C, int m, int width, int window, int di, int64_t n_cap, const int32_t *__restrict__ pos,
     const S *__restrict__ kv_new, int64_t ld_kv, const S *__restrict__ g_new, int64_t ld_g,
     const S *__restrict__ ki_new, int64_t ld_ki, const S *__restrict__ bias, S *entries, S *idx_keys, S *win_kv,
-    S *ring_g, S *ring_ki, int *status) {
+    S *ring_g, S *ring_ki, int *status, LowPrecOut lp) {
     using A = typename Traits<S>::A;
     constexpr int V = Traits<S>::VEC;
     const int b = blockIdx.y;
@@ -339,6 +406,13 @@ __global__ void __launch_bounds__(128) cache_append_kernel(
     }
     A r[V];
     pa.result(r);
+    if constexpr (V == 8) {   // bf16 storage
+        if (lp.on) {
+            store_row_vec(r, is_key, (int64_t)b * n_cap + j, C, di, c0, reinterpret_cast<__nv_bfloat16 *>(entries),
+                          reinterpret_cast<__nv_bfloat16 *>(idx_keys), lp);
+            return;
+        }
+    }
     if (is_key) store_vec(idx_keys + ((int64_t)b * n_cap + j) * di + c0, r);
     else store_vec(entries + ((int64_t)b * n_cap + j) * C + c0, r);
 }
@@ -355,13 +429,13 @@ hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cach
         cache_append_kernel<S><<<grid, 128, 0, st>>>(
             p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
             (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
-            (S *)c.ring_ki, status);
+            (S *)c.ring_ki, status, LowPrecOut{p.lowprec != 0, (int64_t)p.B * p.n_cap});
     } else {
         using S = float;
         cache_append_kernel<S><<<grid, 128, 0, st>>>(
             p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
             (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
-            (S *)c.ring_ki, status);
+            (S *)c.ring_ki, status, LowPrecOut{false, 0});
     }
     count_launch();
     return check_launch();

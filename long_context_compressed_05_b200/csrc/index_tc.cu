@@ -34,6 +34,7 @@
 // over the bitmap words.
 #include <cub/block/block_scan.cuh>
 
+#include "lowprec.cuh"
 #include "tc_common.cuh"
 
 namespace hcsa {
@@ -52,7 +53,15 @@ constexpr int kBTileDec = 64 * 128;  // decode: one token, Hi <= 64 heads
 // epilogue warps: prefill 16 (four per TMEM lane quadrant, 64 columns each: the ReLU-weighted head sum
 // is the busy part), decode 8 (two groups taking alternate accumulators)
 __host__ __device__ constexpr int epi_warps(bool dec) { return dec ? 8 : 16; }
-__host__ __device__ constexpr int cta_threads(bool dec) { return 64 + 32 * epi_warps(dec); }
+// FP4 keys: converter warps (after the epilogue warps) rebuild each staged tile of E2M1 codes as the bf16
+// operand tile, one key row per thread
+__host__ __device__ constexpr int conv_warps(bool dec) { return dec ? 2 : 4; }   // decode: two CTAs per SM
+constexpr int kCodeTile = 128 * 32;   // 128 keys x 64 E2M1 codes
+__host__ __device__ constexpr int cta_threads(bool dec, bool lp = false) {
+    return 64 + 32 * epi_warps(dec) + (lp ? 32 * conv_warps(dec) : 0);
+}
+// key-tile ring stages: fewer with FP4 keys, whose staging ring also takes shared memory
+__host__ __device__ constexpr int ring_stages(bool dec, bool lp) { return dec ? (lp ? 3 : kNSDec) : (lp ? 6 : kNS); }
 
 struct Args {
     int64_t rows;        // prefill: T; decode: B
@@ -69,6 +78,10 @@ struct Args {
     int64_t tps;         // decode: key tiles per sequence (ceil(N / 128))
     int *status;
     uint32_t *bound;     // prefill, or nullptr: per row a lower bound of the order key of its k-th best score
+    // FP4 keys: code pairs [key_rows][32] then int8 exponents [key_rows][2]
+    const uint8_t *codes;
+    const int8_t *kexp;
+    int64_t key_rows;
 };
 
 struct Unit {
@@ -132,29 +145,35 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
     return false;
 }
 
-template <int HI, bool DEC>
-__global__ void __launch_bounds__(cta_threads(DEC), DEC ? kDecCtasPerSm : 1)
+template <int HI, bool DEC, bool LP>
+__global__ void __launch_bounds__(cta_threads(DEC, LP), DEC ? kDecCtasPerSm : 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
                        Args a) {
     // decode: key tiles that share one 128-column TMEM accumulator (Hi columns each)
     constexpr int kTPB = 128 / HI < 4 ? 128 / HI : 4;
     constexpr int kEpiWarps = epi_warps(DEC), kEpiThreads = 32 * kEpiWarps, kGroups = kEpiWarps / 4;
-    constexpr int NS = DEC ? kNSDec : kNS;
+    constexpr int NS = ring_stages(DEC, LP);
     constexpr int BT = DEC ? kBTileDec : kBTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;                       // NS x 16 KB
     uint8_t *sB = sA + NS * kATile;           // 2 x BT
     float *sw = reinterpret_cast<float *>(sB + 2 * BT);   // prefill: 2 x 256 head weights
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sw + (DEC ? 0 : 512));
+    uint8_t *sK8 = reinterpret_cast<uint8_t *>(sw + (DEC ? 0 : 512));   // FP4 keys: NS x 4 KB of staged codes
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sK8 + (LP ? NS * kCodeTile : 0));
     uint64_t *a_full = bars, *a_empty = bars + NS, *b_full = bars + 2 * NS, *b_empty = b_full + 2;
     uint64_t *acc_full = b_empty + 2, *acc_empty = acc_full + 4;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 4);
+    uint64_t *c_full = acc_empty + 4;         // FP4 keys: codes of stage s landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + (LP ? NS : 0));
     uint32_t *shist = tmem_slot + 4;          // decode: [4096] key-bit histogram of the current unit
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; ++i) { tc::mbar_init(&a_full[i], 1); tc::mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < NS; ++i) {
+            tc::mbar_init(&a_full[i], LP ? conv_warps(DEC) : 1);
+            tc::mbar_init(&a_empty[i], 1);
+            if (LP) tc::mbar_init(&c_full[i], 1);
+        }
         for (int i = 0; i < 2; ++i) { tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1); }
         for (int i = 0; i < 4; ++i) { tc::mbar_init(&acc_full[i], 1); tc::mbar_init(&acc_empty[i], kEpiThreads / 32); }
         tc::fence_mbar_init();
@@ -181,8 +200,18 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
                     const int s = ia % NS;
                     if (ia >= NS) ok = ok && tc::mbar_wait(&a_empty[s], ((ia / NS) - 1) & 1, a.status);
-                    tc::mbar_arrive_expect_tx(&a_full[s], kATile);
-                    tc::tma_load_3d(tc::smem_u32(sA + s * kATile), &tm_keys, 0, kt * 128, (int)x.b, &a_full[s]);
+                    if (!ok) break;
+                    if (LP) {
+                        // the tile's codes: 128 consecutive key rows, cut at the end of the array
+                        const int64_t r0 = x.b * a.N + (int64_t)kt * 128;
+                        const int64_t nr = a.key_rows - r0 < 128 ? a.key_rows - r0 : 128;
+                        tc::mbar_arrive_expect_tx(&c_full[s], (uint32_t)nr * 32);
+                        tc::bulk_load(tc::smem_u32(sK8 + s * kCodeTile), a.codes + r0 * 32, (uint32_t)nr * 32,
+                                      &c_full[s]);
+                    } else {
+                        tc::mbar_arrive_expect_tx(&a_full[s], kATile);
+                        tc::tma_load_3d(tc::smem_u32(sA + s * kATile), &tm_keys, 0, kt * 128, (int)x.b, &a_full[s]);
+                    }
                 }
             }
         }
@@ -206,6 +235,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                         const int s0 = ia % NS, s1 = (ia + 1) % NS, ab = iacc % a.nbuf;
                         ok = ok && tc::mbar_wait(&a_full[s0], (ia / NS) & 1, a.status);
                         if (two) ok = ok && tc::mbar_wait(&a_full[s1], ((ia + 1) / NS) & 1, a.status);
+                        if (LP) tc::fence_async_smem();   // converter writes (generic proxy) -> MMA
                         if (slot == 0 && iacc >= (uint32_t)a.nbuf)
                             ok = ok && tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
                         tc::tc_fence_after();
@@ -234,6 +264,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
                     const int s = ia % NS, ab = iacc % a.nbuf;
                     ok = ok && tc::mbar_wait(&a_full[s], (ia / NS) & 1, a.status);
+                    if (LP) tc::fence_async_smem();   // converter writes (generic proxy) -> MMA
                     if (iacc >= (uint32_t)a.nbuf)
                         ok = ok && tc::mbar_wait(&acc_empty[ab], ((iacc / a.nbuf) - 1) & 1, a.status);
                     tc::tc_fence_after();
@@ -248,6 +279,43 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 }
                 tc::mma_commit(&b_empty[bb]);
                 ++ib;
+            }
+        }
+    } else if (LP && warp >= 2 + kEpiWarps) {
+        // ------------------------------------------------ FP4 keys: staged codes -> bf16 operand tile
+        // One key row per thread: 32 code bytes (64 E2M1 values) and the row's two block exponents become
+        // the row's 128-byte swizzled bf16 line (exact: every stored key is a bf16 number).
+        constexpr int kConvThreads = 32 * conv_warps(DEC);
+        const int ct = threadIdx.x - 32 * (2 + kEpiWarps);   // 0 .. kConvThreads - 1
+        uint32_t ia = 0;
+        Unit x;
+        for (Iter it = iter_begin(a); ok && iter_next(a, it, x);) {
+            for (int kt = x.kt0; kt < x.kt1 && ok; ++kt, ++ia) {
+                const int s = ia % NS;
+                ok = ok && tc::mbar_wait(&c_full[s], (ia / NS) & 1, a.status);
+                if (!ok) break;
+                uint8_t *dst = sA + s * kATile;
+#pragma unroll
+                for (int kr = ct; kr < 128; kr += kConvThreads) {   // key row of the tile
+                    const int64_t row = x.b * a.N + (int64_t)kt * 128 + kr;
+                    int e0 = 0, e1 = 0;
+                    if (row < a.key_rows) {
+                        e0 = a.kexp[row * 2];
+                        e1 = a.kexp[row * 2 + 1];
+                    }
+                    const uint4 *src = reinterpret_cast<const uint4 *>(sK8 + s * kCodeTile + kr * 32);
+                    const uint4 c01 = src[0], c23 = src[1];
+                    const uint32_t cw[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
+                    const float s0 = lp::pow2f(e0), s1 = lp::pow2f(e1);
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {   // 16-byte chunk g = channels 8 g .. 8 g + 7
+                        const uint4 v = lp::fp4x8_to_bf16x8(cw[g], g < 4 ? s0 : s1);
+                        *reinterpret_cast<uint4 *>(dst + tc::sw128_offset((uint32_t)kr, (uint32_t)g)) = v;
+                    }
+                }
+                tc::fence_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&a_full[s]);
             }
         }
     } else if (DEC) {
@@ -942,18 +1010,19 @@ static int num_sms() {
     return n;
 }
 
-template <int HI, bool DEC>
+template <int HI, bool DEC, bool LP>
 static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, const CUtensorMap &tq, Args a,
                                  cudaStream_t st) {
-    constexpr int NS = DEC ? kNSDec : kNS;
+    constexpr int NS = ring_stages(DEC, LP);
     constexpr size_t smem = 1024 + NS * kATile + 2 * (DEC ? kBTileDec : kBTile) + (DEC ? 0 : 512 * sizeof(float)) +
-                            (2 * NS + 12) * sizeof(uint64_t) + 16 + (DEC ? 4096 * sizeof(uint32_t) : 128 * sizeof(uint32_t));
+                            (LP ? NS * kCodeTile : 0) + (3 * NS + 12) * sizeof(uint64_t) + 16 +
+                            (DEC ? 4096 * sizeof(uint32_t) : 128 * sizeof(uint32_t));
     static_assert(smem <= 232448, "shared memory per CTA");
     static bool configured[64] = {};   // kernel attributes are set per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(index_scores_tc_kernel<HI, DEC, LP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess)
             return HCSA_ERR_CUDA;
         configured[dev] = true;
@@ -961,9 +1030,27 @@ static hcsa_status launch_scores(const IndexArgs &ia, const CUtensorMap &tk, con
     const int64_t slots = (int64_t)num_sms() * (DEC ? kDecCtasPerSm : 1);
     const int64_t grid = a.n_units < slots ? a.n_units : slots;
     if (grid <= 0) return HCSA_OK;
-    index_scores_tc_kernel<HI, DEC><<<(unsigned)grid, cta_threads(DEC), smem, st>>>(tk, tq, a);
+    index_scores_tc_kernel<HI, DEC, LP><<<(unsigned)grid, cta_threads(DEC, LP), smem, st>>>(tk, tq, a);
     count_launch();
     return check_launch();
+}
+
+template <bool LP>
+static hcsa_status dispatch_scores(const IndexArgs &ia, bool decode, const CUtensorMap &tk, const CUtensorMap &tq,
+                                   const Args &a, cudaStream_t st) {
+    if (decode) {
+        switch (ia.Hi) {
+            case 16: return launch_scores<16, true, LP>(ia, tk, tq, a, st);
+            case 32: return launch_scores<32, true, LP>(ia, tk, tq, a, st);
+            default: return launch_scores<64, true, LP>(ia, tk, tq, a, st);
+        }
+    }
+    switch (ia.Hi) {
+        case 8: return launch_scores<8, false, LP>(ia, tk, tq, a, st);
+        case 16: return launch_scores<16, false, LP>(ia, tk, tq, a, st);
+        case 32: return launch_scores<32, false, LP>(ia, tk, tq, a, st);
+        default: return launch_scores<64, false, LP>(ia, tk, tq, a, st);
+    }
 }
 
 hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
@@ -975,17 +1062,26 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
     // rows read as zeros, so a row-range caller need not have gathered them)
     const int64_t last_vis = ia.row1 > 0 ? (ia.row1 - 1) / ia.m : 0;
     const uint64_t key_rows = decode ? (uint64_t)ia.N : (uint64_t)std::max<int64_t>(1, std::min<int64_t>(ia.N, last_vis));
-    if (!make_tmap_bf16_3d(&tk, ia.keys, 64, key_rows, (uint64_t)nseq, 128, (uint64_t)ia.N * 128, 64, 128, 1,
-                           true))
-        return HCSA_ERR_CUDA;
     if (!make_tmap_bf16_3d(&tq_map, ia.qi, 64, (uint64_t)ia.Hi, (uint64_t)ia.rows, 128, (uint64_t)ia.ld_qi * 2, 64,
                            (uint32_t)ia.Hi, (uint32_t)tq, true))
         return HCSA_ERR_CUDA;
+    if (ia.lowprec) {
+        tk = tq_map;   // unused: FP4 key tiles are bulk copies of their code rows
+    } else if (!make_tmap_bf16_3d(&tk, ia.keys, 64, key_rows, (uint64_t)nseq, 128, (uint64_t)ia.N * 128, 64, 128, 1,
+                                  true)) {
+        return HCSA_ERR_CUDA;
+    }
     Args a{};
     a.rows = ia.rows; a.N = ia.N; a.m = ia.m; a.tq = tq; a.ncols = tq * ia.Hi; a.decode = decode; a.pos = ia.pos;
     a.nbuf = 2;                                   // prefill: 2 x 256 columns; decode: 2 x 128 columns
     a.stride = a.ncols <= 128 ? 128 : 256;
     a.w = (const __nv_bfloat16 *)ia.w; a.ld_w = ia.ld_w; a.scores = (float *)ia.ws; a.status = device_status_ptr();
+    if (ia.lowprec) {
+        // code rows [nseq * N][32], then their exponents; prefill loads stop at the range's last visible key
+        a.codes = (const uint8_t *)ia.keys;
+        a.kexp = (const int8_t *)(a.codes + nseq * ia.N * 32);
+        a.key_rows = decode ? nseq * ia.N : (int64_t)key_rows;
+    }
     // long decode rows: multi-CTA select, whose histogram the scores kernel fills; scratch after the scores
     const bool rows_path = ia.N > 32768 && topk_rows_supported(ia);
     uint8_t *scratch = (uint8_t *)ia.ws + (((size_t)ia.rows * ia.N * sizeof(float) + 255) & ~(size_t)255);
@@ -1008,21 +1104,8 @@ hcsa_status launch_index_tc(const IndexArgs &ia, cudaStream_t st) {
         a.n_units = a.n_qtiles - ia.row0 / tq;
         a.tps = 0;
     }
-    hcsa_status s;
-    if (decode) {
-        switch (ia.Hi) {
-            case 16: s = launch_scores<16, true>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, true>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, true>(ia, tk, tq_map, a, st); break;
-        }
-    } else {
-        switch (ia.Hi) {
-            case 8: s = launch_scores<8, false>(ia, tk, tq_map, a, st); break;
-            case 16: s = launch_scores<16, false>(ia, tk, tq_map, a, st); break;
-            case 32: s = launch_scores<32, false>(ia, tk, tq_map, a, st); break;
-            default: s = launch_scores<64, false>(ia, tk, tq_map, a, st); break;
-        }
-    }
+    hcsa_status s = ia.lowprec ? dispatch_scores<true>(ia, decode, tk, tq_map, a, st)
+                               : dispatch_scores<false>(ia, decode, tk, tq_map, a, st);
     if (s != HCSA_OK) return s;
     // top-k over the materialised scores
     const int64_t nrows = ia.row1 - ia.row0;

@@ -189,6 +189,7 @@ hcsa_status launch_topk_generic(const IndexArgs &a, cudaStream_t st) {
 hcsa_status launch_index_topk(const IndexArgs &a, cudaStream_t st) {
     if (a.rows == 0) return HCSA_OK;
     if (index_tc_supported(a)) return launch_index_tc(a, st);
+    if (a.lowprec) return HCSA_ERR_UNSUPPORTED;   // FP4 keys: tensor-core shapes only
     // CUDA-core scores + generic select: the scores are materialised in the workspace
     if (a.ws_bytes < index_topk_ws_bytes(a.dtype, a.rows, a.N)) return HCSA_ERR_WORKSPACE;
     const int qt = a.pos ? 1 : kQT;

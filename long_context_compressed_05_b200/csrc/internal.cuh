@@ -69,7 +69,11 @@ hcsa_status check_launch();         // maps cudaGetLastError() to a status
 // are truncated to the sequence [0, T) and read kv / g / ki by global token index
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
-                            void *entries, void *idx_keys, int64_t j0, int64_t j1, cudaStream_t st);
+                            void *entries, void *idx_keys, int64_t j0, int64_t j1, bool lowprec, int64_t rows,
+                            cudaStream_t st);
+
+// bf16 rows [rows, ch] -> block-scaled FP8 (keys = false) or FP4 (keys = true) storage
+hcsa_status launch_quantize_rows(const void *src, int64_t rows, int ch, bool keys, void *dst, cudaStream_t st);
 
 hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cache &c, const int32_t *pos,
                                 const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
@@ -90,6 +94,7 @@ struct IndexArgs {
     void *ws; size_t ws_bytes;
     const int32_t *only_rows;   // if set: the generic select handles only rows r with only_rows[4 r + 3] != 0
     int64_t row0, row1;         // query rows computed (prefill row range; decode: 0, rows)
+    bool lowprec;               // keys: E2M1 code pairs [rows][di / 2], then int8 exponents [rows][di / 32]
 };
 size_t index_topk_ws_bytes(int dtype, int64_t rows, int64_t N);
 // multi-CTA exact top-k for long decode rows (N > 32768); scratch after the scores.  The scratch starts
@@ -131,6 +136,7 @@ struct AttendArgs {
     void *out;
     void *ws; size_t ws_bytes;
     int64_t row0, row1;              // query rows computed (prefill row range; decode: 0, rows)
+    bool lowprec;                    // entries: E4M3 codes [rows][C], then int8 exponents [rows][C / 32]
 };
 size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, int dh, int topk, int window,
                        int64_t N);

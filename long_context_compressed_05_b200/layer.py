@@ -16,13 +16,13 @@ def torch_dtype(dtype: str):
     return torch.bfloat16 if dtype == "bf16" else torch.float32
 
 
-def params_for(spec, *, T=None, B=1, n_cap=0, row0=0, row1=0) -> L.Params:
+def params_for(spec, *, T=None, B=1, n_cap=0, row0=0, row1=0, lowprec=False) -> L.Params:
     """Params from any object with the layer fields (kind, D, m, width, C, di, Hi, topk, window, H, dh, scale, dtype).
-    row0 / row1: the prefill row range (both 0: the whole sequence)."""
+    row0 / row1: the prefill row range (both 0: the whole sequence).  lowprec: FP8 entries, FP4 indexer keys."""
     return L.make_params(T=spec.T if T is None else T, D=spec.D, m=spec.m, width=spec.width, C=spec.C,
                          di=getattr(spec, "di", 0), Hi=getattr(spec, "Hi", 0), topk=getattr(spec, "topk", 0),
                          window=spec.window, H=spec.H, dh=spec.dh, scale=spec.scale, dtype=spec.dtype, B=B,
-                         n_cap=n_cap, row0=row0, row1=row1)
+                         n_cap=n_cap, row0=row0, row1=row1, lowprec=lowprec)
 
 
 def _col_offsets(spec):
@@ -40,21 +40,25 @@ def _col_offsets(spec):
 class PrefillLayer:
     """One CSA or HCA layer over a sequence of T tokens, buffers allocated once."""
 
-    def __init__(self, spec, device="cuda"):
+    def __init__(self, spec, device="cuda", lowprec=False):
         self.spec = spec
         self.csa = spec.kind == "csa"
         self.kind = L.KIND_CSA if self.csa else L.KIND_HCA
-        self.p = params_for(spec)
+        self.lowprec = lowprec
+        self.p = params_for(spec, lowprec=lowprec)
         dt = torch_dtype(spec.dtype)
         T, N = spec.T, -(-spec.T // spec.m)
         self.cols, ncols = _col_offsets(spec)
         assert ncols == L.hcsa_proj_cols(self.p, self.kind)
         self.y = torch.empty((T, ncols), dtype=dt, device=device)
-        self.entries = torch.empty((N, spec.C), dtype=dt, device=device)
+        # FP8 / FP4 storage: byte arrays of codes followed by the block exponents
+        self.entries = (torch.empty(L.hcsa_entry_bytes(self.p, N), dtype=torch.uint8, device=device) if lowprec
+                        else torch.empty((N, spec.C), dtype=dt, device=device))
         self.out = torch.empty((T, spec.H * spec.dh), dtype=dt, device=device)
         self.ws_proj = self._ws(L.OP_PROJECT, device)
         if self.csa:
-            self.idx_keys = torch.empty((N, spec.di), dtype=dt, device=device)
+            self.idx_keys = (torch.empty(L.hcsa_key_bytes(self.p, N), dtype=torch.uint8, device=device) if lowprec
+                             else torch.empty((N, spec.di), dtype=dt, device=device))
             self.sel = torch.empty((T, spec.topk), dtype=torch.int32, device=device)
             self.ws_index = self._ws(L.OP_CSA_INDEX_TOPK, device)
             self.ws_attend = self._ws(L.OP_CSA_ATTEND, device)
@@ -101,11 +105,14 @@ class PrefillLayer:
 class DecodeLayer:
     """One layer's decode step for B sequences over a caller-provided cache."""
 
-    def __init__(self, spec, B, n_cap, cache: dict, device="cuda"):
+    def __init__(self, spec, B, n_cap, cache: dict, device="cuda", lowprec=False):
+        """cache: device tensors entries, win_kv, ring_g (+ idx_keys, ring_ki for CSA); with lowprec the
+        entries and idx_keys are byte arrays in the FP8 / FP4 layout (hcsa_quantize_rows converts bf16 rows)."""
         self.spec = spec
         self.csa = spec.kind == "csa"
         self.kind = L.KIND_CSA if self.csa else L.KIND_HCA
-        self.p = params_for(spec, T=0, B=B, n_cap=n_cap)
+        self.lowprec = lowprec
+        self.p = params_for(spec, T=0, B=B, n_cap=n_cap, lowprec=lowprec)
         dt = torch_dtype(spec.dtype)
         self.cols, ncols = _col_offsets(spec)
         self.cache_t = cache
