@@ -112,6 +112,13 @@ typedef struct {
      * shapes: di = 64; H = 64, dh = 512 for the attention) and hca_decode_attend (same shape);
      * hca_attend and the fp32 / CUDA-core paths return HCSA_ERR_UNSUPPORTED. */
     int32_t lowprec;
+    /* Entry-sharded decode (a cache too large for one GPU split by entry index over ranks; the split of
+     * the decode path is that of the CSA / HCA sections of the KV-cache page).  ent_shard = 1: the decode cache holds entries [ent0, ent0 + n_cap) of
+     * each sequence (row b * n_cap + j - ent0); hcsa_cache_append writes a formed entry only when it
+     * falls in that range, and the *_shard calls below work on it.  0 (the default): the cache holds
+     * entries [0, n_cap) and ent0 must be 0. */
+    int32_t ent0;
+    int32_t ent_shard;
 } hcsa_params;
 
 /* Decode cache of one layer (device pointers, caller-owned).
@@ -138,7 +145,10 @@ typedef enum {
     HCSA_OP_HCA_ATTEND = 3,
     HCSA_OP_CSA_DECODE_INDEX_TOPK = 4,
     HCSA_OP_CSA_DECODE_ATTEND = 5,
-    HCSA_OP_HCA_DECODE_ATTEND = 6
+    HCSA_OP_HCA_DECODE_ATTEND = 6,
+    HCSA_OP_CSA_DECODE_INDEX_TOPK_SHARD = 7,
+    HCSA_OP_CSA_DECODE_ATTEND_SHARD = 8,
+    HCSA_OP_HCA_DECODE_ATTEND_SHARD = 9
 } hcsa_op;
 
 /* Library version (major * 10000 + minor * 100 + patch). */
@@ -262,6 +272,48 @@ hcsa_status csa_decode_attend(const hcsa_params *p, const hcsa_cache *cache, con
 /* Decode: HCA attention over entries j < pos[b] / m and the raw window. */
 hcsa_status hca_decode_attend(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
                               int64_t ld_q, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* ---- entry-sharded decode (p->ent_shard = 1; the cache is one shard: entries [ent0, ent0 + n_cap)).
+ * A step: every shard runs csa_decode_index_topk_shard; the ranks all-gather (sel, sel_scores); every
+ * rank runs csa_topk_merge (the exact global top-k: each global top-k entry is in its own shard's top-k),
+ * then csa_decode_attend_shard (or hca_decode_attend_shard) on its shard; the ranks all-gather the
+ * partials and hcsa_merge_partials combines them.  Tensor-core shapes only (di = 64; H = 64, dh = 512,
+ * C = 1024, window 128), bf16 storage; others return HCSA_ERR_UNSUPPORTED.
+ *
+ * Partial layout (part): acc [B, H, dh] fp32 (the unnormalized softmax-weighted value sum), then
+ * ml [B, H, 2] fp32 (max logit in natural units, sum of exp(logit - max)); a head with no key has
+ * max = -inf and sum = 0.  B * H * (dh + 2) floats. */
+
+/* Indexer + exact top-k over the shard's visible entries (global j < pos[b] / m); sel [B, topk] gets
+ * global indices in ascending order (-1 padding), sel_scores [B, topk] their scores (-inf padding).
+ * ws: hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK_SHARD). */
+hcsa_status csa_decode_index_topk_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                        const void *qi, int64_t ld_qi, const void *w, int64_t ld_w, int32_t *sel,
+                                        float *sel_scores, void *ws, size_t ws_bytes, void *stream);
+
+/* Exact top-k (p->topk) of n_cand candidates per row (B = p->B rows): cand_sel [B, n_cand] indices (-1:
+ * none), cand_scores [B, n_cand]; the k best by (score desc, index asc), emitted in ascending index order
+ * into sel [B, topk] (-1 padding).  n_cand <= 8192.  Candidates must be distinct per row. */
+hcsa_status csa_topk_merge(const hcsa_params *p, const int32_t *cand_sel, const float *cand_scores, int32_t n_cand,
+                           int32_t *sel, void *stream);
+
+/* Attention over the entries of sel [B, topk] (global indices) that this shard holds, plus the raw window
+ * when with_window != 0 (exactly one shard attends it); writes the partial (layout above).
+ * ws: hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_ATTEND_SHARD). */
+hcsa_status csa_decode_attend_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                                    int64_t ld_q, const int32_t *sel, int32_t with_window, float *part, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/* HCA: attention over the shard's visible entries (global j < pos[b] / m) plus the window when
+ * with_window != 0; writes the partial.  ws: hcsa_workspace_bytes(p, HCSA_OP_HCA_DECODE_ATTEND_SHARD). */
+hcsa_status hca_decode_attend_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                                    int64_t ld_q, int32_t with_window, float *part, void *ws, size_t ws_bytes,
+                                    void *stream);
+
+/* Log-sum-exp merge of n_parts partials (consecutive blocks of B * H * (dh + 2) floats) into the output
+ * out [B, ld_out] bf16 (out[b, h * dh + d]). */
+hcsa_status hcsa_merge_partials(const hcsa_params *p, const float *parts, int32_t n_parts, void *out,
+                                int64_t ld_out, void *stream);
 
 /* Decode: csa_decode_index_topk without a caller workspace, for callers that cannot allocate
  * device memory (for example code inside a serving engine or host framework that owns every

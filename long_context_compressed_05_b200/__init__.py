@@ -7,4 +7,4 @@ allocate device buffers with torch and issue the calls in order.
 from ._lib import *  # noqa: F401,F403
 from ._lib import EXPORTS, HcsaError, load, make_cache, make_params  # noqa: F401
 from .layer import DecodeLayer, PrefillLayer, params_for, torch_dtype  # noqa: F401
-from .sharded import ShardedPrefillLayer, entry_range, zigzag_chunks  # noqa: F401
+from .sharded import ShardedDecodeLayer, ShardedPrefillLayer, entry_range, shard_cache, zigzag_chunks  # noqa: F401

@@ -18,6 +18,7 @@ HCSA_F32, HCSA_BF16 = 0, 1
 KIND_CSA, KIND_HCA = 0, 1
 OP_PROJECT, OP_CSA_INDEX_TOPK, OP_CSA_ATTEND, OP_HCA_ATTEND = 0, 1, 2, 3
 OP_CSA_DECODE_INDEX_TOPK, OP_CSA_DECODE_ATTEND, OP_HCA_DECODE_ATTEND = 4, 5, 6
+OP_CSA_DECODE_INDEX_TOPK_SHARD, OP_CSA_DECODE_ATTEND_SHARD, OP_HCA_DECODE_ATTEND_SHARD = 7, 8, 9
 
 STATUS = {0: "HCSA_OK", 1: "HCSA_ERR_NULL", 2: "HCSA_ERR_SHAPE", 3: "HCSA_ERR_DTYPE", 4: "HCSA_ERR_ALIGN",
           5: "HCSA_ERR_WORKSPACE", 6: "HCSA_ERR_CUDA", 7: "HCSA_ERR_TIMEOUT", 8: "HCSA_ERR_UNSUPPORTED",
@@ -29,7 +30,9 @@ EXPORTS = ["hcsa_version", "hcsa_status_string", "hcsa_workspace_bytes", "hcsa_p
            "csa_compress", "hca_compress", "csa_index_topk", "csa_attend", "hca_attend", "hcsa_cache_append",
            "csa_decode_index_topk", "csa_decode_attend", "hca_decode_attend", "csa_decode_index_topk_noalloc",
            "hcsa_get_device_status", "hcsa_selftest_wait_timeout",
-           "hcsa_launch_count", "hcsa_entry_bytes", "hcsa_key_bytes", "hcsa_quantize_rows"]
+           "hcsa_launch_count", "hcsa_entry_bytes", "hcsa_key_bytes", "hcsa_quantize_rows",
+           "csa_decode_index_topk_shard", "csa_topk_merge", "csa_decode_attend_shard", "hca_decode_attend_shard",
+           "hcsa_merge_partials"]
 STORE_ENTRIES, STORE_KEYS = 0, 1
 
 
@@ -43,7 +46,8 @@ class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "T", "D", "m", "width", "C", "di", "Hi", "topk", "window",
                                               "H", "dh")] + [("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
                                                              ("n_cap", ctypes.c_int32), ("row0", ctypes.c_int32),
-                                                             ("row1", ctypes.c_int32), ("lowprec", ctypes.c_int32)]
+                                                             ("row1", ctypes.c_int32), ("lowprec", ctypes.c_int32),
+                                                             ("ent0", ctypes.c_int32), ("ent_shard", ctypes.c_int32)]
 
 
 class Cache(ctypes.Structure):
@@ -87,6 +91,11 @@ def load():
         "hcsa_entry_bytes": (SZ, [P, I64]),
         "hcsa_key_bytes": (SZ, [P, I64]),
         "hcsa_quantize_rows": (I32, [P, I32, V, I64, V, V]),
+        "csa_decode_index_topk_shard": (I32, [P, CP, V, V, I64, V, I64, V, V, V, SZ, V]),
+        "csa_topk_merge": (I32, [P, V, V, I32, V, V]),
+        "csa_decode_attend_shard": (I32, [P, CP, V, V, I64, V, I32, V, V, SZ, V]),
+        "hca_decode_attend_shard": (I32, [P, CP, V, V, I64, I32, V, V, SZ, V]),
+        "hcsa_merge_partials": (I32, [P, V, I32, V, I64, V]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -116,10 +125,10 @@ def _stream(stream):
 
 
 def make_params(*, T=0, D=0, m=4, width=8, C=0, di=0, Hi=0, topk=0, window=128, H=1, dh=0, scale=1.0,
-                dtype="bf16", B=1, n_cap=0, row0=0, row1=0, lowprec=0) -> Params:
+                dtype="bf16", B=1, n_cap=0, row0=0, row1=0, lowprec=0, ent0=0, ent_shard=0) -> Params:
     return Params(B=B, T=T, D=D, m=m, width=width, C=C, di=di, Hi=Hi, topk=topk, window=window, H=H, dh=dh,
                   scale=scale, dtype=HCSA_BF16 if dtype == "bf16" else HCSA_F32, n_cap=n_cap, row0=row0,
-                  row1=row1, lowprec=int(lowprec))
+                  row1=row1, lowprec=int(lowprec), ent0=ent0, ent_shard=int(ent_shard))
 
 
 def make_cache(entries, win_kv, ring_g, idx_keys=None, ring_ki=None) -> Cache:
@@ -239,6 +248,36 @@ def hcsa_quantize_rows(p, what, src, dst, stream=None):
     """src: [rows, C] (entries) or [rows, di] (keys) bf16; dst: a byte buffer of the matching size."""
     _check("hcsa_quantize_rows", load().hcsa_quantize_rows(ctypes.byref(p), what, _ptr(src), src.shape[0],
                                                            _ptr(dst), _stream(stream)))
+
+
+def csa_decode_index_topk_shard(p, cache: Cache, pos, qi, w, sel, sel_scores, ws, stream=None):
+    _check("csa_decode_index_topk_shard", load().csa_decode_index_topk_shard(
+        ctypes.byref(p), ctypes.byref(cache), _ptr(pos), _ptr(qi), _ld(qi), _ptr(w), _ld(w), _ptr(sel),
+        _ptr(sel_scores), _ptr(ws), _wsz(ws), _stream(stream)))
+
+
+def csa_topk_merge(p, cand_sel, cand_scores, sel, stream=None):
+    """cand_sel / cand_scores: [B, n_cand] (one row per sequence); sel: [B, topk]."""
+    _check("csa_topk_merge", load().csa_topk_merge(ctypes.byref(p), _ptr(cand_sel), _ptr(cand_scores),
+                                                   cand_sel.shape[1], _ptr(sel), _stream(stream)))
+
+
+def csa_decode_attend_shard(p, cache: Cache, pos, q, sel, with_window, part, ws=None, stream=None):
+    _check("csa_decode_attend_shard", load().csa_decode_attend_shard(
+        ctypes.byref(p), ctypes.byref(cache), _ptr(pos), _ptr(q), _ld(q), _ptr(sel), int(with_window), _ptr(part),
+        _ptr(ws), _wsz(ws), _stream(stream)))
+
+
+def hca_decode_attend_shard(p, cache: Cache, pos, q, with_window, part, ws=None, stream=None):
+    _check("hca_decode_attend_shard", load().hca_decode_attend_shard(
+        ctypes.byref(p), ctypes.byref(cache), _ptr(pos), _ptr(q), _ld(q), int(with_window), _ptr(part), _ptr(ws),
+        _wsz(ws), _stream(stream)))
+
+
+def hcsa_merge_partials(p, parts, n_parts, out, stream=None):
+    """parts: n_parts consecutive partial blocks of B * H * (dh + 2) floats; out: [B, H * dh]."""
+    _check("hcsa_merge_partials", load().hcsa_merge_partials(ctypes.byref(p), _ptr(parts), n_parts, _ptr(out),
+                                                             _ld(out), _stream(stream)))
 
 
 def hcsa_launch_count(reset: bool = False) -> int:

@@ -71,6 +71,8 @@ hcsa_status check_csa(const hcsa_params *p) {
 
 hcsa_status check_decode(const hcsa_params *p, const hcsa_cache *c, const int32_t *pos, bool csa) {
     if (!c || !pos || !c->entries || !c->win_kv || !c->ring_g) return HCSA_ERR_NULL;
+    if (p->ent0 < 0 || (p->ent_shard != 0 && p->ent_shard != 1) || (!p->ent_shard && p->ent0 != 0))
+        return HCSA_ERR_SHAPE;
     if (csa && (!c->idx_keys || !c->ring_ki)) return HCSA_ERR_NULL;
     if (p->B < 1 || p->n_cap < 1 || p->window < p->width) return HCSA_ERR_SHAPE;
     if (!aligned(c->entries) || !aligned(c->win_kv) || !aligned(c->ring_g) || !aligned(pos)) return HCSA_ERR_ALIGN;
@@ -79,6 +81,13 @@ hcsa_status check_decode(const hcsa_params *p, const hcsa_cache *c, const int32_
 }
 
 int64_t n_entries(const hcsa_params *p) { return ((int64_t)p->T + p->m - 1) / p->m; }
+
+size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// segment partials of a sharded decode attention (before their merge into the caller's partial)
+size_t shard_part_ws(const hcsa_params *p, bool dense) {
+    return attend_ws_bytes(HCSA_BF16, true, dense, p->B, p->H, p->dh, dense ? 0 : p->topk, p->window, p->n_cap);
+}
 
 // Prefill row range [r0, r1) of the T query rows (both fields 0: all rows).
 hcsa_status row_range(const hcsa_params *p, int64_t *r0, int64_t *r1) {
@@ -175,6 +184,11 @@ size_t hcsa_workspace_bytes(const hcsa_params *p, int32_t op) {
                                                                p->window, p->n_cap);
         case HCSA_OP_HCA_DECODE_ATTEND: return attend_ws_bytes(p->dtype, true, true, p->B, p->H, p->dh, 0,
                                                                p->window, p->n_cap);
+        case HCSA_OP_CSA_DECODE_INDEX_TOPK_SHARD:
+            return align256(hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK)) + (size_t)p->B * sizeof(int32_t);
+        case HCSA_OP_CSA_DECODE_ATTEND_SHARD:
+            return align256((size_t)p->B * p->topk * sizeof(int32_t)) + shard_part_ws(p, false);
+        case HCSA_OP_HCA_DECODE_ATTEND_SHARD: return shard_part_ws(p, true);
     }
     return 0;
 }
@@ -354,6 +368,109 @@ hcsa_status hcsa_quantize_rows(const hcsa_params *p, int32_t what, const void *s
     if (rows < 0) return HCSA_ERR_SHAPE;
     if (!aligned(src) || !aligned(dst)) return HCSA_ERR_ALIGN;
     return launch_quantize_rows(src, rows, keys ? p->di : p->C, keys, dst, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------- entry-sharded decode
+static hcsa_status check_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, bool csa) {
+    HCSA_TRY(csa ? check_csa(p) : check_common(p));
+    HCSA_TRY(check_decode(p, cache, pos, csa));
+    if (!p->ent_shard) return HCSA_ERR_SHAPE;
+    if (p->dtype != HCSA_BF16 || p->lowprec) return HCSA_ERR_UNSUPPORTED;
+    return HCSA_OK;
+}
+
+hcsa_status csa_decode_index_topk_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
+                                        const void *qi, int64_t ld_qi, const void *w, int64_t ld_w, int32_t *sel,
+                                        float *sel_scores, void *ws, size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_shard(p, cache, pos, true));
+    HCSA_TRY(hcsa::check_decode_index_topk_args(p, cache, pos, qi, ld_qi, w, ld_w, sel));
+    if (!sel_scores) return HCSA_ERR_NULL;
+    if (!aligned(sel_scores)) return HCSA_ERR_ALIGN;
+    const size_t idx_ws = hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK);
+    if (!ws || ws_bytes < hcsa_workspace_bytes(p, HCSA_OP_CSA_DECODE_INDEX_TOPK_SHARD)) return HCSA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the shard's entries are local rows 0 .. n_cap - 1: its visible count is that at position pos - m ent0
+    int32_t *pos_l = reinterpret_cast<int32_t *>((uint8_t *)ws + align256(idx_ws));
+    HCSA_TRY(launch_shift_pos(pos, p->B, (int64_t)p->m * p->ent0, pos_l, st));
+    IndexArgs a{p->dtype, p->B, p->Hi, p->di, p->topk, p->m, p->n_cap, qi, ld_qi, w, ld_w, cache->idx_keys,
+                pos_l, sel, ws, idx_ws, nullptr, 0, p->B, false};
+    HCSA_TRY(launch_index_topk(a, st));
+    return launch_shard_finish(sel, p->B, p->topk, (const float *)ws, p->n_cap, p->ent0, sel_scores, st);
+}
+
+hcsa_status csa_topk_merge(const hcsa_params *p, const int32_t *cand_sel, const float *cand_scores, int32_t n_cand,
+                           int32_t *sel, void *stream) {
+    if (!p) return HCSA_ERR_NULL;
+    if (!cand_sel || !cand_scores || !sel) return HCSA_ERR_NULL;
+    if (p->B < 1 || p->topk < 1) return HCSA_ERR_SHAPE;
+    if (!topk_merge_supported(n_cand, p->topk)) return HCSA_ERR_UNSUPPORTED;
+    return launch_topk_merge(cand_sel, cand_scores, p->B, n_cand, p->topk, sel, (cudaStream_t)stream);
+}
+
+static hcsa_status attend_shard(const hcsa_params *p, bool dense, const hcsa_cache *cache, const int32_t *pos,
+                                const void *q, int64_t ld_q, const int32_t *sel, int32_t with_window, float *part,
+                                void *ws, size_t ws_bytes, cudaStream_t st) {
+    if (!q || !part || (!dense && !sel)) return HCSA_ERR_NULL;
+    if (!aligned(q) || !aligned(part)) return HCSA_ERR_ALIGN;
+    if (ld_q < (int64_t)p->H * p->dh) return HCSA_ERR_SHAPE;
+    const size_t need = hcsa_workspace_bytes(p, dense ? HCSA_OP_HCA_DECODE_ATTEND_SHARD : HCSA_OP_CSA_DECODE_ATTEND_SHARD);
+    if (need && (!ws || ws_bytes < need)) return HCSA_ERR_WORKSPACE;
+    AttendArgs a{};
+    a.dtype = p->dtype; a.rows = p->B; a.H = p->H; a.dh = p->dh; a.C = p->C; a.window = p->window; a.m = p->m;
+    a.topk = dense ? 0 : p->topk; a.scale = p->scale; a.dense = dense; a.N = p->n_cap;
+    a.q = q; a.ld_q = ld_q; a.kv = cache->win_kv; a.ld_kv = p->C; a.entries = cache->entries; a.pos = pos;
+    a.row0 = 0; a.row1 = p->B; a.ent0 = p->ent0; a.no_window = with_window == 0;
+    if (!attend_tc_supported(a)) return HCSA_ERR_UNSUPPORTED;
+    uint8_t *w8 = (uint8_t *)ws;
+    if (!dense) {   // the selection in the shard's local rows
+        int32_t *sel_l = reinterpret_cast<int32_t *>(w8);
+        HCSA_TRY(launch_localize_sel(sel, (int64_t)p->B * p->topk, p->ent0, p->n_cap, sel_l, st));
+        a.sel = sel_l;
+        w8 += align256((size_t)p->B * p->topk * sizeof(int32_t));
+    }
+    const int ns = attend_tc_segments(a);
+    const int64_t nacc = (int64_t)p->B * p->H * p->dh;
+    if (ns == 1) {   // one segment per row: the kernel writes the partial itself
+        a.ws = part;
+        a.ws_bytes = (size_t)(nacc + 2 * (int64_t)p->B * p->H) * sizeof(float);
+        a.partial_out = true;
+        return launch_attend_tc(a, st);
+    }
+    a.ws = w8;
+    a.ws_bytes = shard_part_ws(p, dense);
+    a.partial_out = true;
+    HCSA_TRY(launch_attend_tc(a, st));
+    const float *acc = (const float *)w8;
+    const float *ml = acc + (int64_t)p->B * ns * p->H * p->dh;
+    return launch_merge_parts(acc, ml, (int64_t)p->H * p->dh, (int64_t)ns * p->H * p->dh, p->H, (int64_t)ns * p->H,
+                              ns, p->B, p->H, p->dh, nullptr, part, part + nacc, st);
+}
+
+hcsa_status csa_decode_attend_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                                    int64_t ld_q, const int32_t *sel, int32_t with_window, float *part, void *ws,
+                                    size_t ws_bytes, void *stream) {
+    HCSA_TRY(check_shard(p, cache, pos, true));
+    if (sel && !aligned(sel)) return HCSA_ERR_ALIGN;
+    return attend_shard(p, false, cache, pos, q, ld_q, sel, with_window, part, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+hcsa_status hca_decode_attend_shard(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos, const void *q,
+                                    int64_t ld_q, int32_t with_window, float *part, void *ws, size_t ws_bytes,
+                                    void *stream) {
+    HCSA_TRY(check_shard(p, cache, pos, false));
+    return attend_shard(p, true, cache, pos, q, ld_q, nullptr, with_window, part, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+hcsa_status hcsa_merge_partials(const hcsa_params *p, const float *parts, int32_t n_parts, void *out, int64_t ld_out,
+                                void *stream) {
+    if (!p) return HCSA_ERR_NULL;
+    if (!parts || !out) return HCSA_ERR_NULL;
+    if (p->B < 1 || p->H < 1 || p->dh < 1 || n_parts < 1) return HCSA_ERR_SHAPE;
+    if (ld_out != (int64_t)p->H * p->dh) return HCSA_ERR_SHAPE;   // rows are written contiguously
+    if (!aligned(parts) || !aligned(out)) return HCSA_ERR_ALIGN;
+    const int64_t nacc = (int64_t)p->B * p->H * p->dh, blk = nacc + 2 * (int64_t)p->B * p->H;
+    return launch_merge_parts(parts, parts + nacc, blk, (int64_t)p->H * p->dh, blk / 2, p->H, n_parts, p->B, p->H,
+                              p->dh, out, nullptr, nullptr, (cudaStream_t)stream);
 }
 
 hcsa_status hcsa_get_device_status(void *stream) {

@@ -75,6 +75,8 @@ struct Params {
     float *part;         // partials: acc [nq][nseg][H][dh], then (max, sum) [nq][nseg][H][2]
     int64_t n_units;
     int64_t q0;          // first query of the row range
+    int64_t ent0;        // decode shard: global index of the cache's first entry
+    bool no_window;      // decode shard: the raw window is attended by another shard
     int *status;
 };
 
@@ -88,7 +90,10 @@ __device__ __forceinline__ Unit unit_of(const Params &a, int64_t u) {
     x.q = a.q0 + u / a.nseg;
     x.seg = (int)(u % a.nseg);
     x.p = a.decode ? (int64_t)a.pos[x.q] : x.q;
-    x.nvis = x.p < 0 ? 0 : (x.p / a.m < a.N ? x.p / a.m : a.N);
+    {   // visible entries held here: global j < p / m, local j - ent0 in [0, N)
+        int64_t v = x.p < 0 ? 0 : x.p / a.m - a.ent0;
+        x.nvis = v < 0 ? 0 : (v < a.N ? v : a.N);
+    }
     x.E = a.dense ? (int)((x.nvis + kKT - 1) / kKT) * kKT : a.topk;
     const int ntiles = x.E / kKT + 1;
     x.t0 = x.seg * a.seg_tiles;
@@ -105,7 +110,7 @@ __device__ __forceinline__ int key_row(const Params &a, const Unit &x, int kk) {
         return (int)(a.decode ? x.q * a.N + j : j);
     }
     const int64_t pp = x.p - (kKT - 1) + (kk - x.E);
-    if (pp < 0) return -1;
+    if (pp < 0 || a.no_window) return -1;
     return (int)(a.decode ? x.q * kKT + pp % kKT : pp);
 }
 
@@ -232,7 +237,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                                                         // neither padding nor visible
                     } else {
                         const int64_t pp = x.p - (kKT - 1) + (kk - x.E);
-                        if (pp >= 0) ptr = a.raw + (a.decode ? x.q * kKT + pp % kKT : pp) * a.ld_raw;
+                        if (pp >= 0 && !a.no_window) ptr = a.raw + (a.decode ? x.q * kKT + pp % kKT : pp) * a.ld_raw;
                     }
                     rp[loc] = ptr;
                 }
@@ -466,7 +471,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             const int64_t j = a.dense ? (int64_t)kk : (int64_t)jsel[t];
                             v = j >= 0 && j < x.nvis;
                         } else {
-                            v = x.p - (kKT - 1) + (kk - x.E) >= 0;
+                            v = !a.no_window && x.p - (kKT - 1) + (kk - x.E) >= 0;
                         }
                     }
                     valid[t] = v;
@@ -677,8 +682,10 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.scale = a.scale;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out = (__nv_bfloat16 *)a.out;
-    p.part = p.nseg > 1 ? (float *)a.ws : nullptr;
+    p.part = (p.nseg > 1 || a.partial_out) ? (float *)a.ws : nullptr;
     p.q0 = a.row0;
+    p.ent0 = a.ent0;
+    p.no_window = a.no_window;
     p.n_units = (a.row1 - a.row0) * p.nseg;
     p.status = device_status_ptr();
     if (p.n_units <= 0) return HCSA_OK;

@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(128) cache_append_kernel(
     int C, int m, int width, int window, int di, int64_t n_cap, const int32_t *__restrict__ pos,
     const S *__restrict__ kv_new, int64_t ld_kv, const S *__restrict__ g_new, int64_t ld_g,
     const S *__restrict__ ki_new, int64_t ld_ki, const S *__restrict__ bias, S *entries, S *idx_keys, S *win_kv,
-    S *ring_g, S *ring_ki, int *status, LowPrecOut lp) {
+    S *ring_g, S *ring_ki, int *status, LowPrecOut lp, int64_t ent0, bool shard) {
     using A = typename Traits<S>::A;
     constexpr int V = Traits<S>::VEC;
     const int b = blockIdx.y;
@@ -388,9 +388,11 @@ __global__ void __launch_bounds__(128) cache_append_kernel(
     }
     // 2) entry completion
     if ((P + 1) % m != 0) return;
-    const int64_t j = (P + 1) / m - 1;
+    const int64_t jg = (P + 1) / m - 1;   // the entry the token closes
+    if (shard && (jg < ent0 || jg >= ent0 + n_cap)) return;   // held by another shard
+    const int64_t j = jg - ent0;
     if (j >= n_cap) { report(status, kStatusBounds); return; }
-    const int64_t lo = (int64_t)m * j - (width - m);
+    const int64_t lo = (int64_t)m * jg - (width - m);
     PoolAcc<A, V> pa;
     pa.init();
     for (int64_t i = lo < 0 ? 0 : lo; i <= P; ++i) {
@@ -429,13 +431,14 @@ hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cach
         cache_append_kernel<S><<<grid, 128, 0, st>>>(
             p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
             (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
-            (S *)c.ring_ki, status, LowPrecOut{p.lowprec != 0, (int64_t)p.B * p.n_cap});
+            (S *)c.ring_ki, status, LowPrecOut{p.lowprec != 0, (int64_t)p.B * p.n_cap}, (int64_t)p.ent0,
+            p.ent_shard != 0);
     } else {
         using S = float;
         cache_append_kernel<S><<<grid, 128, 0, st>>>(
             p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
             (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
-            (S *)c.ring_ki, status, LowPrecOut{false, 0});
+            (S *)c.ring_ki, status, LowPrecOut{false, 0}, (int64_t)p.ent0, p.ent_shard != 0);
     }
     count_launch();
     return check_launch();

@@ -72,6 +72,19 @@ hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const
                             void *entries, void *idx_keys, int64_t j0, int64_t j1, bool lowprec, int64_t rows,
                             cudaStream_t st);
 
+// entry-sharded decode (shard.cu)
+hcsa_status launch_shift_pos(const int32_t *pos, int64_t B, int64_t delta, int32_t *out, cudaStream_t st);
+hcsa_status launch_shard_finish(int32_t *sel, int64_t B, int k, const float *scores, int64_t N, int64_t ent0,
+                                float *sel_scores, cudaStream_t st);
+hcsa_status launch_localize_sel(const int32_t *sel, int64_t n, int64_t ent0, int64_t n_cap, int32_t *out,
+                                cudaStream_t st);
+bool topk_merge_supported(int n_cand, int k);
+hcsa_status launch_topk_merge(const int32_t *cand_sel, const float *cand_scores, int64_t rows, int n_cand, int k,
+                              int32_t *sel, cudaStream_t st);
+hcsa_status launch_merge_parts(const float *acc, const float *ml, int64_t ss, int64_t sr, int64_t ms, int64_t mr,
+                               int n_parts, int64_t rows, int H, int dh, void *out, float *pacc, float *pml,
+                               cudaStream_t st);
+
 // bf16 rows [rows, ch] -> block-scaled FP8 (keys = false) or FP4 (keys = true) storage
 hcsa_status launch_quantize_rows(const void *src, int64_t rows, int ch, bool keys, void *dst, cudaStream_t st);
 
@@ -137,6 +150,9 @@ struct AttendArgs {
     void *ws; size_t ws_bytes;
     int64_t row0, row1;              // query rows computed (prefill row range; decode: 0, rows)
     bool lowprec;                    // entries: E4M3 codes [rows][C], then int8 exponents [rows][C / 32]
+    int64_t ent0;                    // decode shard: global index of the cache's first entry (else 0)
+    bool no_window;                  // decode shard: skip the raw window (another shard attends it)
+    bool partial_out;                // tensor-core decode: write per-segment partials to ws even for one segment
 };
 size_t attend_ws_bytes(int dtype, bool decode, bool dense, int64_t rows, int H, int dh, int topk, int window,
                        int64_t N);

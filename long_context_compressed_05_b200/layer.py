@@ -16,13 +16,13 @@ def torch_dtype(dtype: str):
     return torch.bfloat16 if dtype == "bf16" else torch.float32
 
 
-def params_for(spec, *, T=None, B=1, n_cap=0, row0=0, row1=0, lowprec=False) -> L.Params:
+def params_for(spec, *, T=None, B=1, n_cap=0, row0=0, row1=0, lowprec=False, ent0=0, ent_shard=False) -> L.Params:
     """Params from any object with the layer fields (kind, D, m, width, C, di, Hi, topk, window, H, dh, scale, dtype).
     row0 / row1: the prefill row range (both 0: the whole sequence).  lowprec: FP8 entries, FP4 indexer keys."""
     return L.make_params(T=spec.T if T is None else T, D=spec.D, m=spec.m, width=spec.width, C=spec.C,
                          di=getattr(spec, "di", 0), Hi=getattr(spec, "Hi", 0), topk=getattr(spec, "topk", 0),
                          window=spec.window, H=spec.H, dh=spec.dh, scale=spec.scale, dtype=spec.dtype, B=B,
-                         n_cap=n_cap, row0=row0, row1=row1, lowprec=lowprec)
+                         n_cap=n_cap, row0=row0, row1=row1, lowprec=lowprec, ent0=ent0, ent_shard=ent_shard)
 
 
 def _col_offsets(spec):

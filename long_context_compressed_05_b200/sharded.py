@@ -1,4 +1,6 @@
-"""Sequence-sharded prefill of one CSA / HCA layer over the ranks of a process group.
+"""Sequence-sharded prefill and entry-sharded decode of one CSA / HCA layer over the ranks of a process group.
+
+Prefill (ShardedPrefillLayer):
 
 The sequence of T tokens is cut into 2R chunks of equal length (a multiple of 128; the last one takes the
 remainder) and rank r of R takes chunks r and 2R - 1 - r: the zig-zag assignment, which gives every rank
@@ -24,9 +26,9 @@ from __future__ import annotations
 import torch
 
 from . import _lib as L
-from .layer import PrefillLayer, params_for
+from .layer import PrefillLayer, _col_offsets, params_for, torch_dtype
 
-__all__ = ["zigzag_chunks", "entry_range", "ShardedPrefillLayer"]
+__all__ = ["zigzag_chunks", "entry_range", "ShardedPrefillLayer", "ShardedDecodeLayer", "shard_cache"]
 
 ALIGN = 128   # chunk boundaries: the library's row-range granularity
 
@@ -133,3 +135,112 @@ class ShardedPrefillLayer(PrefillLayer):
         self.compute_entries(x, W_cat, bias)
         self.exchange_entries(group)
         return self.attend_local()
+
+
+# ====================================================================================================== decode
+
+def shard_cache(cache: dict, rank: int, world: int) -> dict:
+    """This rank's shard of a decode cache: entries (and indexer keys) [ent0, ent0 + n_shard) of every
+    sequence, n_shard = ceil(n_cap / world) (the last shard zero-padded); the rings are copied whole."""
+    B, n_cap = cache["entries"].shape[:2]
+    n_shard = -(-n_cap // world)
+    a, b = rank * n_shard, min((rank + 1) * n_shard, n_cap)
+    out = {}
+    for k in ("entries", "idx_keys"):
+        if k in cache:
+            t = cache[k]
+            sh = torch.zeros((B, n_shard) + tuple(t.shape[2:]), dtype=t.dtype, device=t.device)
+            if b > a:
+                sh[:, :b - a] = t[:, a:b]
+            out[k] = sh
+    for k in ("win_kv", "ring_g", "ring_ki"):
+        if k in cache:
+            out[k] = cache[k].clone()
+    return out
+
+
+class ShardedDecodeLayer:
+    """One layer's decode step for B sequences whose compressed caches are split by entry index over the
+    ranks: rank r holds entries [r n_shard, (r + 1) n_shard) of every sequence (shard_cache), every rank
+    holds the rings and the weights.  A step:
+
+      1. every rank projects the new token and appends it (the rings everywhere; a formed entry only on the
+         rank that holds it);
+      2. CSA: the indexer and an exact top-k over the rank's own entries, with their scores; one all-gather
+         of the (index, score) candidates; the exact global top-k of their union on every rank (a global
+         top-k entry is always in the top-k of its own shard);
+      3. attention over the rank's part of the keys (its selected / visible entries; the raw window on rank
+         0) as an unnormalized partial per head; one all-gather of the partials and their log-sum-exp merge.
+
+    Every step runs in libhcsa.so; torch.distributed moves the candidates and the partials."""
+
+    def __init__(self, spec, B, n_total, cache: dict, rank: int = 0, world: int = 1, device="cuda"):
+        self.spec = spec
+        self.csa = spec.kind == "csa"
+        self.kind = L.KIND_CSA if self.csa else L.KIND_HCA
+        self.rank, self.world = rank, world
+        self.n_shard = -(-n_total // world)
+        self.ent0 = rank * self.n_shard
+        self.p = params_for(spec, T=0, B=B, n_cap=self.n_shard, ent0=self.ent0, ent_shard=True)
+        self.cache_t = cache
+        self.cache = L.make_cache(cache["entries"], cache["win_kv"], cache["ring_g"], cache.get("idx_keys"),
+                                  cache.get("ring_ki"))
+        dt = torch_dtype(spec.dtype)
+        self.cols, ncols = _col_offsets(spec)
+        self.y = torch.empty((B, ncols), dtype=dt, device=device)
+        self.out = torch.empty((B, spec.H * spec.dh), dtype=dt, device=device)
+        self.part = torch.empty(B * spec.H * (spec.dh + 2), dtype=torch.float32, device=device)
+        self.ws_proj = self._ws(L.OP_PROJECT, device)
+        if self.csa:
+            self.sel_l = torch.empty((B, spec.topk), dtype=torch.int32, device=device)
+            self.score_l = torch.empty((B, spec.topk), dtype=torch.float32, device=device)
+            self.sel = torch.empty((B, spec.topk), dtype=torch.int32, device=device)
+            self.ws_index = self._ws(L.OP_CSA_DECODE_INDEX_TOPK_SHARD, device)
+            self.ws_attend = self._ws(L.OP_CSA_DECODE_ATTEND_SHARD, device)
+        else:
+            self.ws_attend = self._ws(L.OP_HCA_DECODE_ATTEND_SHARD, device)
+
+    def _ws(self, op, device):
+        n = L.hcsa_workspace_bytes(self.p, op)
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n else None
+
+    def view(self, name):
+        a, b = self.cols[name]
+        return self.y[:, a:b]
+
+    def _gather(self, t, group):
+        if self.world == 1:
+            return [t]
+        import torch.distributed as dist
+        bufs = [torch.empty_like(t) for _ in range(self.world)]
+        dist.all_gather(bufs, t.contiguous(), group=group)
+        return bufs
+
+    def select(self, group=None):
+        """Step 2: the global top-k of every sequence in self.sel."""
+        L.csa_decode_index_topk_shard(self.p, self.cache, self.pos, self.view("qi"), self.view("w"), self.sel_l,
+                                      self.score_l, self.ws_index)
+        cs = torch.cat(self._gather(self.sel_l, group), dim=1)
+        cv = torch.cat(self._gather(self.score_l, group), dim=1)
+        L.csa_topk_merge(self.p, cs, cv, self.sel)
+
+    def attend(self, group=None):
+        """Step 3: this rank's partial, the all-gather and the merge into self.out."""
+        if self.csa:
+            L.csa_decode_attend_shard(self.p, self.cache, self.pos, self.view("q"), self.sel, self.rank == 0,
+                                      self.part, self.ws_attend)
+        else:
+            L.hca_decode_attend_shard(self.p, self.cache, self.pos, self.view("q"), self.rank == 0, self.part,
+                                      self.ws_attend)
+        parts = torch.stack(self._gather(self.part, group))
+        L.hcsa_merge_partials(self.p, parts, self.world, self.out)
+        return self.out
+
+    def step(self, x, W_cat, bias, pos, group=None):
+        self.pos = pos
+        L.hcsa_project(self.p, self.kind, x, W_cat, self.y, self.ws_proj)
+        L.hcsa_cache_append(self.p, self.cache, pos, self.view("kv"), self.view("g"),
+                            self.view("ki") if self.csa else None, bias)
+        if self.csa:
+            self.select(group)
+        return self.attend(group)

@@ -119,3 +119,30 @@ def test_row_range_is_checked_before_launch(h):
                                 V(FAKE), V(FAKE), None) == 2, (r0, r1)
         assert lib.hca_attend(ctypes.byref(p), V(FAKE), 36960, V(FAKE), 36960, V(FAKE), V(FAKE), None, 0,
                               None) == 2, (r0, r1)
+
+
+def test_shard_and_lowprec_arguments_are_checked_before_launch(h):
+    lib = h.load()
+    V = ctypes.c_void_p
+    cache = h.Cache(entries=FAKE, idx_keys=FAKE, win_kv=FAKE, ring_g=FAKE, ring_ki=FAKE)
+    C = ctypes.byref(cache)
+    # a non-zero entry offset on an unsharded cache
+    p = _params(h, T=0, B=2, n_cap=1000, ent0=500)
+    assert lib.hcsa_cache_append(ctypes.byref(p), C, V(FAKE), V(FAKE), 36960, V(FAKE), 36960, V(FAKE), 36960,
+                                 V(FAKE), None) == 2
+    # the *_shard calls need a sharded cache
+    p = _params(h, T=0, B=2, n_cap=1000)
+    assert lib.csa_decode_index_topk_shard(ctypes.byref(p), C, V(FAKE), V(FAKE), 36960, V(FAKE), 36960, V(FAKE),
+                                           V(FAKE), V(FAKE), 1 << 30, None) == 2
+    # the merge: candidates per row within 8192 and at least k
+    p = _params(h, T=0, B=2, n_cap=1000)
+    assert lib.csa_topk_merge(ctypes.byref(p), V(FAKE), V(FAKE), 9000, V(FAKE), None) == 8
+    assert lib.csa_topk_merge(ctypes.byref(p), V(FAKE), V(FAKE), 100, V(FAKE), None) == 8   # fewer than k = 512
+    assert lib.hcsa_merge_partials(ctypes.byref(p), V(FAKE), 2, V(FAKE), 12345, None) == 2
+    # low precision: bf16 only, and not for the HCA prefill attention
+    p = _params(h, lowprec=1, dtype=0)
+    assert lib.hcsa_quantize_rows(ctypes.byref(p), 0, V(FAKE), 10, V(FAKE), None) == 8
+    p = _params(h, lowprec=2)
+    assert lib.hcsa_quantize_rows(ctypes.byref(p), 0, V(FAKE), 10, V(FAKE), None) == 2
+    p = _params(h, lowprec=1)
+    assert h.hcsa_entry_bytes(p, 10) == 10 * (1024 + 32) and h.hcsa_key_bytes(p, 10) == 10 * (32 + 2)
