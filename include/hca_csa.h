@@ -257,6 +257,17 @@ hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, con
                               const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
                               int64_t ld_ki, const void *bias, void *stream);
 
+/* Decode: the projection of the new tokens with the cache append done in the GEMM's epilogue (the
+ * compressor of "CSA: compresion 4x" / "HCA: compresion 128x" fed straight from the projection tile).
+ * Same results as hcsa_project followed by hcsa_cache_append: y [B, ncols] (ld ncols) is written, the
+ * rings get the new token and a closed entry is pooled into the cache (FP8 / FP4 with p->lowprec, only
+ * on its shard with p->ent_shard).  x [B, D], W_cat [D, ncols], bias [width, C].  Shapes outside the
+ * fused kernel (fp32 storage, B > 16, C not a multiple of 64, CSA with di != 64) run the two calls'
+ * kernels instead; ws as for hcsa_project. */
+hcsa_status hcsa_project_append(const hcsa_params *p, int32_t kind, const hcsa_cache *cache, const int32_t *pos,
+                                const void *x, const void *W_cat, const void *bias, void *y, void *ws, size_t ws_bytes,
+                                void *stream);
+
 /* Decode: CSA indexer + top-k for the new token of each sequence over entries j < pos[b] / m.
  *   qi [B, ld_qi], w [B, ld_w]; sel [B, topk]. */
 hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,

@@ -315,6 +315,31 @@ hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, con
                                (cudaStream_t)stream);
 }
 
+hcsa_status hcsa_project_append(const hcsa_params *p, int32_t kind, const hcsa_cache *cache, const int32_t *pos,
+                                const void *x, const void *W_cat, const void *bias, void *y, void *ws, size_t ws_bytes,
+                                void *stream) {
+    const bool csa = kind == HCSA_KIND_CSA;
+    if (kind != HCSA_KIND_CSA && kind != HCSA_KIND_HCA) return HCSA_ERR_SHAPE;
+    HCSA_TRY(csa ? check_csa(p) : check_common(p));
+    HCSA_TRY(check_decode(p, cache, pos, csa));
+    if (!x || !W_cat || !y || !bias) return HCSA_ERR_NULL;
+    if (p->D < 1) return HCSA_ERR_SHAPE;
+    if (!aligned(x) || !aligned(W_cat) || !aligned(y) || !aligned(bias)) return HCSA_ERR_ALIGN;
+    const int64_t nc = hcsa_proj_cols(p, kind);
+    if ((p->D * esize(p->dtype)) % 16 || (nc * esize(p->dtype)) % 16) return HCSA_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (project_append_supported(*p, csa))
+        return launch_project_append(*p, csa, *cache, pos, x, W_cat, nc, y, bias, st);
+    // other shapes: the projection, then the append kernel
+    if (p->dtype == HCSA_BF16 && ws && ws_bytes < project_ws_bytes(p->dtype)) return HCSA_ERR_WORKSPACE;
+    HCSA_TRY(launch_project(p->dtype, p->B, p->D, nc, x, W_cat, y, ws, ws_bytes, st));
+    const int64_t ld = nc;
+    const uint8_t *y8 = (const uint8_t *)y;
+    const int es = esize(p->dtype);
+    return launch_cache_append(p->dtype, *p, *cache, pos, y8, ld, y8 + (int64_t)p->C * es, ld,
+                               csa ? y8 + 2 * (int64_t)p->C * es : nullptr, ld, bias, st);
+}
+
 hcsa_status csa_decode_index_topk(const hcsa_params *p, const hcsa_cache *cache, const int32_t *pos,
                                   const void *qi, int64_t ld_qi, const void *w, int64_t ld_w, int32_t *sel,
                                   void *ws, size_t ws_bytes, void *stream) {

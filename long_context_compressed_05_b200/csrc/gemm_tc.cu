@@ -21,6 +21,15 @@
 // projection: 2048 columns, K = 32768), the k range is split; every split writes fp32 partials, and the
 // CTA that finishes a tile last (an atomic ticket per tile, no waiting) sums them, adds the residual
 // and rounds once.
+//
+// Decode step with the cache append in the epilogue (the compressor fed straight from the projection
+// tile).  The pooled columns are tiled in pairs: a tile's first 64 accumulator lanes hold 64 value
+// channels (kv, or the 64 indexer-key channels) and its last 64 lanes the gate channels of the same
+// index.  The gate lanes pass their bf16 values through shared memory; the value lanes then write the
+// new token into the rings and, when the token closes an entry, pool it from the rings and the tile
+// (the same online softmax as the append kernel, so the results are identical).  The other columns
+// (indexer queries, head weights, queries) are tiled as usual.
+#include "lowprec.cuh"
 #include "tc_common.cuh"
 
 namespace hcsa {
@@ -38,8 +47,9 @@ __host__ __device__ constexpr int stage_bytes(int ntok) { return 2 * kBoxW + nto
 __host__ __device__ constexpr uint32_t tmem_cols(int ntok) {
     return 2 * ntok <= 32 ? 32 : 2 * ntok <= 64 ? 64 : 2 * ntok <= 128 ? 128 : 2 * ntok <= 256 ? 256 : 512;
 }
-__host__ __device__ constexpr size_t smem_bytes(int ntok) {
-    return 1024 + (size_t)stages_for(ntok) * stage_bytes(ntok) + (2 * stages_for(ntok) + 8) * sizeof(uint64_t) + 16;
+__host__ __device__ constexpr size_t smem_bytes(int ntok, bool pool = false) {
+    return 1024 + (size_t)stages_for(ntok) * stage_bytes(ntok) + (2 * stages_for(ntok) + 8) * sizeof(uint64_t) + 16 +
+           (pool ? 64 * ntok * sizeof(float) : 0);
 }
 
 struct GemmArgs {
@@ -57,6 +67,40 @@ struct GemmArgs {
     int *tickets;              // S > 1: one arrival counter per (token tile, column tile), zero at launch
     int *status;
 };
+
+// Fused cache append (decode, S = 1): the first pool_tiles column tiles pair value and gate channels.
+struct PoolArgs {
+    int pool_tiles;            // 0: a plain GEMM
+    int plain0;                // first column of the plain tiles
+    const int32_t *pos;        // position of each row's new token
+    int C, di, m, width, window;
+    int64_t n_cap, ent0, rows_total;
+    bool shard, lowprec;
+    const __nv_bfloat16 *bias; // [width, C]
+    __nv_bfloat16 *entries, *idx_keys, *win_kv, *ring_g, *ring_ki;
+};
+
+// Columns of the two 64-column boxes of column tile nt (box 0 -> TMEM lanes 0..63, box 1 -> 64..127).
+template <bool POOL>
+__device__ __forceinline__ void tile_cols(const PoolArgs &a, int nt, int &ca, int &cb) {
+    if (!POOL) {   // the kernels of larger token tiles are never pooled
+        ca = nt * 128;
+        cb = ca + 64;
+        return;
+    }
+    if (nt < a.pool_tiles) {
+        if (nt < a.C / 64) {
+            ca = nt * 64;           // kv channels
+            cb = a.C + nt * 64;     // their gate channels
+        } else {
+            ca = 2 * a.C;           // the indexer-key channels 0..63
+            cb = a.C;               // gate channels 0..63
+        }
+    } else {
+        ca = a.plain0 + (nt - a.pool_tiles) * 128;
+        cb = ca + 64;
+    }
+}
 
 struct Unit {
     int n_tile, m_tile, split;
@@ -80,9 +124,102 @@ __device__ __forceinline__ Unit unit_of(const GemmArgs &a, int64_t u) {
     return x;
 }
 
+// The cache append of one pooled tile's 64 channels for the tile's tokens (one decode sequence each).  Called
+// by the four epilogue warps of the tile together (warp quad holds TMEM lanes 32 quad .. 32 quad + 31):
+// the gate lanes (quads 2, 3) publish their bf16 gate values, the value lanes (quads 0, 1) append.
 template <int NTOK>
+__device__ void fused_append(const GemmArgs &g, const PoolArgs &a, const float *v, int quad, int lane, int64_t t0,
+                             int nt, int ca, int cb, float *sgate) {
+    const int l = (quad & 1) * 32 + lane;   // channel within the 64-channel pair
+    if (quad >= 2) {
+#pragma unroll
+        for (int i = 0; i < NTOK; ++i) sgate[l * NTOK + i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+    }
+    tc::named_bar_sync(1, 128);
+    if (quad < 2) {
+        const bool key = nt >= a.C / 64;                  // indexer-key channels (gates 0..63)
+        const int c = key ? l : ca + l;                   // value channel (key: indexer-key channel)
+        const int gc = cb - a.C + l;                      // gate channel
+        for (int i = 0; i < NTOK; ++i) {
+            const int64_t b = t0 + i;
+            if (b >= g.M) break;
+            const int64_t P = a.pos[b];
+            if (P < 0) {
+                if (l == 0) report(g.status, kStatusBounds);
+                continue;
+            }
+            float vi = 0.f;   // v[i] by an unrolled select: v stays in registers
+#pragma unroll
+            for (int k = 0; k < NTOK; ++k) vi = k == i ? v[k] : vi;
+            const float vnew = __bfloat162float(__float2bfloat16_rn(vi)), gnew = sgate[l * NTOK + i];
+            if (key) {
+                a.ring_ki[(b * a.width + P % a.width) * a.di + c] = __float2bfloat16_rn(vnew);
+            } else {
+                a.win_kv[(b * a.window + P % a.window) * a.C + c] = __float2bfloat16_rn(vnew);
+                a.ring_g[(b * a.width + P % a.width) * a.C + c] = __float2bfloat16_rn(gnew);
+            }
+            if ((P + 1) % a.m != 0) continue;
+            const int64_t jg = (P + 1) / a.m - 1;         // the entry the token closes
+            if (a.shard && (jg < a.ent0 || jg >= a.ent0 + a.n_cap)) continue;
+            const int64_t j = jg - a.ent0;
+            if (j >= a.n_cap) {
+                if (l == 0) report(g.status, kStatusBounds);
+                continue;
+            }
+            const int64_t lo = (int64_t)a.m * jg - (a.width - a.m);
+            float mx = -INFINITY, z = 0.f, acc = 0.f;
+            for (int64_t t = lo < 0 ? 0 : lo; t <= P; ++t) {
+                const float g = t == P ? gnew : __bfloat162float(a.ring_g[(b * a.width + t % a.width) * a.C + gc]);
+                const float val = t == P ? vnew
+                                  : key ? __bfloat162float(a.ring_ki[(b * a.width + t % a.width) * a.di + c])
+                                        : __bfloat162float(a.win_kv[(b * a.window + t % a.window) * a.C + c]);
+                const float lg = g + __bfloat162float(a.bias[(t - lo) * a.C + gc]);
+                if (lg > mx) {
+                    const float sc = expf(mx - lg);
+                    acc = acc * sc + val;
+                    z = z * sc + 1.f;
+                    mx = lg;
+                } else {
+                    const float p = expf(lg - mx);
+                    acc += p * val;
+                    z += p;
+                }
+            }
+            const float e = __bfloat162float(__float2bfloat16_rn(acc / z));
+            const int64_t row = b * a.n_cap + j;
+            if (!a.lowprec) {
+                if (key) a.idx_keys[row * a.di + c] = __float2bfloat16_rn(e);
+                else a.entries[row * a.C + c] = __float2bfloat16_rn(e);
+                continue;
+            }
+            // block-scaled storage: the warp's 32 lanes are one 32-channel block
+            float am = fabsf(e);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+            if (key) {
+                uint8_t *codes = reinterpret_cast<uint8_t *>(a.idx_keys);
+                int8_t *ex = reinterpret_cast<int8_t *>(codes + a.rows_total * (a.di / 2));
+                const int ee = lp::block_exponent(am, 1.5f, 2);
+                const uint32_t cd = __nv_cvt_float_to_fp4(scalbnf(e, -ee), __NV_E2M1, cudaRoundNearest) & 0xFu;
+                const uint32_t hi = __shfl_down_sync(0xffffffffu, cd, 1);
+                if ((lane & 1) == 0) codes[row * (a.di / 2) + c / 2] = (uint8_t)(cd | (hi << 4));
+                if (lane == 0) ex[row * (a.di / 32) + c / 32] = (int8_t)ee;
+            } else {
+                uint8_t *codes = reinterpret_cast<uint8_t *>(a.entries);
+                int8_t *ex = reinterpret_cast<int8_t *>(codes + a.rows_total * a.C);
+                const int ee = lp::block_exponent(am, 1.75f, 8);
+                codes[row * a.C + c] = (uint8_t)__nv_cvt_float_to_fp8(scalbnf(e, -ee), __NV_SATFINITE, __NV_E4M3);
+                if (lane == 0) ex[row * (a.C / 32) + c / 32] = (int8_t)ee;
+            }
+        }
+    }
+    tc::named_bar_sync(1, 128);   // the gate buffer is reused by the next tile
+}
+
+template <int NTOK, bool POOL>
 __global__ void __launch_bounds__(64 + 32 * epi_warps(NTOK), ctas_per_sm(NTOK))
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GemmArgs a) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GemmArgs a,
+               const __grid_constant__ PoolArgs pa) {
     constexpr int NS = stages_for(NTOK), SB = stage_bytes(NTOK), E = epi_warps(NTOK), ET = 32 * E;
     constexpr int kColsPerWarp = NTOK / (E / 4);   // accumulator columns (tokens) each epilogue warp drains
     extern __shared__ uint8_t smem_raw[];
@@ -91,6 +228,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     uint64_t *full = bars, *empty = bars + NS, *acc_full = bars + 2 * NS, *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     int *s_last = reinterpret_cast<int *>(tmem_slot + 1);
+    float *sgate = reinterpret_cast<float *>(tmem_slot + 4);   // fused append: [64][NTOK] gate values
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -111,8 +249,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             uint32_t it = 0;
             for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
                 const Unit x = unit_of(a, u);
-                const int n0 = x.n_tile * kBN;
-                const bool two = n0 + 64 < a.N;   // the second 64-column box holds at least one column
+                int n0, n1;
+                tile_cols<POOL>(pa, x.n_tile, n0, n1);
+                const bool two = n1 < a.N;   // the second 64-column box holds at least one column
                 const uint32_t bytes = (two ? 2 : 1) * kBoxW + NTOK * 128;
                 for (int ks = x.k0; ks < x.k1 && ok; ++ks, ++it) {
                     const int s = it % NS;
@@ -121,7 +260,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     uint8_t *st = base + s * SB;
                     tc::mbar_arrive_expect_tx(&full[s], bytes);
                     tc::tma_load_2d(tc::smem_u32(st), &tm_w, n0, ks * 64, &full[s]);
-                    if (two) tc::tma_load_2d(tc::smem_u32(st + kBoxW), &tm_w, n0 + 64, ks * 64, &full[s]);
+                    if (two) tc::tma_load_2d(tc::smem_u32(st + kBoxW), &tm_w, n1, ks * 64, &full[s]);
                     tc::tma_load_2d(tc::smem_u32(st + 2 * kBoxW), &tm_x, ks * 64, x.m_tile * NTOK, &full[s]);
                 }
             }
@@ -166,10 +305,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             const Unit x = unit_of(a, u);
             const int ab = iacc & 1;
             ok = ok && tc::mbar_wait(&acc_full[ab], (iacc >> 1) & 1, a.status);
-            if (a.S > 1) ok = tc::named_bar_and(1, ET, ok);   // the split-K path meets at barriers below
+            // the split-K path and the fused append meet at barriers below
+            if (a.S > 1 || POOL) ok = tc::named_bar_and(1, ET, ok);
             if (!ok) break;
             tc::tc_fence_after();
-            const int n = x.n_tile * kBN + quad * 32 + lane;
+            int ca = 0, cb = 0;
+            int n = x.n_tile * kBN + quad * 32 + lane;
+            if constexpr (POOL) {
+                tile_cols<POOL>(pa, x.n_tile, ca, cb);
+                n = quad < 2 ? ca + quad * 32 + lane : cb + (quad - 2) * 32 + lane;
+            }
             const int64_t t0 = (int64_t)x.m_tile * NTOK;
             const uint32_t tl = tmem + ab * NTOK + ((uint32_t)(quad * 32) << 16);
             constexpr int CH = kColsPerWarp < 32 ? kColsPerWarp : 32;   // columns per TMEM load
@@ -198,6 +343,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                         if (t < a.M) pp[t * a.N + n] = v[i];
                     }
                 }
+                if constexpr (POOL) {
+                    if (x.n_tile < pa.pool_tiles)
+                        fused_append<NTOK>(a, pa, v, quad, lane, t0, x.n_tile, ca, cb, sgate);
+                }
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -217,7 +366,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     __threadfence();
                     // thread -> (column, token group): the 128 columns of the tile, ET / 128 token groups
                     constexpr int G = ET / 128;
-                    const int nn = x.n_tile * kBN + (et & 127);
+                    const int nn = x.n_tile * kBN + (et & 127);   // split-K never runs with the fused append
                     if (nn < a.N) {
                         for (int64_t t = t0 + (et >> 7); t < t0 + NTOK && t < a.M; t += G) {
                             float r = 0.f;
@@ -253,22 +402,23 @@ int num_sms() {
 constexpr size_t kPartFloats = (size_t)4 << 20;
 constexpr size_t kTicketBytes = 4096;
 
-template <int NTOK>
-hcsa_status launch_ntok(const CUtensorMap &tw, const CUtensorMap &tx, GemmArgs a, cudaStream_t st) {
-    constexpr size_t smem = smem_bytes(NTOK);
+template <int NTOK, bool POOL = false>
+hcsa_status launch_ntok(const CUtensorMap &tw, const CUtensorMap &tx, GemmArgs a, cudaStream_t st,
+                        const PoolArgs &pa = PoolArgs{}) {
+    constexpr size_t smem = smem_bytes(NTOK, POOL);
     static_assert(smem <= 232448, "shared memory per CTA");
     static bool configured[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        if (cudaFuncSetAttribute(gemm_tc_kernel<NTOK, POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return HCSA_ERR_CUDA;
         configured[dev] = true;
     }
     const int64_t slots = (int64_t)num_sms() * ctas_per_sm(NTOK);
     const int64_t grid = a.n_units < slots ? a.n_units : slots;
-    gemm_tc_kernel<NTOK><<<(unsigned)grid, 64 + 32 * epi_warps(NTOK), smem, st>>>(tw, tx, a);
+    gemm_tc_kernel<NTOK, POOL><<<(unsigned)grid, 64 + 32 * epi_warps(NTOK), smem, st>>>(tw, tx, a, pa);
     count_launch();
     return check_launch();
 }
@@ -276,6 +426,45 @@ hcsa_status launch_ntok(const CUtensorMap &tw, const CUtensorMap &tx, GemmArgs a
 }  // namespace
 
 size_t gemm_tc_ws_bytes() { return kPartFloats * sizeof(float) + kTicketBytes; }
+
+// Fused only up to one 16-token tile: the value lanes append the tile's tokens one after another, and at
+// 32 sequences that serial loop costs more than the separate append kernel (measured: 161 vs 143 us per
+// CSA layer at 32 sequences, 106.5 vs 107.8 us at 4).
+bool project_append_supported(const hcsa_params &p, bool csa) {
+    return p.dtype == HCSA_BF16 && p.B >= 1 && p.B <= 16 && p.C % 64 == 0 && (!csa || p.di == 64) && p.D % 8 == 0;
+}
+
+hcsa_status launch_project_append(const hcsa_params &p, bool csa, const hcsa_cache &c, const int32_t *pos,
+                                  const void *x, const void *W, int64_t ncols, void *y, const void *bias,
+                                  cudaStream_t st) {
+    const int64_t M = p.B;
+    const int N = (int)ncols, K = p.D;
+    constexpr int ntok = 16;
+    CUtensorMap tw, tx;
+    if (!make_tmap_bf16_2d(&tw, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64, 64, true)) return HCSA_ERR_CUDA;
+    if (!make_tmap_bf16_2d(&tx, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)ntok, true))
+        return HCSA_ERR_CUDA;
+    GemmArgs a{};
+    a.M = M; a.N = N; a.K = K;
+    a.ksteps = (K + 63) / 64;
+    a.S = 1; a.kper = a.ksteps;
+    PoolArgs pa{};
+    pa.pool_tiles = p.C / 64 + (csa ? 1 : 0);
+    pa.plain0 = 2 * p.C + (csa ? p.di : 0);
+    a.n_tiles = pa.pool_tiles + (N - pa.plain0 + kBN - 1) / kBN;
+    a.m_tiles = (int)((M + ntok - 1) / ntok);
+    a.n_units = (int64_t)a.n_tiles * a.m_tiles;
+    a.y = (__nv_bfloat16 *)y; a.ld_y = N;
+    a.status = device_status_ptr();
+    pa.pos = pos;
+    pa.C = p.C; pa.di = p.di; pa.m = p.m; pa.width = p.width; pa.window = p.window;
+    pa.n_cap = p.n_cap; pa.ent0 = p.ent0; pa.rows_total = (int64_t)p.B * p.n_cap;
+    pa.shard = p.ent_shard != 0; pa.lowprec = p.lowprec != 0;
+    pa.bias = (const __nv_bfloat16 *)bias;
+    pa.entries = (__nv_bfloat16 *)c.entries; pa.idx_keys = (__nv_bfloat16 *)c.idx_keys;
+    pa.win_kv = (__nv_bfloat16 *)c.win_kv; pa.ring_g = (__nv_bfloat16 *)c.ring_g; pa.ring_ki = (__nv_bfloat16 *)c.ring_ki;
+    return launch_ntok<16, true>(tw, tx, a, st, pa);
+}
 
 bool gemm_tc_supported(int64_t M, int N, int K, const void *x, int64_t ld_x, const void *W, int64_t ld_w,
                        const void *y, int64_t ld_y) {

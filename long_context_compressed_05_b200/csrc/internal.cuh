@@ -165,6 +165,11 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st);
 bool hca_attend_tc_supported(const AttendArgs &a);
 hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st);
 
+// decode projection with the cache append in the GEMM epilogue (gemm_tc.cu): y [B, ncols] and the cache update
+bool project_append_supported(const hcsa_params &p, bool csa);
+hcsa_status launch_project_append(const hcsa_params &p, bool csa, const hcsa_cache &c, const int32_t *pos,
+                                  const void *x, const void *W, int64_t ncols, void *y, const void *bias,
+                                  cudaStream_t st);
 // tcgen05 GEMM y[M, N] = x[M, K] W[K, N] (+ res), bf16 (gemm_tc.cu); ws (optional) enables split-K
 size_t gemm_tc_ws_bytes();
 bool gemm_tc_supported(int64_t M, int N, int K, const void *x, int64_t ld_x, const void *W, int64_t ld_w,

@@ -105,9 +105,11 @@ class PrefillLayer:
 class DecodeLayer:
     """One layer's decode step for B sequences over a caller-provided cache."""
 
-    def __init__(self, spec, B, n_cap, cache: dict, device="cuda", lowprec=False):
+    def __init__(self, spec, B, n_cap, cache: dict, device="cuda", lowprec=False, fused_append=True):
         """cache: device tensors entries, win_kv, ring_g (+ idx_keys, ring_ki for CSA); with lowprec the
-        entries and idx_keys are byte arrays in the FP8 / FP4 layout (hcsa_quantize_rows converts bf16 rows)."""
+        entries and idx_keys are byte arrays in the FP8 / FP4 layout (hcsa_quantize_rows converts bf16 rows).
+        fused_append: the projection and the cache append in one kernel (hcsa_project_append) instead of two."""
+        self.fused_append = fused_append
         self.spec = spec
         self.csa = spec.kind == "csa"
         self.kind = L.KIND_CSA if self.csa else L.KIND_HCA
@@ -137,9 +139,12 @@ class DecodeLayer:
         return self.y[:, a:b]
 
     def step(self, x, W_cat, bias, pos):
-        L.hcsa_project(self.p, self.kind, x, W_cat, self.y, self.ws_proj)
-        L.hcsa_cache_append(self.p, self.cache, pos, self.view("kv"), self.view("g"),
-                            self.view("ki") if self.csa else None, bias)
+        if self.fused_append:
+            L.hcsa_project_append(self.p, self.kind, self.cache, pos, x, W_cat, bias, self.y, self.ws_proj)
+        else:
+            L.hcsa_project(self.p, self.kind, x, W_cat, self.y, self.ws_proj)
+            L.hcsa_cache_append(self.p, self.cache, pos, self.view("kv"), self.view("g"),
+                                self.view("ki") if self.csa else None, bias)
         if self.csa:
             L.csa_decode_index_topk(self.p, self.cache, pos, self.view("qi"), self.view("w"), self.sel,
                                     self.ws_index)

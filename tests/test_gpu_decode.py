@@ -191,3 +191,54 @@ def test_decode_residual_stack():
         torch.cuda.synchronize()
         want = oracle.round_to(x_in + out @ oracle.to_f64(inp["W_o"]), oracle.ST_BF16)
         np.testing.assert_allclose(host64(x), want, rtol=2 ** -7, atol=2 ** -10)
+
+
+@pytest.mark.parametrize("spec,pos,n_cap,lowprec", [
+    (CSA_D, [515, 1023, 2000, 3, 7], 520, False),
+    (CSA_TC, [515, 1023, 60], 300, False),
+    (CSA_TC, [515, 1023, 60], 300, True),
+    (HCA_D, [255, 1000, 383], 16, False),
+    (HCA_TC, [255, 3000, 100, 127], 30, True),
+    (CSA_TC, list(range(3, 3 + 4 * 20, 4)), 40, False),   # 20 sequences: the 32-token tile
+    (CSA_D, list(range(3, 3 + 4 * 40, 4)), 50, False),    # 40 sequences: the two separate kernels
+])
+def test_fused_projection_append_matches_separate_calls(spec, pos, n_cap, lowprec):
+    """hcsa_project_append (the append in the projection's epilogue) writes exactly what hcsa_project then
+    hcsa_cache_append write: the projections, the rings and the closed entries."""
+    import long_context_compressed_05_b200 as h
+    d = synth.DecodeSpec(layers=(spec,), B=len(pos), P=max(pos), seed=spec.seed)
+    inp = synth.decode_inputs(d, 0, n_cap=n_cap)
+    B = len(pos)
+    p = h.params_for(spec, T=0, B=B, n_cap=n_cap, lowprec=lowprec)
+    kind = h.KIND_CSA if spec.kind == "csa" else h.KIND_HCA
+
+    def fresh():
+        c = {k: dev(inp[k]) for k in ("entries", "win_kv", "ring_g", "idx_keys", "ring_ki") if k in inp}
+        if lowprec:
+            rows = B * n_cap
+            for key, what, nb in (("entries", h.STORE_ENTRIES, h.hcsa_entry_bytes(p, rows)),
+                                  ("idx_keys", h.STORE_KEYS, h.hcsa_key_bytes(p, rows))):
+                if key in c:
+                    buf = torch.empty(nb, dtype=torch.uint8, device="cuda")
+                    h.hcsa_quantize_rows(p, what, c[key].reshape(rows, -1), buf)
+                    c[key] = buf
+        return c
+
+    x, W, Bb = dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"])
+    pos_t = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    ncols = h.hcsa_proj_cols(p, kind)
+    c1, c2 = fresh(), fresh()
+    y1 = torch.empty((B, ncols), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty_like(y1)
+    h.hcsa_project(p, kind, x, W, y1)   # no workspace: no split-K, the fused kernel's summation order
+    C = spec.C
+    h.hcsa_cache_append(p, h.make_cache(c1["entries"], c1["win_kv"], c1["ring_g"], c1.get("idx_keys"),
+                                        c1.get("ring_ki")), pos_t, y1[:, :C], y1[:, C:2 * C],
+                        y1[:, 2 * C:2 * C + spec.di] if spec.kind == "csa" else None, Bb)
+    h.hcsa_project_append(p, kind, h.make_cache(c2["entries"], c2["win_kv"], c2["ring_g"], c2.get("idx_keys"),
+                                                c2.get("ring_ki")), pos_t, x, W, Bb, y2)
+    torch.cuda.synchronize()
+    assert h.hcsa_get_device_status() == 0
+    assert torch.equal(y1, y2)
+    for k in c1:
+        assert torch.equal(c1[k], c2[k]), k

@@ -115,9 +115,7 @@ def test_sharded_decode_emulated_ranks(name, world):
     ranks = [h.ShardedDecodeLayer(spec, B, n_cap, h.shard_cache(full, r, world), r, world) for r in range(world)]
     for lay in ranks:
         lay.pos = pos_t
-        h.hcsa_project(lay.p, lay.kind, x, W, lay.y, lay.ws_proj)
-        h.hcsa_cache_append(lay.p, lay.cache, pos_t, lay.view("kv"), lay.view("g"),
-                            lay.view("ki") if lay.csa else None, Bb)
+        h.hcsa_project_append(lay.p, lay.kind, lay.cache, pos_t, x, W, Bb, lay.y, lay.ws_proj)
     if spec.kind == "csa":
         for lay in ranks:
             h.csa_decode_index_topk_shard(lay.p, lay.cache, pos_t, lay.view("qi"), lay.view("w"), lay.sel_l,
