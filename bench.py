@@ -370,6 +370,18 @@ def run_prefill(args, spec_name, ws, rank, lowprec=False):
             traffic = ATTEND_TC_DRAM_BYTES_PER_TOKEN * spec.T
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_sus, "unit": "TFLOP/s", "frac": ach / tc_sus,
                 "traffic": traffic, "kernel": dom, "peak_kind": f"{src} bf16 sustained"}
+        if dom == "attend" and spec.kind == "csa":
+            # what binds this kernel: gathered 128-byte segments of entry rows, against the gather rate a
+            # microbenchmark measured on this B200 for a table of the entries' size (16-byte cp.async,
+            # 148 CTAs: 9.6 TB/s up to 32 MB, 4.6 TB/s at 64 MB, 3.6 TB/s from 256 MB)
+            ent_mb = -(-spec.T // spec.m) * spec.C * (1 if lowprec else 2) / 2 ** 20
+            ceiling = 9600.0 if ent_mb <= 32 else 4600.0 if ent_mb <= 64 else 3600.0
+            t = np.arange(spec.T, dtype=np.float64)
+            rows = np.minimum(np.minimum(t // spec.m, -(-spec.T // spec.m)), spec.topk).sum()
+            gathered = rows * spec.C * (1 + 1 / 32 if lowprec else 2)
+            gbs = gathered / (ours[dom] / 1e3) / 1e9
+            roof["gather"] = {"achieved": gbs, "ceiling": ceiling, "unit": "GB/s", "frac": gbs / ceiling,
+                              "bytes": gathered, "entries_MB": ent_mb}
     else:
         ach = wk["bytes"] / (ours[dom] / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,

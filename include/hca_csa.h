@@ -257,6 +257,18 @@ hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, con
                               const void *kv, int64_t ld_kv, const void *g, int64_t ld_g, const void *ki,
                               int64_t ld_ki, const void *bias, void *stream);
 
+/* Prefill: the projection with the compressor done in the GEMM's epilogue (the compressor of "CSA:
+ * compresion 4x" fed straight from the projection tile).  Same results as hcsa_project followed by
+ * csa_compress / hca_compress with the same params: y [T, ncols] (ld ncols), entries and idx_keys (CSA;
+ * NULL for HCA) as documented for the compressors (bf16, or FP8 / FP4 with p->lowprec; a row range forms
+ * the range's entries).  The fused kernel covers CSA layers (m = 4, width = 8, di = 64, C a multiple
+ * of 64, bf16) over the whole sequence: pools inside a 128-token half of a 256-token tile are formed in
+ * the epilogue, the one per half boundary afterwards from the stored projections; other shapes and row
+ * ranges run the two calls' kernels.  ws as for hcsa_project. */
+hcsa_status hcsa_project_compress(const hcsa_params *p, int32_t kind, const void *x, const void *W_cat,
+                                  const void *bias, void *y, void *entries, void *idx_keys, void *ws, size_t ws_bytes,
+                                  void *stream);
+
 /* Decode: the projection of the new tokens with the cache append done in the GEMM's epilogue (the
  * compressor of "CSA: compresion 4x" / "HCA: compresion 128x" fed straight from the projection tile).
  * Same results as hcsa_project followed by hcsa_cache_append: y [B, ncols] (ld ncols) is written, the

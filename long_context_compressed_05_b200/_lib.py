@@ -32,7 +32,7 @@ EXPORTS = ["hcsa_version", "hcsa_status_string", "hcsa_workspace_bytes", "hcsa_p
            "hcsa_get_device_status", "hcsa_selftest_wait_timeout",
            "hcsa_launch_count", "hcsa_entry_bytes", "hcsa_key_bytes", "hcsa_quantize_rows",
            "csa_decode_index_topk_shard", "csa_topk_merge", "csa_decode_attend_shard", "hca_decode_attend_shard",
-           "hcsa_merge_partials", "hcsa_project_append"]
+           "hcsa_merge_partials", "hcsa_project_append", "hcsa_project_compress"]
 STORE_ENTRIES, STORE_KEYS = 0, 1
 
 
@@ -97,6 +97,7 @@ def load():
         "hca_decode_attend_shard": (I32, [P, CP, V, V, I64, I32, V, V, SZ, V]),
         "hcsa_merge_partials": (I32, [P, V, I32, V, I64, V]),
         "hcsa_project_append": (I32, [P, I32, CP, V, V, V, V, V, V, SZ, V]),
+        "hcsa_project_compress": (I32, [P, I32, V, V, V, V, V, V, V, SZ, V]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -249,6 +250,12 @@ def hcsa_quantize_rows(p, what, src, dst, stream=None):
     """src: [rows, C] (entries) or [rows, di] (keys) bf16; dst: a byte buffer of the matching size."""
     _check("hcsa_quantize_rows", load().hcsa_quantize_rows(ctypes.byref(p), what, _ptr(src), src.shape[0],
                                                            _ptr(dst), _stream(stream)))
+
+
+def hcsa_project_compress(p, kind, x, W_cat, bias, y, entries, idx_keys, ws=None, stream=None):
+    _check("hcsa_project_compress", load().hcsa_project_compress(
+        ctypes.byref(p), kind, _ptr(x), _ptr(W_cat), _ptr(bias), _ptr(y), _ptr(entries), _ptr(idx_keys), _ptr(ws),
+        _wsz(ws), _stream(stream)))
 
 
 def hcsa_project_append(p, kind, cache: Cache, pos, x, W_cat, bias, y, ws=None, stream=None):

@@ -315,6 +315,36 @@ hcsa_status hcsa_cache_append(const hcsa_params *p, const hcsa_cache *cache, con
                                (cudaStream_t)stream);
 }
 
+hcsa_status hcsa_project_compress(const hcsa_params *p, int32_t kind, const void *x, const void *W_cat,
+                                  const void *bias, void *y, void *entries, void *idx_keys, void *ws, size_t ws_bytes,
+                                  void *stream) {
+    const bool csa = kind == HCSA_KIND_CSA;
+    if (kind != HCSA_KIND_CSA && kind != HCSA_KIND_HCA) return HCSA_ERR_SHAPE;
+    HCSA_TRY(csa ? check_csa(p) : check_common(p));
+    if (!x || !W_cat || !y || !bias || !entries || (csa && !idx_keys)) return HCSA_ERR_NULL;
+    if (p->T < 0 || p->D < 1) return HCSA_ERR_SHAPE;
+    if (!aligned(x) || !aligned(W_cat) || !aligned(y) || !aligned(bias) || !aligned(entries) ||
+        (csa && !aligned(idx_keys)))
+        return HCSA_ERR_ALIGN;
+    const int64_t nc = hcsa_proj_cols(p, kind);
+    if ((p->D * esize(p->dtype)) % 16 || (nc * esize(p->dtype)) % 16) return HCSA_ERR_ALIGN;
+    int64_t r0, r1, j0, j1;
+    HCSA_TRY(row_range(p, &r0, &r1));
+    entry_range(p, r0, r1, &j0, &j1);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (p->T == 0) return HCSA_OK;
+    if (r0 == 0 && r1 == p->T && project_compress_supported(*p, csa))
+        return launch_project_compress(*p, x, W_cat, nc, y, bias, entries, idx_keys, st);
+    // other shapes and row ranges: the projection, then the compressor kernel
+    if (p->dtype == HCSA_BF16 && ws && ws_bytes < project_ws_bytes(p->dtype)) return HCSA_ERR_WORKSPACE;
+    HCSA_TRY(launch_project(p->dtype, p->T, p->D, nc, x, W_cat, y, ws, ws_bytes, st));
+    const uint8_t *y8 = (const uint8_t *)y;
+    const int es = esize(p->dtype);
+    return launch_compress(p->dtype, p->T, p->C, p->m, p->width, y8, nc, y8 + (int64_t)p->C * es, nc,
+                           csa ? y8 + 2 * (int64_t)p->C * es : nullptr, nc, csa ? p->di : 0, bias, entries,
+                           csa ? idx_keys : nullptr, j0, j1, p->lowprec != 0, n_entries(p), st);
+}
+
 hcsa_status hcsa_project_append(const hcsa_params *p, int32_t kind, const hcsa_cache *cache, const int32_t *pos,
                                 const void *x, const void *W_cat, const void *bias, void *y, void *ws, size_t ws_bytes,
                                 void *stream) {

@@ -26,6 +26,7 @@ namespace hcsa {
 struct LowPrecOut {
     bool on;
     int64_t rows;   // rows of the whole array: the exponents follow rows x ch code bytes
+    int jstride;    // entries j0, j0 + jstride, ... (1: a contiguous range)
 };
 
 __device__ __forceinline__ void store_row_vec(const float *r, bool is_key, int64_t row, int C, int di, int c0,
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(256) compress_kernel(int64_t T, int C, int m, 
     if (gid >= N * slots) return;   // entries j0 .. j0 + N - 1
     const int64_t jl = gid / slots;
     const int s = (int)(gid - jl * slots);
-    const int64_t j = j0 + jl;
+    const int64_t j = j0 + jl * lp.jstride;
     const bool is_key = s >= slots_c;
     const int c0 = (is_key ? s - slots_c : s) * V;   // value channel; also the gate channel
     const S *val = is_key ? ki : kv;
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(256) compress_narrow_bf16_kernel(
     const int gid = blockIdx.x * 256 + threadIdx.x;
     if (gid >= N * slots) return;   // entries j0 .. j0 + N - 1
     const int jl = gid / slots, s = gid - jl * slots;
-    const int j = j0 + jl;
+    const int j = j0 + jl * lp.jstride;
     const bool is_key = s >= slots_c;
     const int c0 = (is_key ? s - slots_c : s) * 8;   // value channel, also the gate channel
     const __nv_bfloat16 *val = is_key ? ki : kv;
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
     const int slots_c = C >> 3;
     const int slots = slots_c + (ki ? di >> 3 : 0);
     const int s = blockIdx.x * 32 + lane;
-    const int j = j0 + blockIdx.y;
+    const int j = j0 + (int)blockIdx.y * lp.jstride;
     const bool active = s < slots;
     const bool is_key = s >= slots_c;
     const int c0 = (is_key ? s - slots_c : s) * 8;
@@ -291,10 +292,10 @@ __global__ void __launch_bounds__(32 * kWideWarps) compress_wide_bf16_kernel(
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
                             void *entries, void *idx_keys, int64_t j0, int64_t j1, bool lowprec, int64_t rows,
-                            cudaStream_t st) {
-    const int64_t N = j1 - j0;   // entries j0 .. j1 - 1 of the sequence
+                            cudaStream_t st, int jstride) {
+    const int64_t N = (j1 - j0 + jstride - 1) / jstride;   // entries j0, j0 + jstride, ... below j1
     if (N <= 0) return HCSA_OK;
-    const LowPrecOut lp{lowprec, rows};
+    const LowPrecOut lp{lowprec, rows, jstride};
     const int threads = 256;
     if (dtype == HCSA_BF16) {
         using S = __nv_bfloat16;
@@ -320,7 +321,7 @@ hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const
         const int64_t blocks = (N * slots + threads - 1) / threads;
         compress_kernel<float><<<(unsigned)blocks, threads, 0, st>>>(
             T, C, m, width, (const float *)kv, ld_kv, (const float *)g, ld_g, (const float *)ki, ld_ki, di,
-            (const float *)bias, (float *)entries, (float *)idx_keys, j0, N, LowPrecOut{false, 0});
+            (const float *)bias, (float *)entries, (float *)idx_keys, j0, N, LowPrecOut{false, 0, jstride});
     }
     count_launch();
     return check_launch();
@@ -431,14 +432,14 @@ hcsa_status launch_cache_append(int dtype, const hcsa_params &p, const hcsa_cach
         cache_append_kernel<S><<<grid, 128, 0, st>>>(
             p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
             (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
-            (S *)c.ring_ki, status, LowPrecOut{p.lowprec != 0, (int64_t)p.B * p.n_cap}, (int64_t)p.ent0,
+            (S *)c.ring_ki, status, LowPrecOut{p.lowprec != 0, (int64_t)p.B * p.n_cap, 1}, (int64_t)p.ent0,
             p.ent_shard != 0);
     } else {
         using S = float;
         cache_append_kernel<S><<<grid, 128, 0, st>>>(
             p.C, p.m, p.width, p.window, p.di, p.n_cap, pos, (const S *)kv, ld_kv, (const S *)g, ld_g,
             (const S *)ki, ld_ki, (const S *)bias, (S *)c.entries, (S *)c.idx_keys, (S *)c.win_kv, (S *)c.ring_g,
-            (S *)c.ring_ki, status, LowPrecOut{false, 0}, (int64_t)p.ent0, p.ent_shard != 0);
+            (S *)c.ring_ki, status, LowPrecOut{false, 0, 1}, (int64_t)p.ent0, p.ent_shard != 0);
     }
     count_launch();
     return check_launch();

@@ -47,9 +47,10 @@ __host__ __device__ constexpr int stage_bytes(int ntok) { return 2 * kBoxW + nto
 __host__ __device__ constexpr uint32_t tmem_cols(int ntok) {
     return 2 * ntok <= 32 ? 32 : 2 * ntok <= 64 ? 64 : 2 * ntok <= 128 ? 128 : 2 * ntok <= 256 ? 256 : 512;
 }
-__host__ __device__ constexpr size_t smem_bytes(int ntok, bool pool = false) {
+__host__ __device__ constexpr size_t smem_bytes(int ntok, int pool = 0) {
+    // pool 1 (decode append): gates [64][ntok]; pool 2 (prefill compressor): gates [2 halves][64][32]
     return 1024 + (size_t)stages_for(ntok) * stage_bytes(ntok) + (2 * stages_for(ntok) + 8) * sizeof(uint64_t) + 16 +
-           (pool ? 64 * ntok * sizeof(float) : 0);
+           (pool == 1 ? 64 * ntok * sizeof(float) : pool == 2 ? 2 * 64 * 32 * sizeof(float) : 0);
 }
 
 struct GemmArgs {
@@ -80,10 +81,104 @@ struct PoolArgs {
     __nv_bfloat16 *entries, *idx_keys, *win_kv, *ring_g, *ring_ki;
 };
 
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Store one entry value e (a bf16 number) of channel c of row j, bf16 or block-scaled (the warp's 32 lanes
+// are one 32-channel block; every lane of the warp calls this together).
+__device__ __forceinline__ void store_entry_value(float e, bool key, int64_t j, int c, int lane, int64_t rows_total,
+                                                  int C, int di, bool lowprec, __nv_bfloat16 *entries,
+                                                  __nv_bfloat16 *idx_keys) {
+    if (!lowprec) {
+        if (key) idx_keys[j * di + c] = __float2bfloat16_rn(e);
+        else entries[j * C + c] = __float2bfloat16_rn(e);
+        return;
+    }
+    float am = fabsf(e);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if (key) {
+        uint8_t *codes = reinterpret_cast<uint8_t *>(idx_keys);
+        int8_t *ex = reinterpret_cast<int8_t *>(codes + rows_total * (di / 2));
+        const int ee = lp::block_exponent(am, 1.5f, 2);
+        const uint32_t cd = __nv_cvt_float_to_fp4(scalbnf(e, -ee), __NV_E2M1, cudaRoundNearest) & 0xFu;
+        const uint32_t hi = __shfl_down_sync(0xffffffffu, cd, 1);
+        if ((lane & 1) == 0) codes[j * (di / 2) + c / 2] = (uint8_t)(cd | (hi << 4));
+        if (lane == 0) ex[j * (di / 32) + c / 32] = (int8_t)ee;
+    } else {
+        uint8_t *codes = reinterpret_cast<uint8_t *>(entries);
+        int8_t *ex = reinterpret_cast<int8_t *>(codes + rows_total * C);
+        const int ee = lp::block_exponent(am, 1.75f, 8);
+        codes[j * C + c] = (uint8_t)__nv_cvt_float_to_fp8(scalbnf(e, -ee), __NV_SATFINITE, __NV_E4M3);
+        if (lane == 0) ex[j * (C / 32) + c / 32] = (int8_t)ee;
+    }
+}
+
+// Prefill: the CSA compressor (pools of 8 tokens at stride 4) on one 32-token chunk of a pooled tile.  The
+// four warps of a 128-token half call this together: the gate lanes publish the chunk's bf16 gates, each
+// value lane appends the chunk's tokens to its 8-token ring and closes the entries whose last token is in
+// the chunk, with the compressor kernel's two-pass softmax in its row order (so the entries are
+// identical).  Entries whose pool reaches into the previous half are left to the seam pass.
+__device__ void fused_compress_chunk(const GemmArgs &g, const PoolArgs &a, const float *v, int quad, int lane,
+                                     int64_t tb, int64_t hs, int nt, int ca, float *sg, int bar_id, float (&kr)[8],
+                                     float (&gr)[8], const float (&b8)[8]) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    const int l = (quad & 1) * 32 + lane;
+    if (quad >= 2) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sg[l * 32 + i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+    }
+    tc::named_bar_sync(bar_id, 128);
+    if (quad < 2) {
+        const bool key = nt >= a.C / 64;
+        const int c = key ? l : ca + l;
+        const int64_t T = g.M;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int64_t t = tb + i;
+            if (t < T) {
+                kr[i & 7] = __bfloat162float(__float2bfloat16_rn(v[i]));
+                gr[i & 7] = sg[l * 32 + i];
+            }
+            // entry j = t / 4 closes at its last token (4 j + 3, or the sequence's last)
+            if (t < T && ((i & 3) == 3 || t == T - 1)) {
+                const int64_t j = t >> 2;
+                const int64_t lo = 4 * j - 4;
+                if ((lo < 0 ? 0 : lo) >= hs) {
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int64_t tok = lo + r;
+                        const int sl = ((i & 7) - (i & 3) - 4 + r) & 7;   // ring slot of token lo + r
+                        if (tok >= 0 && tok <= t) mx = fmaxf(mx, gr[sl] + b8[r]);
+                    }
+                    float z = 0.f, acc = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int64_t tok = lo + r;
+                        const int sl = ((i & 7) - (i & 3) - 4 + r) & 7;
+                        if (tok >= 0 && tok <= t) {
+                            const float p = ex2_approx((gr[sl] + b8[r] - mx) * kLog2e);
+                            z += p;
+                            acc = fmaf(p, kr[sl], acc);
+                        }
+                    }
+                    const float e = __bfloat162float(__float2bfloat16_rn(acc / z));
+                    store_entry_value(e, key, j, c, lane, a.rows_total, a.C, a.di, a.lowprec, a.entries, a.idx_keys);
+                }
+            }
+        }
+    }
+    tc::named_bar_sync(bar_id, 128);   // the gate buffer is rewritten by the next chunk
+}
+
 // Columns of the two 64-column boxes of column tile nt (box 0 -> TMEM lanes 0..63, box 1 -> 64..127).
-template <bool POOL>
+template <int POOL>
 __device__ __forceinline__ void tile_cols(const PoolArgs &a, int nt, int &ca, int &cb) {
-    if (!POOL) {   // the kernels of larger token tiles are never pooled
+    if (!POOL) {   // a plain GEMM
         ca = nt * 128;
         cb = ca + 64;
         return;
@@ -216,7 +311,7 @@ __device__ void fused_append(const GemmArgs &g, const PoolArgs &a, const float *
     tc::named_bar_sync(1, 128);   // the gate buffer is reused by the next tile
 }
 
-template <int NTOK, bool POOL>
+template <int NTOK, int POOL>
 __global__ void __launch_bounds__(64 + 32 * epi_warps(NTOK), ctas_per_sm(NTOK))
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, GemmArgs a,
                const __grid_constant__ PoolArgs pa) {
@@ -228,7 +323,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     uint64_t *full = bars, *empty = bars + NS, *acc_full = bars + 2 * NS, *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     int *s_last = reinterpret_cast<int *>(tmem_slot + 1);
-    float *sgate = reinterpret_cast<float *>(tmem_slot + 4);   // fused append: [64][NTOK] gate values
+    float *sgate = reinterpret_cast<float *>(tmem_slot + 4);   // fused append / compressor: gate values
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -306,14 +401,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             const int ab = iacc & 1;
             ok = ok && tc::mbar_wait(&acc_full[ab], (iacc >> 1) & 1, a.status);
             // the split-K path and the fused append meet at barriers below
-            if (a.S > 1 || POOL) ok = tc::named_bar_and(1, ET, ok);
+            if (a.S > 1 || POOL != 0) ok = tc::named_bar_and(1, ET, ok);
             if (!ok) break;
             tc::tc_fence_after();
             int ca = 0, cb = 0;
             int n = x.n_tile * kBN + quad * 32 + lane;
-            if constexpr (POOL) {
+            if constexpr (POOL != 0) {
                 tile_cols<POOL>(pa, x.n_tile, ca, cb);
                 n = quad < 2 ? ca + quad * 32 + lane : cb + (quad - 2) * 32 + lane;
+            }
+            // prefill compressor state of a value lane: the last 8 tokens (value, gate) and the 8 bias rows
+            float kr[8], gr[8], b8[8];
+            const bool pooled = POOL == 2 && x.n_tile < pa.pool_tiles;
+            if constexpr (POOL == 2) {
+                if (pooled && quad < 2) {
+                    const int gc = cb - pa.C + (quad & 1) * 32 + lane;
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) b8[r] = __bfloat162float(pa.bias[r * pa.C + gc]);
+                }
             }
             const int64_t t0 = (int64_t)x.m_tile * NTOK;
             const uint32_t tl = tmem + ab * NTOK + ((uint32_t)(quad * 32) << 16);
@@ -343,9 +448,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                         if (t < a.M) pp[t * a.N + n] = v[i];
                     }
                 }
-                if constexpr (POOL) {
+                if constexpr (POOL == 1) {
                     if (x.n_tile < pa.pool_tiles)
                         fused_append<NTOK>(a, pa, v, quad, lane, t0, x.n_tile, ca, cb, sgate);
+                }
+                if constexpr (POOL == 2 && CH == 32) {
+                    if (pooled)
+                        fused_compress_chunk(a, pa, v, quad, lane, t0 + c0, t0 + c_begin, x.n_tile, ca,
+                                             sgate + (c_begin / 128) * 64 * 32, 2 + c_begin / 128, kr, gr, b8);
                 }
             }
             tc::tc_fence_before();
@@ -402,7 +512,7 @@ int num_sms() {
 constexpr size_t kPartFloats = (size_t)4 << 20;
 constexpr size_t kTicketBytes = 4096;
 
-template <int NTOK, bool POOL = false>
+template <int NTOK, int POOL = 0>
 hcsa_status launch_ntok(const CUtensorMap &tw, const CUtensorMap &tx, GemmArgs a, cudaStream_t st,
                         const PoolArgs &pa = PoolArgs{}) {
     constexpr size_t smem = smem_bytes(NTOK, POOL);
@@ -430,6 +540,51 @@ size_t gemm_tc_ws_bytes() { return kPartFloats * sizeof(float) + kTicketBytes; }
 // Fused only up to one 16-token tile: the value lanes append the tile's tokens one after another, and at
 // 32 sequences that serial loop costs more than the separate append kernel (measured: 161 vs 143 us per
 // CSA layer at 32 sequences, 106.5 vs 107.8 us at 4).
+// Prefill: the CSA compressor (m = 4, width = 8) in the epilogue of the projection's 256-token tiles.  Pools
+// inside a 128-token half of a tile are formed there; the one pool per half boundary that reaches into the
+// previous half (entry 32 s) is formed afterwards from the stored projections by the compressor kernel.
+// Measured at T = 131072: 18.0-19.5 ms against 17.4-18.9 ms for the projection and the compressor kernel
+// (the pooled tiles' epilogue costs more than the 0.4 ms pass it replaces).
+bool project_compress_supported(const hcsa_params &p, bool csa) {
+    return csa && p.dtype == HCSA_BF16 && p.m == 4 && p.width == 8 && p.C % 64 == 0 && p.di == 64 &&
+           p.D % 8 == 0 && p.T >= 1 && p.T <= INT32_MAX;
+}
+
+hcsa_status launch_project_compress(const hcsa_params &p, const void *x, const void *W, int64_t ncols, void *y,
+                                    const void *bias, void *entries, void *idx_keys, cudaStream_t st) {
+    const int64_t M = p.T;
+    const int N = (int)ncols, K = p.D;
+    constexpr int ntok = 256;
+    CUtensorMap tw, tx;
+    if (!make_tmap_bf16_2d(&tw, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64, 64, true)) return HCSA_ERR_CUDA;
+    if (!make_tmap_bf16_2d(&tx, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)ntok, true))
+        return HCSA_ERR_CUDA;
+    GemmArgs a{};
+    a.M = M; a.N = N; a.K = K;
+    a.ksteps = (K + 63) / 64;
+    a.S = 1; a.kper = a.ksteps;
+    PoolArgs pa{};
+    pa.pool_tiles = p.C / 64 + 1;
+    pa.plain0 = 2 * p.C + p.di;
+    a.n_tiles = pa.pool_tiles + (N - pa.plain0 + kBN - 1) / kBN;
+    a.m_tiles = (int)((M + ntok - 1) / ntok);
+    a.n_units = (int64_t)a.n_tiles * a.m_tiles;
+    a.y = (__nv_bfloat16 *)y; a.ld_y = N;
+    a.status = device_status_ptr();
+    const int64_t n_ent = (p.T + p.m - 1) / p.m;
+    pa.C = p.C; pa.di = p.di; pa.m = p.m; pa.width = p.width;
+    pa.rows_total = n_ent; pa.lowprec = p.lowprec != 0;
+    pa.bias = (const __nv_bfloat16 *)bias;
+    pa.entries = (__nv_bfloat16 *)entries; pa.idx_keys = (__nv_bfloat16 *)idx_keys;
+    const hcsa_status s = launch_ntok<ntok, 2>(tw, tx, a, st, pa);
+    if (s != HCSA_OK) return s;
+    // seams: entries 32, 64, ... (pools across a 128-token boundary), from the stored projections
+    const uint8_t *y8 = (const uint8_t *)y;
+    return launch_compress(HCSA_BF16, p.T, p.C, p.m, p.width, y8, N, y8 + 2 * (int64_t)p.C, N,
+                           y8 + 4 * (int64_t)p.C, N, p.di, bias, entries, idx_keys, 32, n_ent, p.lowprec != 0, n_ent,
+                           st, 32);
+}
+
 bool project_append_supported(const hcsa_params &p, bool csa) {
     return p.dtype == HCSA_BF16 && p.B >= 1 && p.B <= 16 && p.C % 64 == 0 && (!csa || p.di == 64) && p.D % 8 == 0;
 }
@@ -463,7 +618,7 @@ hcsa_status launch_project_append(const hcsa_params &p, bool csa, const hcsa_cac
     pa.bias = (const __nv_bfloat16 *)bias;
     pa.entries = (__nv_bfloat16 *)c.entries; pa.idx_keys = (__nv_bfloat16 *)c.idx_keys;
     pa.win_kv = (__nv_bfloat16 *)c.win_kv; pa.ring_g = (__nv_bfloat16 *)c.ring_g; pa.ring_ki = (__nv_bfloat16 *)c.ring_ki;
-    return launch_ntok<16, true>(tw, tx, a, st, pa);
+    return launch_ntok<16, 1>(tw, tx, a, st, pa);
 }
 
 bool gemm_tc_supported(int64_t M, int N, int K, const void *x, int64_t ld_x, const void *W, int64_t ld_w,

@@ -70,7 +70,7 @@ hcsa_status check_launch();         // maps cudaGetLastError() to a status
 hcsa_status launch_compress(int dtype, int64_t T, int C, int m, int width, const void *kv, int64_t ld_kv,
                             const void *g, int64_t ld_g, const void *ki, int64_t ld_ki, int di, const void *bias,
                             void *entries, void *idx_keys, int64_t j0, int64_t j1, bool lowprec, int64_t rows,
-                            cudaStream_t st);
+                            cudaStream_t st, int jstride = 1);
 
 // entry-sharded decode (shard.cu)
 hcsa_status launch_shift_pos(const int32_t *pos, int64_t B, int64_t delta, int32_t *out, cudaStream_t st);
@@ -165,6 +165,10 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st);
 bool hca_attend_tc_supported(const AttendArgs &a);
 hcsa_status launch_hca_attend_tc(const AttendArgs &a, cudaStream_t st);
 
+// prefill projection with the CSA compressor in the GEMM epilogue (gemm_tc.cu): y [T, ncols], entries, keys
+bool project_compress_supported(const hcsa_params &p, bool csa);
+hcsa_status launch_project_compress(const hcsa_params &p, const void *x, const void *W, int64_t ncols, void *y,
+                                    const void *bias, void *entries, void *idx_keys, cudaStream_t st);
 // decode projection with the cache append in the GEMM epilogue (gemm_tc.cu): y [B, ncols] and the cache update
 bool project_append_supported(const hcsa_params &p, bool csa);
 hcsa_status launch_project_append(const hcsa_params &p, bool csa, const hcsa_cache &c, const int32_t *pos,

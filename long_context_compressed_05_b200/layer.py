@@ -93,6 +93,12 @@ class PrefillLayer:
         else:
             L.hca_attend(self.p, self.view("q"), self.view("kv"), self.entries, self.out, self.ws_attend)
 
+    def project_compress(self, x, W_cat, bias):
+        """The projection with the compressor in its epilogue (one GEMM + a seam pass for CSA layers).  Same
+        results as project + compress; at T = 131072 about 0.6 ms slower, so forward() keeps the two calls."""
+        L.hcsa_project_compress(self.p, self.kind, x, W_cat, bias, self.y, self.entries,
+                                self.idx_keys if self.csa else None, self.ws_proj)
+
     def forward(self, x, W_cat, bias):
         self.project(x, W_cat)
         self.compress(bias)

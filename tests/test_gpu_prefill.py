@@ -121,3 +121,30 @@ def test_prefill_full_size_sampled(name):
     rows = sample_rows(spec.T, spec.m, max(spec.topk, 1), n_random=24 if spec.kind == "csa" else 64)
     ref = oracle.prefill(spec, inp, rows=rows)
     compare(spec, inp, layer, rows, ref)
+
+
+@pytest.mark.parametrize("name,lowprec", [("csa_bf16_small", False), ("csa_bf16_tc_k128", False),
+                                          ("csa_bf16_tc_k128", True), ("csa_bf16_t3", False),
+                                          ("csa_bf16_vis_lt_k", False), ("hca_bf16_small", False),
+                                          ("csa_f32_ragged", False)])
+def test_fused_projection_compressor_matches_separate_calls(name, lowprec):
+    """hcsa_project_compress (the compressor in the projection's epilogue, seams after) writes exactly
+    what hcsa_project then csa_compress / hca_compress write."""
+    import long_context_compressed_05_b200 as h
+    spec = CASES[name]
+    for T in sorted({spec.T, 257, 640, 1023} if spec.T > 100 else {spec.T}):
+        sp = spec.replace(T=T)
+        inp = synth.prefill_inputs(sp)
+        x, W, B = dev(inp["x"]), dev(inp["W_cat"]), dev(inp["B"])
+        a, b = h.PrefillLayer(sp, lowprec=lowprec), h.PrefillLayer(sp, lowprec=lowprec)
+        a.y.fill_(0)
+        L = h
+        L.hcsa_project(a.p, a.kind, x, W, a.y)                     # no workspace: no split-K
+        a.compress(B)
+        L.hcsa_project_compress(b.p, b.kind, x, W, B, b.y, b.entries, b.idx_keys if b.csa else None)
+        torch.cuda.synchronize()
+        assert h.hcsa_get_device_status() == 0
+        assert torch.equal(a.y, b.y), T
+        assert torch.equal(a.entries, b.entries), T
+        if sp.kind == "csa":
+            assert torch.equal(a.idx_keys, b.idx_keys), T
