@@ -69,6 +69,7 @@ struct Params {
     int64_t nq;          // queries (prefill T, decode B)
     int64_t N;           // entries per sequence (prefill ceil(T/m), decode n_cap)
     int m, topk, seg_tiles, nseg;
+    int dq_split;        // decode: units per (query, segment), each taking 4 / dq_split of the 128-dh value blocks
     const int32_t *sel, *pos;
     float scale, scale_log2;
     __nv_bfloat16 *out;  // direct output [nq, H*dh] (nseg == 1)
@@ -83,12 +84,17 @@ struct Params {
 struct Unit {
     int64_t q, p, nvis;
     int seg, E, t0, nt;
+    int dp0, dp1;        // value blocks [dp0, dp1) of 128 dh this unit accumulates and writes
 };
 
 __device__ __forceinline__ Unit unit_of(const Params &a, int64_t u) {
     Unit x;
+    const int dq = (int)(u % a.dq_split);
+    u /= a.dq_split;
     x.q = a.q0 + u / a.nseg;
     x.seg = (int)(u % a.nseg);
+    x.dp0 = dq * (4 / a.dq_split);
+    x.dp1 = x.dp0 + 4 / a.dq_split;
     x.p = a.decode ? (int64_t)a.pos[x.q] : x.q;
     {   // visible entries held here: global j < p / m, local j - ent0 in [0, N)
         int64_t v = x.p < 0 ? 0 : x.p / a.m - a.ent0;
@@ -349,7 +355,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     load_chunk(4, dc * 64);
                 }
             for (int t = 0; t < x.nt; ++t)            // P V: value halves, 64-dh chunks in pairs
-                for (int c = 0; c < 8; ++c) load_chunk(t, kDh + c * 64);
+                for (int c = 2 * x.dp0; c < 2 * x.dp1; ++c) load_chunk(t, kDh + c * 64);
         }
         tc::cp_async_wait_all();
         if (!ok && pt == 0) {
@@ -412,7 +418,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 ok = ok && tc::mbar_wait(&bars->p_full, iu & 1, a.status);
                 tc::tc_fence_after();
                 for (int t = 0; t < x.nt; ++t)
-                    for (int dp = 0; dp < 4; ++dp, ic += 2) {
+                    for (int dp = x.dp0; dp < x.dp1; ++dp, ic += 2) {
                         const int s0 = ic % kNS, s1 = (ic + 1) % kNS;
                         ok = ok && tc::mbar_wait(&bars->rf[s0], (ic / kNS) & 1, a.status);
                         ok = ok && tc::mbar_wait(&bars->rf[s1], ((ic + 1) / kNS) & 1, a.status);
@@ -447,7 +453,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const Unit x = unit_of(a, u);
             const int64_t slot = x.q * a.nseg + x.seg;
             if (x.nt <= 0) {
-                if (a.part && et < kH) {
+                if (a.part && et < kH && x.dp0 == 0) {
                     float *pml = a.part + a.nq * (int64_t)a.nseg * kH * kDh;
                     pml[(slot * kH + et) * 2] = -INFINITY;
                     pml[(slot * kH + et) * 2 + 1] = 0.f;
@@ -545,7 +551,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ---- output
             ok = ok && tc::mbar_wait(&bars->o_full, iu & 1, a.status);
             tc::tc_fence_after();
-            for (int dp = 0; dp < 4; ++dp) {
+            for (int dp = x.dp0; dp < x.dp1; ++dp) {
                 float o[32];
                 tc::tmem_ld32(tl + kColB + dp * kH + hh * 32, o);
                 tc::tmem_ld_wait();
@@ -563,7 +569,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int i = 0; i < 32; ++i) pacc[(int64_t)(hh * 32 + i) * kDh] = o[i];
                 }
             }
-            if (a.part && et < kH) {
+            if (a.part && et < kH && x.dp0 == 0) {   // the value-block units of a slot share its (max, sum)
                 float *pml = a.part + a.nq * (int64_t)a.nseg * kH * kDh;
                 pml[(slot * kH + et) * 2] = mnat[et];
                 pml[(slot * kH + et) * 2 + 1] = znat[et];
@@ -677,6 +683,15 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.topk = a.topk;
     p.nseg = attend_tc_segments(a);
     p.seg_tiles = decode ? decode_seg_tiles(a) : kMaxTiles;
+    // decode units that leave most SMs idle split their value blocks over 2 or 4 CTAs (each recomputes the
+    // scores from the same key rows, an L2 hit after the first, and gathers and writes a part of the values)
+    p.dq_split = 1;
+    if (decode)
+        for (int s = 4; s >= 2; s /= 2)
+            if ((a.row1 - a.row0) * p.nseg * s <= num_sms()) {
+                p.dq_split = s;
+                break;
+            }
     p.sel = a.sel;
     p.pos = a.pos;
     p.scale = a.scale;
@@ -686,7 +701,7 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.q0 = a.row0;
     p.ent0 = a.ent0;
     p.no_window = a.no_window;
-    p.n_units = (a.row1 - a.row0) * p.nseg;
+    p.n_units = (a.row1 - a.row0) * p.nseg * p.dq_split;
     p.status = device_status_ptr();
     if (p.n_units <= 0) return HCSA_OK;
     const int64_t grid = p.n_units < num_sms() ? p.n_units : num_sms();
