@@ -145,6 +145,14 @@ __device__ __forceinline__ bool iter_next(const Args &a, Iter &it, Unit &x) {
     return false;
 }
 
+// c += a * b on two fp32 lanes at once (one packed FMA instruction)
+__device__ __forceinline__ void fma2(float &c0, float &c1, float a0, float a1, float b0, float b1) {
+    asm("{.reg .b64 ra, rb, rc; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; mov.b64 rc, {%0, %1};"
+        " fma.rn.f32x2 rc, ra, rb, rc; mov.b64 {%0, %1}, rc;}"
+        : "+f"(c0), "+f"(c1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 template <int HI, bool DEC, bool LP>
 __global__ void __launch_bounds__(cta_threads(DEC, LP), DEC ? kDecCtasPerSm : 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_qi,
@@ -421,9 +429,10 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 const int ab = iacc % a.nbuf;
                 ok = ok && tc::mbar_wait(&acc_full[ab], (iacc / a.nbuf) & 1, a.status);
                 tc::tc_fence_after();
-                float s[TPH];
+                // two partial sums per token, updated by packed FMAs (even / odd head of each pair)
+                float s[TPH], s1[TPH];
 #pragma unroll
-                for (int i = 0; i < TPH; ++i) s[i] = 0.f;
+                for (int i = 0; i < TPH; ++i) { s[i] = 0.f; s1[i] = 0.f; }
                 const uint32_t tl = tmem + ab * a.stride + ((uint32_t)(quad * 32) << 16);
                 // the head weights are read as float4 (the same address in every lane: a broadcast)
                 constexpr int LB = 1;
@@ -441,9 +450,11 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                             const float4 wq = wv[i4];
                             const float wl[4] = {wq.x, wq.y, wq.z, wq.w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
+                            for (int e = 0; e < 4; e += 2) {
                                 const int c = (c0 + l) * 32 + i4 * 4 + e;   // column within this group's 64
-                                s[c / HI < TPH ? c / HI : TPH - 1] += wl[e] * fmaxf(v[l][i4 * 4 + e], 0.f);
+                                const int ti = c / HI < TPH ? c / HI : TPH - 1;   // c, c + 1: the same token
+                                fma2(s[ti], s1[ti], wl[e], wl[e + 1], fmaxf(v[l][i4 * 4 + e], 0.f),
+                                     fmaxf(v[l][i4 * 4 + e + 1], 0.f));
                             }
                         }
                     }
@@ -451,6 +462,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_keys, const __grid
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
+#pragma unroll
+                for (int i = 0; i < TPH; ++i) s[i] += s1[i];
                 const int64_t j = (int64_t)kt * 128 + row;
 #pragma unroll
                 for (int i = 0; i < TPH; ++i)
