@@ -18,9 +18,13 @@
 //   exact softmax over all keys of the unit (per-head max / sum across lanes)
 //   P^T (bf16) -> shared memory as an MN-major operand
 //   O^T[dh, head] = V^T . P^T  4 blocks of 128 dh in columns [256, 512)
-// Prefill streams Q in 64-dim chunks next to the key chunks, so the scores of the next unit
-// (columns [0, 256)) accumulate while this unit's P V runs and its output drains; decode loads a
-// unit's whole query at once into the P region, which is free until the softmax writes P.
+// Decode writes all of P^T, then runs P V.  Prefill writes P^T one tile at a time into two 16 KB slots,
+// the window tile first (its score columns are the accumulator's), and P V of a tile starts as soon as
+// that tile is written; the smaller P region leaves room for 10 ring stages instead of 6.
+// Prefill streams Q in 64-dim chunks, each next to the key chunks of every tile (one pass over Q per
+// unit), so the scores of the next unit accumulate while this unit's output drains; tile 4, whose
+// columns the output accumulator reuses, starts once the drain is done.  Decode loads a unit's whole
+// query at once into the P region, which is free until the softmax writes P.
 //
 // Warp roles (persistent CTAs, 16 warps): warps 0-6 load (gathered entry rows and the decode window
 // ring with 16-byte cp.async whose completion arrives on the stage's mbarrier by itself; Q chunks and
@@ -40,11 +44,15 @@ constexpr int kDh = 512;
 constexpr int kC = 1024;
 constexpr int kKT = 128;          // keys per tile (MMA M)
 constexpr int kMaxTiles = 5;
-constexpr int kNS = 6;            // key/value ring stages (even: P V pairs sit in adjacent stages)
+// Key/value ring stages (even: P V pairs sit in adjacent stages).  Decode keeps all of P^T (and, until
+// the softmax, the whole query) in one 80 KB region; prefill keeps two 16 KB P^T tile slots, which
+// leaves room for more stages: more gathered bytes in flight per SM, which is what sets the gather rate.
+constexpr int ring_stages(bool dec) { return dec ? 6 : 10; }
+constexpr int kNSMax = 10;
 constexpr int kStage = 16384;     // 128 rows x 64 bf16
 constexpr int kGatherDepth = 4;   // gathered chunks in flight per producer thread
 constexpr int kQStage = kH * 128; // 64 heads x 64 bf16
-constexpr int kPBytes = kMaxTiles * kKT * 128;
+constexpr int p_bytes(bool dec) { return dec ? kMaxTiles * kKT * 128 : 2 * kKT * 128; }
 // The gather rate of cp.async grows with the number of warps issuing it, so most of the CTA's warps are
 // producers (the warps take 128 registers each either way).
 constexpr int kProdWarps = 7;
@@ -122,6 +130,11 @@ __device__ __forceinline__ int key_row(const Params &a, const Unit &x, int kk) {
 
 __device__ __forceinline__ uint32_t s_col(int t) { return t < 4 ? (uint32_t)(t * kH) : kColB; }
 
+// Tile of the i-th step of the P V phase.  Prefill hands P^T over tile by tile, and the first P V overwrites
+// the output accumulator's columns, which hold tile 4's scores: so the last tile goes first there.
+template <bool DEC>
+__device__ __forceinline__ int pv_tile(int i, int nt) { return DEC ? i : (i == 0 ? nt - 1 : i - 1); }
+
 template <bool kMax>
 __device__ __forceinline__ float warp_transpose_reduce32(float *v, int lane) {
     // 32 values per lane -> lane l holds the warp-wide reduction of value l
@@ -152,17 +165,20 @@ __device__ __forceinline__ const __nv_bfloat16 *key_ptr(const Params &a, const U
 }
 
 struct Bars {
-    uint64_t rf[kNS], re[kNS], qf[2], qe[2];
+    uint64_t rf[kNSMax], re[kNSMax], qf[2], qe[2];
     uint64_t s_full, s_free, p_full, o_full, o_free, fin;
+    uint64_t pt_full[2], pt_empty[2];   // prefill: P^T tile slots (written by the softmax, read by P V)
 };
 
+template <bool DEC>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ent,
                  const __grid_constant__ CUtensorMap tm_raw, Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sP = base;                         // P^T: 640 rows x 128 B
-    uint8_t *sRing = sP + kPBytes;              // kNS x 16 KB
+    constexpr int kNS = ring_stages(DEC);
+    uint8_t *sP = base;                         // P^T: 640 rows x 128 B (decode), 2 x 128 rows x 128 B (prefill)
+    uint8_t *sRing = sP + p_bytes(DEC);         // kNS x 16 KB
     uint8_t *sQ = sRing + kNS * kStage;         // 2 x 8 KB
     float *red = reinterpret_cast<float *>(sQ + 2 * kQStage);   // [4][64]
     float *mx = red + 4 * kH;                   // [64] scaled max
@@ -181,6 +197,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc::mbar_init(&bars->o_full, 1);
         tc::mbar_init(&bars->s_free, kSoftThreads / 32);
         tc::mbar_init(&bars->p_full, kSoftThreads / 32);
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&bars->pt_full[i], kSoftThreads / 32); tc::mbar_init(&bars->pt_empty[i], 1); }
         tc::mbar_init(&bars->o_free, kSoftThreads / 32);
         tc::mbar_init(&bars->fin, 1);
         tc::fence_mbar_init();
@@ -344,18 +361,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 ++iq;
             };
-            const int n1 = x.nt < 4 ? x.nt : 4;
-            for (int dc = 0; dc < 8; ++dc) {          // S phase 1: tiles 0..3
+            for (int dc = 0; dc < 8; ++dc) {          // S: every tile's key chunk next to its Q chunk
                 if (!a.decode) load_q(dc);
-                for (int t = 0; t < n1; ++t) load_chunk(t, dc * 64);
+                for (int t = 0; t < x.nt; ++t) load_chunk(t, dc * 64);
             }
-            if (x.nt == 5)
-                for (int dc = 0; dc < 8; ++dc) {      // S phase 2: tile 4
-                    if (!a.decode) load_q(dc);
-                    load_chunk(4, dc * 64);
-                }
-            for (int t = 0; t < x.nt; ++t)            // P V: value halves, 64-dh chunks in pairs
-                for (int c = 2 * x.dp0; c < 2 * x.dp1; ++c) load_chunk(t, kDh + c * 64);
+            for (int i = 0; i < x.nt; ++i)            // P V: value halves, 64-dh chunks in pairs
+                for (int c = 2 * x.dp0; c < 2 * x.dp1; ++c) load_chunk(pv_tile<DEC>(i, x.nt), kDh + c * 64);
         }
         tc::cp_async_wait_all();
         if (!ok && pt == 0) {
@@ -368,18 +379,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             uint32_t ic = 0, iq = 0, iu = 0;
+            uint32_t puse[2] = {0u, 0u};   // prefill: uses of each P^T tile slot so far
             for (int64_t u = blockIdx.x; u < a.n_units && ok; u += gridDim.x) {
                 const Unit x = unit_of(a, u);
                 if (x.nt <= 0) continue;
-                const int n1 = x.nt < 4 ? x.nt : 4;
                 if (iu >= 1) ok = ok && tc::mbar_wait(&bars->s_free, (iu - 1) & 1, a.status);
                 if (a.decode) ok = ok && tc::mbar_wait(&bars->qf[0], iu & 1, a.status);   // whole query in P
                 for (int dc = 0; dc < 8; ++dc) {
                     const int qb = iq & 1;
                     if (!a.decode) ok = ok && tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
                     const uint32_t qsm = a.decode ? P + dc * kQStage : Qs + qb * kQStage;
-                    for (int t = 0; t < n1; ++t, ++ic) {
+                    for (int t = 0; t < x.nt; ++t, ++ic) {
                         const int s = ic % kNS;
+                        // tile 4's scores share TMEM columns with the previous unit's output accumulator
+                        if (t == 4 && dc == 0 && iu >= 1) ok = ok && tc::mbar_wait(&bars->o_free, (iu - 1) & 1, a.status);
                         ok = ok && tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
                         tc::fence_async_smem();   // cp.async data (generic proxy) -> MMA (async proxy)
                         tc::tc_fence_after();
@@ -394,44 +407,37 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         ++iq;
                     }
                 }
-                if (x.nt == 5) {
-                    if (iu >= 1) ok = ok && tc::mbar_wait(&bars->o_free, (iu - 1) & 1, a.status);
-                    for (int dc = 0; dc < 8; ++dc, ++ic) {
-                        const int qb = iq & 1, s = ic % kNS;
-                        if (!a.decode) ok = ok && tc::mbar_wait(&bars->qf[qb], (iq >> 1) & 1, a.status);
-                        const uint32_t qsm = a.decode ? P + dc * kQStage : Qs + qb * kQStage;
-                        ok = ok && tc::mbar_wait(&bars->rf[s], (ic / kNS) & 1, a.status);
-                        tc::fence_async_smem();
-                        tc::tc_fence_after();
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            tc::mma_bf16(tmem + kColB, tc::sdesc_sw128(ring + s * kStage + 32 * k, 16, 1024),
-                                         tc::sdesc_sw128(qsm + 32 * k, 16, 1024), kIdescS, (dc | k) != 0);
-                        tc::mma_commit(&bars->re[s]);
-                        if (!a.decode) {
-                            tc::mma_commit(&bars->qe[qb]);
-                            ++iq;
-                        }
-                    }
-                }
                 tc::mma_commit(&bars->s_full);
-                ok = ok && tc::mbar_wait(&bars->p_full, iu & 1, a.status);
-                tc::tc_fence_after();
-                for (int t = 0; t < x.nt; ++t)
+                if (DEC) {   // all of P^T at once
+                    ok = ok && tc::mbar_wait(&bars->p_full, iu & 1, a.status);
+                    tc::tc_fence_after();
+                }
+                for (int i = 0; i < x.nt; ++i) {
+                    const int t = pv_tile<DEC>(i, x.nt);
+                    const int ps = i & 1;   // prefill: the P^T slot of step i
+                    if (!DEC) {
+                        ok = ok && tc::mbar_wait(&bars->pt_full[ps], puse[ps] & 1, a.status);
+                        tc::tc_fence_after();
+                    }
                     for (int dp = x.dp0; dp < x.dp1; ++dp, ic += 2) {
                         const int s0 = ic % kNS, s1 = (ic + 1) % kNS;
                         ok = ok && tc::mbar_wait(&bars->rf[s0], (ic / kNS) & 1, a.status);
                         ok = ok && tc::mbar_wait(&bars->rf[s1], ((ic + 1) / kNS) & 1, a.status);
                         tc::fence_async_smem();
                         tc::tc_fence_after();
-                        const uint32_t av = ring + s0 * kStage, bp = P + t * kKT * 128;
+                        const uint32_t av = ring + s0 * kStage, bp = P + (DEC ? t : ps) * kKT * 128;
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             tc::mma_bf16(tmem + kColB + dp * kH, tc::sdesc_sw128(av + 2048 * k, kStage, 1024),
-                                         tc::sdesc_sw128(bp + 2048 * k, kStage, 1024), kIdescPV, (t | k) != 0);
+                                         tc::sdesc_sw128(bp + 2048 * k, kStage, 1024), kIdescPV, (i | k) != 0);
                         tc::mma_commit(&bars->re[s0]);
                         tc::mma_commit(&bars->re[s1]);
                     }
+                    if (!DEC) {
+                        tc::mma_commit(&bars->pt_empty[ps]);
+                        ++puse[ps];
+                    }
+                }
                 tc::mma_commit(&bars->o_full);
                 ++iu;
             }
@@ -446,6 +452,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int r = quad * 32 + lane;                  // key row in a tile; dh row in an output block
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         uint32_t iu = 0;
+        uint32_t puse[2] = {0u, 0u};   // prefill: uses of each P^T tile slot so far
         for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
             // the softmax warps meet at named barriers within a unit: they leave the loop together
             ok = tc::named_bar_and(1, kSoftThreads, ok);
@@ -508,12 +515,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             float mloc[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) { mloc[i] = mx[hh * 32 + i]; v[i] = 0.f; }
-            for (int t = 0; t < x.nt; ++t) {
+            for (int i = 0; i < x.nt; ++i) {
+                const int t = pv_tile<DEC>(i, x.nt);
+                const int ps = i & 1;   // prefill: step i's tile goes to slot i % 2 once P V of step i - 2 has read it
+                if (!DEC && puse[ps] >= 1)
+                    ok = ok && tc::mbar_wait(&bars->pt_empty[ps], (puse[ps] - 1) & 1, a.status);
                 float s[32];
                 tc::tmem_ld32(tl + s_col(t) + hh * 32, s);
                 tc::tmem_ld_wait();
                 const bool vt = valid[t];
-                const uint32_t rowaddr = P + (uint32_t)(t * kKT + r) * 128u;
+                const uint32_t rowaddr = P + (uint32_t)((DEC ? t : ps) * kKT + r) * 128u;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     uint32_t w[4];
@@ -532,6 +543,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                  "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                                  : "memory");
                 }
+                if (!DEC) {   // this warp's part of the tile -> the MMA's async proxy; P V of tile t may start
+                    tc::fence_async_smem();
+                    tc::tc_fence_before();   // and its TMEM reads of the scores before P V writes those columns
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&bars->pt_full[ps]);
+                    ++puse[ps];
+                }
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -546,8 +564,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 znat[et] = Z;
             }
             tc::fence_async_smem();
-            tc::named_bar_sync(1, kSoftThreads);
-            if (lane == 0) tc::mbar_arrive(&bars->p_full);
+            tc::named_bar_sync(1, kSoftThreads);     // zinv / znat visible to every epilogue thread
+            if (DEC && lane == 0) tc::mbar_arrive(&bars->p_full);
             // ---- output
             ok = ok && tc::mbar_wait(&bars->o_full, iu & 1, a.status);
             tc::tc_fence_after();
@@ -588,8 +606,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
-constexpr size_t kSmemBytes = 1024 + kPBytes + kNS * kStage + 2 * kQStage + sizeof(float) * 8 * kH +
-                              sizeof(void *) * 2 * kMaxTiles * kKT + sizeof(Bars) + 16;
+constexpr size_t smem_bytes(bool dec) {
+    return 1024 + p_bytes(dec) + (size_t)ring_stages(dec) * kStage + 2 * kQStage + sizeof(float) * 8 * kH +
+           sizeof(void *) * 2 * kMaxTiles * kKT + sizeof(Bars) + 16;
+}
+static_assert(smem_bytes(false) <= 232448 && smem_bytes(true) <= 232448, "shared memory per CTA");
 
 int num_sms() {
     static int n = 0;
@@ -645,8 +666,10 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HCSA_ERR_CUDA;
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(attend_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes(true)) != cudaSuccess ||
+            cudaFuncSetAttribute(attend_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_bytes(false)) != cudaSuccess)
             return HCSA_ERR_CUDA;
         configured[dev] = true;
     }
@@ -705,7 +728,10 @@ hcsa_status launch_attend_tc(const AttendArgs &a, cudaStream_t st) {
     p.status = device_status_ptr();
     if (p.n_units <= 0) return HCSA_OK;
     const int64_t grid = p.n_units < num_sms() ? p.n_units : num_sms();
-    attend_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tq, te, tr, p);
+    if (decode)
+        attend_tc_kernel<true><<<(unsigned)grid, kThreads, smem_bytes(true), st>>>(tq, te, tr, p);
+    else
+        attend_tc_kernel<false><<<(unsigned)grid, kThreads, smem_bytes(false), st>>>(tq, te, tr, p);
     count_launch();
     return check_launch();
 }
