@@ -64,6 +64,10 @@ def peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum = 1076.9 MB (7 producer warps); linear in T.
 ATTEND_TC_DRAM_BYTES_PER_TOKEN = 1076.9e6 / 8192
 
+# Rate at which 148 CTAs gather random 128-byte row segments into shared memory with 16-byte cp.async,
+# measured on this B200 (the same for tables of 32 to 256 MB).
+GATHER_CEILING_GBS = 7340.0
+
 
 def prefill_work(spec):
     """Algorithmic flops / bytes of each call of a prefill layer (visible pairs only)."""
@@ -371,11 +375,12 @@ def run_prefill(args, spec_name, ws, rank, lowprec=False):
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_sus, "unit": "TFLOP/s", "frac": ach / tc_sus,
                 "traffic": traffic, "kernel": dom, "peak_kind": f"{src} bf16 sustained"}
         if dom == "attend" and spec.kind == "csa":
-            # what binds this kernel: gathered 128-byte segments of entry rows, against the gather rate a
-            # microbenchmark measured on this B200 for a table of the entries' size (16-byte cp.async,
-            # 148 CTAs: 9.6 TB/s up to 32 MB, 4.6 TB/s at 64 MB, 3.6 TB/s from 256 MB)
+            # the kernel's gathered 128-byte segments of entry rows, against the rate a microbenchmark
+            # measured on this B200 for random 128-byte segments moved by 16-byte cp.async into a
+            # swizzled ring (148 CTAs, row indices from shared memory): 7.33-7.35 TB/s for any table
+            # size from 32 to 256 MB
             ent_mb = -(-spec.T // spec.m) * spec.C * (1 if lowprec else 2) / 2 ** 20
-            ceiling = 9600.0 if ent_mb <= 32 else 4600.0 if ent_mb <= 64 else 3600.0
+            ceiling = GATHER_CEILING_GBS
             t = np.arange(spec.T, dtype=np.float64)
             rows = np.minimum(np.minimum(t // spec.m, -(-spec.T // spec.m)), spec.topk).sum()
             gathered = rows * spec.C * (1 + 1 / 32 if lowprec else 2)
