@@ -61,8 +61,8 @@ def peaks():
 
 # DRAM bytes per query token of the tensor-core attention kernel (query rows in, output rows out; the
 # gathered key/value rows are served by L2), from an ncu capture of the same kernel at T=8192 with
-# dram__bytes_read.sum + dram__bytes_write.sum = 1076.9 MB (7 producer warps); linear in T.
-ATTEND_TC_DRAM_BYTES_PER_TOKEN = 1076.9e6 / 8192
+# dram__bytes_read.sum + dram__bytes_write.sum = 576.9 + 499.8 MB; linear in T.
+ATTEND_TC_DRAM_BYTES_PER_TOKEN = 1076.7e6 / 8192
 
 # Rate at which 148 CTAs gather random 128-byte row segments into shared memory with 16-byte cp.async,
 # measured on this B200 (the same for tables of 32 to 256 MB).
