@@ -21,6 +21,9 @@ HCA_F32 = HCA_SMALL.replace(dtype="f32", T=700, seed=24)
 CSA_TC_K128 = synth.LayerSpec(kind="csa", T=900, D=256, m=4, width=8, C=1024, di=64, Hi=8, topk=128, window=128,
                               H=64, dh=512, scale=512 ** -0.5, dtype="bf16", seed=41)
 CSA_TC_K512 = CSA_TC_K128.replace(T=2600, topk=512, seed=42)
+# the same kernel over a dense entry list (64 heads of 512, pools of 8): units of 1 to 5 tiles as t grows
+HCA_TC_DENSE = synth.LayerSpec(kind="hca", T=3500, D=128, m=8, width=8, C=1024, window=128, H=64, dh=512,
+                               scale=512 ** -0.5, dtype="bf16", seed=46)
 
 CASES = {
     "csa_f32_t2048": synth.PREFILL["csa_f32_t2048"],
@@ -37,9 +40,14 @@ CASES = {
     "csa_bf16_tc_k128": CSA_TC_K128,
     "csa_bf16_tc_k512": CSA_TC_K512,
     "csa_bf16_tc_t5": CSA_TC_K128.replace(T=5, seed=43),
+    # units of 3 and 4 tiles (the window tile is the last one, outside the output accumulator's columns)
+    "csa_bf16_tc_k256": CSA_TC_K128.replace(T=1400, topk=256, seed=44),
+    "csa_bf16_tc_k384": CSA_TC_K128.replace(T=2000, topk=384, seed=45),
+    "hca_bf16_tc_dense": HCA_TC_DENSE,
 }
 # query rows checked per case (default: all)
-SAMPLED = {"csa_bf16_tc_k128": 48, "csa_bf16_tc_k512": 48}
+SAMPLED = {"csa_bf16_tc_k128": 48, "csa_bf16_tc_k512": 48, "csa_bf16_tc_k256": 48, "csa_bf16_tc_k384": 48,
+           "hca_bf16_tc_dense": 64}
 
 
 def run_gpu(spec):
@@ -97,7 +105,8 @@ def test_prefill_parity(name):
     inp, layer = run_gpu(spec)
     rows = np.arange(spec.T, dtype=np.int64)
     if name in SAMPLED:
-        rows = sample_rows(spec.T, spec.m, spec.topk, n_random=SAMPLED[name], seed=spec.seed)
+        # dense layers: rows around the first change of tile count (t = 128 m) stand in for the top-k crossing
+        rows = sample_rows(spec.T, spec.m, spec.topk or 128, n_random=SAMPLED[name], seed=spec.seed)
     ref = oracle.prefill(spec, inp, rows=rows)
     compare(spec, inp, layer, rows, ref)
 
