@@ -86,12 +86,14 @@ class PrefillLayer:
     def index_topk(self):
         L.csa_index_topk(self.p, self.view("qi"), self.view("w"), self.idx_keys, self.sel, self.ws_index)
 
-    def attend(self, sel=None):
+    def attend(self, sel=None, p=None):
+        """Attention for all rows, or for the row range of `p` (params with row0 / row1 set)."""
+        p = self.p if p is None else p
         if self.csa:
-            L.csa_attend(self.p, self.view("q"), self.view("kv"), self.entries, self.sel if sel is None else sel,
+            L.csa_attend(p, self.view("q"), self.view("kv"), self.entries, self.sel if sel is None else sel,
                          self.out, self.ws_attend)
         else:
-            L.hca_attend(self.p, self.view("q"), self.view("kv"), self.entries, self.out, self.ws_attend)
+            L.hca_attend(p, self.view("q"), self.view("kv"), self.entries, self.out, self.ws_attend)
 
     def project_compress(self, x, W_cat, bias):
         """The projection with the compressor in its epilogue (one GEMM + a seam pass for CSA layers).  Same
@@ -106,6 +108,45 @@ class PrefillLayer:
             self.index_topk()
         self.attend()
         return self.out
+
+    def forward_host(self, x_host, W_cat, bias, out_host, chunks=8):
+        """forward() with the input x and the output in (pinned) host memory.
+
+        The attention runs in at most `chunks` row ranges (multiples of 128 rows), and each range's output
+        rows go back on a copy stream as soon as they are written, so the device-to-host copy overlaps the
+        rest of the attention.  The copies of one call also overlap the next call's input copy, projection,
+        compressor and indexer; only its attention, which rewrites `out`, waits for them.  Call wait_host()
+        before reading out_host."""
+        T = self.spec.T
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream(device=self.y.device)
+            self._x = torch.empty(x_host.shape, dtype=x_host.dtype, device=self.y.device)
+            self._copied = None
+        cur = torch.cuda.current_stream(self.y.device)
+        self._x.copy_(x_host, non_blocking=True)
+        self.project(self._x, W_cat)
+        self.compress(bias)
+        if self.csa:
+            self.index_topk()
+        if self._copied is not None:
+            cur.wait_event(self._copied)   # the previous call's copies have read `out`
+        step = -(-max(1, -(-T // max(1, chunks))) // 128) * 128   # row ranges start on 128-row boundaries
+        for a in range(0, T, step):
+            b = min(T, a + step)
+            self.attend(p=params_for(self.spec, row0=a, row1=b, lowprec=self.lowprec))
+            done = torch.cuda.Event()
+            done.record(cur)
+            self._copy_stream.wait_event(done)
+            with torch.cuda.stream(self._copy_stream):
+                out_host[a:b].copy_(self.out[a:b], non_blocking=True)
+        self._copied = torch.cuda.Event()
+        self._copied.record(self._copy_stream)
+        return out_host
+
+    def wait_host(self):
+        """Make the current stream wait for the output copies of the last forward_host() call."""
+        if getattr(self, "_copied", None) is not None:
+            torch.cuda.current_stream(self.y.device).wait_event(self._copied)
 
 
 class DecodeLayer:

@@ -157,3 +157,26 @@ def test_fused_projection_compressor_matches_separate_calls(name, lowprec):
         assert torch.equal(a.entries, b.entries), T
         if sp.kind == "csa":
             assert torch.equal(a.idx_keys, b.idx_keys), T
+
+
+@pytest.mark.parametrize("name,chunks", [("csa_bf16_tc_k512", 3), ("csa_bf16_tc_t5", 8), ("hca_bf16_tc_dense", 5),
+                                         ("csa_bf16_small", 7), ("hca_bf16_small", 8)])
+def test_forward_host_matches_forward(name, chunks):
+    """The host-buffer call (attention by row ranges, output rows copied back on a second stream) returns
+    the device call's output; a second call, whose attention waits for the first call's copies, too.
+    Per-token attention kernels are bit-exact by range; the HCA kernel for dh = 128 tiles the window from
+    each query block's first token, so a range boundary inside a block may change rounding by an ulp."""
+    spec = CASES[name]
+    inp, layer = run_gpu(spec)
+    ref = layer.out.detach().cpu().clone()
+    W, B = dev(inp["W_cat"]), dev(inp["B"])
+    xh = dev(inp["x"]).cpu().pin_memory()
+    for _ in range(2):
+        oh = torch.full(tuple(layer.out.shape), float("nan"), dtype=layer.out.dtype).pin_memory()
+        layer.forward_host(xh, W, B, oh, chunks=chunks)
+        layer.wait_host()
+        torch.cuda.synchronize()
+        if spec.kind == "hca" and spec.dh == 128:
+            torch.testing.assert_close(oh.float(), ref.float(), rtol=2 ** -7, atol=2 ** -9)
+        else:
+            assert torch.equal(oh, ref)
