@@ -461,7 +461,7 @@ def run_decode(args, spec_name, ws, rank, lowprec=False):
     stream = torch.cuda.current_stream()
     xw = torch.empty_like(xs)   # the residual stream of a chained stack (restarts from xs every step)
 
-    def step():
+    def step(xw=xw):
         if d.residual:
             xw.copy_(xs)
             for L, W, B, Wo in zip(layers, Ws, Bs, Wos):
@@ -503,21 +503,49 @@ def run_decode(args, spec_name, ws, rank, lowprec=False):
     ach = total_bytes / (us / 1e6) / 1e9
     roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
             "kernel": "whole decode step (CUDA graph)", "peak_kind": f"{src} hbm"}
+    # End to end: the step's input from pinned host memory and its result (the hidden state of a chained
+    # stack, else the last layer's output) back to pinned host memory, every step.  The result buffer is
+    # double-buffered (a second graph writes the other one), so step i's copy back overlaps step i + 1;
+    # the replay of step i + 2 waits for it.
     xh = torch.empty(xs.shape, dtype=xs.dtype, pin_memory=True)
     xh.copy_(xs)
-    result = xw if d.residual else layers[-1].out   # the step's result: hidden state or last layer's output
-    oh = torch.empty(result.shape, dtype=result.dtype, pin_memory=True)
+    if d.residual:
+        res = (xw, torch.empty_like(xw))
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2):
+            step(res[1])
+    else:
+        res = (layers[-1].out, torch.empty_like(layers[-1].out))
+        layers[-1].out = res[1]
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2):
+            step()
+        layers[-1].out = res[0]
+    graphs = (g, g2)
+    oh = torch.empty(res[0].shape, dtype=res[0].dtype, pin_memory=True)
+    cs = torch.cuda.Stream()
+    copied = [None, None]
     torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        k = i & 1
         xs.copy_(xh, non_blocking=True)
-        g.replay()
-        oh.copy_(result, non_blocking=True)
+        if copied[k] is not None:
+            stream.wait_event(copied[k])
+        graphs[k].replay()
+        done = torch.cuda.Event()
+        done.record(stream)
+        cs.wait_event(done)
+        with torch.cuda.stream(cs):
+            oh.copy_(res[k], non_blocking=True)
+        copied[k] = torch.cuda.Event()
+        copied[k].record(cs)
+    stream.wait_stream(cs)
     a1.record(stream)
     torch.cuda.synchronize()
     eus = max_over_ranks(a0.elapsed_time(a1), ws) / args.steps * 1e3
-    del g
+    del g, g2, graphs
     line = {"metric": METRIC, "value": us, "unit": "us/step", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) caches and inputs)",
