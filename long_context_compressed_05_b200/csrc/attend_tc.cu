@@ -30,8 +30,9 @@
 // ring with 16-byte cp.async whose completion arrives on the stage's mbarrier by itself; Q chunks and
 // the prefill window tile -- 128 consecutive raw rows -- with TMA box loads), warp 7 issues the MMAs,
 // warps 8..15 run the softmax and the output epilogue (two warps per TMEM lane quadrant, 32 heads
-// each).  Gathered 128-byte row segments are what bounds this kernel: the gather rate per SM, not the
-// tensor core, sets its speed, and that rate grows with the number of warps issuing the copies.
+// each).  The producers' copy path bounds this kernel: without its MMAs, softmax arithmetic and output
+// stores it keeps 82% of its time, and gathering from a few hot rows instead is no faster; its rate
+// grows with the number of warps issuing the copies.
 #include "lowprec.cuh"
 #include "tc_common.cuh"
 
@@ -46,7 +47,7 @@ constexpr int kKT = 128;          // keys per tile (MMA M)
 constexpr int kMaxTiles = 5;
 // Key/value ring stages (even: P V pairs sit in adjacent stages).  Decode keeps all of P^T (and, until
 // the softmax, the whole query) in one 80 KB region; prefill keeps two 16 KB P^T tile slots, which
-// leaves room for more stages: more gathered bytes in flight per SM, which is what sets the gather rate.
+// leaves room for 10 stages (6, 8 and 10 measured the same: the stage count is not what limits it).
 constexpr int ring_stages(bool dec) { return dec ? 6 : 10; }
 constexpr int kNSMax = 10;
 constexpr int kStage = 16384;     // 128 rows x 64 bf16
