@@ -9,7 +9,7 @@ import torch
 
 from . import _lib as L
 
-__all__ = ["params_for", "torch_dtype", "PrefillLayer", "DecodeLayer"]
+__all__ = ["params_for", "torch_dtype", "row_ranges", "PrefillLayer", "DecodeLayer"]
 
 
 def torch_dtype(dtype: str):
@@ -23,6 +23,13 @@ def params_for(spec, *, T=None, B=1, n_cap=0, row0=0, row1=0, lowprec=False, ent
                          di=getattr(spec, "di", 0), Hi=getattr(spec, "Hi", 0), topk=getattr(spec, "topk", 0),
                          window=spec.window, H=spec.H, dh=spec.dh, scale=spec.scale, dtype=spec.dtype, B=B,
                          n_cap=n_cap, row0=row0, row1=row1, lowprec=lowprec, ent0=ent0, ent_shard=ent_shard)
+
+
+def row_ranges(T, chunks):
+    """At most `chunks` contiguous row ranges covering [0, T), each starting on a 128-row boundary (the
+    prefill calls' row-range rule)."""
+    step = -(-max(1, -(-T // max(1, chunks))) // 128) * 128
+    return [(a, min(T, a + step)) for a in range(0, T, step)]
 
 
 def _col_offsets(spec):
@@ -130,9 +137,7 @@ class PrefillLayer:
             self.index_topk()
         if self._copied is not None:
             cur.wait_event(self._copied)   # the previous call's copies have read `out`
-        step = -(-max(1, -(-T // max(1, chunks))) // 128) * 128   # row ranges start on 128-row boundaries
-        for a in range(0, T, step):
-            b = min(T, a + step)
+        for a, b in row_ranges(T, chunks):
             self.attend(p=params_for(self.spec, row0=a, row1=b, lowprec=self.lowprec))
             done = torch.cuda.Event()
             done.record(cur)
